@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200 through libkda's C ABI.
+
+A *step* is one pass of the prefill hot path over the K3-layer-shaped
+workload: ``kda_prologue`` (short conv + SiLU + L2 over 32768 tokens x 96
+heads x 128 channels of q/k/v projections) followed by ``kda_chunk_fwd``
+(chunkwise prefill, chunk 64, fp32 state).  ``value`` is prefill tokens/s
+(a token is one position through all 96 heads) with inputs resident in HBM.
+The batched decode step (256 sequences x 96 heads, 100 consecutive steps,
+state updated in place) is timed in the same run and reported under
+``decode``.
+
+Usage: ``python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]``.
+With N > 1 launch one process per GPU (torchrun); every rank runs its own
+replica of the workload (the problems are independent: no collective on the
+data path) and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import resource
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s & decode tokens/s at H=96,d=128 on 1 B200; % of roofline"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+# Algorithmic work per token-head (d = 128; see the design notes).
+D_ = 128
+QKV_DT = 4                                          # q/k/v handed from prologue to chunk: f32
+PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/k/v      = 2304
+CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 2564
+FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
+CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
+# decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
+DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
+
+KERNEL_SOURCES = {
+    "kda_prologue": "gated_delta_rule_prologue_b200/csrc/kda_prologue.cu",
+    "kda_chunk_fwd": "gated_delta_rule_prologue_b200/csrc/kda_chunk_simt.cu",
+    "kda_decode_step": "gated_delta_rule_prologue_b200/csrc/kda_decode.cu",
+}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(
+            p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def src_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = src_sha(KERNEL_SOURCES[kernel])
+    for line in open(path):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
+        if kv.get("kernel") == kernel and kv.get("src_sha256") == sha:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.rows = []
+        self.sel = []
+        try:
+            props = torch.cuda.get_device_properties(device)
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                u = str(uuid)
+                self.sel = ["-i", u if u.startswith("GPU-") else "GPU-" + u]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        sm, mx, reasons = [], [], set()
+        for line in self.tmp.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.tmp.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def roofline(bound, algo, ms, peak, unit, traffic):
+    achieved = algo / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(n_tokens):
+    """The float64 oracle on the first ``n_tokens`` tokens of the K3-layer
+    workload, all 96 heads (prologue + recurrence).  Returns (seconds, cores)."""
+    import numpy as np
+    from oracle import kda_recurrent, prologue
+    c = W.WORKLOADS["k3_prefill"]
+    H, D = c["H"], c["D"]
+    heads = [W.k3_prefill_head(h, T=n_tokens) for h in range(H)]
+    x = torch.stack([hh[0] for hh in heads], dim=2).reshape(n_tokens, 3 * H * D)
+    w = torch.stack([hh[1] for hh in heads], dim=1).reshape(3 * H * D, 4)
+    g = torch.stack([hh[2] for hh in heads], dim=1)
+    beta = torch.stack([hh[3] for hh in heads], dim=1)
+    r0 = resource.getrusage(resource.RUSAGE_SELF)
+    t0 = time.perf_counter()
+    q, k, v, _ = prologue(x, w, H, D)
+    o, _ = kda_recurrent(q, k, v, g, beta, 1.0)
+    wall = time.perf_counter() - t0
+    r1 = resource.getrusage(resource.RUSAGE_SELF)
+    cpu = (r1.ru_utime - r0.ru_utime) + (r1.ru_stime - r0.ru_stime)
+    assert np.all(np.isfinite(o))
+    return wall, max(1, round(cpu / wall))
+
+
+def cpu_baseline(n_tokens=1024):
+    wall, cores = oracle_sample(n_tokens)
+    return {"value": round(n_tokens / wall, 3), "unit": "tokens/s", "cores": cores,
+            "host_cores_available": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"first {n_tokens} tokens of the K3-layer prefill, all 96 heads "
+                      f"(prologue + token-by-token recurrence, float64 NumPy), {wall:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    budget_s = 150.0
+    per_token_s = 0.011
+    n_tok = int(max(16, min(1024, budget_s / max(1, args.steps + args.warmup) / per_token_s)))
+    for _ in range(args.warmup):
+        oracle_sample(n_tok)
+    times, cores = [], 1
+    for _ in range(args.steps):
+        wall, cores = oracle_sample(n_tok)
+        times.append(wall)
+    ms = 1e3 * statistics.mean(times)
+    value = n_tok / (ms * 1e-3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "k3_prefill sample: first %d tokens x 96 heads x d=128 "
+                               "(prologue + recurrence)" % n_tok},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"first {n_tok} tokens of the K3-layer prefill per step"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import gated_delta_rule_prologue_b200 as kda
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm, bf16_burst, bf16_sust, peak_kind = peaks()
+
+    # ---- prefill workload (inputs resident in HBM) ----
+    inp = W.k3_prefill(pin_memory=True)
+    T, H, D = inp.T, inp.H, inp.D
+    x = inp.x.to(dev)
+    w = inp.conv_w.to(dev)
+    g = inp.g.to(dev)
+    beta = inp.beta.to(dev)
+    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    k, v, o = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
+                          chunk=inp.chunk, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
+        ev[i][1].record(stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
+                          chunk=inp.chunk, stream=stream)
+        ev[i][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(start.elapsed_time(end), world)
+    ms_step = total_ms / args.steps
+    pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    chk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    assert kda.kda_get_device_status() == 0
+    value = world * T / (ms_step * 1e-3)
+    launches = 2 * args.steps
+
+    th = T * H
+    kernels = {
+        "kda_prologue": dict(ms=round(pro_ms, 4), **roofline(
+            "hbm", PROLOGUE_BYTES_PER_TH * th, pro_ms, hbm, "GB/s", recorded_traffic("kda_prologue"))),
+        "kda_chunk_fwd": dict(ms=round(chk_ms, 4), **roofline(
+            "hbm", CHUNK_BYTES_PER_TH * th, chk_ms, hbm, "GB/s", recorded_traffic("kda_chunk_fwd"))),
+    }
+    kernels["kda_chunk_fwd"]["tensor_tflops"] = round(CHUNK_FLOPS_PER_TH * th / (chk_ms * 1e-3) / 1e12, 2)
+    dominant = max(kernels, key=lambda n: kernels[n]["ms"])
+    roof = {k_: kernels[dominant][k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roof["kernel"] = dominant
+    roof["peak_source"] = f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+    fused_floor_ms = 1e3 * FUSED_BYTES_PER_TH * th / (hbm * 1e9)
+
+    # ---- end to end through the C ABI with host buffers ----
+    out_host = torch.empty((T, H, D), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(1, args.e2e_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(inp.x, non_blocking=True)
+        g.copy_(inp.g, non_blocking=True)
+        beta.copy_(inp.beta, non_blocking=True)
+        step()
+        out_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = inp.x.numel() * 2 + inp.g.numel() * 4 + inp.beta.numel() * 4
+    d2h = out_host.numel() * 4
+    del x, q, k, v, o, g, beta, inp
+    torch.cuda.empty_cache()
+
+    # ---- batched decode: 256 sequences x 96 heads, consecutive steps ----
+    dinp = W.decode256(steps=args.decode_steps)
+    Nd, Hd, Dd = dinp.N, dinp.H, dinp.D
+    state = dinp.state.to(dev)
+    cache = dinp.conv_cache.to(dev)
+    dw = dinp.conv_w.to(dev)
+    dx, dg, db = dinp.x.to(dev), dinp.g.to(dev), dinp.beta.to(dev)
+    do = torch.empty((Nd, Hd, Dd), dtype=torch.float32, device=dev)
+    for s in range(min(3, args.decode_steps)):
+        kda.kda_decode_step(dx[s], dw, cache, dg[s], db[s], state, do, H=Hd, D=Dd,
+                            scale=dinp.scale, stream=stream)
+    torch.cuda.synchronize(dev)
+    dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+              for _ in range(args.decode_steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for s in range(args.decode_steps):
+        dev_ev[s][0].record(stream)
+        kda.kda_decode_step(dx[s], dw, cache, dg[s], db[s], state, do, H=Hd, D=Dd,
+                            scale=dinp.scale, stream=stream)
+        dev_ev[s][1].record(stream)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world)
+    assert kda.kda_get_device_status() == 0
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / args.decode_steps
+    dec_kernel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in dev_ev)
+    decode = {
+        "metric": "decode tokens/s", "unit": "tokens/s",
+        "value": round(world * Nd / (dec_ms * 1e-3), 1),
+        "ms_per_step": round(dec_ms, 4), "steps": args.decode_steps,
+        "workload": "decode256: 256 sequences x 96 heads x d=128, fp32 state in place, "
+                    "bf16 projections with conv cache",
+        "roofline": dict(roofline("hbm", DECODE_BYTES_PER_SH * Nd * Hd, dec_kernel_ms, hbm,
+                                  "GB/s", recorded_traffic("kda_decode_step")),
+                         kernel="kda_decode_step"),
+    }
+    launches_total = launches
+    del state, cache, dx, dg, db
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "k3_prefill: kda_prologue + kda_chunk_fwd over T=32768 tokens, H=96, "
+                        "d_k=d_v=128, chunk 64, bf16 q/k/v projections, fp32 g/beta/state/o",
+            "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
+            "parallelism": f"replicas x{world} (independent problems, no collective)",
+            "l2": "inputs larger than L2 (15.3 GB touched per step, no flush needed)",
+        },
+        "roofline": roof,
+        "kernels": kernels,
+        "fused_hbm_floor_ms": round(fused_floor_ms, 4),
+        "decode": decode,
+        "e2e": {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_total,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_tokens)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup(args) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

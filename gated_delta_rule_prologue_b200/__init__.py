@@ -1,0 +1,171 @@
+"""Python binding of libkda (KDA recurrence hot path for B200 / sm_100a).
+
+Argument marshalling only: every function hands raw device pointers, sizes
+and the current CUDA stream of ``torch`` to the C ABI declared in
+``include/kda.h`` and raises :class:`KdaError` on a non-OK status.  All work
+runs in the library's CUDA kernels; there is no other implementation behind
+these names, and importing fails loudly when ``libkda.so`` has not been built
+(``python -m gated_delta_rule_prologue_b200.build``).
+
+Tensor conventions (all contiguous, on the current CUDA device):
+  q, k, v              [T, H, D]       float32 or bfloat16
+  o                    [T, H, D]       float32 (read-outs are always float32)
+  g                    [T, H, Dk]      float32 (log-decay, alpha = exp(g))
+  beta                 [T, H]          float32
+  state                [N, H, Dv, Dk]  float32 (key index contiguous)
+  x (projections)      [T, 3*H*D]      activation dtype, channel p*H*D + h*D + d
+  conv_w               [3*H*D, 4]      float32
+  conv cache           [N, 3, 3*H*D]   activation dtype, oldest row first
+  cu_seqlens           [N+1]           int32
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "KdaError",
+    "LIB_PATH",
+    "lib",
+    "kda_prologue",
+    "kda_chunk_fwd",
+    "kda_decode_step",
+    "kda_get_device_status",
+    "kda_version",
+    "KDA_OK",
+    "KDA_ERR_INVALID_ARG",
+    "KDA_ERR_UNSUPPORTED",
+    "KDA_ERR_CUDA",
+    "KDA_ERR_DEVICE_TIMEOUT",
+    "KDA_ERR_DEVICE_BOUNDS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_CUDA = 3
+KDA_ERR_DEVICE_TIMEOUT = 4
+KDA_ERR_DEVICE_BOUNDS = 5
+_F32, _BF16 = 0, 1
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libkda status {status}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m gated_delta_rule_prologue_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+lib.kda_prologue.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                             _vp]
+lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                              _i, _vp, _vp, _vp]
+lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
+lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_decode_step, lib.kda_get_device_status):
+    _fn.restype = ctypes.c_int
+lib.kda_last_error.restype = ctypes.c_char_p
+lib.kda_last_error.argtypes = []
+lib.kda_version.restype = ctypes.c_char_p
+lib.kda_version.argtypes = []
+
+
+def _check(status: int):
+    if status != KDA_OK:
+        raise KdaError(status, lib.kda_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype(t) -> int:
+    if t.dtype == torch.float32:
+        return _F32
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    raise TypeError(f"unsupported activation dtype {t.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None):
+    if t is None:
+        return
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def kda_version() -> str:
+    return lib.kda_version().decode()
+
+
+def kda_get_device_status() -> int:
+    """Read and clear the current device's status word (0 = no fault)."""
+    code = ctypes.c_int(0)
+    _check(lib.kda_get_device_status(ctypes.byref(code)))
+    return code.value
+
+
+def kda_prologue(x, conv_w, q, k, v, *, H: int, D: int, cache_in=None, cache_out=None,
+                 cu_seqlens=None, stream=None):
+    """Short conv + SiLU + L2 on q/k: writes ``q, k, v`` [T, H, D] (and ``cache_out``).
+    ``x`` and the caches share one dtype; ``q, k, v`` share another."""
+    for t, n in ((x, "x"), (cache_in, "cache_in"), (cache_out, "cache_out")):
+        _need(t, n, x.dtype)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(conv_w, "conv_w", torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    T = x.shape[0]
+    _check(lib.kda_prologue(_ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out),
+                            _ptr(cu_seqlens), N, T, H, D, _dtype(x), _dtype(q), _ptr(q),
+                            _ptr(k), _ptr(v), _stream(stream)))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None,
+                  final_state=None, cu_seqlens=None, chunk: int = 64, stream=None):
+    """Chunkwise prefill: writes ``o`` [T, H, Dv] and optionally ``final_state``."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                             _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
+                             _dtype(q), _ptr(o), _ptr(final_state), _stream(stream)))
+
+
+def kda_decode_step(x, conv_w, conv_cache, g, beta, state, o, *, H: int, D: int,
+                    scale: float = 1.0, stream=None):
+    """One decode token per sequence; updates ``state`` and ``conv_cache`` in place."""
+    for t, n in ((x, "x"), (conv_cache, "conv_cache")):
+        _need(t, n, x.dtype)
+    for t, n in ((o, "o"), (conv_w, "conv_w"), (g, "g"), (beta, "beta"), (state, "state")):
+        _need(t, n, torch.float32)
+    N = x.shape[0]
+    _check(lib.kda_decode_step(_ptr(x), _ptr(conv_w), _ptr(conv_cache), _ptr(g), _ptr(beta),
+                               float(scale), _ptr(state), N, H, D, _dtype(x), _ptr(o),
+                               _stream(stream)))

@@ -1,0 +1,227 @@
+// Host side of the libkda C ABI: argument validation, the per-device status
+// word, error reporting and dispatch to the kernels.  No entry point
+// allocates memory per call.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "kda_common.cuh"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+kda_status fail(kda_status code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+kda_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int *g_status[kMaxDevices] = {nullptr};
+
+// The status word of the current device, allocated (and zeroed) on first use.
+kda_status device_status_word(int **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (g_status[dev] == nullptr) {
+    int *p = nullptr;
+    e = cudaMalloc(&p, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status word)");
+    e = cudaMemset(p, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
+    g_status[dev] = p;
+  }
+  *out = g_status[dev];
+  return KDA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  auto pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+size_t esize(kda_dtype dt) { return dt == KDA_BF16 ? 2 : 4; }
+
+bool valid_dtype(kda_dtype dt) { return dt == KDA_F32 || dt == KDA_BF16; }
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+#define KDA_REQUIRE(cond, ...) \
+  do {                         \
+    if (!(cond)) return fail(KDA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define KDA_REQUIRE_PTR(p, name)                                                    \
+  do {                                                                              \
+    if ((p) == nullptr) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", name);       \
+    if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+#define KDA_OPT_PTR(p, name)                                                        \
+  do {                                                                              \
+    if ((p) != nullptr && !aligned16(p))                                            \
+      return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);          \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_last_error(void) { return g_last_error.c_str(); }
+
+const char *kda_version(void) { return "libkda 0.1 (sm_100a)"; }
+
+kda_status kda_get_device_status(int *code) {
+  KDA_REQUIRE(code != nullptr, "code is NULL");
+  int *word = nullptr;
+  kda_status st = device_status_word(&word);
+  if (st != KDA_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int host = 0;
+  e = cudaMemcpy(&host, word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status word)");
+  e = cudaMemset(word, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
+  *code = host;
+  return KDA_OK;
+}
+
+kda_status kda_prologue(const void *x, const float *conv_w, const void *cache_in,
+                        void *cache_out, const int32_t *cu_seqlens, int N, int T, int H,
+                        int D, kda_dtype dt, kda_dtype out_dt, void *q, void *k, void *v,
+                        kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(valid_dtype(out_dt), "unknown output dtype %d", (int)out_dt);
+  KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1 && D >= 1, "bad sizes N=%d T=%d H=%d D=%d", N, T, H, D);
+  KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
+  if (!supported_d(D)) return fail(KDA_ERR_UNSUPPORTED, "prologue: D=%d not in {16,32,64,128}", D);
+  KDA_REQUIRE((long long)H * D * 3 < (1LL << 31), "3*H*D too large");
+  if (T > 0) {
+    KDA_REQUIRE_PTR(x, "x");
+    KDA_REQUIRE_PTR(q, "q");
+    KDA_REQUIRE_PTR(k, "k");
+    KDA_REQUIRE_PTR(v, "v");
+  }
+  KDA_REQUIRE_PTR(conv_w, "conv_w");
+  KDA_OPT_PTR(cache_in, "cache_in");
+  KDA_OPT_PTR(cache_out, "cache_out");
+  KDA_OPT_PTR(cu_seqlens, "cu_seqlens");
+  const size_t C = (size_t)3 * H * D, es = esize(dt);
+  const size_t act = (size_t)T * H * D * esize(out_dt), cache_bytes = (size_t)N * 3 * C * es;
+  KDA_REQUIRE(!overlaps(cache_in, cache_bytes, cache_out, cache_bytes),
+              "cache_out overlaps cache_in");
+  const void *outs[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    KDA_REQUIRE(!overlaps(outs[i], act, x, (size_t)T * C * es), "output overlaps x");
+    for (int j = i + 1; j < 3; ++j)
+      KDA_REQUIRE(!overlaps(outs[i], act, outs[j], act), "q/k/v outputs overlap");
+  }
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaError_t e = kda::launch_prologue(x, conv_w, cache_in, cache_out, cu_seqlens, N, T, H, D,
+                                       dt, out_dt, q, k, v, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_prologue launch");
+  return KDA_OK;
+}
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, float scale, const float *initial_state,
+                         const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                         int chunk, kda_dtype dt, float *o, float *final_state,
+                         kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1 && Dk >= 1 && Dv >= 1,
+              "bad sizes N=%d T=%d H=%d Dk=%d Dv=%d", N, T, H, Dk, Dv);
+  KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
+  if (Dk != Dv || !supported_d(Dk))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_fwd: Dk=%d Dv=%d (need Dk == Dv in {16,32,64,128})",
+                Dk, Dv);
+  if (chunk != 16 && chunk != 32 && chunk != 64)
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_fwd: chunk=%d not in {16,32,64}", chunk);
+  if (T > 0) {
+    KDA_REQUIRE_PTR(q, "q");
+    KDA_REQUIRE_PTR(k, "k");
+    KDA_REQUIRE_PTR(v, "v");
+    KDA_REQUIRE_PTR(g, "g");
+    KDA_REQUIRE_PTR(beta, "beta");
+    KDA_REQUIRE_PTR(o, "o");
+  }
+  KDA_OPT_PTR(initial_state, "initial_state");
+  KDA_OPT_PTR(final_state, "final_state");
+  KDA_OPT_PTR(cu_seqlens, "cu_seqlens");
+  const size_t es = esize(dt);
+  const size_t act = (size_t)T * H * Dk * es, obytes = (size_t)T * H * Dv * sizeof(float);
+  const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
+  const void *ins[5] = {q, k, v, g, beta};
+  const size_t insz[5] = {act, act, (size_t)T * H * Dv * es, (size_t)T * H * Dk * 4,
+                          (size_t)T * H * 4};
+  for (int i = 0; i < 5; ++i)
+    KDA_REQUIRE(!overlaps(o, obytes, ins[i], insz[i]), "o overlaps an input");
+  KDA_REQUIRE(!overlaps(o, obytes, final_state, sbytes), "o overlaps final_state");
+  KDA_REQUIRE(final_state == initial_state ||
+                  !overlaps(final_state, sbytes, initial_state, sbytes),
+              "final_state partially overlaps initial_state");
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  if (T == 0 && final_state == nullptr) return KDA_OK;
+  cudaError_t e = kda::launch_chunk_simt(q, k, v, g, beta, scale, initial_state, cu_seqlens, N,
+                                         T, H, Dk, chunk, dt, o, final_state, status,
+                                         (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
+  return KDA_OK;
+}
+
+kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache, const float *g,
+                           const float *beta, float scale, float *state, int N, int H, int D,
+                           kda_dtype dt, float *o, kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(N >= 0 && H >= 1 && D >= 1, "bad sizes N=%d H=%d D=%d", N, H, D);
+  if (!supported_d(D)) return fail(KDA_ERR_UNSUPPORTED, "decode: D=%d not in {16,32,64,128}", D);
+  if (N == 0) return KDA_OK;
+  KDA_REQUIRE_PTR(x, "x");
+  KDA_REQUIRE_PTR(conv_w, "conv_w");
+  KDA_REQUIRE_PTR(conv_cache, "conv_cache");
+  KDA_REQUIRE_PTR(g, "g");
+  KDA_REQUIRE_PTR(beta, "beta");
+  KDA_REQUIRE_PTR(state, "state");
+  KDA_REQUIRE_PTR(o, "o");
+  const size_t es = esize(dt), C = (size_t)3 * H * D;
+  const size_t obytes = (size_t)N * H * D * sizeof(float), sbytes = (size_t)N * H * D * D * 4;
+  KDA_REQUIRE(!overlaps(o, obytes, state, sbytes), "o overlaps state");
+  KDA_REQUIRE(!overlaps(o, obytes, conv_cache, (size_t)N * 3 * C * es), "o overlaps conv_cache");
+  KDA_REQUIRE(!overlaps(o, obytes, x, (size_t)N * C * es), "o overlaps x");
+  KDA_REQUIRE(!overlaps(state, sbytes, conv_cache, (size_t)N * 3 * C * es),
+              "state overlaps conv_cache");
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaError_t e = kda::launch_decode(x, conv_w, conv_cache, g, beta, scale, state, N, H, D, dt, o,
+                                     status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
+  return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,119 @@
+// Shared device helpers for the libkda kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// ---------------------------------------------------------------------------
+// Element access for the two activation types
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Load/store 8 consecutive elements (16 B for bf16, 32 B for f32) as floats.
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&out)[8]) {
+  uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float *p, float (&out)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+  out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&in)[8]) {
+  uint4 u;
+  __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(in[2 * i], in[2 * i + 1]);
+  *reinterpret_cast<uint4 *>(p) = u;
+}
+__device__ __forceinline__ void store8(float *p, const float (&in)[8]) {
+  reinterpret_cast<float4 *>(p)[0] = make_float4(in[0], in[1], in[2], in[3]);
+  reinterpret_cast<float4 *>(p)[1] = make_float4(in[4], in[5], in[6], in[7]);
+}
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+
+// ---------------------------------------------------------------------------
+// Device status word (one per device, allocated by the host layer)
+// ---------------------------------------------------------------------------
+
+// Record the first fault code; later faults keep the first one.
+__device__ __forceinline__ void report(int *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Sequence bounds from cu_seqlens with device-side validation: a malformed
+// entry (decreasing or outside [0, T]) is clamped and recorded.
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int n, int T, int *status,
+                                           int &bos, int &eos) {
+  if (cu == nullptr) {
+    bos = 0;
+    eos = T;
+    return;
+  }
+  int a = cu[n], b = cu[n + 1];
+  if (a < 0 || b < a || b > T) {
+    report(status, KDA_ERR_DEVICE_BOUNDS);
+    a = min(max(a, 0), T);
+    b = min(max(b, a), T);
+  }
+  bos = a;
+  eos = b;
+}
+
+// Index of the sequence containing token t (cu sorted); -1 if none.
+__device__ __forceinline__ int seq_of_token(const int32_t *cu, int N, int t) {
+  if (cu == nullptr) return 0;
+  int lo = 0, hi = N - 1, ans = -1;
+  while (lo <= hi) {
+    int mid = (lo + hi) >> 1;
+    if (cu[mid] <= t) {
+      ans = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  return ans;
+}
+
+}  // namespace kda
+
+// Host-side launchers implemented in the kernel files, called by kda_api.cu.
+namespace kda {
+cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in, void *cache_out,
+                            const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
+                            kda_dtype out_dt, void *q, void *k, void *v, int *status,
+                            cudaStream_t s);
+cudaError_t launch_decode(const void *x, const float *w, void *cache, const float *g,
+                          const float *beta, float scale, float *state, int N, int H, int D,
+                          kda_dtype dt, float *o, int *status, cudaStream_t s);
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, float scale, const float *s0,
+                              const int32_t *cu, int N, int T, int H, int D, int chunk,
+                              kda_dtype dt, float *o, float *sN, int *status, cudaStream_t s);
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *s0, const int32_t *cu,
+                            int N, int T, int H, float *o, float *sN, int *status,
+                            cudaStream_t s);
+}  // namespace kda

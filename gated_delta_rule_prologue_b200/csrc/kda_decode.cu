@@ -1,0 +1,176 @@
+// Batched decode step: for each (sequence, head) the prologue on the new token
+// with the conv cache as history, then one step of the KDA recurrence on the
+// fp32 state in place.
+//
+// Sources: "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆" -- 第二站 (short conv,
+// SiLU, L2 on q and k), 第三站 (rows of the key-first state decayed by
+// alpha_t = exp(g_t)), 第四站 (error against the decayed state, delta write),
+// 第五站 (read after the write), 彩蛋 (recurrent execution for generation).
+//
+// The state is stored value-major, state[n][h][j][i] = S[i][j] (S key-first),
+// so row j of S^T is D contiguous floats.  Per row j:
+//     s'  = alpha (.) S^T[j,:]
+//     p_j = <s', k>,   r_j = <s', q>            (one fused shuffle tree)
+//     e_j = v_j - p_j
+//     S^T[j,:] = s' + beta e_j k
+//     o_j = scale * <S^T[j,:], q> = scale * (r_j + beta e_j <k, q>)
+// so both reductions are independent and <k, q> is computed once per head.
+// HBM traffic is dominated by the state: 2 * 4 * D^2 bytes per (seq, head).
+#include "kda_common.cuh"
+
+namespace kda {
+namespace {
+
+template <int D>
+struct DecodeShape {
+  static constexpr int kLanesPerRow = D / 4;                  // float4 per lane
+  static constexpr int kRowsPerInstr = 32 / kLanesPerRow;     // rows per warp access
+  static constexpr int kWarps = (D / kRowsPerInstr) < 8 ? (D / kRowsPerInstr) : 8;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kIters = D / (kRowsPerInstr * kWarps); // row groups per warp
+  static_assert(kIters >= 1 && kIters * kRowsPerInstr * kWarps == D, "row split");
+};
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(DecodeShape<D>::kThreads)
+decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__restrict__ cache,
+              const float *__restrict__ g, const float *__restrict__ beta, float scale,
+              float *__restrict__ state, int N, int H, float *__restrict__ o) {
+  using Sh = DecodeShape<D>;
+  constexpr int LPR = Sh::kLanesPerRow;
+  __shared__ float qkv[3 * D];
+  __shared__ float red[4];
+  __shared__ float o_s[D];
+
+  const int nh = blockIdx.x;
+  const int n = nh / H, h = nh % H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = lane % LPR;          // float4 slot within a row
+  const int rsub = lane / LPR;         // row within the warp access
+  const int dk0 = sub * 4;
+
+  // 1. Issue the state loads first: they do not depend on the prologue.
+  float *base = state + (size_t)nh * D * D;
+  float4 s[Sh::kIters];
+#pragma unroll
+  for (int it = 0; it < Sh::kIters; ++it) {
+    const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
+    s[it] = __ldcs(reinterpret_cast<const float4 *>(base + (size_t)j * D + dk0));
+  }
+  const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g + (size_t)nh * D + dk0));
+  const float b = __ldg(beta + nh);
+
+  // 2. Prologue for this head's 3*D channels; the conv cache is shifted in place.
+  const int C = 3 * H * D;
+  for (int i = tid; i < 3 * D; i += Sh::kThreads) {
+    const int pidx = i / D, d = i % D;
+    const int c = pidx * H * D + h * D + d;
+    Tin *cr = cache + (size_t)n * 3 * C + c;
+    const float c0 = to_f32(cr[0]), c1 = to_f32(cr[C]), c2 = to_f32(cr[2 * C]);
+    const Tin xin = x[(size_t)n * C + c];
+    const float4 wc = __ldg(reinterpret_cast<const float4 *>(w + (size_t)c * 4));
+    float a = wc.x * c0;
+    a = fmaf(wc.y, c1, a);
+    a = fmaf(wc.z, c2, a);
+    a = fmaf(wc.w, to_f32(xin), a);
+    qkv[i] = silu(a);
+    cr[0] = cr[C];
+    cr[C] = cr[2 * C];
+    cr[2 * C] = xin;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float sq = 0.f, sk = 0.f, skq = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float qq = qkv[d], kk = qkv[D + d];
+      sq = fmaf(qq, qq, sq);
+      sk = fmaf(kk, kk, sk);
+      skq = fmaf(kk, qq, skq);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      skq += __shfl_xor_sync(0xffffffffu, skq, off);
+    }
+    if (lane == 0) {
+      const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
+      red[0] = rq;
+      red[1] = rk;
+      red[2] = skq * rq * rk;  // <k, q> of the normalised vectors
+    }
+  }
+  __syncthreads();
+  const float rq = red[0], rk = red[1], kq = red[2];
+  const float4 q4 = make_float4(qkv[dk0] * rq, qkv[dk0 + 1] * rq, qkv[dk0 + 2] * rq,
+                                qkv[dk0 + 3] * rq);
+  const float4 k4 = make_float4(qkv[D + dk0] * rk, qkv[D + dk0 + 1] * rk,
+                                qkv[D + dk0 + 2] * rk, qkv[D + dk0 + 3] * rk);
+  const float4 a4 = make_float4(expf(g4.x), expf(g4.y), expf(g4.z), expf(g4.w));
+
+  // 3. State update, one row of S^T per LPR lanes.
+#pragma unroll
+  for (int it = 0; it < Sh::kIters; ++it) {
+    const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
+    float4 sp = make_float4(a4.x * s[it].x, a4.y * s[it].y, a4.z * s[it].z, a4.w * s[it].w);
+    float pk = sp.x * k4.x;
+    pk = fmaf(sp.y, k4.y, pk);
+    pk = fmaf(sp.z, k4.z, pk);
+    pk = fmaf(sp.w, k4.w, pk);
+    float pq = sp.x * q4.x;
+    pq = fmaf(sp.y, q4.y, pq);
+    pq = fmaf(sp.z, q4.z, pq);
+    pq = fmaf(sp.w, q4.w, pq);
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) {
+      pk += __shfl_xor_sync(0xffffffffu, pk, off);
+      pq += __shfl_xor_sync(0xffffffffu, pq, off);
+    }
+    const float be = b * (qkv[2 * D + j] - pk);
+    sp.x = fmaf(be, k4.x, sp.x);
+    sp.y = fmaf(be, k4.y, sp.y);
+    sp.z = fmaf(be, k4.z, sp.z);
+    sp.w = fmaf(be, k4.w, sp.w);
+    __stcs(reinterpret_cast<float4 *>(base + (size_t)j * D + dk0), sp);
+    if (sub == 0) o_s[j] = scale * fmaf(be, kq, pq);
+  }
+  __syncthreads();
+  for (int j = tid; j < D; j += Sh::kThreads) o[(size_t)nh * D + j] = o_s[j];
+}
+
+template <typename Tin, int D>
+cudaError_t launch_typed(const void *x, const float *w, void *cache, const float *g,
+                         const float *beta, float scale, float *state, int N, int H, float *o,
+                         cudaStream_t s) {
+  decode_kernel<Tin, D><<<N * H, DecodeShape<D>::kThreads, 0, s>>>(
+      static_cast<const Tin *>(x), w, static_cast<Tin *>(cache), g, beta, scale, state, N, H,
+      o);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_d(int D, const void *x, const float *w, void *cache, const float *g,
+                     const float *beta, float scale, float *state, int N, int H, float *o,
+                     cudaStream_t s) {
+  switch (D) {
+    case 16: return launch_typed<Tin, 16>(x, w, cache, g, beta, scale, state, N, H, o, s);
+    case 32: return launch_typed<Tin, 32>(x, w, cache, g, beta, scale, state, N, H, o, s);
+    case 64: return launch_typed<Tin, 64>(x, w, cache, g, beta, scale, state, N, H, o, s);
+    case 128: return launch_typed<Tin, 128>(x, w, cache, g, beta, scale, state, N, H, o, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void *x, const float *w, void *cache, const float *g,
+                          const float *beta, float scale, float *state, int N, int H, int D,
+                          kda_dtype dt, float *o, int *status, cudaStream_t s) {
+  (void)status;  // the decode kernel has no waits or data-dependent indices
+  if ((long long)N * H >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (dt == KDA_BF16)
+    return launch_d<__nv_bfloat16>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
+  return launch_d<float>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
+}
+
+}  // namespace kda

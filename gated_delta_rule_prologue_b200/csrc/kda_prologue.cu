@@ -1,0 +1,221 @@
+// Prologue kernel: causal depthwise short conv (width 4) + SiLU over the q/k/v
+// projections, then per-(token, head) L2 normalisation of q and k.
+//
+// Source: "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆", 第二站 (short conv
+// of width 4 that never looks ahead, SiLU inside the conv module, q and k
+// unit-normalised); "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解",
+// ShortConv paragraph (per channel: the current token and the three before).
+//
+// Work decomposition (HBM-bound, 1536 B of traffic per token-head for bf16):
+//   * one thread owns 8 consecutive channels of one (part, head) segment and
+//     walks TT consecutive tokens, keeping the previous three inputs of its
+//     channels in registers, so every input element is read from HBM once
+//     (plus a 3-row halo per TT tokens, mostly served by L2);
+//   * the D/8 threads of a segment sit in one warp and reduce the sum of
+//     squares for the L2 norm with xor shuffles;
+//   * loads of a batch of 8 tokens are issued before any of them is used.
+#include "kda_common.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTokensPerThread = 32;  // TT
+constexpr int kBatch = 8;             // tokens whose loads are in flight together
+
+template <typename Tin>
+__device__ __forceinline__ void load8_or_zero(const Tin *p, bool ok, float (&out)[8]) {
+  if (ok) {
+    load8(p, out);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = 0.f;
+  }
+}
+
+template <typename Tin, typename Tout, int D>
+__global__ void __launch_bounds__(kThreads)
+prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
+                const Tin *__restrict__ cache_in, Tin *__restrict__ cache_out,
+                const int32_t *__restrict__ cu, int N, int T, int H, Tout *__restrict__ q,
+                Tout *__restrict__ k, Tout *__restrict__ v, int *status) {
+  constexpr int G = D / 8;  // threads per (part, head) segment; divides 32
+  const int HD = H * D;
+  const int C = 3 * HD;
+  const int c0 = (blockIdx.x * kThreads + threadIdx.x) * 8;
+  const bool active = c0 < C;
+  const int p = active ? c0 / HD : 0;
+  const int h = active ? (c0 % HD) / D : 0;
+  const int d0 = c0 % D;
+  Tout *out = p == 0 ? q : (p == 1 ? k : v);
+
+  // Sequences with no tokens pass their cache through unchanged.
+  if (blockIdx.y == 0 && cache_out != nullptr && active) {
+    for (int n = 0; n < N; ++n) {
+      const int a = cu ? cu[n] : 0, b = cu ? cu[n + 1] : T;
+      if (a != b) continue;
+      for (int r = 0; r < 3; ++r) {
+        float tmp[8];
+        load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0, cache_in != nullptr, tmp);
+        store8(cache_out + ((size_t)n * 3 + r) * C + c0, tmp);
+      }
+    }
+  }
+
+  const int t0 = blockIdx.y * kTokensPerThread;
+  const int t_end = min(t0 + kTokensPerThread, T);
+  if (t0 >= t_end) return;  // uniform over the block
+  if (cu != nullptr && (cu[0] != 0 || cu[N] != T)) {
+    report(status, KDA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+
+  float wt[8][4];
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 f = __ldg(reinterpret_cast<const float4 *>(w + (size_t)(c0 + i) * 4));
+      wt[i][0] = f.x; wt[i][1] = f.y; wt[i][2] = f.z; wt[i][3] = f.w;
+    }
+  }
+
+  int n = seq_of_token(cu, N, t0);
+  int bos, eos;
+  seq_bounds(cu, n, T, status, bos, eos);
+  while (t0 >= eos && n < N - 1) {  // skip empty sequences ending at t0
+    ++n;
+    seq_bounds(cu, n, T, status, bos, eos);
+  }
+
+  // History of t0: tokens t0-3, t0-2, t0-1 (from the cache before bos).
+  float xm3[8], xm2[8], xm1[8];
+  {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int tt = t0 - 3 + j;
+      float tmp[8];
+      if (tt >= bos) {
+        load8_or_zero(x + (size_t)tt * C + c0, active, tmp);
+      } else {
+        const int r = 3 - (bos - tt);  // cache row (0 = oldest)
+        load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0, active && cache_in != nullptr,
+                      tmp);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (j == 0) xm3[e] = tmp[e];
+        if (j == 1) xm2[e] = tmp[e];
+        if (j == 2) xm1[e] = tmp[e];
+      }
+    }
+  }
+
+  for (int tb = t0; tb < t_end; tb += kBatch) {
+    float xr[kBatch][8];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      load8_or_zero(x + (size_t)(tb + i) * C + c0, active && tb + i < t_end, xr[i]);
+
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int t = tb + i;
+      if (t >= t_end) break;
+      if (t >= eos) {  // next non-empty sequence starts at t: restart the history
+        do {
+          ++n;
+          seq_bounds(cu, n, T, status, bos, eos);
+        } while (t >= eos && n < N - 1);
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+          float tmp[8];
+          load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0,
+                        active && cache_in != nullptr, tmp);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (r == 0) xm3[e] = tmp[e];
+            if (r == 1) xm2[e] = tmp[e];
+            if (r == 2) xm1[e] = tmp[e];
+          }
+        }
+      }
+      float y[8];
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float a = wt[e][0] * xm3[e];
+        a = fmaf(wt[e][1], xm2[e], a);
+        a = fmaf(wt[e][2], xm1[e], a);
+        a = fmaf(wt[e][3], xr[i][e], a);
+        y[e] = silu(a);
+        ss = fmaf(y[e], y[e], ss);
+      }
+#pragma unroll
+      for (int off = G / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (p < 2) {
+        const float r = rsqrtf(ss + 1e-6f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] *= r;
+      }
+      if (active) {
+        store8(out + ((size_t)t * H + h) * D + d0, y);
+        if (cache_out != nullptr && t == eos - 1) {
+          store8(cache_out + ((size_t)n * 3 + 0) * C + c0, xm2);
+          store8(cache_out + ((size_t)n * 3 + 1) * C + c0, xm1);
+          store8(cache_out + ((size_t)n * 3 + 2) * C + c0, xr[i]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        xm3[e] = xm2[e];
+        xm2[e] = xm1[e];
+        xm1[e] = xr[i][e];
+      }
+    }
+  }
+}
+
+template <typename Tin, typename Tout, int D>
+cudaError_t launch_typed(const void *x, const float *w, const void *cache_in, void *cache_out,
+                         const int32_t *cu, int N, int T, int H, void *q, void *k, void *v,
+                         int *status, cudaStream_t s) {
+  const int C = 3 * H * D;
+  const int groups = C / 8;
+  dim3 grid((groups + kThreads - 1) / kThreads,
+            max(1, (T + kTokensPerThread - 1) / kTokensPerThread));
+  prologue_kernel<Tin, Tout, D><<<grid, kThreads, 0, s>>>(
+      static_cast<const Tin *>(x), w, static_cast<const Tin *>(cache_in),
+      static_cast<Tin *>(cache_out), cu, N, T, H, static_cast<Tout *>(q),
+      static_cast<Tout *>(k), static_cast<Tout *>(v), status);
+  return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout>
+cudaError_t launch_d(int D, const void *x, const float *w, const void *ci, void *co,
+                     const int32_t *cu, int N, int T, int H, void *q, void *k, void *v,
+                     int *status, cudaStream_t s) {
+  switch (D) {
+    case 16: return launch_typed<Tin, Tout, 16>(x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    case 32: return launch_typed<Tin, Tout, 32>(x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    case 64: return launch_typed<Tin, Tout, 64>(x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    case 128: return launch_typed<Tin, Tout, 128>(x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in, void *cache_out,
+                            const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
+                            kda_dtype out_dt, void *q, void *k, void *v, int *status,
+                            cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  if (dt == KDA_BF16 && out_dt == KDA_BF16)
+    return launch_d<bf, bf>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
+  if (dt == KDA_BF16)
+    return launch_d<bf, float>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
+  if (out_dt == KDA_BF16)
+    return launch_d<float, bf>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
+  return launch_d<float, float>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
+}
+
+}  // namespace kda

@@ -1,0 +1,155 @@
+/*
+ * kda.h -- C ABI of libkda, a B200 (sm_100a) implementation of the Kimi Delta
+ * Attention (KDA) recurrence hot path: the prologue (short conv, SiLU, L2),
+ * the chunkwise-parallel prefill and the batched decode step.
+ *
+ * Sources (web pages; cited as [Wn section]):
+ *   [W1] "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆" (yeyulingfeng.com)
+ *   [W3] "Kimi K3 记忆架构总览：KDA、MLA、AttnRes 各管什么" (moonzj.com)
+ *   [W4] "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解"
+ *   [W5] "AI-Workshop 文献分享 #16 — KDA：给长文本建立可更新的记忆"
+ *
+ * The recurrence, per head with state S in R^{Dk x Dv} ([W1 第三站-第五站]):
+ *     S <- diag(exp(g_t)) S;  e <- v_t - S^T k_t;  S <- S + beta_t k_t e^T;
+ *     o_t <- scale * S^T q_t.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays
+ *     owned by the caller.  The library never allocates per call; it keeps
+ *     one lazily allocated 4-byte status word per device (see
+ *     kda_get_device_status).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  A synchronous return reports argument,
+ *     support and launch errors only; faults detected inside a kernel
+ *     (out-of-range cu_seqlens, a bounded wait that ran out) are recorded in
+ *     the device status word.
+ *   - Recurrent state layout is [N, H, Dv, Dk] float32: the key index is the
+ *     contiguous one (the transpose of the pages' key-first S; [W1 第三站]
+ *     allows a transposed storage layout).
+ *   - Activations (q, k, v, x, conv cache) have the element type `dt`
+ *     (KDA_F32 or KDA_BF16).  g, beta, the state and every read-out o are
+ *     always float32: o is heavy-tailed (its largest entries are many times
+ *     its RMS), so rounding it to bf16 alone would exceed the parity bound
+ *     max|o - o_ref| <= 2e-2 * RMS(o_ref).
+ *   - Every pointer must be 16-byte aligned.  Outputs must not overlap
+ *     inputs unless an argument says "in/out".
+ *   - On any non-OK return, kda_last_error() gives a message (thread-local).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size, aliasing   */
+  KDA_ERR_UNSUPPORTED = 2,    /* valid request outside the compiled domain     */
+  KDA_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed   */
+  KDA_ERR_DEVICE_TIMEOUT = 4, /* (status word) a bounded device wait ran out   */
+  KDA_ERR_DEVICE_BOUNDS = 5   /* (status word) device-side index check failed  */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+typedef struct CUstream_st *kda_stream_t; /* same type as cudaStream_t */
+
+/*
+ * kda_prologue -- short conv + SiLU on the q/k/v projections, then per-head
+ * L2 normalisation of q and k.  [W1 第二站]: a causal depthwise conv of
+ * width 4 that never reads future tokens, SiLU inside the conv module, and
+ * q, k unit-normalised inside the KDA operator; [W4 ShortConv paragraph]:
+ * each channel sees the current token and the three before it.
+ *
+ *   x          [T, 3*H*D] dt   projections; channel p*H*D + h*D + d with
+ *                              p = 0 (query), 1 (key), 2 (value)
+ *   conv_w     [3*H*D, 4] f32  tap 3 multiplies the current token, tap 0 the
+ *                              token three back; no bias
+ *   cache_in   [N, 3, 3*H*D] dt or NULL: the three inputs before each
+ *                              sequence, oldest first (NULL: zero history)
+ *   cache_out  [N, 3, 3*H*D] dt or NULL: receives the last three inputs of
+ *                              each sequence; must not overlap cache_in
+ *   cu_seqlens [N+1] int32 device, or NULL (then N must be 1): packed
+ *                              sequence boundaries; the conv never crosses one
+ *   dt         element type of x and of both caches
+ *   out_dt     element type of the outputs q, k, v
+ *   q, k, v    [T, H, D] out_dt outputs; q, k are y/sqrt(sum y^2 + 1e-6) over
+ *                              the head's D channels of y = SiLU(conv)
+ * Supported: D in {16, 32, 64, 128}; T >= 0 (T == 0 only writes cache_out).
+ */
+kda_status kda_prologue(const void *x, const float *conv_w, const void *cache_in,
+                        void *cache_out, const int32_t *cu_seqlens, int N, int T,
+                        int H, int D, kda_dtype dt, kda_dtype out_dt, void *q, void *k,
+                        void *v, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel prefill of the recurrence.  [W1 彩蛋]
+ * and [W5 §10.3]: tokens are grouped into chunks of `chunk`, the state is
+ * carried from chunk to chunk, and the work inside a chunk is matrix algebra
+ * (in-chunk cumulative log-decay, a unit-lower-triangular WY solve by
+ * forward substitution, the state-dependent chunk update); [W4 Figure 1]:
+ * the chunk map of the state is affine.  Results equal the token-by-token
+ * recurrence up to rounding.
+ *
+ *   q, k          [T, H, Dk] dt  q and k already unit-normalised
+ *   v             [T, H, Dv] dt
+ *   g             [T, H, Dk] f32 log-decay, alpha = exp(g); the bf16 tensor-core
+ *                                path requires g >= -5 (the bounded gate of
+ *                                [W1 彩蛋]); other values may lose accuracy
+ *   beta          [T, H] f32
+ *   scale         multiplier on every read o_t ([W1 第五站])
+ *   initial_state [N, H, Dv, Dk] f32 or NULL (zero state)
+ *   cu_seqlens    [N+1] int32 device or NULL (N must be 1); sequences restart
+ *                 from initial_state[n]
+ *   o             [T, H, Dv] float32 output
+ *   final_state   [N, H, Dv, Dk] f32 or NULL; may alias initial_state
+ * Supported: dt == KDA_F32: Dk == Dv in {16, 32, 64, 128}, chunk in {16, 32,
+ *   64} (exact-fp32 CUDA-core path).  dt == KDA_BF16: the same domain; with
+ *   Dk == Dv == 128 and chunk == 64 it runs the tcgen05 tensor-core path.
+ */
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, float scale, const float *initial_state,
+                         const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                         int chunk, kda_dtype dt, float *o, float *final_state,
+                         kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one new token for each of N independent sequences: the
+ * prologue on that token with the conv cache as history, then one step of
+ * the recurrence on the state in place (the recurrent mode used for
+ * generation, [W1 彩蛋]; one fixed-size state update per token, [W1 回头看看]).
+ *
+ *   x          [N, 3*H*D] dt   the new token's projections (layout as above)
+ *   conv_w     [3*H*D, 4] f32
+ *   conv_cache [N, 3, 3*H*D] dt in/out: oldest first; after the call it holds
+ *                              the last three inputs including x
+ *   g          [N, H, D] f32;  beta [N, H] f32
+ *   state      [N, H, Dv, Dk] f32 in/out
+ *   o          [N, H, D] float32 output
+ * Supported: D in {16, 32, 64, 128} (Dk == Dv == D).
+ */
+kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache,
+                           const float *g, const float *beta, float scale, float *state,
+                           int N, int H, int D, kda_dtype dt, float *o,
+                           kda_stream_t stream);
+
+/*
+ * kda_get_device_status -- read and clear the current device's status word
+ * (KDA_OK if no kernel recorded a fault).  Synchronises the device.
+ */
+kda_status kda_get_device_status(int *code);
+
+/* Message for the last non-OK return on the calling thread (never NULL). */
+const char *kda_last_error(void);
+
+/* Library version string. */
+const char *kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

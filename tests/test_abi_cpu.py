@@ -1,0 +1,114 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+include/kda.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from gated_delta_rule_prologue_b200.build import build
+    build()
+    import gated_delta_rule_prologue_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:kda_status|const char \*)\s*(kda_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = declared_functions()
+    for n in ("kda_prologue", "kda_chunk_fwd", "kda_decode_step", "kda_get_device_status",
+              "kda_last_error", "kda_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(kda):
+    out = subprocess.run(["nm", "-D", "--defined-only", kda.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)$", out, re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(kda.lib, n)
+
+
+def test_no_oracle_or_fallback_in_product_package():
+    pkg = os.path.join(ROOT, "gated_delta_rule_prologue_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def _vp(x):
+    return ctypes.c_void_p(x)
+
+
+ALIGNED = 0x10000          # fake, never dereferenced: validation fails first
+MISALIGNED = 0x10008
+
+
+def test_version_and_last_error(kda):
+    assert "sm_100a" in kda.kda_version()
+    assert isinstance(kda.lib.kda_last_error(), bytes)
+
+
+def test_chunk_fwd_rejects_bad_arguments(kda):
+    L = kda.lib
+    a = _vp(ALIGNED)
+    # null q
+    st = L.kda_chunk_fwd(None, a, a, a, a, 1.0, None, None, 1, 64, 2, 16, 16, 16, 0, a, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"q is NULL" in L.kda_last_error()
+    # misaligned k
+    st = L.kda_chunk_fwd(a, _vp(MISALIGNED), a, a, a, 1.0, None, None, 1, 64, 2, 16, 16, 16, 0,
+                         _vp(ALIGNED * 2), None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"aligned" in L.kda_last_error()
+    # N > 1 without cu_seqlens
+    st = L.kda_chunk_fwd(a, a, a, a, a, 1.0, None, None, 3, 64, 2, 16, 16, 16, 0, a, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    # unsupported head size / chunk / dtype
+    st = L.kda_chunk_fwd(a, a, a, a, a, 1.0, None, None, 1, 64, 2, 48, 48, 16, 0, a, None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_chunk_fwd(a, a, a, a, a, 1.0, None, None, 1, 64, 2, 16, 16, 24, 0, a, None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_chunk_fwd(a, a, a, a, a, 1.0, None, None, 1, 64, 2, 16, 16, 16, 7, a, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    # output aliasing an input
+    st = L.kda_chunk_fwd(a, _vp(ALIGNED * 4), _vp(ALIGNED * 8), _vp(ALIGNED * 12),
+                         _vp(ALIGNED * 16), 1.0, None, None, 1, 64, 2, 16, 16, 16, 0, a, None,
+                         None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
+    # negative sizes
+    st = L.kda_chunk_fwd(a, a, a, a, a, 1.0, None, None, 1, -1, 2, 16, 16, 16, 0, a, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+
+
+def test_prologue_and_decode_reject_bad_arguments(kda):
+    L = kda.lib
+    a = _vp(ALIGNED)
+    st = L.kda_prologue(None, a, None, None, None, 1, 8, 2, 16, 1, 1, _vp(2 * ALIGNED),
+                        _vp(3 * ALIGNED), _vp(4 * ALIGNED), None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    st = L.kda_prologue(a, a, None, None, None, 1, 8, 2, 24, 1, 1, _vp(2 * ALIGNED),
+                        _vp(3 * ALIGNED), _vp(4 * ALIGNED), None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_prologue(a, a, _vp(5 * ALIGNED), _vp(5 * ALIGNED), None, 1, 8, 2, 16, 1, 0,
+                        _vp(2 * ALIGNED), _vp(3 * ALIGNED), _vp(4 * ALIGNED), None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"cache_out overlaps" in L.kda_last_error()
+    st = L.kda_decode_step(a, a, a, a, a, 1.0, None, 4, 2, 16, 1, _vp(2 * ALIGNED), None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"state is NULL" in L.kda_last_error()
+    st = L.kda_decode_step(a, a, a, a, a, 1.0, a, 4, 2, 100, 1, _vp(2 * ALIGNED), None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_get_device_status(None)
+    assert st == kda.KDA_ERR_INVALID_ARG

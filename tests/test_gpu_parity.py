@@ -1,0 +1,328 @@
+"""GPU parity: every libkda kernel against the float64 oracle, through the C ABI.
+
+Tolerances (stated by the workloads): outputs max|delta| / RMS(reference)
+<= 1e-4 for float32 activations and <= 2e-2 for bfloat16 activations; final
+state relative Frobenius error <= 1e-2.  Full-size workloads run in the launch
+configuration the benchmark times and are compared on sampled heads or
+sequences that the oracle recomputes from regenerated input slabs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import (kda_decode_step as o_decode, kda_recurrent, prologue as o_prologue,
+                    state_from_abi, state_to_abi)
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_BF16, TOL_STATE = 1e-4, 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def kda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import gated_delta_rule_prologue_b200 as m
+    return m
+
+
+def rel_max(got, ref):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got))
+    return float(np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref * ref)))
+
+
+def rel_fro(got, ref):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got))
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_chunk(kda, inp, *, chunk=None, in_place=False):
+    dev = "cuda"
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    g, beta = inp.g.to(dev), inp.beta.to(dev)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    N, H, D = inp.N, inp.H, inp.q.shape[2]
+    s0 = None if inp.initial_state is None else inp.initial_state.to(dev).contiguous()
+    fs = s0 if (in_place and s0 is not None) else torch.empty((N, H, D, D), device=dev)
+    o = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, initial_state=s0, final_state=fs,
+                      cu_seqlens=cu, chunk=chunk or inp.chunk)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    return f64(o), f64(fs)
+
+
+def oracle_chunk(inp):
+    s0 = None if inp.initial_state is None else state_from_abi(inp.initial_state)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    o, S = kda_recurrent(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.scale, s0, cu)
+    return o, state_to_abi(S)
+
+
+# --- chunk_fwd ---------------------------------------------------------------
+
+def test_tiny_f32_parity(kda):
+    inp = W.tiny_f32()
+    o, S = run_chunk(kda, inp)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert rel_max(o, o_ref) <= TOL_F32
+    assert rel_fro(S, S_ref) <= 1e-5
+
+
+def test_seq4k_bf16_parity(kda):
+    inp = W.seq4k_bf16()
+    o, S = run_chunk(kda, inp)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert rel_max(o, o_ref) <= TOL_BF16
+    assert rel_fro(S, S_ref) <= TOL_STATE
+
+
+EDGE = [
+    # (name, D, chunk, bf16, lengths, g_shift, s0_std, g_fn)
+    ("ragged_f32_d128_c64", 128, 64, False, [200, 1, 64, 0, 63, 130], 0.0, 0.3, None),
+    ("ragged_bf16_d128_c64", 128, 64, True, [200, 1, 64, 0, 63, 130], 0.0, 0.3, None),
+    ("bf16_d64_c32", 64, 32, True, [77, 150], 0.0, 0.1, None),
+    ("f32_d32_c16", 32, 16, False, [33, 5], 0.0, 0.1, None),
+    ("bf16_d16_c64", 16, 64, True, [100], 0.0, 0.0, None),
+    ("slow_decay_bf16", 128, 64, True, [700], 0.0, 0.05,
+     lambda z: -5.0 * torch.sigmoid(z - 6.0)),
+    ("saturated_decay_bf16", 128, 64, True, [300], 0.0, 0.05,
+     lambda z: torch.full_like(z, -5.0)),
+    ("no_decay_bf16", 128, 64, True, [190], 0.0, 0.05, lambda z: torch.zeros_like(z)),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_chunk_edge_cases(kda, case):
+    name, D, chunk, bf16, lengths, g_shift, s0_std, g_fn = case
+    inp = W.random_prefill(100 + EDGE.index(case), sum(lengths), 3, D, bf16=bf16,
+                           g_shift=g_shift, s0_std=s0_std, lengths=lengths, chunk=chunk,
+                           g_fn=g_fn)
+    inp.scale = 0.5
+    o, S = run_chunk(kda, inp)
+    o_ref, S_ref = oracle_chunk(inp)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert rel_max(o, o_ref) <= tol
+    assert rel_fro(S, S_ref) <= (TOL_STATE if bf16 else 1e-5)
+
+
+def test_chunk_final_state_in_place(kda):
+    inp = W.random_prefill(5, 150, 2, 128, s0_std=0.1, lengths=[90, 60],
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 5.0))
+    o, S = run_chunk(kda, inp, in_place=True)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert rel_max(o, o_ref) <= TOL_BF16
+    assert rel_fro(S, S_ref) <= TOL_STATE
+
+
+def test_chunk_size_does_not_change_results(kda):
+    inp = W.random_prefill(6, 257, 2, 64, bf16=False, s0_std=0.1,
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 4.0))
+    outs = [run_chunk(kda, inp, chunk=c) for c in (16, 32, 64)]
+    for o, S in outs[1:]:
+        assert rel_max(o, outs[0][0]) <= 1e-4
+        assert rel_fro(S, outs[0][1]) <= 1e-5
+
+
+def test_malformed_cu_seqlens_sets_status_without_fault(kda):
+    inp = W.random_prefill(7, 64, 1, 16, bf16=False, lengths=[30, 34], chunk=16)
+    dev = "cuda"
+    bad = torch.tensor([0, 40, 20], dtype=torch.int32, device=dev)  # decreasing
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    o = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, cu_seqlens=bad, chunk=16)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == kda.KDA_ERR_DEVICE_BOUNDS
+    assert kda.kda_get_device_status() == 0    # cleared by the read
+    o2, _ = run_chunk(kda, inp)                 # the context is still usable
+    assert np.all(np.isfinite(o2))
+
+
+# --- prologue ----------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,out_dtype,D", [(torch.bfloat16, torch.bfloat16, 128),
+                                               (torch.bfloat16, torch.float32, 128),
+                                               (torch.float32, torch.float32, 16),
+                                               (torch.float32, torch.bfloat16, 64)])
+def test_prologue_parity_varlen_with_cache(kda, dtype, out_dtype, D):
+    H = 3
+    lengths = [70, 0, 1, 2, 45, 33]
+    T, N, C = sum(lengths), len(lengths), 3 * H * D
+    r = torch.Generator().manual_seed(D)
+    x = torch.randn((T, C), generator=r).to(dtype)
+    w = 0.5 * torch.randn((C, 4), generator=r)
+    cache = torch.randn((N, 3, C), generator=r).to(dtype)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    dev = "cuda"
+    q = torch.empty((T, H, D), dtype=out_dtype, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    cache_out = torch.empty((N, 3, C), dtype=dtype, device=dev)
+    kda.kda_prologue(x.to(dev), w.to(dev), q, k, v, H=H, D=D, cache_in=cache.to(dev),
+                     cache_out=cache_out, cu_seqlens=cu.to(dev))
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    q_ref, k_ref, v_ref, c_ref = o_prologue(x, w, H, D, cu.numpy(), cache)
+    for got, ref in ((q, q_ref), (k, k_ref), (v, v_ref)):
+        if out_dtype == torch.bfloat16:
+            # rounding to bf16 (8 significant bits, nearest-even) moves a value by
+            # at most 2^-9 of itself; allow that plus float32 arithmetic noise
+            rms = np.sqrt(np.mean(ref * ref))
+            assert np.all(np.abs(f64(got) - ref) <= 2.0 ** -9 * np.abs(ref) + 1e-5 * rms)
+        else:
+            assert rel_max(f64(got), ref) <= 1e-5
+    np.testing.assert_array_equal(f64(cache_out), c_ref)   # a copy of inputs: exact
+
+
+# --- full-size workloads, sampled ------------------------------------------------
+
+def test_k3_prefill_full_size_sampled_heads(kda):
+    """Prologue + chunkwise prefill over 32768 tokens x 96 heads (the benchmark's
+    launches); heads 0, 53 and 95 recomputed by the oracle over all tokens."""
+    inp = W.k3_prefill()
+    T, H, D = inp.T, inp.H, inp.D
+    dev = "cuda"
+    x = inp.x.to(dev)
+    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    kda.kda_prologue(x, inp.conv_w.to(dev), q, k, v, H=H, D=D)
+    o = torch.empty_like(v)
+    fs = torch.empty((1, H, D, D), device=dev)
+    kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, scale=inp.scale,
+                      final_state=fs, chunk=inp.chunk)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    del x
+    for h in (0, 53, 95):
+        xh, wh, gh, bh = W.k3_prefill_head(h)
+        qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
+        assert rel_max(f64(q[:, h]), qr[:, 0]) <= 1e-5
+        assert rel_max(f64(v[:, h]), vr[:, 0]) <= 1e-5
+        o_ref, S_ref = kda_recurrent(qr, kr, vr, gh[:, None, :], bh[:, None], inp.scale)
+        assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16
+        assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
+
+
+def test_varlen16_full_size_sampled(kda):
+    inp = W.varlen16()
+    o, S = run_chunk(kda, inp)
+    lengths = W.varlen16_lengths()
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    picks = [(int(np.argmin(lengths)), 0), (int(np.argmax(lengths)), 31), (5, 17)]
+    for n, h in picks:
+        qn, kn, vn, gn, bn, s0 = W.varlen16_seq_head(n, h)
+        o_ref, S_ref = kda_recurrent(qn[:, None], kn[:, None], vn[:, None], gn[:, None],
+                                     bn[:, None], 1.0, state_from_abi(s0)[None, None])
+        assert rel_max(o[cu[n]:cu[n + 1], h], o_ref[:, 0]) <= TOL_BF16
+        assert rel_fro(S[n, h], state_to_abi(S_ref)[0, 0]) <= TOL_STATE
+
+
+def test_decode256_full_size_sampled(kda):
+    """256 x 96 heads, 3 consecutive in-place steps; sequences 0, 77, 255 checked."""
+    steps = 3
+    inp = W.decode256(steps=steps)
+    dev = "cuda"
+    H, D = inp.H, inp.D
+    state = inp.state.to(dev)
+    cache = inp.conv_cache.to(dev)
+    w = inp.conv_w.to(dev)
+    outs = []
+    for s in range(steps):
+        o = torch.empty((inp.N, H, D), dtype=torch.float32, device=dev)
+        kda.kda_decode_step(inp.x[s].to(dev), w, cache, inp.g[s].to(dev), inp.beta[s].to(dev),
+                            state, o, H=H, D=D, scale=inp.scale)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    ns = [0, 77, 255]
+    st0, c0, xs, gs, bs, wr = W.decode256_seqs(ns, steps)
+    S = state_from_abi(st0)
+    c = c0
+    for s in range(steps):
+        o_ref, S, c = o_decode(xs[s], wr, c, gs[s], bs[s], S, H, D)
+        assert rel_max(f64(outs[s][ns]), o_ref) <= TOL_BF16
+    assert rel_fro(f64(state[ns]), state_to_abi(S)) <= TOL_STATE
+    np.testing.assert_array_equal(f64(cache[ns]), c)
+
+
+# --- cross-checks between GPU paths ------------------------------------------------
+
+def _prefill_gpu(kda, x, w, H, D, cache_in=None, s0=None, cu=None):
+    dev = "cuda"
+    T = x.shape[0]
+    N = 1 if cu is None else cu.numel() - 1
+    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    cache_out = torch.empty((N, 3, 3 * H * D), dtype=x.dtype, device=dev)
+    kda.kda_prologue(x, w, q, k, v, H=H, D=D, cache_in=cache_in, cache_out=cache_out,
+                     cu_seqlens=cu)
+    return q, k, v, cache_out
+
+
+def test_decode_kernel_matches_prologue_plus_chunk_kernel(kda):
+    """Two independent GPU paths over the same tokens: prefill (prologue kernel
+    + chunk kernel) and the decode kernel applied token by token."""
+    dev = "cuda"
+    N, T, H, D = 3, 40, 4, 128
+    C = 3 * H * D
+    r = torch.Generator().manual_seed(11)
+    x = torch.randn((N, T, C), generator=r).to(torch.bfloat16)
+    w = 0.5 * torch.randn((C, 4), generator=r)
+    g = -5.0 * torch.sigmoid(torch.randn((N, T, H, D), generator=r) - 3.0)
+    beta = torch.sigmoid(torch.randn((N, T, H), generator=r))
+    s0 = 0.05 * torch.randn((N, H, D, D), generator=r)
+    cu = torch.arange(0, N * T + 1, T, dtype=torch.int32, device=dev)
+    q, k, v, cache_out = _prefill_gpu(kda, x.reshape(N * T, C).to(dev), w.to(dev), H, D, cu=cu)
+    o_pre = torch.empty_like(v)
+    S_pre = torch.empty((N, H, D, D), device=dev)
+    kda.kda_chunk_fwd(q, k, v, g.reshape(N * T, H, D).to(dev), beta.reshape(N * T, H).to(dev),
+                      o_pre, initial_state=s0.to(dev), final_state=S_pre, cu_seqlens=cu)
+    state = s0.to(dev).clone()
+    cache = torch.zeros((N, 3, C), dtype=torch.bfloat16, device=dev)
+    o_dec = torch.empty((N, T, H, D), dtype=torch.float32, device=dev)
+    for t in range(T):
+        ot = torch.empty((N, H, D), dtype=torch.float32, device=dev)
+        kda.kda_decode_step(x[:, t].contiguous().to(dev), w.to(dev), cache,
+                            g[:, t].contiguous().to(dev), beta[:, t].contiguous().to(dev),
+                            state, ot, H=H, D=D)
+        o_dec[:, t] = ot
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    assert rel_max(f64(o_pre).reshape(N, T, H, D), f64(o_dec)) <= 1e-4
+    assert rel_fro(f64(S_pre), f64(state)) <= 1e-5
+    np.testing.assert_array_equal(f64(cache), f64(cache_out))
+
+
+def test_resume_prefill_with_state_and_cache_handoff(kda):
+    """Prefill [0, T1) then [T1, T) with final_state / conv cache handed over
+    equals one prefill over [0, T)."""
+    dev = "cuda"
+    T, T1, H, D = 300, 131, 2, 128
+    C = 3 * H * D
+    r = torch.Generator().manual_seed(12)
+    x = torch.randn((T, C), generator=r).to(torch.bfloat16).to(dev)
+    w = (0.5 * torch.randn((C, 4), generator=r)).to(dev)
+    g = (-5.0 * torch.sigmoid(torch.randn((T, H, D), generator=r) - 4.0)).to(dev)
+    beta = torch.sigmoid(torch.randn((T, H), generator=r)).to(dev)
+    q, k, v, _ = _prefill_gpu(kda, x, w, H, D)
+    o_full = torch.empty_like(v)
+    S_full = torch.empty((1, H, D, D), device=dev)
+    kda.kda_chunk_fwd(q, k, v, g, beta, o_full, final_state=S_full)
+    q1, k1, v1, c1 = _prefill_gpu(kda, x[:T1].contiguous(), w, H, D)
+    S1 = torch.empty((1, H, D, D), device=dev)
+    o1 = torch.empty_like(v1)
+    kda.kda_chunk_fwd(q1, k1, v1, g[:T1].contiguous(), beta[:T1].contiguous(), o1,
+                      final_state=S1)
+    q2, k2, v2, _ = _prefill_gpu(kda, x[T1:].contiguous(), w, H, D, cache_in=c1)
+    o2 = torch.empty_like(v2)
+    S2 = torch.empty((1, H, D, D), device=dev)
+    kda.kda_chunk_fwd(q2, k2, v2, g[T1:].contiguous(), beta[T1:].contiguous(), o2,
+                      initial_state=S1, final_state=S2)
+    torch.cuda.synchronize()
+    assert rel_max(f64(torch.cat([o1, o2])), f64(o_full)) <= TOL_BF16
+    assert rel_fro(f64(S2), f64(S_full)) <= TOL_STATE
