@@ -40,9 +40,9 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 # Algorithmic work per token-head (d = 128; see the design notes).
 D_ = 128
-QKV_DT = 4                                          # q/k/v handed from prologue to chunk: f32
-PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/k/v      = 2304
-CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 2564
+QKV_DT = 2                                          # q/k/v handed from prologue to chunk: f16
+PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/k/v      = 1536
+CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 1796
 FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
 CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 # decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
@@ -50,7 +50,7 @@ DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4
 
 KERNEL_SOURCES = {
     "kda_prologue": "gated_delta_rule_prologue_b200/csrc/kda_prologue.cu",
-    "kda_chunk_fwd": "gated_delta_rule_prologue_b200/csrc/kda_chunk_simt.cu",
+    "kda_chunk_fwd": "gated_delta_rule_prologue_b200/csrc/kda_chunk_tc.cu",
     "kda_decode_step": "gated_delta_rule_prologue_b200/csrc/kda_decode.cu",
 }
 
@@ -262,8 +262,9 @@ def run_ours(args, world, rank, local):
     w = inp.conv_w.to(dev)
     g = inp.g.to(dev)
     beta = inp.beta.to(dev)
-    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
-    k, v, o = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
     fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -385,10 +386,11 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": "k3_prefill: kda_prologue + kda_chunk_fwd over T=32768 tokens, H=96, "
-                        "d_k=d_v=128, chunk 64, bf16 q/k/v projections, fp32 g/beta/state/o",
+                        "d_k=d_v=128, chunk 64, bf16 q/k/v projections, fp16 q/k/v handed "
+                        "from prologue to chunk, fp32 g/beta/state/o",
             "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
             "parallelism": f"replicas x{world} (independent problems, no collective)",
-            "l2": "inputs larger than L2 (15.3 GB touched per step, no flush needed)",
+            "l2": "inputs larger than L2 (10.5 GB touched per step, no flush needed)",
         },
         "roofline": roof,
         "kernels": kernels,

@@ -8,7 +8,7 @@ these names, and importing fails loudly when ``libkda.so`` has not been built
 (``python -m gated_delta_rule_prologue_b200.build``).
 
 Tensor conventions (all contiguous, on the current CUDA device):
-  q, k, v              [T, H, D]       float32 or bfloat16
+  q, k, v              [T, H, D]       float32, bfloat16 or float16
   o                    [T, H, D]       float32 (read-outs are always float32)
   g                    [T, H, Dk]      float32 (log-decay, alpha = exp(g))
   beta                 [T, H]          float32
@@ -40,6 +40,7 @@ __all__ = [
     "KDA_ERR_CUDA",
     "KDA_ERR_DEVICE_TIMEOUT",
     "KDA_ERR_DEVICE_BOUNDS",
+    "KDA_ERR_DEVICE_RANGE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -50,7 +51,8 @@ KDA_ERR_UNSUPPORTED = 2
 KDA_ERR_CUDA = 3
 KDA_ERR_DEVICE_TIMEOUT = 4
 KDA_ERR_DEVICE_BOUNDS = 5
-_F32, _BF16 = 0, 1
+KDA_ERR_DEVICE_RANGE = 6
+_F32, _BF16, _F16 = 0, 1, 2
 
 
 class KdaError(RuntimeError):
@@ -93,6 +95,8 @@ def _dtype(t) -> int:
         return _F32
     if t.dtype == torch.bfloat16:
         return _BF16
+    if t.dtype == torch.float16:
+        return _F16
     raise TypeError(f"unsupported activation dtype {t.dtype}")
 
 

@@ -60,9 +60,9 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
   return pa < pb + nb && pb < pa + na;
 }
 
-size_t esize(kda_dtype dt) { return dt == KDA_BF16 ? 2 : 4; }
+size_t esize(kda_dtype dt) { return dt == KDA_F32 ? 4 : 2; }
 
-bool valid_dtype(kda_dtype dt) { return dt == KDA_F32 || dt == KDA_BF16; }
+bool valid_dtype(kda_dtype dt) { return dt == KDA_F32 || dt == KDA_BF16 || dt == KDA_F16; }
 
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
@@ -75,6 +75,20 @@ bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
   do {                                                                              \
     if ((p) == nullptr) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", name);       \
     if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+// Arrays read element by element (beta, cu_seqlens) only need 4-byte alignment.
+#define KDA_REQUIRE_PTR4(p, name)                                                   \
+  do {                                                                              \
+    if ((p) == nullptr) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", name);       \
+    if (reinterpret_cast<uintptr_t>(p) & 3u)                                        \
+      return fail(KDA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);           \
+  } while (0)
+
+#define KDA_OPT_PTR4(p, name)                                                       \
+  do {                                                                              \
+    if ((p) != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u))                    \
+      return fail(KDA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);           \
   } while (0)
 
 #define KDA_OPT_PTR(p, name)                                                        \
@@ -126,7 +140,7 @@ kda_status kda_prologue(const void *x, const float *conv_w, const void *cache_in
   KDA_REQUIRE_PTR(conv_w, "conv_w");
   KDA_OPT_PTR(cache_in, "cache_in");
   KDA_OPT_PTR(cache_out, "cache_out");
-  KDA_OPT_PTR(cu_seqlens, "cu_seqlens");
+  KDA_OPT_PTR4(cu_seqlens, "cu_seqlens");
   const size_t C = (size_t)3 * H * D, es = esize(dt);
   const size_t act = (size_t)T * H * D * esize(out_dt), cache_bytes = (size_t)N * 3 * C * es;
   KDA_REQUIRE(!overlaps(cache_in, cache_bytes, cache_out, cache_bytes),
@@ -165,12 +179,12 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
     KDA_REQUIRE_PTR(k, "k");
     KDA_REQUIRE_PTR(v, "v");
     KDA_REQUIRE_PTR(g, "g");
-    KDA_REQUIRE_PTR(beta, "beta");
+    KDA_REQUIRE_PTR4(beta, "beta");
     KDA_REQUIRE_PTR(o, "o");
   }
   KDA_OPT_PTR(initial_state, "initial_state");
   KDA_OPT_PTR(final_state, "final_state");
-  KDA_OPT_PTR(cu_seqlens, "cu_seqlens");
+  KDA_OPT_PTR4(cu_seqlens, "cu_seqlens");
   const size_t es = esize(dt);
   const size_t act = (size_t)T * H * Dk * es, obytes = (size_t)T * H * Dv * sizeof(float);
   const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
@@ -187,9 +201,14 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
   kda_status st = device_status_word(&status);
   if (st != KDA_OK) return st;
   if (T == 0 && final_state == nullptr) return KDA_OK;
-  cudaError_t e = kda::launch_chunk_simt(q, k, v, g, beta, scale, initial_state, cu_seqlens, N,
-                                         T, H, Dk, chunk, dt, o, final_state, status,
-                                         (cudaStream_t)stream);
+  cudaError_t e;
+  if (dt != KDA_F32 && Dk == 128 && chunk == 64 && T > 0) {
+    e = kda::launch_chunk_tc(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, dt, o,
+                             final_state, status, (cudaStream_t)stream);
+  } else {
+    e = kda::launch_chunk_simt(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk,
+                               chunk, dt, o, final_state, status, (cudaStream_t)stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
   return KDA_OK;
 }
@@ -205,7 +224,7 @@ kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache,
   KDA_REQUIRE_PTR(conv_w, "conv_w");
   KDA_REQUIRE_PTR(conv_cache, "conv_cache");
   KDA_REQUIRE_PTR(g, "g");
-  KDA_REQUIRE_PTR(beta, "beta");
+  KDA_REQUIRE_PTR4(beta, "beta");
   KDA_REQUIRE_PTR(state, "state");
   KDA_REQUIRE_PTR(o, "o");
   const size_t es = esize(dt), C = (size_t)3 * H * D;

@@ -217,6 +217,8 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
   if (dt == KDA_BF16)
     return launch_d<__nv_bfloat16>(D, chunk, q, k, v, g, beta, scale, s0, cu, N, T, H, o, sN,
                                    status, s);
+  if (dt == KDA_F16)
+    return launch_d<__half>(D, chunk, q, k, v, g, beta, scale, s0, cu, N, T, H, o, sN, status, s);
   return launch_d<float>(D, chunk, q, k, v, g, beta, scale, s0, cu, N, T, H, o, sN, status, s);
 }
 

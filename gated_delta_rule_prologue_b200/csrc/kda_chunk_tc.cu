@@ -1,0 +1,625 @@
+// Chunkwise KDA prefill on the 5th-generation tensor cores (tcgen05 + TMEM,
+// TMA tile loads), bf16 or fp16 q/k/v, d_k = d_v = 128, chunk 64, fp32 state
+// and fp32 read-out.
+//
+// Sources: "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆", 彩蛋 (chunked
+// execution; the K3 report's observation that inside a 16-token block the
+// cumulative log-decay of the bounded gate stays in [-80, 0], so the
+// reciprocal scaling fits the bf16 range and the diagonal blocks can use dense
+// tensor-core products); "AI-Workshop 文献分享 #16 — KDA：给长文本建立可更新的记忆",
+// §10.3; "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解",
+// Figure 1 (the chunk map of the state is affine).
+//
+// Per chunk (entry state S key-first; gamma = inclusive in-chunk cumsum of g).
+// The 64 tokens form two halves, each with a reference in its middle:
+// c_A = gamma_15 for tokens 0..31 and c_B = gamma_47 for tokens 32..63.  With
+// g >= -5 a half spans at most 16 tokens on either side of its reference, so
+// E_r = exp(gamma_r - c(r)) lies in [e^-80, e^75] and every factor below fits
+// fp32/bf16:
+//   Gram  D_G = [K*E ; Q*E] . [ver_A ; ver_B]^T          (M=128, N=96, K=128)
+//         ver_A_i = k_i / E_i                     (i < 32, reference c_A)
+//         ver_B_i = k_i / E_i * exp(c_B - c(i))   (i < 64, reference c_B; for i < 32
+//                   the factor is applied as two halves: it alone can underflow
+//                   while the product with the row factor of token 32 cannot)
+//         rows of the first half read ver_A, rows of the second half ver_B.
+//         A[r,i] = beta_r D_G[r, i] (i < r);  P[r,i] = D_G[64+r, i] (i < r)
+//         P[r,r] = <q_r, k_r> is taken in fp32 from the unscaled tiles.
+//   WY    T = (I + A)^{-1} (fp32, blocked over 16x16 blocks)
+//         W^T = (beta K G)^T T^T,  Ut^T = (beta V)^T T^T           (G_r = exp(gamma_r))
+//   state U^T = Ut^T - S^T W^T,   O^T = S^T (Q G)^T + U^T P_strict^T
+//         S <- diag(G_last) S + U^T (K * G_last / G)    (value-major registers)
+//   Operand types: the Gram operands are bf16 (they need the e^+-80 range);
+//   every other operand (T, beta K G, beta V, S^T, W, Q G, U^T, P, K') has a
+//   modest range and is fp16, whose 11-bit significand keeps the read-out
+//   within the parity bound when the decay is slow.  A value that would not
+//   fit fp16 (|x| >= 2^15) is recorded in the status word.
+//   fp32 diagonal terms: u_r gets beta_r v_r - f16(beta_r v_r) back, and
+//   o_r gets <q_r, k_r> u_r in fp32, so a token's own (dominant) contribution
+//   to its read-out is never rounded to bf16.
+// One CTA (256 threads) per (sequence, head); the chunks of a sequence run in
+// order, the next chunk's tiles stream in by TMA during the current one.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kda_common.cuh"
+#include "kda_tcgen05.cuh"
+
+namespace kda {
+namespace {
+using namespace tc;
+
+constexpr int kThreads = 256;
+
+// ---- shared memory plan (byte offsets from a 1024-aligned base) ----------------
+constexpr uint32_t SM_Q = 0;                // raw q tile [64][128] bf16
+constexpr uint32_t SM_K = SM_Q + 16384;     // raw k tile
+constexpr uint32_t SM_V = SM_K + 16384;     // raw v tile
+constexpr uint32_t SM_G = SM_V + 16384;     // raw g [64][128] f32 -> gamma -> E -> (A^T, T)
+constexpr uint32_t SM_X = SM_G + 32768;     // 64 KB, reused within a chunk:
+constexpr uint32_t SM_GA = SM_X;            //   Gram A operand (K-major 128 x 128)  32 KB
+constexpr uint32_t SM_GB = SM_X + 32768;    //   Gram B operand (K-major  96 x 128)  24 KB
+constexpr uint32_t SM_BKG = SM_X;           //   beta K G (MN-major, 64 k-rows)     16 KB; then W op
+constexpr uint32_t SM_BV = SM_X + 16384;    //   beta V   (MN-major)                16 KB
+constexpr uint32_t SM_QG = SM_X + 32768;    //   Q G      (K-major 64 x 128)        16 KB
+constexpr uint32_t SM_KP = SM_X + 49152;    //   K G_last/G (MN-major)              16 KB
+constexpr uint32_t SM_TOP = SM_X + 65536;   // T operand (K-major 64 x 64) 8 KB; before it is
+constexpr uint32_t SM_XS = SM_TOP;          //   written: scratch (cumsum totals, inverse blocks)
+constexpr uint32_t SM_POP = SM_TOP + 8192;  // P operand (K-major 64 x 64)          8 KB
+constexpr uint32_t SM_ST = SM_POP + 8192;   // S^T operand (K-major 128 x 128) 32 KB; then U^T
+constexpr uint32_t SM_F = SM_ST + 32768;    // per-channel fp32 factors [128] each:
+constexpr uint32_t F_CA = SM_F;             //   c_A = gamma_15
+constexpr uint32_t F_CB = F_CA + 512;       //   c_B = gamma_47
+constexpr uint32_t F_ECA = F_CB + 512;      //   exp(c_A)
+constexpr uint32_t F_ECB = F_ECA + 512;     //   exp(c_B)
+constexpr uint32_t F_EBA = F_ECB + 512;     //   exp((c_B - c_A) / 2): applied twice, so no
+                                            //   partial product underflows (c_B - c_A >= -160)
+constexpr uint32_t F_ELA = F_EBA + 512;     //   exp(gamma_last - c_A)
+constexpr uint32_t F_ELB = F_ELA + 512;     //   exp(gamma_last - c_B)
+constexpr uint32_t F_EGC = F_ELB + 512;     //   exp(gamma_last)
+constexpr uint32_t SM_BETA = F_EGC + 512;   // beta of the chunk     [64]
+constexpr uint32_t SM_PDIAG = SM_BETA + 256;// <q_r, k_r> in fp32    [64]
+constexpr uint32_t SM_BAR = SM_PDIAG + 256; // two mbarriers
+constexpr uint32_t SM_SLOT = SM_BAR + 16;   // TMEM base address
+constexpr uint32_t SM_TOTAL = SM_SLOT + 16;
+constexpr uint32_t SM_ALLOC = SM_TOTAL + 1024;  // slack for 1024-byte alignment
+static_assert(SM_ALLOC <= 232448, "shared memory budget");
+
+// ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
+constexpr uint32_t TM_G = 0;     // Gram, 96 columns
+constexpr uint32_t TM_W = 160;   // W^T, 64
+constexpr uint32_t TM_U = 224;   // U^T, 64
+constexpr uint32_t TM_O = 288;   // O^T, 64
+constexpr uint32_t TM_S = 352;   // delta S^T, 128
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t kTmaBytes = 3 * 16384 + 32768;
+
+
+// 8 consecutive 16-bit activations of a raw tile (bf16 or fp16) as floats.
+template <typename Tin>
+__device__ __forceinline__ void ld8_in(const uint8_t *p, float (&f)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const Tin *h = reinterpret_cast<const Tin *>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = to_f32(h[i]);
+}
+
+__device__ __forceinline__ void ld8_f32(const float *p, float (&f)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0];
+  const float4 b = reinterpret_cast<const float4 *>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// All threads wait for a barrier phase; false (and a recorded timeout) if any
+// thread gave up.  Also acts as a CTA-wide barrier.
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *status) {
+  const bool ok = mbar_wait(bar, parity);
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
+    return false;
+  }
+  return true;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const float *__restrict__ beta, float scale, const float *s0,
+                const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
+                int *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);
+  uint64_t *bar_mma = bar_tma + 1;
+  uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SM_SLOT);
+  float *Gf = reinterpret_cast<float *>(sm + SM_G);
+  float *beta_s = reinterpret_cast<float *>(sm + SM_BETA);
+  float *pdiag = reinterpret_cast<float *>(sm + SM_PDIAG);
+  float *fca = reinterpret_cast<float *>(sm + F_CA);
+  float *fcb = reinterpret_cast<float *>(sm + F_CB);
+  float *feca = reinterpret_cast<float *>(sm + F_ECA);
+  float *fecb = reinterpret_cast<float *>(sm + F_ECB);
+  float *feba = reinterpret_cast<float *>(sm + F_EBA);
+  float *fela = reinterpret_cast<float *>(sm + F_ELA);
+  float *felb = reinterpret_cast<float *>(sm + F_ELB);
+  float *fegc = reinterpret_cast<float *>(sm + F_EGC);
+
+  int bos, eos;
+  seq_bounds(cu, n, T, status, bos, eos);
+  const int nchunks = (eos - bos + 63) / 64;
+
+  if (warp == 0) tmem_alloc(slot, TM_COLS);
+  if (tid == 0) {
+    mbar_init(bar_tma, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_g);
+  }
+
+  // State rows held in registers: row j of S^T, key columns [dk0, dk0 + 64).
+  const int j = 32 * quad + lane;
+  const int dk0 = 64 * half;
+  float S[64];
+  {
+    const float *src = s0 ? s0 + (((size_t)n * H + h) * 128 + j) * 128 + dk0 : nullptr;
+#pragma unroll
+    for (int x = 0; x < 64; x += 4) {
+      float4 f = src ? *reinterpret_cast<const float4 *>(src + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+      S[x] = f.x; S[x + 1] = f.y; S[x + 2] = f.z; S[x + 3] = f.w;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t lane_addr = static_cast<uint32_t>(32 * quad) << 16;
+
+  auto issue_tma = [&](int t) {
+    mbar_arrive_expect_tx(bar_tma, kTmaBytes);
+    tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
+    tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, h, t);
+    tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
+    tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, h, t);
+  };
+  if (tid == 0 && nchunks > 0) issue_tma(bos);
+
+  uint32_t tma_par = 0, mma_par = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    const int t0 = bos + c * 64;
+    const int Lc = min(64, eos - t0);
+
+    // ---- P0: raw tiles of this chunk ---------------------------------------------
+    if (!wait_all(bar_tma, tma_par, status)) break;
+    tma_par ^= 1;
+
+    // ---- P1: beta, in-chunk cumulative log-decay, per-channel factors, E ------------
+    if (tid < 64) beta_s[tid] = tid < Lc ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    {
+      const int d = tid & 127, part = tid >> 7;
+      float vals[32];
+      float acc = 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const int rr = 32 * part + r;
+        const float gv = Gf[rr * 128 + d];
+        acc += rr < Lc ? gv : 0.f;
+        vals[r] = acc;
+      }
+      float *tot = reinterpret_cast<float *>(sm + SM_XS);
+      if (part == 0) tot[d] = acc;
+      __syncthreads();
+      const float off = part ? tot[d] : 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) Gf[(32 * part + r) * 128 + d] = vals[r] + off;
+    }
+    __syncthreads();
+    if (tid < 128) {
+      const int d = tid;
+      const float ca = Gf[15 * 128 + d], cb = Gf[47 * 128 + d], cl = Gf[63 * 128 + d];
+      fca[d] = ca;
+      fcb[d] = cb;
+      feca[d] = expf(ca);
+      fecb[d] = expf(cb);
+      feba[d] = expf(0.5f * (cb - ca));
+      fela[d] = expf(cl - ca);
+      felb[d] = expf(cl - cb);
+      fegc[d] = expf(cl);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < 64 * 128; idx += kThreads) {
+      const int r = idx >> 7, d = idx & 127;
+      Gf[idx] = expf(Gf[idx] - (r < 32 ? fca[d] : fcb[d]));  // E_r in [e^-80, e^75]
+    }
+    __syncthreads();
+
+    // ---- P2: Gram operands -------------------------------------------------------------
+#pragma unroll 1
+    for (int m = 0; m < 4; ++m) {
+      const int p = tid + kThreads * m;
+      const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
+      const bool valid = r < Lc;
+      float k8[8], q8[8], e8[8];
+      ld8_in<Tin>(sm + SM_K + r * 256 + c8 * 16, k8);
+      ld8_in<Tin>(sm + SM_Q + r * 256 + c8 * 16, q8);
+      ld8_f32(Gf + r * 128 + d0, e8);
+      float a[8], b[8], ki[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f;
+        a[e] = kk * e8[e];
+        b[e] = qq * e8[e];
+        ki[e] = kk * __frcp_rn(e8[e]);
+      }
+      st_shared_16(sm + SM_GA, kmaj_off(128, r, c8), pack8_bf16(a));
+      st_shared_16(sm + SM_GA, kmaj_off(128, 64 + r, c8), pack8_bf16(b));
+      if (r < 32) {
+        st_shared_16(sm + SM_GB, kmaj_off(96, r, c8), pack8_bf16(ki));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * feba[d0 + e]) * feba[d0 + e];
+      }
+      st_shared_16(sm + SM_GB, kmaj_off(96, 32 + r, c8), pack8_bf16(ki));
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---- P3: Gram MMA ------------------------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
+      constexpr uint32_t id = idesc_bf16(128, 96, false, false);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, mma_par, status)) break;
+    mma_par ^= 1;
+    tc_fence_after();
+
+    // ---- P4a: WY / output operands (the Gram operands are dead) -------------------------
+#pragma unroll 1
+    for (int m = 0; m < 4; ++m) {
+      const int p = tid + kThreads * m;
+      const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
+      const bool valid = r < Lc;
+      const float bt = beta_s[r];
+      const float *fec = r < 32 ? feca : fecb;
+      const float *fel = r < 32 ? fela : felb;
+      float k8[8], q8[8], v8[8], e8[8];
+      ld8_in<Tin>(sm + SM_K + r * 256 + c8 * 16, k8);
+      ld8_in<Tin>(sm + SM_Q + r * 256 + c8 * 16, q8);
+      ld8_in<Tin>(sm + SM_V + r * 256 + c8 * 16, v8);
+      ld8_f32(Gf + r * 128 + d0, e8);
+      float bkg[8], bv[8], qg[8], kp[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f, vv = valid ? v8[e] : 0.f;
+        const float ec = fec[d0 + e];
+        bkg[e] = bt * kk * e8[e] * ec;
+        bv[e] = bt * vv;
+        qg[e] = qq * e8[e] * ec;
+        kp[e] = kk * __frcp_rn(e8[e]) * fel[d0 + e];
+      }
+      st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
+      st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
+      st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
+      st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
+    }
+    __syncthreads();
+
+    // ---- P4b: <q_r, k_r> in fp32; Gram read-out -> A^T (fp32), strict P operand ---------
+    float *AT = Gf;           // AT[i*64 + r] = A[r][i]
+    float *TT = Gf + 4096;    // TT[r*64 + c] = T[r][c]
+    for (int idx = tid; idx < 4096 / 4; idx += kThreads)
+      reinterpret_cast<float4 *>(AT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int idx = tid; idx < 8192 / 16; idx += kThreads)
+      reinterpret_cast<uint4 *>(sm + SM_POP)[idx] = make_uint4(0u, 0u, 0u, 0u);
+    {
+      const int r = tid >> 2, part = tid & 3;
+      float acc = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float q8[8], k8[8];
+        ld8_in<Tin>(sm + SM_Q + r * 256 + (part * 4 + c8) * 16, q8);
+        ld8_in<Tin>(sm + SM_K + r * 256 + (part * 4 + c8) * 16, k8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = fmaf(q8[e], k8[e], acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (part == 0) pdiag[r] = r < Lc ? acc : 0.f;
+    }
+    __syncthreads();
+    {
+      const bool isP = quad >= 2;
+      const int r = 32 * (quad & 1) + lane;
+      // first half: columns [0, 32) (i = col); second half: [32, 96) (i = col - 32)
+      const bool active = (quad & 1) || half == 0;
+      if (active) {
+        const int col0 = (quad & 1) ? 32 + 32 * half : 0;
+        const int ibase = (quad & 1) ? 32 * half : 0;
+        float v[32];
+        tmem_ld32(tmem + lane_addr + TM_G + col0, v);
+        const float br = beta_s[r];
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          const int i0 = ibase + 8 * g8;
+          if (!isP) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
+          } else if (i0 < r) {
+            float p8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
+            st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 --------------------------------------
+    if (tid < 64) {
+      const int base = 16 * (tid >> 4), jj = tid & 15;
+      float x[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        float acc = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < rr; ++ii) acc = fmaf(AT[(base + ii) * 64 + base + rr], x[ii], acc);
+        x[rr] = rr == jj ? 1.f : (rr < jj ? 0.f : -acc);
+      }
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = x[rr];
+    }
+    __syncthreads();
+    {
+      float *XS = reinterpret_cast<float *>(sm + SM_XS);
+      for (int dlt = 1; dlt <= 3; ++dlt) {
+        const int nblk = 4 - dlt;
+        for (int idx = tid; idx < nblk * 256; idx += kThreads) {
+          const int s = dlt + (idx >> 8), sp = s - dlt, a = (idx >> 4) & 15, b = idx & 15;
+          float acc = 0.f;
+          for (int mb = sp; mb < s; ++mb) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              acc = fmaf(AT[(16 * mb + t) * 64 + 16 * s + a], TT[(16 * mb + t) * 64 + 16 * sp + b], acc);
+          }
+          XS[idx] = acc;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < nblk * 256; idx += kThreads) {
+          const int s = dlt + (idx >> 8), sp = s - dlt, a = (idx >> 4) & 15, b = idx & 15;
+          float acc = 0.f;
+          for (int t = 0; t <= a; ++t)
+            acc = fmaf(TT[(16 * s + a) * 64 + 16 * s + t], XS[(idx & ~255) + t * 16 + b], acc);
+          TT[(16 * s + a) * 64 + 16 * sp + b] = -acc;
+        }
+        __syncthreads();
+      }
+    }
+    for (int p = tid; p < 512; p += kThreads) {
+      const int r = p >> 3, c8 = p & 7;
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int cc = 8 * c8 + e;
+        f[e] = cc < r ? TT[r * 64 + cc] : (cc == r ? 1.f : 0.f);
+      }
+      st_shared_16(sm + SM_TOP, kmaj_off(64, r, c8), pack8_f16(f));
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> bf16 operand ------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t top = smem_u32(sm + SM_TOP), bkg = smem_u32(sm + SM_BKG);
+      const uint32_t bv = smem_u32(sm + SM_BV);
+      constexpr uint32_t id = idesc_fp16(128, 64, true, false);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16(tmem + TM_W, desc_mnmajor(bkg, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16(tmem + TM_U, desc_mnmajor(bv, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
+      mma_commit(bar_mma);
+    }
+    {
+      float amax = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          f[e] = S[8 * cc + e];
+          amax = fmaxf(amax, fabsf(f[e]));
+        }
+        st_shared_16(sm + SM_ST, kmaj_off(128, j, 8 * half + cc), pack8_f16(f));
+      }
+      if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+    }
+    fence_async_smem();
+    if (!wait_all(bar_mma, mma_par, status)) break;
+    mma_par ^= 1;
+    tc_fence_after();
+
+    // ---- P7: W^T read-out -> -W operand (MN-major, over beta K G) --------------------------
+    {
+      float v[32];
+      tmem_ld32(tmem + lane_addr + TM_W + 32 * half, v);
+      const int dk = 32 * quad + lane;
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = -v[8 * g8 + e];
+        st_shared_16(sm + SM_BKG, mnmaj_off(128, dk, 4 * half + g8), pack8_f16(f));
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- P8: U^T = Ut^T - S^T W^T ;  O^T = S^T (Q G)^T -------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t st = smem_u32(sm + SM_ST), wop = smem_u32(sm + SM_BKG);
+      const uint32_t qg = smem_u32(sm + SM_QG);
+      constexpr uint32_t idU = idesc_fp16(128, 64, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TM_U, desc_kmajor(st, 128, ks), desc_mnmajor(wop, 128, ks), idU, 1);
+      constexpr uint32_t idO = idesc_fp16(128, 64, false, false);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TM_O, desc_kmajor(st, 128, ks), desc_kmajor(qg, 64, ks), idO, ks > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, mma_par, status)) break;
+    mma_par ^= 1;
+    tc_fence_after();
+
+    // ---- P9: U read-out (+ fp32 diagonal), U^T operand -----------------------------------
+    float u[32];
+    tmem_ld32(tmem + lane_addr + TM_U + 32 * half, u);
+    {
+      const Tin *Vr = reinterpret_cast<const Tin *>(sm + SM_V);
+#pragma unroll
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * half + i;
+        const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
+        const float bvv = beta_s[r] * vv;
+        u[i] += bvv - __half2float(__float2half_rn(bvv));
+        amax = fmaxf(amax, fmaxf(fabsf(u[i]), fabsf(bvv)));
+      }
+      if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = u[8 * g8 + e];
+        st_shared_16(sm + SM_ST, kmaj_off(128, j, 4 * half + g8), pack8_f16(f));
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- P10: O^T += U^T P^T ; delta S^T = U^T K' ; next chunk's tiles ------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ut = smem_u32(sm + SM_ST), pop = smem_u32(sm + SM_POP);
+      const uint32_t kp = smem_u32(sm + SM_KP);
+      constexpr uint32_t idO = idesc_fp16(128, 64, false, false);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16(tmem + TM_O, desc_kmajor(ut, 128, ks), desc_kmajor(pop, 64, ks), idO, 1);
+      constexpr uint32_t idS = idesc_fp16(128, 128, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16(tmem + TM_S, desc_kmajor(ut, 128, ks), desc_mnmajor(kp, 64, ks), idS, ks > 0);
+      mma_commit(bar_mma);
+      if (c + 1 < nchunks) issue_tma(t0 + 64);
+    }
+    if (!wait_all(bar_mma, mma_par, status)) break;
+    mma_par ^= 1;
+    tc_fence_after();
+
+    // ---- P11: outputs and state update ----------------------------------------------------
+    {
+      float ov[32];
+      tmem_ld32(tmem + lane_addr + TM_O + 32 * half, ov);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * half + i;
+        if (r < Lc) o[((size_t)(t0 + r) * H + h) * 128 + j] = scale * fmaf(pdiag[r], u[i], ov[i]);
+      }
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        float dv[32];
+        tmem_ld32(tmem + lane_addr + TM_S + 64 * half + 32 * l, dv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          S[32 * l + i] = fmaf(S[32 * l + i], fegc[dk0 + 32 * l + i], dv[i]);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (sN) {
+    float *dst = sN + (((size_t)n * H + h) * 128 + j) * 128 + dk0;
+#pragma unroll
+    for (int x = 0; x < 64; x += 4)
+      *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a [T, H, 128] tensor: box = 64 tokens x 1 head x 128 channels.
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esz, int H, int T) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)H * 128 * esz};
+  cuuint32_t box[3] = {128, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *s0, const int32_t *cu,
+                            int N, int T, int H, kda_dtype dt, float *o, float *sN, int *status,
+                            cudaStream_t s) {
+  const CUtensorMapDataType act =
+      dt == KDA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tq, tk, tv, tg;
+  if (!make_map(&tq, q, act, 2, H, T) || !make_map(&tk, k, act, 2, H, T) ||
+      !make_map(&tv, v, act, 2, H, T) ||
+      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+    return cudaErrorInvalidValue;
+  auto kern = dt == KDA_BF16 ? chunk_tc_kernel<__nv_bfloat16> : chunk_tc_kernel<__half>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SM_ALLOC);
+  if (e != cudaSuccess) return e;
+  const long long blocks = (long long)N * H;
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
+                                                    sN, status);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

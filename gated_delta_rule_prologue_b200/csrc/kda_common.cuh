@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -15,12 +16,14 @@ namespace kda {
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
 
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
 
 // Load/store 8 consecutive elements (16 B for bf16, 32 B for f32) as floats.
 __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&out)[8]) {
@@ -29,6 +32,16 @@ __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&out)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float2 f = __bfloat1622float2(h[i]);
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const __half *p, float (&out)[8]) {
+  uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
     out[2 * i] = f.x;
     out[2 * i + 1] = f.y;
   }
@@ -44,6 +57,13 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&in)[8]) {
   __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
 #pragma unroll
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(in[2 * i], in[2 * i + 1]);
+  *reinterpret_cast<uint4 *>(p) = u;
+}
+__device__ __forceinline__ void store8(__half *p, const float (&in)[8]) {
+  uint4 u;
+  __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(in[2 * i], in[2 * i + 1]);
   *reinterpret_cast<uint4 *>(p) = u;
 }
 __device__ __forceinline__ void store8(float *p, const float (&in)[8]) {
@@ -114,6 +134,6 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               kda_dtype dt, float *o, float *sN, int *status, cudaStream_t s);
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, float scale, const float *s0, const int32_t *cu,
-                            int N, int T, int H, float *o, float *sN, int *status,
+                            int N, int T, int H, kda_dtype dt, float *o, float *sN, int *status,
                             cudaStream_t s);
 }  // namespace kda

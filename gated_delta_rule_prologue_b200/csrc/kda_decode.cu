@@ -170,6 +170,7 @@ cudaError_t launch_decode(const void *x, const float *w, void *cache, const floa
   if ((long long)N * H >= (1LL << 31)) return cudaErrorInvalidValue;
   if (dt == KDA_BF16)
     return launch_d<__nv_bfloat16>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
+  if (dt == KDA_F16) return launch_d<__half>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
   return launch_d<float>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
 }
 

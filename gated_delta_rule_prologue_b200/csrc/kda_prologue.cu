@@ -202,20 +202,35 @@ cudaError_t launch_d(int D, const void *x, const float *w, const void *ci, void 
   }
 }
 
+template <typename Tin>
+cudaError_t launch_out(kda_dtype out_dt, int D, const void *x, const float *w, const void *ci,
+                       void *co, const int32_t *cu, int N, int T, int H, void *q, void *k,
+                       void *v, int *status, cudaStream_t s) {
+  switch (out_dt) {
+    case KDA_BF16:
+      return launch_d<Tin, __nv_bfloat16>(D, x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    case KDA_F16: return launch_d<Tin, __half>(D, x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+    default: return launch_d<Tin, float>(D, x, w, ci, co, cu, N, T, H, q, k, v, status, s);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in, void *cache_out,
                             const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
                             kda_dtype out_dt, void *q, void *k, void *v, int *status,
                             cudaStream_t s) {
-  using bf = __nv_bfloat16;
-  if (dt == KDA_BF16 && out_dt == KDA_BF16)
-    return launch_d<bf, bf>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
-  if (dt == KDA_BF16)
-    return launch_d<bf, float>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
-  if (out_dt == KDA_BF16)
-    return launch_d<float, bf>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
-  return launch_d<float, float>(D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v, status, s);
+  switch (dt) {
+    case KDA_BF16:
+      return launch_out<__nv_bfloat16>(out_dt, D, x, w, cache_in, cache_out, cu, N, T, H, q, k,
+                                       v, status, s);
+    case KDA_F16:
+      return launch_out<__half>(out_dt, D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v,
+                                status, s);
+    default:
+      return launch_out<float>(out_dt, D, x, w, cache_in, cache_out, cu, N, T, H, q, k, v,
+                               status, s);
+  }
 }
 
 }  // namespace kda

@@ -27,12 +27,13 @@
  *     contiguous one (the transpose of the pages' key-first S; [W1 第三站]
  *     allows a transposed storage layout).
  *   - Activations (q, k, v, x, conv cache) have the element type `dt`
- *     (KDA_F32 or KDA_BF16).  g, beta, the state and every read-out o are
+ *     (KDA_F32, KDA_BF16 or KDA_F16).  g, beta, the state and every read-out o are
  *     always float32: o is heavy-tailed (its largest entries are many times
  *     its RMS), so rounding it to bf16 alone would exceed the parity bound
  *     max|o - o_ref| <= 2e-2 * RMS(o_ref).
- *   - Every pointer must be 16-byte aligned.  Outputs must not overlap
- *     inputs unless an argument says "in/out".
+ *   - Every pointer must be 16-byte aligned, except beta and cu_seqlens
+ *     (4-byte aligned).  Outputs must not overlap inputs unless an argument
+ *     says "in/out".
  *   - On any non-OK return, kda_last_error() gives a message (thread-local).
  */
 #ifndef KDA_H_
@@ -50,10 +51,12 @@ typedef enum {
   KDA_ERR_UNSUPPORTED = 2,    /* valid request outside the compiled domain     */
   KDA_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed   */
   KDA_ERR_DEVICE_TIMEOUT = 4, /* (status word) a bounded device wait ran out   */
-  KDA_ERR_DEVICE_BOUNDS = 5   /* (status word) device-side index check failed  */
+  KDA_ERR_DEVICE_BOUNDS = 5,  /* (status word) device-side index check failed  */
+  KDA_ERR_DEVICE_RANGE = 6    /* (status word) a value left the range of the
+                                 fp16 tensor-core operands (|x| >= 2^15)      */
 } kda_status;
 
-typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1, KDA_F16 = 2 } kda_dtype;
 
 typedef struct CUstream_st *kda_stream_t; /* same type as cudaStream_t */
 
@@ -106,9 +109,10 @@ kda_status kda_prologue(const void *x, const float *conv_w, const void *cache_in
  *                 from initial_state[n]
  *   o             [T, H, Dv] float32 output
  *   final_state   [N, H, Dv, Dk] f32 or NULL; may alias initial_state
- * Supported: dt == KDA_F32: Dk == Dv in {16, 32, 64, 128}, chunk in {16, 32,
- *   64} (exact-fp32 CUDA-core path).  dt == KDA_BF16: the same domain; with
- *   Dk == Dv == 128 and chunk == 64 it runs the tcgen05 tensor-core path.
+ * Supported: Dk == Dv in {16, 32, 64, 128}, chunk in {16, 32, 64}.  With
+ *   dt == KDA_BF16 or KDA_F16, Dk == Dv == 128 and chunk == 64 the call runs
+ *   the tcgen05 tensor-core path; every other case runs the exact-fp32
+ *   CUDA-core path.
  */
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                          const float *beta, float scale, const float *initial_state,

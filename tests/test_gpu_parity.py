@@ -42,6 +42,21 @@ def f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+# Unit roundoff of each storage type: rounding to nearest moves a value by at
+# most this fraction of itself (bf16: 8 significant bits, fp16: 11).
+UNIT_ROUNDOFF = {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}
+
+
+def check_rounded(got, ref, dtype):
+    """Elementwise check of a stored activation: the rounding of the storage
+    type plus float32 arithmetic noise (1e-5 of the RMS)."""
+    rms = np.sqrt(np.mean(ref * ref))
+    if dtype in UNIT_ROUNDOFF:
+        assert np.all(np.abs(f64(got) - ref) <= UNIT_ROUNDOFF[dtype] * np.abs(ref) + 1e-5 * rms)
+    else:
+        assert rel_max(f64(got), ref) <= 1e-5
+
+
 def run_chunk(kda, inp, *, chunk=None, in_place=False):
     dev = "cuda"
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
@@ -130,6 +145,17 @@ def test_chunk_size_does_not_change_results(kda):
         assert rel_fro(S, outs[0][1]) <= 1e-5
 
 
+def test_tensor_core_and_cuda_core_paths_agree(kda):
+    """bf16, d=128: chunk 64 runs the tcgen05 kernel, chunk 32 the fp32
+    CUDA-core kernel; both within the bf16 bound of each other."""
+    inp = W.random_prefill(9, 333, 2, 128, s0_std=0.1, lengths=[200, 133],
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 1.0))
+    o_tc, S_tc = run_chunk(kda, inp, chunk=64)
+    o_cc, S_cc = run_chunk(kda, inp, chunk=32)
+    assert rel_max(o_tc, o_cc) <= TOL_BF16
+    assert rel_fro(S_tc, S_cc) <= TOL_STATE
+
+
 def test_malformed_cu_seqlens_sets_status_without_fault(kda):
     inp = W.random_prefill(7, 64, 1, 16, bf16=False, lengths=[30, 34], chunk=16)
     dev = "cuda"
@@ -148,6 +174,7 @@ def test_malformed_cu_seqlens_sets_status_without_fault(kda):
 
 @pytest.mark.parametrize("dtype,out_dtype,D", [(torch.bfloat16, torch.bfloat16, 128),
                                                (torch.bfloat16, torch.float32, 128),
+                                               (torch.bfloat16, torch.float16, 128),
                                                (torch.float32, torch.float32, 16),
                                                (torch.float32, torch.bfloat16, 64)])
 def test_prologue_parity_varlen_with_cache(kda, dtype, out_dtype, D):
@@ -169,13 +196,7 @@ def test_prologue_parity_varlen_with_cache(kda, dtype, out_dtype, D):
     assert kda.kda_get_device_status() == 0
     q_ref, k_ref, v_ref, c_ref = o_prologue(x, w, H, D, cu.numpy(), cache)
     for got, ref in ((q, q_ref), (k, k_ref), (v, v_ref)):
-        if out_dtype == torch.bfloat16:
-            # rounding to bf16 (8 significant bits, nearest-even) moves a value by
-            # at most 2^-9 of itself; allow that plus float32 arithmetic noise
-            rms = np.sqrt(np.mean(ref * ref))
-            assert np.all(np.abs(f64(got) - ref) <= 2.0 ** -9 * np.abs(ref) + 1e-5 * rms)
-        else:
-            assert rel_max(f64(got), ref) <= 1e-5
+        check_rounded(got, ref, out_dtype)
     np.testing.assert_array_equal(f64(cache_out), c_ref)   # a copy of inputs: exact
 
 
@@ -188,10 +209,10 @@ def test_k3_prefill_full_size_sampled_heads(kda):
     T, H, D = inp.T, inp.H, inp.D
     dev = "cuda"
     x = inp.x.to(dev)
-    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
     k, v = torch.empty_like(q), torch.empty_like(q)
     kda.kda_prologue(x, inp.conv_w.to(dev), q, k, v, H=H, D=D)
-    o = torch.empty_like(v)
+    o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
     fs = torch.empty((1, H, D, D), device=dev)
     kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, scale=inp.scale,
                       final_state=fs, chunk=inp.chunk)
@@ -201,8 +222,8 @@ def test_k3_prefill_full_size_sampled_heads(kda):
     for h in (0, 53, 95):
         xh, wh, gh, bh = W.k3_prefill_head(h)
         qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
-        assert rel_max(f64(q[:, h]), qr[:, 0]) <= 1e-5
-        assert rel_max(f64(v[:, h]), vr[:, 0]) <= 1e-5
+        check_rounded(q[:, h], qr[:, 0], torch.float16)
+        check_rounded(v[:, h], vr[:, 0], torch.float16)
         o_ref, S_ref = kda_recurrent(qr, kr, vr, gh[:, None, :], bh[:, None], inp.scale)
         assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16
         assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
@@ -252,11 +273,11 @@ def test_decode256_full_size_sampled(kda):
 
 # --- cross-checks between GPU paths ------------------------------------------------
 
-def _prefill_gpu(kda, x, w, H, D, cache_in=None, s0=None, cu=None):
+def _prefill_gpu(kda, x, w, H, D, cache_in=None, s0=None, cu=None, act=torch.float32):
     dev = "cuda"
     T = x.shape[0]
     N = 1 if cu is None else cu.numel() - 1
-    q = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    q = torch.empty((T, H, D), dtype=act, device=dev)
     k, v = torch.empty_like(q), torch.empty_like(q)
     cache_out = torch.empty((N, 3, 3 * H * D), dtype=x.dtype, device=dev)
     kda.kda_prologue(x, w, q, k, v, H=H, D=D, cache_in=cache_in, cache_out=cache_out,
@@ -278,7 +299,7 @@ def test_decode_kernel_matches_prologue_plus_chunk_kernel(kda):
     s0 = 0.05 * torch.randn((N, H, D, D), generator=r)
     cu = torch.arange(0, N * T + 1, T, dtype=torch.int32, device=dev)
     q, k, v, cache_out = _prefill_gpu(kda, x.reshape(N * T, C).to(dev), w.to(dev), H, D, cu=cu)
-    o_pre = torch.empty_like(v)
+    o_pre = torch.empty(v.shape, dtype=torch.float32, device=dev)
     S_pre = torch.empty((N, H, D, D), device=dev)
     kda.kda_chunk_fwd(q, k, v, g.reshape(N * T, H, D).to(dev), beta.reshape(N * T, H).to(dev),
                       o_pre, initial_state=s0.to(dev), final_state=S_pre, cu_seqlens=cu)
@@ -298,31 +319,33 @@ def test_decode_kernel_matches_prologue_plus_chunk_kernel(kda):
     np.testing.assert_array_equal(f64(cache), f64(cache_out))
 
 
-def test_resume_prefill_with_state_and_cache_handoff(kda):
-    """Prefill [0, T1) then [T1, T) with final_state / conv cache handed over
-    equals one prefill over [0, T)."""
+@pytest.mark.parametrize("act", [torch.float32, torch.float16])
+def test_resume_prefill_with_state_and_cache_handoff(kda, act):
+    """Prefill [0, T1) then [T1, T) with final_state / conv cache handed over:
+    both halves match the oracle's single pass over [0, T) (float32 hand-off:
+    CUDA-core chunk kernel; float16 hand-off: tensor-core chunk kernel)."""
     dev = "cuda"
     T, T1, H, D = 300, 131, 2, 128
     C = 3 * H * D
     r = torch.Generator().manual_seed(12)
-    x = torch.randn((T, C), generator=r).to(torch.bfloat16).to(dev)
-    w = (0.5 * torch.randn((C, 4), generator=r)).to(dev)
-    g = (-5.0 * torch.sigmoid(torch.randn((T, H, D), generator=r) - 4.0)).to(dev)
-    beta = torch.sigmoid(torch.randn((T, H), generator=r)).to(dev)
-    q, k, v, _ = _prefill_gpu(kda, x, w, H, D)
-    o_full = torch.empty_like(v)
-    S_full = torch.empty((1, H, D, D), device=dev)
-    kda.kda_chunk_fwd(q, k, v, g, beta, o_full, final_state=S_full)
-    q1, k1, v1, c1 = _prefill_gpu(kda, x[:T1].contiguous(), w, H, D)
+    x = torch.randn((T, C), generator=r).to(torch.bfloat16)
+    w = 0.5 * torch.randn((C, 4), generator=r)
+    g = -5.0 * torch.sigmoid(torch.randn((T, H, D), generator=r) - 4.0)
+    beta = torch.sigmoid(torch.randn((T, H), generator=r))
+    xd, wd, gd, bd = x.to(dev), w.to(dev), g.to(dev), beta.to(dev)
+    q1, k1, v1, c1 = _prefill_gpu(kda, xd[:T1].contiguous(), wd, H, D, act=act)
     S1 = torch.empty((1, H, D, D), device=dev)
-    o1 = torch.empty_like(v1)
-    kda.kda_chunk_fwd(q1, k1, v1, g[:T1].contiguous(), beta[:T1].contiguous(), o1,
-                      final_state=S1)
-    q2, k2, v2, _ = _prefill_gpu(kda, x[T1:].contiguous(), w, H, D, cache_in=c1)
-    o2 = torch.empty_like(v2)
+    o1 = torch.empty(v1.shape, dtype=torch.float32, device=dev)
+    kda.kda_chunk_fwd(q1, k1, v1, gd[:T1].contiguous(), bd[:T1].contiguous(), o1, final_state=S1)
+    q2, k2, v2, _ = _prefill_gpu(kda, xd[T1:].contiguous(), wd, H, D, cache_in=c1, act=act)
+    o2 = torch.empty(v2.shape, dtype=torch.float32, device=dev)
     S2 = torch.empty((1, H, D, D), device=dev)
-    kda.kda_chunk_fwd(q2, k2, v2, g[T1:].contiguous(), beta[T1:].contiguous(), o2,
+    kda.kda_chunk_fwd(q2, k2, v2, gd[T1:].contiguous(), bd[T1:].contiguous(), o2,
                       initial_state=S1, final_state=S2)
     torch.cuda.synchronize()
-    assert rel_max(f64(torch.cat([o1, o2])), f64(o_full)) <= TOL_BF16
-    assert rel_fro(f64(S2), f64(S_full)) <= TOL_STATE
+    assert kda.kda_get_device_status() == 0
+    qr, kr, vr, _ = o_prologue(x, w, H, D)
+    o_ref, S_ref = kda_recurrent(qr, kr, vr, g, beta, 1.0)
+    tol = TOL_BF16 if act != torch.float32 else TOL_F32
+    assert rel_max(f64(torch.cat([o1, o2])), o_ref) <= tol
+    assert rel_fro(f64(S2), state_to_abi(S_ref)) <= (TOL_STATE if act != torch.float32 else 1e-5)
