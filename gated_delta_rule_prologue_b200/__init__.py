@@ -32,6 +32,7 @@ __all__ = [
     "kda_prologue",
     "kda_chunk_fwd",
     "kda_decode_step",
+    "kda_prologue_chunk_fwd",
     "kda_get_device_status",
     "kda_version",
     "KDA_OK",
@@ -72,8 +73,11 @@ lib.kda_prologue.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _v
 lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               _i, _vp, _vp, _vp]
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
+lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
+                                       _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
-for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_decode_step, lib.kda_get_device_status):
+for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_decode_step, lib.kda_prologue_chunk_fwd,
+            lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
 lib.kda_last_error.argtypes = []
@@ -160,6 +164,25 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
     _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
                              _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
                              _dtype(q), _ptr(o), _ptr(final_state), _stream(stream)))
+
+
+def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: float = 1.0,
+                           cache_in=None, cache_out=None, initial_state=None, final_state=None,
+                           cu_seqlens=None, stream=None):
+    """Prologue fused into the chunkwise prefill (chunk 64): ``x`` [T, 3*H*D]
+    bf16/fp16 projections in, ``o`` [T, H, D] float32 out; q, k, v stay on chip."""
+    for t, n in ((x, "x"), (cache_in, "cache_in"), (cache_out, "cache_out")):
+        _need(t, n, x.dtype)
+    for t, n in ((conv_w, "conv_w"), (o, "o"), (g, "g"), (beta, "beta"),
+                 (initial_state, "initial_state"), (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    T = x.shape[0]
+    _check(lib.kda_prologue_chunk_fwd(_ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out),
+                                      _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                                      _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
+                                      _ptr(final_state), _stream(stream)))
 
 
 def kda_decode_step(x, conv_w, conv_cache, g, beta, state, o, *, H: int, D: int,

@@ -1,7 +1,7 @@
 """Build ``libkda.so`` in-tree with nvcc for sm_100a.
 
-Usage: ``python -m gated_delta_rule_prologue_b200.build`` (or call
-:func:`build`).  Every ``csrc/*.cu`` file is compiled to an object under
+Usage: ``python gated_delta_rule_prologue_b200/build.py`` (run as a script, so
+that the package, which loads the library at import, is not imported first).  Every ``csrc/*.cu`` file is compiled to an object under
 ``_build/`` in parallel and linked into ``gated_delta_rule_prologue_b200/libkda.so``
 (CUDA runtime linked statically).  Objects are rebuilt when their source or
 any header is newer.

@@ -213,6 +213,51 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
   return KDA_OK;
 }
 
+kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void *cache_in,
+                                  void *cache_out, const float *g, const float *beta,
+                                  float scale, const float *initial_state,
+                                  const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                  kda_dtype dt, float *o, float *final_state,
+                                  kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(N >= 1 && T >= 1 && H >= 1 && D >= 1, "bad sizes N=%d T=%d H=%d D=%d", N, T, H, D);
+  KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
+  if (D != 128 || dt == KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "prologue_chunk_fwd: needs D=128 and bf16/f16 x (D=%d)", D);
+  KDA_REQUIRE((long long)H * D * 3 < (1LL << 31), "3*H*D too large");
+  KDA_REQUIRE_PTR(x, "x");
+  KDA_REQUIRE_PTR(conv_w, "conv_w");
+  KDA_REQUIRE_PTR(g, "g");
+  KDA_REQUIRE_PTR4(beta, "beta");
+  KDA_REQUIRE_PTR(o, "o");
+  KDA_OPT_PTR(cache_in, "cache_in");
+  KDA_OPT_PTR(cache_out, "cache_out");
+  KDA_OPT_PTR(initial_state, "initial_state");
+  KDA_OPT_PTR(final_state, "final_state");
+  KDA_OPT_PTR4(cu_seqlens, "cu_seqlens");
+  const size_t C = (size_t)3 * H * D, es = esize(dt);
+  const size_t obytes = (size_t)T * H * D * sizeof(float);
+  const size_t sbytes = (size_t)N * H * D * D * sizeof(float);
+  const size_t cache_bytes = (size_t)N * 3 * C * es;
+  KDA_REQUIRE(!overlaps(o, obytes, x, (size_t)T * C * es), "o overlaps x");
+  KDA_REQUIRE(!overlaps(o, obytes, g, (size_t)T * H * D * 4), "o overlaps g");
+  KDA_REQUIRE(!overlaps(o, obytes, beta, (size_t)T * H * 4), "o overlaps beta");
+  KDA_REQUIRE(!overlaps(o, obytes, final_state, sbytes), "o overlaps final_state");
+  KDA_REQUIRE(!overlaps(cache_in, cache_bytes, cache_out, cache_bytes),
+              "cache_out overlaps cache_in");
+  KDA_REQUIRE(final_state == initial_state ||
+                  !overlaps(final_state, sbytes, initial_state, sbytes),
+              "final_state partially overlaps initial_state");
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaError_t e = kda::launch_prologue_chunk_tc(x, conv_w, cache_in, cache_out, g, beta, scale,
+                                                initial_state, cu_seqlens, N, T, H, dt, o,
+                                                final_state, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_prologue_chunk_fwd launch");
+  return KDA_OK;
+}
+
 kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache, const float *g,
                            const float *beta, float scale, float *state, int N, int H, int D,
                            kda_dtype dt, float *o, kda_stream_t stream) {

@@ -24,6 +24,9 @@
 //         rows of the first half read ver_A, rows of the second half ver_B.
 //         A[r,i] = beta_r D_G[r, i] (i < r);  P[r,i] = D_G[64+r, i] (i < r)
 //         P[r,r] = <q_r, k_r> is taken in fp32 from the unscaled tiles.
+//         Each Gram operand x is split as hi = bf16(x), lo = bf16(x - hi) and the
+//         Gram is hi.hi + hi.lo + lo.hi (three MMAs into one accumulator): the
+//         read-out's error is dominated by P, which this makes nearly exact.
 //   WY    T = (I + A)^{-1} (fp32, blocked over 16x16 blocks)
 //         W^T = (beta K G)^T T^T,  Ut^T = (beta V)^T T^T           (G_r = exp(gamma_r))
 //   state U^T = Ut^T - S^T W^T,   O^T = S^T (Q G)^T + U^T P_strict^T
@@ -39,6 +42,7 @@
 // One CTA (256 threads) per (sequence, head); the chunks of a sequence run in
 // order, the next chunk's tiles stream in by TMA during the current one.
 #include <cuda.h>
+#include <type_traits>
 #include <cudaTypedefs.h>
 
 #include "kda_common.cuh"
@@ -55,9 +59,12 @@ constexpr uint32_t SM_Q = 0;                // raw q tile [64][128] bf16
 constexpr uint32_t SM_K = SM_Q + 16384;     // raw k tile
 constexpr uint32_t SM_V = SM_K + 16384;     // raw v tile
 constexpr uint32_t SM_G = SM_V + 16384;     // raw g [64][128] f32 -> gamma -> E -> (A^T, T)
-constexpr uint32_t SM_X = SM_G + 32768;     // 64 KB, reused within a chunk:
-constexpr uint32_t SM_GA = SM_X;            //   Gram A operand (K-major 128 x 128)  32 KB
-constexpr uint32_t SM_GB = SM_X + 32768;    //   Gram B operand (K-major  96 x 128)  24 KB
+constexpr uint32_t SM_X = SM_G + 32768;     // 64 KB, reused within a chunk (the Gram's
+                                            // four tiles also use TOP, POP and ST, 112 KB):
+constexpr uint32_t SM_GA = SM_X;            //   Gram A operand, high bf16 part (K-major 128 x 128)
+constexpr uint32_t SM_GB = SM_X + 32768;    //   Gram B operand, high part (K-major 96 x 128)
+constexpr uint32_t SM_GAL = SM_X + 57344;   //   Gram A operand, low part x - bf16(x)
+constexpr uint32_t SM_GBL = SM_X + 90112;   //   Gram B operand, low part
 constexpr uint32_t SM_BKG = SM_X;           //   beta K G (MN-major, 64 k-rows)     16 KB; then W op
 constexpr uint32_t SM_BV = SM_X + 16384;    //   beta V   (MN-major)                16 KB
 constexpr uint32_t SM_QG = SM_X + 32768;    //   Q G      (K-major 64 x 128)        16 KB
@@ -81,8 +88,15 @@ constexpr uint32_t SM_PDIAG = SM_BETA + 256;// <q_r, k_r> in fp32    [64]
 constexpr uint32_t SM_BAR = SM_PDIAG + 256; // two mbarriers
 constexpr uint32_t SM_SLOT = SM_BAR + 16;   // TMEM base address
 constexpr uint32_t SM_TOTAL = SM_SLOT + 16;
+// Fused prologue only: fp32 correction beta*v - f16(beta*v_tile) kept as bf16
+// [64][128], and two conv histories (3 parts x 3 rows x 128 raw values).
+constexpr uint32_t SM_CORR = (SM_TOTAL + 1023) & ~1023u;
+constexpr uint32_t SM_HIST = SM_CORR + 16384;
+constexpr uint32_t SM_TOTAL_FUSED = SM_HIST + 2 * 3 * 3 * 128 * 2;
 constexpr uint32_t SM_ALLOC = SM_TOTAL + 1024;  // slack for 1024-byte alignment
-static_assert(SM_ALLOC <= 232448, "shared memory budget");
+constexpr uint32_t SM_ALLOC_FUSED = SM_TOTAL_FUSED + 1024;
+static_assert(SM_ALLOC_FUSED <= 232448, "shared memory budget");
+static_assert(SM_GBL + 24576 <= SM_ST + 32768, "Gram tiles stay inside X, TOP, POP and ST");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
 constexpr uint32_t TM_G = 0;     // Gram, 96 columns
@@ -111,6 +125,27 @@ __device__ __forceinline__ void ld8_f32(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// Split 8 floats into bf16 high parts and bf16 residuals.
+__device__ __forceinline__ void pack8_hilo(const float (&f)[8], uint4 &hi, uint4 &lo) {
+  float l[8];
+  __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = __float2bfloat16_rn(f[i]);
+    l[i] = f[i] - __bfloat162float(h[i]);
+  }
+  lo = pack8_bf16(l);
+}
+
+template <typename Tin>
+__device__ __forceinline__ uint4 pack8_in(const float (&f)[8]) {
+  uint4 u;
+  Tin *h = reinterpret_cast<Tin *>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) h[i] = from_f32<Tin>(f[i]);
+  return u;
+}
+
 // All threads wait for a barrier phase; false (and a recorded timeout) if any
 // thread gave up.  Also acts as a CTA-wide barrier.
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *status) {
@@ -122,13 +157,21 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *st
   return true;
 }
 
-template <typename Tin>
+// kFused = false: q, k, v tiles come from HBM as given (already unit-normalised).
+// kFused = true:  the three tiles are the raw projections x (parts q, k, v of
+// head h); the prologue (causal width-4 conv with history, SiLU, L2 on q and
+// k) runs in fp32 in shared memory and overwrites them with q, k, v.
+template <typename Tin, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                 const float *__restrict__ beta, float scale, const float *s0,
                 const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
-                int *status) {
+                int *status, const float *__restrict__ conv_w, const Tin *cache_in,
+                Tin *cache_out) {
+  // Element type of the q/k/v tiles the chunk phases read: the inputs as given,
+  // or fp16 written by the fused prologue (q, k are unit vectors; v is guarded).
+  using Tact = typename std::conditional<kFused, __half, Tin>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -185,11 +228,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   auto issue_tma = [&](int t) {
     mbar_arrive_expect_tx(bar_tma, kTmaBytes);
-    tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
-    tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, h, t);
-    tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
+    if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
+      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
+      tma_load_3d(sm + SM_K, &tm_q, bar_tma, 0, H + h, t);
+      tma_load_3d(sm + SM_V, &tm_q, bar_tma, 0, 2 * H + h, t);
+    } else {
+      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
+      tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, h, t);
+      tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
+    }
     tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, h, t);
   };
+  Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
+  __nv_bfloat16 *corr = reinterpret_cast<__nv_bfloat16 *>(sm + SM_CORR);
+  const int HD = H * 128;
+  if constexpr (kFused) {
+    // conv history before the sequence: the cache rows (oldest first) or zero
+    for (int idx = tid; idx < 9 * 128; idx += kThreads) {
+      const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
+      hist[idx] = cache_in ? cache_in[((size_t)n * 3 + row) * 3 * HD + p * HD + h * 128 + ch]
+                           : from_f32<Tin>(0.f);
+    }
+    __syncthreads();
+  }
   if (tid == 0 && nchunks > 0) issue_tma(bos);
 
   uint32_t tma_par = 0, mma_par = 0;
@@ -203,6 +264,99 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // ---- P1: beta, in-chunk cumulative log-decay, per-channel factors, E ------------
     if (tid < 64) beta_s[tid] = tid < Lc ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    if constexpr (kFused) {
+      // ---- Pc: prologue in place on the x tiles (fp32 arithmetic) ----------------------
+      __syncthreads();  // beta_s visible
+      const Tin *hcur = hist + (c & 1) * 1152;
+      Tin *hnxt = hist + ((c + 1) & 1) * 1152;
+      const int c8 = tid & 15, d0 = c8 * 8;
+      float qn[4][8];
+#pragma unroll 1
+      for (int p = 0; p < 3; ++p) {
+        uint8_t *tile = sm + (p == 0 ? SM_Q : (p == 1 ? SM_K : SM_V));
+        float w4[8][4];
+        {
+          const float *wp = conv_w + ((size_t)p * HD + h * 128 + d0) * 4;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(wp) + e);
+            w4[e][0] = f.x; w4[e][1] = f.y; w4[e][2] = f.z; w4[e][3] = f.w;
+          }
+        }
+        float y[4][8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int r = (tid >> 4) + 16 * m;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int tap = 0; tap < 4; ++tap) {
+            const int rr = r - 3 + tap;
+            float xv[8];
+            if (rr >= 0)
+              ld8_in<Tin>(tile + rr * 256 + c8 * 16, xv);
+            else
+              ld8_in<Tin>(reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + rr) * 128) + c8 * 16, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w4[e][tap], xv[e], acc[e]);
+          }
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            y[m][e] = silu(acc[e]);
+            ss = fmaf(y[m][e], y[m][e], ss);
+          }
+          ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          const float sc = p < 2 ? rsqrtf(ss + 1e-6f) : 1.f;
+          const bool valid = r < Lc;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[m][e] = valid ? y[m][e] * sc : 0.f;
+        }
+        // history for the next chunk: raw rows Lc-3 .. Lc-1 of this part
+        if (tid < 48) {
+          const int hr = tid >> 4, src = Lc - 3 + hr;
+          const uint8_t *from = src >= 0 ? tile + src * 256 + c8 * 16
+                                         : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + src) * 128) + c8 * 16;
+          *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(hnxt + (p * 3 + hr) * 128) + c8 * 16) =
+              *reinterpret_cast<const uint4 *>(from);
+        }
+        __syncthreads();  // every raw value of this part has been read
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int r = (tid >> 4) + 16 * m;
+          st_shared_16(tile, r * 256 + c8 * 16, pack8_in<Tact>(y[m]));
+          if (p == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qn[m][e] = y[m][e];
+          } else if (p == 1) {
+            float qk = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qk = fmaf(qn[m][e], y[m][e], qk);
+            qk += __shfl_xor_sync(0xffffffffu, qk, 8);
+            qk += __shfl_xor_sync(0xffffffffu, qk, 4);
+            qk += __shfl_xor_sync(0xffffffffu, qk, 2);
+            qk += __shfl_xor_sync(0xffffffffu, qk, 1);
+            if (c8 == 0) pdiag[r] = qk;  // <q_r, k_r> of the fp32 prologue outputs
+          } else {
+            float vmax = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) vmax = fmaxf(vmax, fabsf(y[m][e]));
+            if (!(vmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+            const float bt = beta_s[r];
+            float cr[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float stored = to_f32(from_f32<Tact>(y[m][e]));
+              cr[e] = bt * y[m][e] - __half2float(__float2half_rn(bt * stored));
+            }
+            st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
+          }
+        }
+        __syncthreads();
+      }
+    }
     {
       const int d = tid & 127, part = tid >> 7;
       float vals[32];
@@ -248,8 +402,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
       const bool valid = r < Lc;
       float k8[8], q8[8], e8[8];
-      ld8_in<Tin>(sm + SM_K + r * 256 + c8 * 16, k8);
-      ld8_in<Tin>(sm + SM_Q + r * 256 + c8 * 16, q8);
+      ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
+      ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
       ld8_f32(Gf + r * 128 + d0, e8);
       float a[8], b[8], ki[8];
 #pragma unroll
@@ -259,14 +413,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         b[e] = qq * e8[e];
         ki[e] = kk * __frcp_rn(e8[e]);
       }
-      st_shared_16(sm + SM_GA, kmaj_off(128, r, c8), pack8_bf16(a));
-      st_shared_16(sm + SM_GA, kmaj_off(128, 64 + r, c8), pack8_bf16(b));
+      uint4 hi, lo;
+      pack8_hilo(a, hi, lo);
+      st_shared_16(sm + SM_GA, kmaj_off(128, r, c8), hi);
+      st_shared_16(sm + SM_GAL, kmaj_off(128, r, c8), lo);
+      pack8_hilo(b, hi, lo);
+      st_shared_16(sm + SM_GA, kmaj_off(128, 64 + r, c8), hi);
+      st_shared_16(sm + SM_GAL, kmaj_off(128, 64 + r, c8), lo);
       if (r < 32) {
-        st_shared_16(sm + SM_GB, kmaj_off(96, r, c8), pack8_bf16(ki));
+        pack8_hilo(ki, hi, lo);
+        st_shared_16(sm + SM_GB, kmaj_off(96, r, c8), hi);
+        st_shared_16(sm + SM_GBL, kmaj_off(96, r, c8), lo);
 #pragma unroll
         for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * feba[d0 + e]) * feba[d0 + e];
       }
-      st_shared_16(sm + SM_GB, kmaj_off(96, 32 + r, c8), pack8_bf16(ki));
+      pack8_hilo(ki, hi, lo);
+      st_shared_16(sm + SM_GB, kmaj_off(96, 32 + r, c8), hi);
+      st_shared_16(sm + SM_GBL, kmaj_off(96, 32 + r, c8), lo);
     }
     fence_async_smem();
     __syncthreads();
@@ -275,10 +438,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
+      const uint32_t gal = smem_u32(sm + SM_GAL), gbl = smem_u32(sm + SM_GBL);
       constexpr uint32_t id = idesc_bf16(128, 96, false, false);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gbl, 96, ks), id, 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TM_G, desc_kmajor(gal, 128, ks), desc_kmajor(gb, 96, ks), id, 1);
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, mma_par, status)) break;
@@ -295,9 +465,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float *fec = r < 32 ? feca : fecb;
       const float *fel = r < 32 ? fela : felb;
       float k8[8], q8[8], v8[8], e8[8];
-      ld8_in<Tin>(sm + SM_K + r * 256 + c8 * 16, k8);
-      ld8_in<Tin>(sm + SM_Q + r * 256 + c8 * 16, q8);
-      ld8_in<Tin>(sm + SM_V + r * 256 + c8 * 16, v8);
+      ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
+      ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
+      ld8_in<Tact>(sm + SM_V + r * 256 + c8 * 16, v8);
       ld8_f32(Gf + r * 128 + d0, e8);
       float bkg[8], bv[8], qg[8], kp[8];
 #pragma unroll
@@ -323,14 +493,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       reinterpret_cast<float4 *>(AT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int idx = tid; idx < 8192 / 16; idx += kThreads)
       reinterpret_cast<uint4 *>(sm + SM_POP)[idx] = make_uint4(0u, 0u, 0u, 0u);
-    {
+    if constexpr (!kFused) {
       const int r = tid >> 2, part = tid & 3;
       float acc = 0.f;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float q8[8], k8[8];
-        ld8_in<Tin>(sm + SM_Q + r * 256 + (part * 4 + c8) * 16, q8);
-        ld8_in<Tin>(sm + SM_K + r * 256 + (part * 4 + c8) * 16, k8);
+        ld8_in<Tact>(sm + SM_Q + r * 256 + (part * 4 + c8) * 16, q8);
+        ld8_in<Tact>(sm + SM_K + r * 256 + (part * 4 + c8) * 16, k8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc = fmaf(q8[e], k8[e], acc);
       }
@@ -495,7 +665,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float u[32];
     tmem_ld32(tmem + lane_addr + TM_U + 32 * half, u);
     {
-      const Tin *Vr = reinterpret_cast<const Tin *>(sm + SM_V);
+      const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
 #pragma unroll
       float amax = 0.f;
 #pragma unroll
@@ -503,7 +673,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = 32 * half + i;
         const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
         const float bvv = beta_s[r] * vv;
-        u[i] += bvv - __half2float(__float2half_rn(bvv));
+        if constexpr (kFused)
+          u[i] += __bfloat162float(corr[r * 128 + j]);
+        else
+          u[i] += bvv - __half2float(__float2half_rn(bvv));
         amax = fmaxf(amax, fmaxf(fabsf(u[i]), fabsf(bvv)));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
@@ -561,6 +734,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
   }
 
+  if constexpr (kFused) {
+    if (cache_out) {  // the last three raw inputs of the sequence (oldest first)
+      const Tin *hfin = hist + (nchunks & 1) * 1152;
+      for (int idx = tid; idx < 9 * 128; idx += kThreads) {
+        const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
+        cache_out[((size_t)n * 3 + row) * 3 * HD + p * HD + h * 128 + ch] = hfin[idx];
+      }
+    }
+  }
   if (sN) {
     float *dst = sN + (((size_t)n * H + h) * 128 + j) * 128 + dk0;
 #pragma unroll
@@ -611,15 +793,61 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
       !make_map(&tv, v, act, 2, H, T) ||
       !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
     return cudaErrorInvalidValue;
-  auto kern = dt == KDA_BF16 ? chunk_tc_kernel<__nv_bfloat16> : chunk_tc_kernel<__half>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SM_ALLOC);
-  if (e != cudaSuccess) return e;
   const long long blocks = (long long)N * H;
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
-  kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
-                                                    sN, status);
+  if (dt == KDA_BF16) {
+    auto kern = chunk_tc_kernel<__nv_bfloat16, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SM_ALLOC);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
+                                                      sN, status, nullptr, nullptr, nullptr);
+  } else {
+    auto kern = chunk_tc_kernel<__half, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SM_ALLOC);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
+                                                      sN, status, nullptr, nullptr, nullptr);
+  }
   return cudaGetLastError();
+}
+
+namespace {
+template <typename Tin>
+cudaError_t launch_fused_typed(const void *x, const float *conv_w, const void *cache_in,
+                               void *cache_out, const float *g, const float *beta, float scale,
+                               const float *s0, const int32_t *cu, int N, int T, int H,
+                               CUtensorMapDataType act, float *o, float *sN, int *status,
+                               cudaStream_t s) {
+  CUtensorMap tx, tg;
+  if (!make_map(&tx, x, act, 2, 3 * H, T) ||
+      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+    return cudaErrorInvalidValue;
+  const long long blocks = (long long)N * H;
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  auto kern = chunk_tc_kernel<Tin, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SM_ALLOC_FUSED);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)blocks, kThreads, SM_ALLOC_FUSED, s>>>(
+      tx, tx, tx, tg, beta, scale, s0, cu, T, H, o, sN, status, conv_w,
+      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out));
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,
+                                     void *cache_out, const float *g, const float *beta,
+                                     float scale, const float *s0, const int32_t *cu, int N,
+                                     int T, int H, kda_dtype dt, float *o, float *sN,
+                                     int *status, cudaStream_t s) {
+  if (dt == KDA_BF16)
+    return launch_fused_typed<__nv_bfloat16>(x, conv_w, cache_in, cache_out, g, beta, scale, s0,
+                                             cu, N, T, H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, sN,
+                                             status, s);
+  return launch_fused_typed<__half>(x, conv_w, cache_in, cache_out, g, beta, scale, s0, cu, N, T,
+                                    H, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, o, sN, status, s);
 }
 
 }  // namespace kda

@@ -136,4 +136,9 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             const float *beta, float scale, const float *s0, const int32_t *cu,
                             int N, int T, int H, kda_dtype dt, float *o, float *sN, int *status,
                             cudaStream_t s);
+cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,
+                                     void *cache_out, const float *g, const float *beta,
+                                     float scale, const float *s0, const int32_t *cu, int N,
+                                     int T, int H, kda_dtype dt, float *o, float *sN,
+                                     int *status, cudaStream_t s);
 }  // namespace kda

@@ -121,6 +121,28 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
                          kda_stream_t stream);
 
 /*
+ * kda_prologue_chunk_fwd -- the prologue fused into the chunkwise prefill: the
+ * same result as kda_prologue followed by kda_chunk_fwd (chunk 64), with q, k
+ * and v never written to memory.  Each chunk's projections are convolved
+ * (causal width 4 with the carried three-row history), passed through SiLU
+ * and L2-normalised in fp32 on chip ([W1 第二站], [W4 ShortConv paragraph]),
+ * then used by the chunk update of kda_chunk_fwd ([W1 彩蛋]).
+ *
+ *   x             [T, 3*H*D] dt (KDA_BF16 or KDA_F16) projections, layout as in
+ *                 kda_prologue
+ *   conv_w        [3*H*D, 4] f32;  cache_in / cache_out as in kda_prologue
+ *   g, beta, scale, initial_state, cu_seqlens, o, final_state as in
+ *                 kda_chunk_fwd
+ * Supported: D == 128, dt in {KDA_BF16, KDA_F16}; T >= 1.
+ */
+kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void *cache_in,
+                                  void *cache_out, const float *g, const float *beta,
+                                  float scale, const float *initial_state,
+                                  const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                  kda_dtype dt, float *o, float *final_state,
+                                  kda_stream_t stream);
+
+/*
  * kda_decode_step -- one new token for each of N independent sequences: the
  * prologue on that token with the conv cache as history, then one step of
  * the recurrence on the state in place (the recurrent mode used for

@@ -13,8 +13,8 @@ HEADER = os.path.join(ROOT, "include", "kda.h")
 
 @pytest.fixture(scope="module")
 def kda():
-    from gated_delta_rule_prologue_b200.build import build
-    build()
+    import __graft_entry__
+    __graft_entry__.build()
     import gated_delta_rule_prologue_b200 as m
     return m
 
@@ -27,8 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_hot_path_entry_points():
     names = declared_functions()
-    for n in ("kda_prologue", "kda_chunk_fwd", "kda_decode_step", "kda_get_device_status",
-              "kda_last_error", "kda_version"):
+    for n in ("kda_prologue", "kda_chunk_fwd", "kda_decode_step", "kda_prologue_chunk_fwd",
+              "kda_get_device_status", "kda_last_error", "kda_version"):
         assert n in names
 
 
@@ -112,3 +112,25 @@ def test_prologue_and_decode_reject_bad_arguments(kda):
     assert st == kda.KDA_ERR_UNSUPPORTED
     st = L.kda_get_device_status(None)
     assert st == kda.KDA_ERR_INVALID_ARG
+
+
+def test_fused_prefill_rejects_bad_arguments(kda):
+    L = kda.lib
+    a = _vp(ALIGNED)
+    # D != 128 is outside the fused path's domain
+    st = L.kda_prologue_chunk_fwd(a, a, None, None, a, a, 1.0, None, None, 1, 8, 2, 64, 1,
+                                  _vp(2 * ALIGNED), None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    # float32 projections are not supported by the fused path
+    st = L.kda_prologue_chunk_fwd(a, a, None, None, a, a, 1.0, None, None, 1, 8, 2, 128, 0,
+                                  _vp(2 * ALIGNED), None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    # missing g
+    st = L.kda_prologue_chunk_fwd(a, a, None, None, None, a, 1.0, None, None, 1, 8, 2, 128, 1,
+                                  _vp(2 * ALIGNED), None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"g is NULL" in L.kda_last_error()
+    # o aliasing x
+    st = L.kda_prologue_chunk_fwd(a, _vp(8 * ALIGNED), None, None, _vp(4 * ALIGNED),
+                                  _vp(6 * ALIGNED), 1.0, None, None, 1, 8, 2, 128, 1, a, None,
+                                  None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()

@@ -203,30 +203,118 @@ def test_prologue_parity_varlen_with_cache(kda, dtype, out_dtype, D):
 # --- full-size workloads, sampled ------------------------------------------------
 
 def test_k3_prefill_full_size_sampled_heads(kda):
-    """Prologue + chunkwise prefill over 32768 tokens x 96 heads (the benchmark's
-    launches); heads 0, 53 and 95 recomputed by the oracle over all tokens."""
+    """Fused prologue + chunkwise prefill over 32768 tokens x 96 heads (the
+    benchmark's launch); heads 0, 53 and 95 recomputed by the oracle over all
+    tokens."""
     inp = W.k3_prefill()
     T, H, D = inp.T, inp.H, inp.D
     dev = "cuda"
     x = inp.x.to(dev)
-    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
-    k, v = torch.empty_like(q), torch.empty_like(q)
-    kda.kda_prologue(x, inp.conv_w.to(dev), q, k, v, H=H, D=D)
     o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
     fs = torch.empty((1, H, D, D), device=dev)
-    kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, scale=inp.scale,
-                      final_state=fs, chunk=inp.chunk)
+    cache = torch.empty((1, 3, 3 * H * D), dtype=torch.bfloat16, device=dev)
+    kda.kda_prologue_chunk_fwd(x, inp.conv_w.to(dev), inp.g.to(dev), inp.beta.to(dev), o, H=H,
+                               D=D, scale=inp.scale, final_state=fs, cache_out=cache)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
+    np.testing.assert_array_equal(f64(cache[0]), f64(inp.x[-3:]))
     del x
     for h in (0, 53, 95):
         xh, wh, gh, bh = W.k3_prefill_head(h)
         qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
-        check_rounded(q[:, h], qr[:, 0], torch.float16)
-        check_rounded(v[:, h], vr[:, 0], torch.float16)
         o_ref, S_ref = kda_recurrent(qr, kr, vr, gh[:, None, :], bh[:, None], inp.scale)
         assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16
         assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
+
+
+def test_k3_prologue_kernel_full_size_sampled_heads(kda):
+    """The standalone prologue over the full K3-shaped input, fp16 outputs."""
+    inp = W.k3_prefill()
+    T, H, D = inp.T, inp.H, inp.D
+    dev = "cuda"
+    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    kda.kda_prologue(inp.x.to(dev), inp.conv_w.to(dev), q, k, v, H=H, D=D)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    for h in (7, 88):
+        xh, wh, _, _ = W.k3_prefill_head(h)
+        qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
+        for got, ref in ((q[:, h], qr[:, 0]), (k[:, h], kr[:, 0]), (v[:, h], vr[:, 0])):
+            check_rounded(got, ref, torch.float16)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_fused_prefill_varlen_with_cache_and_resume(kda, dtype):
+    """Fused path over packed sequences with conv cache and initial state in,
+    cache and final state out; then a second call continuing every sequence
+    from the first call's cache and state.  Both calls match the oracle run
+    over the concatenated tokens."""
+    dev = "cuda"
+    H, D = 2, 128
+    l1 = [70, 1, 130, 64]
+    l2 = [5, 100, 2, 66]
+    N, C = len(l1), 3 * H * D
+    r = torch.Generator().manual_seed(31)
+    xs = [torch.randn((a + b, C), generator=r).to(dtype) for a, b in zip(l1, l2)]
+    w = 0.5 * torch.randn((C, 4), generator=r)
+    gs = [-5.0 * torch.sigmoid(torch.randn((a + b, H, D), generator=r) - 2.0) for a, b in zip(l1, l2)]
+    bs = [torch.sigmoid(torch.randn((a + b, H), generator=r)) for a, b in zip(l1, l2)]
+    cache0 = torch.randn((N, 3, C), generator=r).to(dtype)
+    s0 = 0.05 * torch.randn((N, H, D, D), generator=r)
+
+    def pack(lists, part):
+        return torch.cat([t[:a] if part == 0 else t[a:] for t, a in zip(lists, l1)]).contiguous()
+
+    outs = []
+    cache_in, state = cache0.to(dev), s0.to(dev)
+    for part, lens in ((0, l1), (1, l2)):
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+        T = sum(lens)
+        o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+        cache_out = torch.empty((N, 3, C), dtype=dtype, device=dev)
+        fs = torch.empty((N, H, D, D), device=dev)
+        kda.kda_prologue_chunk_fwd(pack(xs, part).to(dev), w.to(dev), pack(gs, part).to(dev),
+                                   pack(bs, part).to(dev), o, H=H, D=D, cache_in=cache_in,
+                                   cache_out=cache_out, initial_state=state, final_state=fs,
+                                   cu_seqlens=cu)
+        outs.append((o, cu))
+        cache_in, state = cache_out, fs
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    lens_all = [a + b for a, b in zip(l1, l2)]
+    cu_all = np.concatenate([[0], np.cumsum(lens_all)])
+    qr, kr, vr, c_ref = o_prologue(torch.cat(xs), w, H, D, cu_all, cache0)
+    o_ref, S_ref = kda_recurrent(qr, kr, vr, torch.cat(gs), torch.cat(bs), 1.0,
+                                 state_from_abi(s0), cu_all)
+    got = np.zeros_like(o_ref)
+    for n in range(N):
+        a = cu_all[n]
+        got[a:a + l1[n]] = f64(outs[0][0])[int(outs[0][1][n]):int(outs[0][1][n + 1])]
+        got[a + l1[n]:a + lens_all[n]] = f64(outs[1][0])[int(outs[1][1][n]):int(outs[1][1][n + 1])]
+    assert rel_max(got, o_ref) <= TOL_BF16
+    assert rel_fro(f64(state), state_to_abi(S_ref)) <= TOL_STATE
+    np.testing.assert_array_equal(f64(cache_in), c_ref)
+
+
+def test_fused_and_unfused_prefill_agree(kda):
+    """kda_prologue_chunk_fwd equals kda_prologue (fp16 hand-off) followed by
+    kda_chunk_fwd within the bf16 bound."""
+    dev = "cuda"
+    T, H, D = 400, 3, 128
+    C = 3 * H * D
+    r = torch.Generator().manual_seed(41)
+    x = torch.randn((T, C), generator=r).to(torch.bfloat16).to(dev)
+    w = (0.5 * torch.randn((C, 4), generator=r)).to(dev)
+    g = (-5.0 * torch.sigmoid(torch.randn((T, H, D), generator=r))).to(dev)
+    beta = torch.sigmoid(torch.randn((T, H), generator=r)).to(dev)
+    o1 = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    kda.kda_prologue_chunk_fwd(x, w, g, beta, o1, H=H, D=D)
+    q, k, v, _ = _prefill_gpu(kda, x, w, H, D, act=torch.float16)
+    o2 = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    kda.kda_chunk_fwd(q, k, v, g, beta, o2)
+    torch.cuda.synchronize()
+    assert rel_max(f64(o1), f64(o2)) <= 2 * TOL_BF16
 
 
 def test_varlen16_full_size_sampled(kda):
