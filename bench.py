@@ -423,6 +423,42 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_ncu_case(args):
+    """Launch one kernel twice (warm-up, then the launch to capture) on a slice
+    of the workload, for profiling runs; prints nothing."""
+    import gated_delta_rule_prologue_b200 as kda
+    dev = torch.device("cuda", 0)
+    if args.ncu_case == "decode":
+        d = W.decode256(steps=2)
+        state, cache = d.state.to(dev), d.conv_cache.to(dev)
+        w = d.conv_w.to(dev)
+        o = torch.empty((d.N, d.H, d.D), device=dev)
+        for s_ in range(2):
+            kda.kda_decode_step(d.x[s_].to(dev), w, cache, d.g[s_].to(dev), d.beta[s_].to(dev),
+                                state, o, H=d.H, D=d.D)
+    else:
+        inp = W.k3_prefill()
+        T = min(args.ncu_tokens, inp.T)
+        H, D = inp.H, inp.D
+        x = inp.x[:T].contiguous().to(dev)
+        w = inp.conv_w.to(dev)
+        g = inp.g[:T].contiguous().to(dev)
+        beta = inp.beta[:T].contiguous().to(dev)
+        o = torch.empty((T, H, D), device=dev)
+        q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
+        k, v = torch.empty_like(q), torch.empty_like(q)
+        for _ in range(2):
+            if args.ncu_case == "fused":
+                kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D)
+            elif args.ncu_case == "prologue":
+                kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+            else:
+                kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+                kda.kda_chunk_fwd(q, k, v, g, beta, o)
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -433,7 +469,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "decode"),
+                    help="profiling mode: launch one kernel twice on a workload slice and exit")
+    ap.add_argument("--ncu-tokens", type=int, default=4096)
     args = ap.parse_args()
+    if args.ncu_case:
+        run_ncu_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world, rank, local = dist_setup(args) if args.impl == "ours" else (
