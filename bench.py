@@ -2,9 +2,10 @@
 """Benchmark of the KDA hot path on B200 through libkda's C ABI.
 
 A *step* is one pass of the prefill hot path over the K3-layer-shaped
-workload: ``kda_prologue_chunk_fwd``, the prologue (short conv + SiLU + L2 over
-32768 tokens x 96 heads x 128 channels of q/k/v projections) fused into the
-chunkwise prefill (chunk 64, fp32 state).  ``value`` is prefill tokens/s
+workload: ``kda_prologue`` (short conv + SiLU + L2 over 32768 tokens x 96
+heads x 128 channels of q/k/v projections, fp16 q/k/v out) followed by
+``kda_chunk_fwd`` (tensor-core chunkwise prefill, chunk 64, fp32 state).  The
+fused variant ``kda_prologue_chunk_fwd`` is timed beside it.  ``value`` is prefill tokens/s
 (a token is one position through all 96 heads) with inputs resident in HBM.
 The batched decode step (256 sequences x 96 heads, 100 consecutive steps,
 state updated in place) is timed in the same run and reported under
@@ -265,17 +266,20 @@ def run_ours(args, world, rank, local):
     beta = inp.beta.to(dev)
     o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
     fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D, scale=inp.scale, final_state=fs,
-                                   stream=stream)
+        kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
+                          chunk=inp.chunk, stream=stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     assert kda.kda_get_device_status() == 0
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev)
     barrier(world)
@@ -284,34 +288,32 @@ def run_ours(args, world, rank, local):
     start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        step()
+        kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
         ev[i][1].record(stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
+                          chunk=inp.chunk, stream=stream)
+        ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     total_ms = max_over_ranks(start.elapsed_time(end), world)
     ms_step = total_ms / args.steps
-    fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    chk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     assert kda.kda_get_device_status() == 0
     value = world * T / (ms_step * 1e-3)
-    launches = args.steps
+    launches = 2 * args.steps
 
-    # the standalone prologue and the unfused chunk kernel (rows of the path on
-    # their own; not part of the timed step)
-    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
-    k, v = torch.empty_like(q), torch.empty_like(q)
+    # the fused variant (prologue inside the chunk kernel), timed beside the step
     o2 = torch.empty_like(o)
-    side = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(3)]
+    side = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
     for i in range(3):
         side[i][0].record(stream)
-        kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
+        kda.kda_prologue_chunk_fwd(x, w, g, beta, o2, H=H, D=D, scale=inp.scale, stream=stream)
         side[i][1].record(stream)
-        kda.kda_chunk_fwd(q, k, v, g, beta, o2, scale=inp.scale, chunk=inp.chunk, stream=stream)
-        side[i][2].record(stream)
     torch.cuda.synchronize(dev)
-    pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in side[1:])
-    chk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in side[1:])
-    del q, k, v, o2
+    fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in side[1:])
+    del o2
 
     th = T * H
     kernels = {
@@ -323,9 +325,9 @@ def run_ours(args, world, rank, local):
         "kda_chunk_fwd": dict(ms=round(chk_ms, 4), **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, chk_ms, hbm, "GB/s", recorded_traffic("kda_chunk_fwd"))),
     }
-    kernels["kda_prologue_chunk_fwd"]["tensor_tflops"] = round(
-        CHUNK_FLOPS_PER_TH * th / (fused_ms * 1e-3) / 1e12, 2)
-    dominant = "kda_prologue_chunk_fwd"
+    kernels["kda_chunk_fwd"]["tensor_tflops"] = round(
+        CHUNK_FLOPS_PER_TH * th / (chk_ms * 1e-3) / 1e12, 2)
+    dominant = "kda_chunk_fwd"
     roof = {k_: kernels[dominant][k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dominant
     roof["peak_source"] = f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
@@ -400,12 +402,12 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": "k3_prefill: kda_prologue_chunk_fwd (prologue fused into the chunkwise "
-                        "prefill) over T=32768 tokens, H=96, d_k=d_v=128, chunk 64, bf16 q/k/v "
-                        "projections, fp32 g/beta/state/o",
+            "workload": "k3_prefill: kda_prologue (fp16 q/k/v out) + kda_chunk_fwd over "
+                        "T=32768 tokens, H=96, d_k=d_v=128, chunk 64, bf16 q/k/v projections, "
+                        "fp32 g/beta/state/o",
             "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
             "parallelism": f"replicas x{world} (independent problems, no collective)",
-            "l2": "inputs larger than L2 (5.7 GB touched per step, no flush needed)",
+            "l2": "inputs larger than L2 (10.5 GB touched per step, no flush needed)",
         },
         "roofline": roof,
         "kernels": kernels,

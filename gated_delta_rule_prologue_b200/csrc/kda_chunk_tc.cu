@@ -39,9 +39,10 @@
 //   fp32 diagonal terms: u_r gets beta_r v_r - f16(beta_r v_r) back, and
 //   o_r gets <q_r, k_r> u_r in fp32, so a token's own (dominant) contribution
 //   to its read-out is never rounded to bf16.
-// One CTA (256 threads) per (sequence, head); the chunks of a sequence run in
+// One CTA (512 threads) per (sequence, head); the chunks of a sequence run in
 // order, the next chunk's tiles stream in by TMA during the current one.
 #include <cuda.h>
+#include <cstring>
 #include <type_traits>
 #include <cudaTypedefs.h>
 
@@ -52,7 +53,7 @@ namespace kda {
 namespace {
 using namespace tc;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 // ---- shared memory plan (byte offsets from a 1024-aligned base) ----------------
 constexpr uint32_t SM_Q = 0;                // raw q tile [64][128] bf16
@@ -92,7 +93,8 @@ constexpr uint32_t SM_TOTAL = SM_SLOT + 16;
 // [64][128], and two conv histories (3 parts x 3 rows x 128 raw values).
 constexpr uint32_t SM_CORR = (SM_TOTAL + 1023) & ~1023u;
 constexpr uint32_t SM_HIST = SM_CORR + 16384;
-constexpr uint32_t SM_TOTAL_FUSED = SM_HIST + 2 * 3 * 3 * 128 * 2;
+constexpr uint32_t SM_WCONV = SM_HIST + 2 * 3 * 3 * 128 * 2;  // conv weights of head h [3][4 taps][128] f32
+constexpr uint32_t SM_TOTAL_FUSED = SM_WCONV + 3 * 128 * 4 * 4;
 constexpr uint32_t SM_ALLOC = SM_TOTAL + 1024;  // slack for 1024-byte alignment
 constexpr uint32_t SM_ALLOC_FUSED = SM_TOTAL_FUSED + 1024;
 static_assert(SM_ALLOC_FUSED <= 232448, "shared memory budget");
@@ -108,6 +110,27 @@ constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t kTmaBytes = 3 * 16384 + 32768;
 
+
+// Eight 16-bit values packed in a uint4, widened to floats.
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8], __nv_bfloat16) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8], __half) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 hh;
+    memcpy(&hh, &w[i], 4);
+    const float2 t = __half22float2(hh);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
 
 // 8 consecutive 16-bit activations of a raw tile (bf16 or fp16) as floats.
 template <typename Tin>
@@ -161,6 +184,10 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *st
 // kFused = true:  the three tiles are the raw projections x (parts q, k, v of
 // head h); the prologue (causal width-4 conv with history, SiLU, L2 on q and
 // k) runs in fp32 in shared memory and overwrites them with q, k, v.
+//
+// Thread layout (512 threads, 16 warps): warp w reads TMEM lanes
+// 32*(w%4).. (its "quad") and handles column group w/4 of every accumulator it
+// reads; element-wise phases walk (row, 8-channel chunk) pairs.
 template <typename Tin, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -176,7 +203,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
+  const int quad = warp & 3, grp = warp >> 2;
   const int n = blockIdx.x / H, h = blockIdx.x % H;
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);
   uint64_t *bar_mma = bar_tma + 1;
@@ -192,6 +219,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   float *fela = reinterpret_cast<float *>(sm + F_ELA);
   float *felb = reinterpret_cast<float *>(sm + F_ELB);
   float *fegc = reinterpret_cast<float *>(sm + F_EGC);
+  float *XS = reinterpret_cast<float *>(sm + SM_XS);
 
   int bos, eos;
   seq_bounds(cu, n, T, status, bos, eos);
@@ -208,14 +236,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tma_prefetch_desc(&tm_g);
   }
 
-  // State rows held in registers: row j of S^T, key columns [dk0, dk0 + 64).
+  // State rows held in registers: row j of S^T, key columns [dk0, dk0 + 32).
   const int j = 32 * quad + lane;
-  const int dk0 = 64 * half;
-  float S[64];
+  const int dk0 = 32 * grp;
+  float S[32];
   {
     const float *src = s0 ? s0 + (((size_t)n * H + h) * 128 + j) * 128 + dk0 : nullptr;
 #pragma unroll
-    for (int x = 0; x < 64; x += 4) {
+    for (int x = 0; x < 32; x += 4) {
       float4 f = src ? *reinterpret_cast<const float4 *>(src + x) : make_float4(0.f, 0.f, 0.f, 0.f);
       S[x] = f.x; S[x + 1] = f.y; S[x + 2] = f.z; S[x + 3] = f.w;
     }
@@ -242,7 +270,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
   __nv_bfloat16 *corr = reinterpret_cast<__nv_bfloat16 *>(sm + SM_CORR);
   const int HD = H * 128;
+  float *wconv = reinterpret_cast<float *>(sm + SM_WCONV);
   if constexpr (kFused) {
+    for (int idx = tid; idx < 3 * 128; idx += kThreads) {  // tap-major: lanes read consecutive channels
+      const int p = idx >> 7, ch = idx & 127;
+      const float4 w = __ldg(reinterpret_cast<const float4 *>(conv_w + ((size_t)p * HD + h * 128 + ch) * 4));
+      wconv[(p * 4 + 0) * 128 + ch] = w.x;
+      wconv[(p * 4 + 1) * 128 + ch] = w.y;
+      wconv[(p * 4 + 2) * 128 + ch] = w.z;
+      wconv[(p * 4 + 3) * 128 + ch] = w.w;
+    }
     // conv history before the sequence: the cache rows (oldest first) or zero
     for (int idx = tid; idx < 9 * 128; idx += kThreads) {
       const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
@@ -266,114 +303,124 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid < 64) beta_s[tid] = tid < Lc ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
     if constexpr (kFused) {
       // ---- Pc: prologue in place on the x tiles (fp32 arithmetic) ----------------------
+      // thread: 8 channels (c8) of two consecutive rows r0, r0+1 of all three parts;
+      // all raw values are read before any tile is overwritten.
       __syncthreads();  // beta_s visible
       const Tin *hcur = hist + (c & 1) * 1152;
       Tin *hnxt = hist + ((c + 1) & 1) * 1152;
-      const int c8 = tid & 15, d0 = c8 * 8;
-      float qn[4][8];
-#pragma unroll 1
+      const int c8 = tid & 15, d0 = c8 * 8, r0 = 2 * (tid >> 4);
+      uint4 packed[3][2];      // q, k, v of rows r0, r0+1 as fp16, written after the barrier
+      uint4 corr_pk[2];        // beta*v - f16(beta*f16(v)) as bf16
+      float q32[2][8];         // q in fp32 until k is known
+      float qk[2] = {0.f, 0.f};
+      float vmax = 0.f;
+#pragma unroll
       for (int p = 0; p < 3; ++p) {
-        uint8_t *tile = sm + (p == 0 ? SM_Q : (p == 1 ? SM_K : SM_V));
-        float w4[8][4];
-        {
-          const float *wp = conv_w + ((size_t)p * HD + h * 128 + d0) * 4;
+        const uint8_t *tile = sm + (p == 0 ? SM_Q : (p == 1 ? SM_K : SM_V));
+        float w8[4][8];  // taps x 8 channels
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(wp) + e);
-            w4[e][0] = f.x; w4[e][1] = f.y; w4[e][2] = f.z; w4[e][3] = f.w;
-          }
+        for (int tp = 0; tp < 4; ++tp) ld8_f32(wconv + (p * 4 + tp) * 128 + d0, w8[tp]);
+        uint4 xraw[5];  // raw rows r0-3 .. r0+1, still packed
+#pragma unroll
+        for (int t = 0; t < 5; ++t) {
+          const int rr = r0 - 3 + t;
+          xraw[t] = *reinterpret_cast<const uint4 *>(
+              rr >= 0 ? tile + rr * 256 + c8 * 16
+                      : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + rr) * 128) + c8 * 16);
         }
-        float y[4][8];
+
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int r = (tid >> 4) + 16 * m;
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int q2 = 0; q2 < 2; ++q2) {
+          float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int tap = 0; tap < 4; ++tap) {
-            const int rr = r - 3 + tap;
+          for (int tp = 0; tp < 4; ++tp) {
             float xv[8];
-            if (rr >= 0)
-              ld8_in<Tin>(tile + rr * 256 + c8 * 16, xv);
-            else
-              ld8_in<Tin>(reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + rr) * 128) + c8 * 16, xv);
+            unpack8(xraw[q2 + tp], xv, Tin());
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w4[e][tap], xv[e], acc[e]);
+            for (int e = 0; e < 8; ++e) y[e] = fmaf(w8[tp][e], xv[e], y[e]);
           }
           float ss = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            y[m][e] = silu(acc[e]);
-            ss = fmaf(y[m][e], y[m][e], ss);
+            y[e] = silu(y[e]);
+            ss = fmaf(y[e], y[e], ss);
           }
-          ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          if (p < 2) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          }
           const float sc = p < 2 ? rsqrtf(ss + 1e-6f) : 1.f;
-          const bool valid = r < Lc;
+          const bool valid = r0 + q2 < Lc;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[m][e] = valid ? y[m][e] * sc : 0.f;
-        }
-        // history for the next chunk: raw rows Lc-3 .. Lc-1 of this part
-        if (tid < 48) {
-          const int hr = tid >> 4, src = Lc - 3 + hr;
-          const uint8_t *from = src >= 0 ? tile + src * 256 + c8 * 16
-                                         : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + src) * 128) + c8 * 16;
-          *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(hnxt + (p * 3 + hr) * 128) + c8 * 16) =
-              *reinterpret_cast<const uint4 *>(from);
-        }
-        __syncthreads();  // every raw value of this part has been read
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int r = (tid >> 4) + 16 * m;
-          st_shared_16(tile, r * 256 + c8 * 16, pack8_in<Tact>(y[m]));
+          for (int e = 0; e < 8; ++e) y[e] = valid ? y[e] * sc : 0.f;
+          packed[p][q2] = pack8_in<Tact>(y);
           if (p == 0) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qn[m][e] = y[m][e];
+            for (int e = 0; e < 8; ++e) q32[q2][e] = y[e];
           } else if (p == 1) {
-            float qk = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qk = fmaf(qn[m][e], y[m][e], qk);
-            qk += __shfl_xor_sync(0xffffffffu, qk, 8);
-            qk += __shfl_xor_sync(0xffffffffu, qk, 4);
-            qk += __shfl_xor_sync(0xffffffffu, qk, 2);
-            qk += __shfl_xor_sync(0xffffffffu, qk, 1);
-            if (c8 == 0) pdiag[r] = qk;  // <q_r, k_r> of the fp32 prologue outputs
+            for (int e = 0; e < 8; ++e) qk[q2] = fmaf(q32[q2][e], y[e], qk[q2]);
           } else {
-            float vmax = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) vmax = fmaxf(vmax, fabsf(y[m][e]));
-            if (!(vmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
-            const float bt = beta_s[r];
+            const float bt = beta_s[r0 + q2];
             float cr[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float stored = to_f32(from_f32<Tact>(y[m][e]));
-              cr[e] = bt * y[m][e] - __half2float(__float2half_rn(bt * stored));
+              vmax = fmaxf(vmax, fabsf(y[e]));
+              const float stored = to_f32(from_f32<Tact>(y[e]));
+              cr[e] = bt * y[e] - __half2float(__float2half_rn(bt * stored));
             }
-            st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
+            corr_pk[q2] = pack8_bf16(cr);
           }
         }
-        __syncthreads();
       }
+      if (!(vmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        qk[q2] += __shfl_xor_sync(0xffffffffu, qk[q2], 8);
+        qk[q2] += __shfl_xor_sync(0xffffffffu, qk[q2], 4);
+        qk[q2] += __shfl_xor_sync(0xffffffffu, qk[q2], 2);
+        qk[q2] += __shfl_xor_sync(0xffffffffu, qk[q2], 1);
+      }
+      // history for the next chunk: raw rows Lc-3 .. Lc-1 of every part
+      if (tid < 144) {
+        const int p = tid / 48, hr = (tid % 48) >> 4, cc = tid & 15, src = Lc - 3 + hr;
+        const uint8_t *tile = sm + (p == 0 ? SM_Q : (p == 1 ? SM_K : SM_V));
+        const uint8_t *from = src >= 0 ? tile + src * 256 + cc * 16
+                                       : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + src) * 128) + cc * 16;
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(hnxt + (p * 3 + hr) * 128) + cc * 16) =
+            *reinterpret_cast<const uint4 *>(from);
+      }
+      __syncthreads();  // every raw value has been read
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int r = r0 + q2;
+        st_shared_16(sm + SM_Q, r * 256 + c8 * 16, packed[0][q2]);
+        st_shared_16(sm + SM_K, r * 256 + c8 * 16, packed[1][q2]);
+        st_shared_16(sm + SM_V, r * 256 + c8 * 16, packed[2][q2]);
+        st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, corr_pk[q2]);
+        if (c8 == 0) pdiag[r] = qk[q2];  // <q_r, k_r> of the fp32 prologue outputs
+      }
+      __syncthreads();
     }
-    {
-      const int d = tid & 127, part = tid >> 7;
-      float vals[32];
+    {  // inclusive cumulative log-decay along the chunk, per key channel
+      const int d = tid & 127, part = tid >> 7;  // rows [16*part, 16*part + 16)
+      float vals[16];
       float acc = 0.f;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const int rr = 32 * part + r;
+      for (int r = 0; r < 16; ++r) {
+        const int rr = 16 * part + r;
         const float gv = Gf[rr * 128 + d];
         acc += rr < Lc ? gv : 0.f;
         vals[r] = acc;
       }
-      float *tot = reinterpret_cast<float *>(sm + SM_XS);
-      if (part == 0) tot[d] = acc;
+      XS[part * 128 + d] = acc;
       __syncthreads();
-      const float off = part ? tot[d] : 0.f;
+      float off = 0.f;
+      for (int pp = 0; pp < part; ++pp) off += XS[pp * 128 + d];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) Gf[(32 * part + r) * 128 + d] = vals[r] + off;
+      for (int r = 0; r < 16; ++r) Gf[(16 * part + r) * 128 + d] = vals[r] + off;
     }
     __syncthreads();
     if (tid < 128) {
@@ -381,23 +428,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float ca = Gf[15 * 128 + d], cb = Gf[47 * 128 + d], cl = Gf[63 * 128 + d];
       fca[d] = ca;
       fcb[d] = cb;
-      feca[d] = expf(ca);
-      fecb[d] = expf(cb);
-      feba[d] = expf(0.5f * (cb - ca));
-      fela[d] = expf(cl - ca);
-      felb[d] = expf(cl - cb);
-      fegc[d] = expf(cl);
+      feca[d] = __expf(ca);
+      fecb[d] = __expf(cb);
+      feba[d] = __expf(0.5f * (cb - ca));
+      fela[d] = __expf(cl - ca);
+      felb[d] = __expf(cl - cb);
+      fegc[d] = __expf(cl);
     }
     __syncthreads();
     for (int idx = tid; idx < 64 * 128; idx += kThreads) {
       const int r = idx >> 7, d = idx & 127;
-      Gf[idx] = expf(Gf[idx] - (r < 32 ? fca[d] : fcb[d]));  // E_r in [e^-80, e^75]
+      Gf[idx] = __expf(Gf[idx] - (r < 32 ? fca[d] : fcb[d]));  // E_r in [e^-80, e^75]
     }
     __syncthreads();
 
     // ---- P2: Gram operands -------------------------------------------------------------
-#pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
       const int p = tid + kThreads * m;
       const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
       const bool valid = r < Lc;
@@ -405,13 +452,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
       ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
       ld8_f32(Gf + r * 128 + d0, e8);
-      float a[8], b[8], ki[8];
+      float a[8], b[8], ki[8], hf[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f;
         a[e] = kk * e8[e];
         b[e] = qq * e8[e];
-        ki[e] = kk * __frcp_rn(e8[e]);
+        ki[e] = __fdividef(kk, e8[e]);  // E in [e^-80, e^75]: inside the intrinsic's range
       }
       uint4 hi, lo;
       pack8_hilo(a, hi, lo);
@@ -424,8 +471,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         pack8_hilo(ki, hi, lo);
         st_shared_16(sm + SM_GB, kmaj_off(96, r, c8), hi);
         st_shared_16(sm + SM_GBL, kmaj_off(96, r, c8), lo);
+        ld8_f32(feba + d0, hf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * feba[d0 + e]) * feba[d0 + e];
+        for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * hf[e]) * hf[e];
       }
       pack8_hilo(ki, hi, lo);
       st_shared_16(sm + SM_GB, kmaj_off(96, 32 + r, c8), hi);
@@ -456,8 +504,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
 
     // ---- P4a: WY / output operands (the Gram operands are dead) -------------------------
-#pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
       const int p = tid + kThreads * m;
       const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
       const bool valid = r < Lc;
@@ -469,15 +517,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
       ld8_in<Tact>(sm + SM_V + r * 256 + c8 * 16, v8);
       ld8_f32(Gf + r * 128 + d0, e8);
-      float bkg[8], bv[8], qg[8], kp[8];
+      float bkg[8], bv[8], qg[8], kp[8], ec8[8], el8[8];
+      ld8_f32(fec + d0, ec8);
+      ld8_f32(fel + d0, el8);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f, vv = valid ? v8[e] : 0.f;
-        const float ec = fec[d0 + e];
-        bkg[e] = bt * kk * e8[e] * ec;
+        bkg[e] = bt * kk * e8[e] * ec8[e];
         bv[e] = bt * vv;
-        qg[e] = qq * e8[e] * ec;
-        kp[e] = kk * __frcp_rn(e8[e]) * fel[d0 + e];
+        qg[e] = qq * e8[e] * ec8[e];
+        kp[e] = __fdividef(kk, e8[e]) * el8[e];
       }
       st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
       st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
@@ -491,96 +540,125 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *TT = Gf + 4096;    // TT[r*64 + c] = T[r][c]
     for (int idx = tid; idx < 4096 / 4; idx += kThreads)
       reinterpret_cast<float4 *>(AT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int idx = tid; idx < 8192 / 16; idx += kThreads)
-      reinterpret_cast<uint4 *>(sm + SM_POP)[idx] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4 *>(sm + SM_POP)[tid] = make_uint4(0u, 0u, 0u, 0u);  // 8 KB
     if constexpr (!kFused) {
-      const int r = tid >> 2, part = tid & 3;
+      const int r = tid >> 3, part = tid & 7;
       float acc = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
+      for (int cc = 0; cc < 2; ++cc) {
         float q8[8], k8[8];
-        ld8_in<Tact>(sm + SM_Q + r * 256 + (part * 4 + c8) * 16, q8);
-        ld8_in<Tact>(sm + SM_K + r * 256 + (part * 4 + c8) * 16, k8);
+        ld8_in<Tact>(sm + SM_Q + r * 256 + (part * 2 + cc) * 16, q8);
+        ld8_in<Tact>(sm + SM_K + r * 256 + (part * 2 + cc) * 16, k8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc = fmaf(q8[e], k8[e], acc);
       }
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
       if (part == 0) pdiag[r] = r < Lc ? acc : 0.f;
     }
     __syncthreads();
     {
       const bool isP = quad >= 2;
       const int r = 32 * (quad & 1) + lane;
-      // first half: columns [0, 32) (i = col); second half: [32, 96) (i = col - 32)
-      const bool active = (quad & 1) || half == 0;
-      if (active) {
-        const int col0 = (quad & 1) ? 32 + 32 * half : 0;
-        const int ibase = (quad & 1) ? 32 * half : 0;
-        float v[32];
-        tmem_ld32(tmem + lane_addr + TM_G + col0, v);
-        const float br = beta_s[r];
+      const float br = beta_s[r];
+      // first half: columns [0, 32), i = col, 8 per column group;
+      // second half: columns [32, 96), i = col - 32, 16 per column group
+      float v[16];
+      int i0s;
+      if (quad & 1) {
+        tmem_ld16(tmem + lane_addr + TM_G + 32 + 16 * grp, v);
+        i0s = 16 * grp;
+      } else {
+        float v8[8];
+        tmem_ld8(tmem + lane_addr + TM_G + 8 * grp, v8);
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          const int i0 = ibase + 8 * g8;
-          if (!isP) {
+        for (int e = 0; e < 8; ++e) v[e] = v8[e];
+        i0s = 8 * grp;
+      }
+      const int nch = (quad & 1) ? 2 : 1;
+      for (int g8 = 0; g8 < nch; ++g8) {
+        const int i0 = i0s + 8 * g8;
+        if (!isP) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
-          } else if (i0 < r) {
-            float p8[8];
+          for (int e = 0; e < 8; ++e)
+            if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
+        } else if (i0 < r) {
+          float p8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
-            st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
-          }
+          for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
+          st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
         }
       }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 --------------------------------------
-    if (tid < 64) {
+    // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ------------------------------------
+    // (i) the four diagonal 16x16 blocks by forward substitution, one column per
+    //     thread; (ii) the two 16x16 blocks under them inside each 32x32 half,
+    //     T_{s+1,s} = -T_{s+1,s+1} A_{s+1,s} T_{s,s}; (iii) the lower-left 32x32
+    //     block T_BL = -T_BR (A_BL T_TL).
+    if (tid < 64) {  // column jj of a diagonal block, swept row by row, stored at the end
       const int base = 16 * (tid >> 4), jj = tid & 15;
-      float x[16];
+      float acc[16];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        float acc = 0.f;
+      for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
 #pragma unroll
-        for (int ii = 0; ii < rr; ++ii) acc = fmaf(AT[(base + ii) * 64 + base + rr], x[ii], acc);
-        x[rr] = rr == jj ? 1.f : (rr < jj ? 0.f : -acc);
+      for (int ii = 0; ii < 16; ++ii) {
+        acc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -acc[ii]);
+        const float *arow = AT + (base + ii) * 64 + base;  // A[base+rr][base+ii], rr > ii
+#pragma unroll
+        for (int rr = ii + 1; rr < 16; ++rr) acc[rr] = fmaf(arow[rr], acc[ii], acc[rr]);
       }
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = x[rr];
+      for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = acc[rr];
     }
     __syncthreads();
     {
-      float *XS = reinterpret_cast<float *>(sm + SM_XS);
-      for (int dlt = 1; dlt <= 3; ++dlt) {
-        const int nblk = 4 - dlt;
-        for (int idx = tid; idx < nblk * 256; idx += kThreads) {
-          const int s = dlt + (idx >> 8), sp = s - dlt, a = (idx >> 4) & 15, b = idx & 15;
-          float acc = 0.f;
-          for (int mb = sp; mb < s; ++mb) {
+      const int blk = tid >> 8, a = (tid >> 4) & 15, b = tid & 15, s0b = 32 * blk;
+      float acc = 0.f;  // (ii) X = A_{s+1,s} T_{s,s}
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-              acc = fmaf(AT[(16 * mb + t) * 64 + 16 * s + a], TT[(16 * mb + t) * 64 + 16 * sp + b], acc);
-          }
-          XS[idx] = acc;
-        }
-        __syncthreads();
-        for (int idx = tid; idx < nblk * 256; idx += kThreads) {
-          const int s = dlt + (idx >> 8), sp = s - dlt, a = (idx >> 4) & 15, b = idx & 15;
-          float acc = 0.f;
-          for (int t = 0; t <= a; ++t)
-            acc = fmaf(TT[(16 * s + a) * 64 + 16 * s + t], XS[(idx & ~255) + t * 16 + b], acc);
-          TT[(16 * s + a) * 64 + 16 * sp + b] = -acc;
-        }
-        __syncthreads();
-      }
+      for (int t = 0; t < 16; ++t)
+        acc = fmaf(AT[(s0b + t) * 64 + s0b + 16 + a], TT[(s0b + t) * 64 + s0b + b], acc);
+      XS[blk * 256 + a * 16 + b] = acc;
+      __syncthreads();
+      acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 16; ++t)  // T_{s+1,s+1}[a][t] is zero above the diagonal
+        acc = fmaf(TT[(s0b + 16 + a) * 64 + s0b + 16 + t], XS[blk * 256 + t * 16 + b], acc);
+      TT[(s0b + 16 + a) * 64 + s0b + b] = -acc;
     }
-    for (int p = tid; p < 512; p += kThreads) {
-      const int r = p >> 3, c8 = p & 7;
+    __syncthreads();
+    {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31), two rows per thread
+      const int cc = tid & 31, a0 = tid >> 5;  // rows a0, a0+16
+      float acc[2] = {0.f, 0.f};
+      for (int m = 0; m < 32; ++m) {
+        const float tv = m >= cc ? TT[m * 64 + cc] : 0.f;  // T_TL[m][cc]; its upper blocks are never written
+#pragma unroll
+        for (int q4 = 0; q4 < 2; ++q4) acc[q4] = fmaf(AT[m * 64 + 32 + a0 + 16 * q4], tv, acc[q4]);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 2; ++q4) XS[(a0 + 16 * q4) * 32 + cc] = acc[q4];
+    }
+    __syncthreads();
+    {  // T_BL = -T_BR Y
+      const int cc = tid & 31, a0 = tid >> 5;
+      float acc[2] = {0.f, 0.f};
+      for (int m = 0; m < 32; ++m) {
+        const float yv = XS[m * 32 + cc];
+#pragma unroll
+        for (int q4 = 0; q4 < 2; ++q4) {
+          const int a = a0 + 16 * q4;  // T_BR[a][m], zero for m > a
+          acc[q4] = fmaf(m <= a ? TT[(32 + a) * 64 + 32 + m] : 0.f, yv, acc[q4]);
+        }
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 2; ++q4) TT[(32 + a0 + 16 * q4) * 64 + cc] = -acc[q4];
+    }
+    __syncthreads();
+    {
+      const int r = tid >> 3, c8 = tid & 7;
       float f[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -592,7 +670,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     fence_async_smem();
     __syncthreads();
 
-    // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> bf16 operand ------------------------------
+    // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> fp16 operand ------------------------------
     if (tid == 0) {
       tc_fence_after();
       const uint32_t top = smem_u32(sm + SM_TOP), bkg = smem_u32(sm + SM_BKG);
@@ -609,14 +687,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     {
       float amax = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           f[e] = S[8 * cc + e];
           amax = fmaxf(amax, fabsf(f[e]));
         }
-        st_shared_16(sm + SM_ST, kmaj_off(128, j, 8 * half + cc), pack8_f16(f));
+        st_shared_16(sm + SM_ST, kmaj_off(128, j, 4 * grp + cc), pack8_f16(f));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
     }
@@ -627,15 +705,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // ---- P7: W^T read-out -> -W operand (MN-major, over beta K G) --------------------------
     {
-      float v[32];
-      tmem_ld32(tmem + lane_addr + TM_W + 32 * half, v);
-      const int dk = 32 * quad + lane;
+      float v[16];
+      tmem_ld16(tmem + lane_addr + TM_W + 16 * grp, v);
 #pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
+      for (int g8 = 0; g8 < 2; ++g8) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = -v[8 * g8 + e];
-        st_shared_16(sm + SM_BKG, mnmaj_off(128, dk, 4 * half + g8), pack8_f16(f));
+        st_shared_16(sm + SM_BKG, mnmaj_off(128, j, 2 * grp + g8), pack8_f16(f));
       }
     }
     fence_async_smem();
@@ -662,15 +739,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
 
     // ---- P9: U read-out (+ fp32 diagonal), U^T operand -----------------------------------
-    float u[32];
-    tmem_ld32(tmem + lane_addr + TM_U + 32 * half, u);
+    float u[16];
+    tmem_ld16(tmem + lane_addr + TM_U + 16 * grp, u);
     {
       const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
-#pragma unroll
       float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * half + i;
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * grp + i;
         const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
         const float bvv = beta_s[r] * vv;
         if constexpr (kFused)
@@ -681,11 +757,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
 #pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
+      for (int g8 = 0; g8 < 2; ++g8) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = u[8 * g8 + e];
-        st_shared_16(sm + SM_ST, kmaj_off(128, j, 4 * half + g8), pack8_f16(f));
+        st_shared_16(sm + SM_ST, kmaj_off(128, j, 2 * grp + g8), pack8_f16(f));
       }
     }
     fence_async_smem();
@@ -714,21 +790,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // ---- P11: outputs and state update ----------------------------------------------------
     {
-      float ov[32];
-      tmem_ld32(tmem + lane_addr + TM_O + 32 * half, ov);
+      float ov[16];
+      tmem_ld16(tmem + lane_addr + TM_O + 16 * grp, ov);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * half + i;
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * grp + i;
         if (r < Lc) o[((size_t)(t0 + r) * H + h) * 128 + j] = scale * fmaf(pdiag[r], u[i], ov[i]);
       }
+      float dv[32];
+      tmem_ld32(tmem + lane_addr + TM_S + dk0, dv);
 #pragma unroll
-      for (int l = 0; l < 2; ++l) {
-        float dv[32];
-        tmem_ld32(tmem + lane_addr + TM_S + 64 * half + 32 * l, dv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          S[32 * l + i] = fmaf(S[32 * l + i], fegc[dk0 + 32 * l + i], dv[i]);
-      }
+      for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], fegc[dk0 + i], dv[i]);
     }
     tc_fence_before();
     __syncthreads();
@@ -746,7 +818,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (sN) {
     float *dst = sN + (((size_t)n * H + h) * 128 + j) * 128 + dk0;
 #pragma unroll
-    for (int x = 0; x < 64; x += 4)
+    for (int x = 0; x < 32; x += 4)
       *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
   }
   tc_fence_before();

@@ -71,7 +71,63 @@ __device__ __forceinline__ void store8(float *p, const float (&in)[8]) {
   reinterpret_cast<float4 *>(p)[1] = make_float4(in[4], in[5], in[6], in[7]);
 }
 
-__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+// SiLU(x) = x * sigmoid(x) with the fast exponential and division intrinsics
+// (a few ulp; for x -> -inf the denominator overflows and the result is 0).
+// Eight consecutive elements kept in their storage type (16 bytes for 16-bit
+// types, 32 bytes for float) until they are used.
+template <typename T> struct Raw8 { uint4 u; };
+template <> struct Raw8<float> { float4 a, b; };
+
+__device__ __forceinline__ Raw8<__nv_bfloat16> load_raw8(const __nv_bfloat16 *p) {
+  return {__ldg(reinterpret_cast<const uint4 *>(p))};
+}
+__device__ __forceinline__ Raw8<__half> load_raw8(const __half *p) {
+  return {__ldg(reinterpret_cast<const uint4 *>(p))};
+}
+__device__ __forceinline__ Raw8<float> load_raw8(const float *p) {
+  return {__ldg(reinterpret_cast<const float4 *>(p)), __ldg(reinterpret_cast<const float4 *>(p) + 1)};
+}
+template <typename T> __device__ __forceinline__ Raw8<T> zero_raw8() {
+  Raw8<T> r;
+  r.u = make_uint4(0u, 0u, 0u, 0u);
+  return r;
+}
+template <> __device__ __forceinline__ Raw8<float> zero_raw8<float>() {
+  return {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+}
+__device__ __forceinline__ void widen8(const Raw8<__nv_bfloat16> &r, float (&f)[8]) {
+  const uint32_t w[4] = {r.u.x, r.u.y, r.u.z, r.u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void widen8(const Raw8<__half> &r, float (&f)[8]) {
+  const __half2 *h = reinterpret_cast<const __half2 *>(&r.u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void widen8(const Raw8<float> &r, float (&f)[8]) {
+  f[0] = r.a.x; f[1] = r.a.y; f[2] = r.a.z; f[3] = r.a.w;
+  f[4] = r.b.x; f[5] = r.b.y; f[6] = r.b.z; f[7] = r.b.w;
+}
+__device__ __forceinline__ void store_raw8(__nv_bfloat16 *p, const Raw8<__nv_bfloat16> &r) {
+  *reinterpret_cast<uint4 *>(p) = r.u;
+}
+__device__ __forceinline__ void store_raw8(__half *p, const Raw8<__half> &r) {
+  *reinterpret_cast<uint4 *>(p) = r.u;
+}
+__device__ __forceinline__ void store_raw8(float *p, const Raw8<float> &r) {
+  reinterpret_cast<float4 *>(p)[0] = r.a;
+  reinterpret_cast<float4 *>(p)[1] = r.b;
+}
+
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // ---------------------------------------------------------------------------
 // Device status word (one per device, allocated by the host layer)

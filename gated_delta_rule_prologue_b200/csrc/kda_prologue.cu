@@ -13,7 +13,9 @@
 //     (plus a 3-row halo per TT tokens, mostly served by L2);
 //   * the D/8 threads of a segment sit in one warp and reduce the sum of
 //     squares for the L2 norm with xor shuffles;
-//   * loads of a batch of 8 tokens are issued before any of them is used.
+//   * loads of a batch of 8 tokens are issued before any of them is used, and
+//     rows stay in their storage type until used (4 registers per 16-bit row),
+//     so two 256-thread blocks fit per SM with 64 KB of loads in flight.
 #include "kda_common.cuh"
 
 namespace kda {
@@ -21,20 +23,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTokensPerThread = 32;  // TT
-constexpr int kBatch = 8;             // tokens whose loads are in flight together
-
-template <typename Tin>
-__device__ __forceinline__ void load8_or_zero(const Tin *p, bool ok, float (&out)[8]) {
-  if (ok) {
-    load8(p, out);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = 0.f;
-  }
-}
+// tokens whose loads are in flight together (fewer for 32-byte float rows)
+template <typename Tin> constexpr int batch_of() { return sizeof(Tin) == 2 ? 8 : 4; }
 
 template <typename Tin, typename Tout, int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
                 const Tin *__restrict__ cache_in, Tin *__restrict__ cache_out,
                 const int32_t *__restrict__ cu, int N, int T, int H, Tout *__restrict__ q,
@@ -48,17 +41,16 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
   const int h = active ? (c0 % HD) / D : 0;
   const int d0 = c0 % D;
   Tout *out = p == 0 ? q : (p == 1 ? k : v);
+  auto load_or_zero = [&](const Tin *ptr, bool ok) { return ok ? load_raw8(ptr) : zero_raw8<Tin>(); };
 
   // Sequences with no tokens pass their cache through unchanged.
   if (blockIdx.y == 0 && cache_out != nullptr && active) {
     for (int n = 0; n < N; ++n) {
       const int a = cu ? cu[n] : 0, b = cu ? cu[n + 1] : T;
       if (a != b) continue;
-      for (int r = 0; r < 3; ++r) {
-        float tmp[8];
-        load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0, cache_in != nullptr, tmp);
-        store8(cache_out + ((size_t)n * 3 + r) * C + c0, tmp);
-      }
+      for (int r = 0; r < 3; ++r)
+        store_raw8(cache_out + ((size_t)n * 3 + r) * C + c0,
+                   load_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0, cache_in != nullptr));
     }
   }
 
@@ -87,34 +79,32 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
     seq_bounds(cu, n, T, status, bos, eos);
   }
 
-  // History of t0: tokens t0-3, t0-2, t0-1 (from the cache before bos).
-  float xm3[8], xm2[8], xm1[8];
+  // History of t0: tokens t0-3, t0-2, t0-1 (from the cache before bos), packed.
+  Raw8<Tin> hm3, hm2, hm1;
   {
+    Raw8<Tin> hv[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       const int tt = t0 - 3 + j;
-      float tmp[8];
       if (tt >= bos) {
-        load8_or_zero(x + (size_t)tt * C + c0, active, tmp);
+        hv[j] = load_or_zero(x + (size_t)tt * C + c0, active);
       } else {
         const int r = 3 - (bos - tt);  // cache row (0 = oldest)
-        load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0, active && cache_in != nullptr,
-                      tmp);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (j == 0) xm3[e] = tmp[e];
-        if (j == 1) xm2[e] = tmp[e];
-        if (j == 2) xm1[e] = tmp[e];
+        hv[j] = load_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0,
+                             active && cache_in != nullptr);
       }
     }
+    hm3 = hv[0];
+    hm2 = hv[1];
+    hm1 = hv[2];
   }
 
+  constexpr int kBatch = batch_of<Tin>();
   for (int tb = t0; tb < t_end; tb += kBatch) {
-    float xr[kBatch][8];
+    Raw8<Tin> xr[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i)
-      load8_or_zero(x + (size_t)(tb + i) * C + c0, active && tb + i < t_end, xr[i]);
+      xr[i] = load_or_zero(x + (size_t)(tb + i) * C + c0, active && tb + i < t_end);
 
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
@@ -125,28 +115,27 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
           ++n;
           seq_bounds(cu, n, T, status, bos, eos);
         } while (t >= eos && n < N - 1);
-#pragma unroll
-        for (int r = 0; r < 3; ++r) {
-          float tmp[8];
-          load8_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0,
-                        active && cache_in != nullptr, tmp);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (r == 0) xm3[e] = tmp[e];
-            if (r == 1) xm2[e] = tmp[e];
-            if (r == 2) xm1[e] = tmp[e];
-          }
-        }
+        const Tin *cr = cache_in + (size_t)n * 3 * C + c0;
+        const bool ok = active && cache_in != nullptr;
+        hm3 = load_or_zero(cr, ok);
+        hm2 = load_or_zero(cr + C, ok);
+        hm1 = load_or_zero(cr + 2 * C, ok);
       }
-      float y[8];
+      float y[8], f[8];
+      widen8(hm3, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = wt[e][0] * f[e];
+      widen8(hm2, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][1], f[e], y[e]);
+      widen8(hm1, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][2], f[e], y[e]);
+      widen8(xr[i], f);
       float ss = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        float a = wt[e][0] * xm3[e];
-        a = fmaf(wt[e][1], xm2[e], a);
-        a = fmaf(wt[e][2], xm1[e], a);
-        a = fmaf(wt[e][3], xr[i][e], a);
-        y[e] = silu(a);
+        y[e] = silu(fmaf(wt[e][3], f[e], y[e]));
         ss = fmaf(y[e], y[e], ss);
       }
 #pragma unroll
@@ -159,17 +148,14 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
       if (active) {
         store8(out + ((size_t)t * H + h) * D + d0, y);
         if (cache_out != nullptr && t == eos - 1) {
-          store8(cache_out + ((size_t)n * 3 + 0) * C + c0, xm2);
-          store8(cache_out + ((size_t)n * 3 + 1) * C + c0, xm1);
-          store8(cache_out + ((size_t)n * 3 + 2) * C + c0, xr[i]);
+          store_raw8(cache_out + ((size_t)n * 3 + 0) * C + c0, hm2);
+          store_raw8(cache_out + ((size_t)n * 3 + 1) * C + c0, hm1);
+          store_raw8(cache_out + ((size_t)n * 3 + 2) * C + c0, xr[i]);
         }
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        xm3[e] = xm2[e];
-        xm2[e] = xm1[e];
-        xm1[e] = xr[i][e];
-      }
+      hm3 = hm2;
+      hm2 = hm1;
+      hm1 = xr[i];
     }
   }
 }

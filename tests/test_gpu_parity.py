@@ -227,6 +227,29 @@ def test_k3_prefill_full_size_sampled_heads(kda):
         assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
 
 
+def test_k3_unfused_full_size_sampled_heads(kda):
+    """kda_prologue (fp16 q/k/v) followed by kda_chunk_fwd over the full K3
+    workload; heads 3 and 61 against the oracle."""
+    inp = W.k3_prefill()
+    T, H, D = inp.T, inp.H, inp.D
+    dev = "cuda"
+    q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    kda.kda_prologue(inp.x.to(dev), inp.conv_w.to(dev), q, k, v, H=H, D=D)
+    o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+    fs = torch.empty((1, H, D, D), device=dev)
+    kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, scale=inp.scale,
+                      final_state=fs, chunk=inp.chunk)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    for h in (3, 61):
+        xh, wh, gh, bh = W.k3_prefill_head(h)
+        qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
+        o_ref, S_ref = kda_recurrent(qr, kr, vr, gh[:, None, :], bh[:, None], inp.scale)
+        assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16
+        assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
+
+
 def test_k3_prologue_kernel_full_size_sampled_heads(kda):
     """The standalone prologue over the full K3-shaped input, fp16 outputs."""
     inp = W.k3_prefill()
