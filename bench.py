@@ -164,11 +164,21 @@ def dist_setup(args):
 
 
 def max_over_ranks(x, world):
+    """The largest of the ranks' values (device timings are compared on every
+    rank; the slowest rank defines the job's time)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, units_per_rank, local_ms):
+    """Whole-job units/s for replicas that each process `units_per_rank` units:
+    every rank's units over the slowest rank's time.  Returns (value, max_ms)."""
+    ms = max_over_ranks(local_ms, world)
+    return world * units_per_rank / (ms * 1e-3), ms
 
 
 def barrier(world):
@@ -296,12 +306,10 @@ def run_ours(args, world, rank, local):
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
-    total_ms = max_over_ranks(start.elapsed_time(end), world)
-    ms_step = total_ms / args.steps
+    value, ms_step = job_throughput(world, T, start.elapsed_time(end) / args.steps)
     pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     chk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     assert kda.kda_get_device_status() == 0
-    value = world * T / (ms_step * 1e-3)
     launches = 2 * args.steps
 
     # the fused variant (prologue inside the chunk kernel), timed beside the step
@@ -347,7 +355,7 @@ def run_ours(args, world, rank, local):
         out_host.copy_(o, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e_value, e2e_ms = job_throughput(world, T, e0.elapsed_time(e1) / e2e_steps)
     h2d = inp.x.numel() * 2 + inp.g.numel() * 4 + inp.beta.numel() * 4
     d2h = out_host.numel() * 4
     del x, o, g, beta, inp
@@ -381,11 +389,11 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     barrier(world)
     assert kda.kda_get_device_status() == 0
-    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / args.decode_steps
+    dec_value, dec_ms = job_throughput(world, Nd, d0.elapsed_time(d1) / args.decode_steps)
     dec_kernel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in dev_ev)
     decode = {
         "metric": "decode tokens/s", "unit": "tokens/s",
-        "value": round(world * Nd / (dec_ms * 1e-3), 1),
+        "value": round(dec_value, 1),
         "ms_per_step": round(dec_ms, 4), "steps": args.decode_steps,
         "workload": "decode256: 256 sequences x 96 heads x d=128, fp32 state in place, "
                     "bf16 projections with conv cache",
@@ -413,7 +421,7 @@ def run_ours(args, world, rank, local):
         "kernels": kernels,
         "fused_hbm_floor_ms": round(fused_floor_ms, 4),
         "decode": decode,
-        "e2e": {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_total,

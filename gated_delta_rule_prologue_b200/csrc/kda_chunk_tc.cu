@@ -254,18 +254,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *slot;
   const uint32_t lane_addr = static_cast<uint32_t>(32 * quad) << 16;
 
-  auto issue_tma = [&](int t) {
+  // The next chunk's tiles are requested as soon as each buffer is dead: q and k
+  // after the Gram read-out, g after the inverse, v after the U read-out; one
+  // mbarrier phase counts all four.
+  auto issue_tma_qk = [&](int t) {
     mbar_arrive_expect_tx(bar_tma, kTmaBytes);
     if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
       tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
       tma_load_3d(sm + SM_K, &tm_q, bar_tma, 0, H + h, t);
-      tma_load_3d(sm + SM_V, &tm_q, bar_tma, 0, 2 * H + h, t);
     } else {
       tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
       tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, h, t);
-      tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
     }
-    tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, h, t);
+  };
+  auto issue_tma_g = [&](int t) { tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, h, t); };
+  auto issue_tma_v = [&](int t) {
+    if constexpr (kFused)
+      tma_load_3d(sm + SM_V, &tm_q, bar_tma, 0, 2 * H + h, t);
+    else
+      tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
+  };
+  auto issue_tma = [&](int t) {
+    issue_tma_qk(t);
+    issue_tma_g(t);
+    issue_tma_v(t);
   };
   Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
   __nv_bfloat16 *corr = reinterpret_cast<__nv_bfloat16 *>(sm + SM_CORR);
@@ -404,7 +416,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       __syncthreads();
     }
-    {  // inclusive cumulative log-decay along the chunk, per key channel
+    {  // inclusive cumulative log-decay along the chunk, per key channel, then E in place
       const int d = tid & 127, part = tid >> 7;  // rows [16*part, 16*part + 16)
       float vals[16];
       float acc = 0.f;
@@ -420,25 +432,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float off = 0.f;
       for (int pp = 0; pp < part; ++pp) off += XS[pp * 128 + d];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) Gf[(16 * part + r) * 128 + d] = vals[r] + off;
-    }
-    __syncthreads();
-    if (tid < 128) {
-      const int d = tid;
-      const float ca = Gf[15 * 128 + d], cb = Gf[47 * 128 + d], cl = Gf[63 * 128 + d];
-      fca[d] = ca;
-      fcb[d] = cb;
-      feca[d] = __expf(ca);
-      fecb[d] = __expf(cb);
-      feba[d] = __expf(0.5f * (cb - ca));
-      fela[d] = __expf(cl - ca);
-      felb[d] = __expf(cl - cb);
-      fegc[d] = __expf(cl);
-    }
-    __syncthreads();
-    for (int idx = tid; idx < 64 * 128; idx += kThreads) {
-      const int r = idx >> 7, d = idx & 127;
-      Gf[idx] = __expf(Gf[idx] - (r < 32 ? fca[d] : fcb[d]));  // E_r in [e^-80, e^75]
+      for (int r = 0; r < 16; ++r) vals[r] += off;
+      if (part == 0) fca[d] = vals[15];  // c_A = gamma_15
+      if (part == 2) fcb[d] = vals[15];  // c_B = gamma_47
+      if (part == 3) fegc[d] = vals[15]; // gamma_63 (exponentiated below)
+      __syncthreads();
+      const float ref = part < 2 ? fca[d] : fcb[d];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) Gf[(16 * part + r) * 128 + d] = __expf(vals[r] - ref);
+      if (tid < 128) {
+        const float ca = fca[d], cb = fcb[d], cl = fegc[d];
+        feca[d] = __expf(ca);
+        fecb[d] = __expf(cb);
+        feba[d] = __expf(0.5f * (cb - ca));
+        fela[d] = __expf(cl - ca);
+        felb[d] = __expf(cl - cb);
+      }
+      __syncthreads();
+      if (tid < 128) fegc[d] = __expf(fegc[d]);  // every reader of gamma_63 is past the barrier
     }
     __syncthreads();
 
@@ -593,6 +604,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && c + 1 < nchunks) issue_tma_qk(t0 + 64);  // q, k tiles are dead
 
     // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ------------------------------------
     // (i) the four diagonal 16x16 blocks by forward substitution, one column per
@@ -633,6 +645,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31), two rows per thread
       const int cc = tid & 31, a0 = tid >> 5;  // rows a0, a0+16
       float acc[2] = {0.f, 0.f};
+#pragma unroll 8
       for (int m = 0; m < 32; ++m) {
         const float tv = m >= cc ? TT[m * 64 + cc] : 0.f;  // T_TL[m][cc]; its upper blocks are never written
 #pragma unroll
@@ -645,6 +658,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     {  // T_BL = -T_BR Y
       const int cc = tid & 31, a0 = tid >> 5;
       float acc[2] = {0.f, 0.f};
+#pragma unroll 8
       for (int m = 0; m < 32; ++m) {
         const float yv = XS[m * 32 + cc];
 #pragma unroll
@@ -669,6 +683,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     __syncthreads();
+    if (tid == 0 && c + 1 < nchunks) issue_tma_g(t0 + 64);  // A^T / T (the g tile) are dead
 
     // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> fp16 operand ------------------------------
     if (tid == 0) {
@@ -734,6 +749,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_bf16(tmem + TM_O, desc_kmajor(st, 128, ks), desc_kmajor(qg, 64, ks), idO, ks > 0);
       mma_commit(bar_mma);
     }
+    // ---- P9 (first half, overlapping the MMAs): the fp32 diagonal correction ---------------
+    float dcorr[16], bvmax = 0.f;
+    {
+      const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * grp + i;
+        const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
+        const float bvv = beta_s[r] * vv;
+        if constexpr (kFused)
+          dcorr[i] = __bfloat162float(corr[r * 128 + j]);
+        else
+          dcorr[i] = bvv - __half2float(__float2half_rn(bvv));
+        bvmax = fmaxf(bvmax, fabsf(bvv));
+      }
+    }
     if (!wait_all(bar_mma, mma_par, status)) break;
     mma_par ^= 1;
     tc_fence_after();
@@ -742,18 +773,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float u[16];
     tmem_ld16(tmem + lane_addr + TM_U + 16 * grp, u);
     {
-      const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
-      float amax = 0.f;
+      float amax = bvmax;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int r = 16 * grp + i;
-        const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
-        const float bvv = beta_s[r] * vv;
-        if constexpr (kFused)
-          u[i] += __bfloat162float(corr[r * 128 + j]);
-        else
-          u[i] += bvv - __half2float(__float2half_rn(bvv));
-        amax = fmaxf(amax, fmaxf(fabsf(u[i]), fabsf(bvv)));
+        u[i] += dcorr[i];
+        amax = fmaxf(amax, fabsf(u[i]));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
 #pragma unroll
@@ -767,8 +791,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && c + 1 < nchunks) issue_tma_v(t0 + 64);  // the v tile is dead
 
-    // ---- P10: O^T += U^T P^T ; delta S^T = U^T K' ; next chunk's tiles ------------------
+    // ---- P10: O^T += U^T P^T ; delta S^T = U^T K' ----------------------------------------
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ut = smem_u32(sm + SM_ST), pop = smem_u32(sm + SM_POP);
@@ -782,7 +807,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int ks = 0; ks < 4; ++ks)
         mma_bf16(tmem + TM_S, desc_kmajor(ut, 128, ks), desc_mnmajor(kp, 64, ks), idS, ks > 0);
       mma_commit(bar_mma);
-      if (c + 1 < nchunks) issue_tma(t0 + 64);
     }
     if (!wait_all(bar_mma, mma_par, status)) break;
     mma_par ^= 1;
@@ -790,15 +814,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // ---- P11: outputs and state update ----------------------------------------------------
     {
-      float ov[16];
-      tmem_ld16(tmem + lane_addr + TM_O + 16 * grp, ov);
+      float ov[16], dv[32];
+      tmem_ld16_nowait(tmem + lane_addr + TM_O + 16 * grp, ov);
+      tmem_ld32_nowait(tmem + lane_addr + TM_S + dk0, dv);
+      tmem_wait_ld(ov, dv);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = 16 * grp + i;
         if (r < Lc) o[((size_t)(t0 + r) * H + h) * 128 + j] = scale * fmaf(pdiag[r], u[i], ov[i]);
       }
-      float dv[32];
-      tmem_ld32(tmem + lane_addr + TM_S + dk0, dv);
 #pragma unroll
       for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], fegc[dk0 + i], dv[i]);
     }

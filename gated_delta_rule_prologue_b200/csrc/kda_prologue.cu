@@ -24,7 +24,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTokensPerThread = 32;  // TT
 // tokens whose loads are in flight together (fewer for 32-byte float rows)
-template <typename Tin> constexpr int batch_of() { return sizeof(Tin) == 2 ? 8 : 4; }
+template <typename Tin> __host__ __device__ constexpr int batch_of() { return sizeof(Tin) == 2 ? 8 : 4; }
 
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kThreads, 2)
