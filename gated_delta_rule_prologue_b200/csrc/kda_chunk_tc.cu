@@ -627,57 +627,89 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = acc[rr];
     }
     __syncthreads();
-    {
-      const int blk = tid >> 8, a = (tid >> 4) & 15, b = tid & 15, s0b = 32 * blk;
-      float acc = 0.f;  // (ii) X = A_{s+1,s} T_{s,s}
+    // Blocks below the diagonal, 2x2 output tiles per thread.  A is read through
+    // its transpose (columns of A are contiguous), T and Y by rows, so the
+    // operands of one k-step are float2 loads.
+    if (tid < 128) {  // (ii) X = A_{s+1,s} T_{s,s} for s = 0, 2
+      const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
+      float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        acc = fmaf(AT[(s0b + t) * 64 + s0b + 16 + a], TT[(s0b + t) * 64 + s0b + b], acc);
-      XS[blk * 256 + a * 16 + b] = acc;
-      __syncthreads();
-      acc = 0.f;
-#pragma unroll
-      for (int t = 0; t < 16; ++t)  // T_{s+1,s+1}[a][t] is zero above the diagonal
-        acc = fmaf(TT[(s0b + 16 + a) * 64 + s0b + 16 + t], XS[blk * 256 + t * 16 + b], acc);
-      TT[(s0b + 16 + a) * 64 + s0b + b] = -acc;
-    }
-    __syncthreads();
-    {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31), two rows per thread
-      const int cc = tid & 31, a0 = tid >> 5;  // rows a0, a0+16
-      float acc[2] = {0.f, 0.f};
-#pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float tv = m >= cc ? TT[m * 64 + cc] : 0.f;  // T_TL[m][cc]; its upper blocks are never written
-#pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4) acc[q4] = fmaf(AT[m * 64 + 32 + a0 + 16 * q4], tv, acc[q4]);
+      for (int t = 0; t < 16; ++t) {
+        const float2 av = *reinterpret_cast<const float2 *>(AT + (s0b + t) * 64 + s0b + 16 + a);
+        const float2 tv = *reinterpret_cast<const float2 *>(TT + (s0b + t) * 64 + s0b + b);
+        x00 = fmaf(av.x, tv.x, x00); x01 = fmaf(av.x, tv.y, x01);
+        x10 = fmaf(av.y, tv.x, x10); x11 = fmaf(av.y, tv.y, x11);
       }
-#pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) XS[(a0 + 16 * q4) * 32 + cc] = acc[q4];
+      *reinterpret_cast<float2 *>(XS + blk * 256 + a * 16 + b) = make_float2(x00, x01);
+      *reinterpret_cast<float2 *>(XS + blk * 256 + (a + 1) * 16 + b) = make_float2(x10, x11);
     }
     __syncthreads();
-    {  // T_BL = -T_BR Y
-      const int cc = tid & 31, a0 = tid >> 5;
-      float acc[2] = {0.f, 0.f};
-#pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float yv = XS[m * 32 + cc];
+    if (tid < 128) {  // T_{s+1,s} = -T_{s+1,s+1} X
+      const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
+      const float *t0r = TT + (s0b + 16 + a) * 64 + s0b + 16;  // row a of T_{s+1,s+1}
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4) {
-          const int a = a0 + 16 * q4;  // T_BR[a][m], zero for m > a
-          acc[q4] = fmaf(m <= a ? TT[(32 + a) * 64 + 32 + m] : 0.f, yv, acc[q4]);
+      for (int t4 = 0; t4 < 16; t4 += 4) {  // diagonal blocks were stored with their zeros
+        const float4 ra = *reinterpret_cast<const float4 *>(t0r + t4);
+        const float4 rb = *reinterpret_cast<const float4 *>(t0r + 64 + t4);
+        const float ta[4] = {ra.x, ra.y, ra.z, ra.w}, tb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 xv = *reinterpret_cast<const float2 *>(XS + blk * 256 + (t4 + e) * 16 + b);
+          y00 = fmaf(ta[e], xv.x, y00); y01 = fmaf(ta[e], xv.y, y01);
+          y10 = fmaf(tb[e], xv.x, y10); y11 = fmaf(tb[e], xv.y, y11);
         }
       }
+      *reinterpret_cast<float2 *>(TT + (s0b + 16 + a) * 64 + s0b + b) = make_float2(-y00, -y01);
+      *reinterpret_cast<float2 *>(TT + (s0b + 17 + a) * 64 + s0b + b) = make_float2(-y10, -y11);
+    }
+    __syncthreads();
+    if (tid < 256) {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31)
+      const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const float2 av = *reinterpret_cast<const float2 *>(AT + m * 64 + 32 + a);
+        float2 tv = *reinterpret_cast<const float2 *>(TT + m * 64 + cc);  // T_TL[m][cc..cc+1]
+        tv.x = m >= cc ? tv.x : 0.f;                                      // upper blocks unwritten
+        tv.y = m >= cc + 1 ? tv.y : 0.f;
+        y00 = fmaf(av.x, tv.x, y00); y01 = fmaf(av.x, tv.y, y01);
+        y10 = fmaf(av.y, tv.x, y10); y11 = fmaf(av.y, tv.y, y11);
+      }
+      *reinterpret_cast<float2 *>(XS + a * 32 + cc) = make_float2(y00, y01);
+      *reinterpret_cast<float2 *>(XS + (a + 1) * 32 + cc) = make_float2(y10, y11);
+    }
+    __syncthreads();
+    if (tid < 256) {  // T_BL = -T_BR Y
+      const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
+      const float *tr = TT + (32 + a) * 64 + 32;  // row a of T_BR
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 2
+      for (int m4 = 0; m4 < 32; m4 += 4) {
+        const float4 ra = *reinterpret_cast<const float4 *>(tr + m4);
+        const float4 rb = *reinterpret_cast<const float4 *>(tr + 64 + m4);
+        const float ta4[4] = {ra.x, ra.y, ra.z, ra.w}, tb4[4] = {rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) TT[(32 + a0 + 16 * q4) * 64 + cc] = -acc[q4];
+        for (int e = 0; e < 4; ++e) {  // T_BR's upper-right 16x16 block was never written
+          const int m = m4 + e;
+          const float ta = m <= a ? ta4[e] : 0.f, tb = m <= a + 1 ? tb4[e] : 0.f;
+          const float2 yv = *reinterpret_cast<const float2 *>(XS + m * 32 + cc);
+          y00 = fmaf(ta, yv.x, y00); y01 = fmaf(ta, yv.y, y01);
+          y10 = fmaf(tb, yv.x, y10); y11 = fmaf(tb, yv.y, y11);
+        }
+      }
+      *reinterpret_cast<float2 *>(TT + (32 + a) * 64 + cc) = make_float2(-y00, -y01);
+      *reinterpret_cast<float2 *>(TT + (33 + a) * 64 + cc) = make_float2(-y10, -y11);
     }
     __syncthreads();
     {
       const int r = tid >> 3, c8 = tid & 7;
       float f[8];
+      ld8_f32(TT + r * 64 + 8 * c8, f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int cc = 8 * c8 + e;
-        f[e] = cc < r ? TT[r * 64 + cc] : (cc == r ? 1.f : 0.f);
+        f[e] = cc < r ? f[e] : (cc == r ? 1.f : 0.f);
       }
       st_shared_16(sm + SM_TOP, kmaj_off(64, r, c8), pack8_f16(f));
     }
