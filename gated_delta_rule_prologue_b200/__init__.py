@@ -72,12 +72,16 @@ lib.kda_prologue.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _v
                              _vp]
 lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               _i, _vp, _vp, _vp]
+lib.kda_chunk_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                 _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
-for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_decode_step, lib.kda_prologue_chunk_fwd,
-            lib.kda_get_device_status):
+for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_decode_step,
+            lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
 lib.kda_last_error.argtypes = []
@@ -92,6 +96,9 @@ def _check(status: int):
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 
 def _dtype(t) -> int:
@@ -149,9 +156,21 @@ def kda_prologue(x, conv_w, q, k, v, *, H: int, D: int, cache_in=None, cache_out
                             _ptr(k), _ptr(v), _stream(stream)))
 
 
+def kda_chunk_fwd_workspace_bytes(N: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
+                                  dtype: torch.dtype) -> int:
+    """Scratch bytes of the two-pass tensor-core prefill (0 if it does not apply)."""
+    return int(lib.kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, _DTYPES[dtype]))
+
+
 def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None,
-                  final_state=None, cu_seqlens=None, chunk: int = 64, stream=None):
-    """Chunkwise prefill: writes ``o`` [T, H, Dv] and optionally ``final_state``."""
+                  final_state=None, cu_seqlens=None, chunk: int = 64, workspace="auto",
+                  stream=None):
+    """Chunkwise prefill: writes ``o`` [T, H, Dv] and optionally ``final_state``.
+
+    ``workspace``: ``"auto"`` allocates the two-pass path's scratch from
+    torch's caching allocator; a uint8 CUDA tensor is used as given (at least
+    :func:`kda_chunk_fwd_workspace_bytes`); ``None`` runs the one-pass kernels.
+    """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
     for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
@@ -161,9 +180,21 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
     T, H, Dk = q.shape
     Dv = v.shape[2]
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
-    _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
-                             _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
-                             _dtype(q), _ptr(o), _ptr(final_state), _stream(stream)))
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto', None or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, q.dtype)
+        workspace = (torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None)
+    if workspace is None:
+        _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                 _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
+                                 _dtype(q), _ptr(o), _ptr(final_state), _stream(stream)))
+        return
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_chunk_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
+                                _dtype(q), _ptr(o), _ptr(final_state), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
 
 
 def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: float = 1.0,

@@ -9,6 +9,7 @@
 #include <mutex>
 #include <string>
 
+#include "kda_chunk_record.cuh"
 #include "kda_common.cuh"
 
 namespace {
@@ -160,11 +161,19 @@ kda_status kda_prologue(const void *x, const float *conv_w, const void *cache_in
   return KDA_OK;
 }
 
-kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
-                         const float *beta, float scale, const float *initial_state,
-                         const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
-                         int chunk, kda_dtype dt, float *o, float *final_state,
-                         kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+bool chunk_tc_path(int T, int Dk, int Dv, int chunk, kda_dtype dt) {
+  return dt != KDA_F32 && Dk == 128 && Dv == 128 && chunk == 64 && T > 0;
+}
+
+// Argument checks shared by kda_chunk_fwd and kda_chunk_fwd_ws.
+kda_status check_chunk_args(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *initial_state,
+                            const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                            int chunk, kda_dtype dt, float *o, float *final_state) {
   KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
   KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1 && Dk >= 1 && Dv >= 1,
               "bad sizes N=%d T=%d H=%d Dk=%d Dv=%d", N, T, H, Dk, Dv);
@@ -197,12 +206,27 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
   KDA_REQUIRE(final_state == initial_state ||
                   !overlaps(final_state, sbytes, initial_state, sbytes),
               "final_state partially overlaps initial_state");
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, float scale, const float *initial_state,
+                         const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                         int chunk, kda_dtype dt, float *o, float *final_state,
+                         kda_stream_t stream) {
+  kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                                   chunk, dt, o, final_state);
+  if (st != KDA_OK) return st;
   int *status = nullptr;
-  kda_status st = device_status_word(&status);
+  st = device_status_word(&status);
   if (st != KDA_OK) return st;
   if (T == 0 && final_state == nullptr) return KDA_OK;
   cudaError_t e;
-  if (dt != KDA_F32 && Dk == 128 && chunk == 64 && T > 0) {
+  if (chunk_tc_path(T, Dk, Dv, chunk, dt)) {
     e = kda::launch_chunk_tc(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, dt, o,
                              final_state, status, (cudaStream_t)stream);
   } else {
@@ -210,6 +234,57 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
                                chunk, dt, o, final_state, status, (cudaStream_t)stream);
   }
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
+  return KDA_OK;
+}
+
+size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt) {
+  if (N < 1 || T < 0 || H < 1 || !chunk_tc_path(T, Dk, Dv, chunk, dt)) return 0;
+  return kda::rec::workspace_bytes(N, T, H);
+}
+
+kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *initial_state,
+                            const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                            int chunk, kda_dtype dt, float *o, float *final_state,
+                            void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+  if (workspace == nullptr)
+    return kda_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                         chunk, dt, o, final_state, stream);
+  kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                                   chunk, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, dt);
+  if (need == 0)
+    return kda_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                         chunk, dt, o, final_state, stream);
+  KDA_OPT_PTR(workspace, "workspace");
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {
+    const size_t es = esize(dt), act = (size_t)T * H * Dk * es;
+    const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
+    const void *others[8] = {q, k, v, g, beta, o, initial_state, final_state};
+    const size_t osz[8] = {act, act, act, (size_t)T * H * Dk * 4, (size_t)T * H * 4,
+                           (size_t)T * H * Dv * 4, sbytes, sbytes};
+    for (int i = 0; i < 8; ++i)
+      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
+                  "workspace overlaps another argument");
+    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
+                "workspace overlaps cu_seqlens");
+  }
+  int *status = nullptr;
+  st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+                                final_state, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_ws launch");
   return KDA_OK;
 }
 

@@ -42,10 +42,12 @@
 // One CTA (512 threads) per (sequence, head); the chunks of a sequence run in
 // order, the next chunk's tiles stream in by TMA during the current one.
 #include <cuda.h>
+#include <algorithm>
 #include <cstring>
 #include <type_traits>
 #include <cudaTypedefs.h>
 
+#include "kda_chunk_record.cuh"
 #include "kda_common.cuh"
 #include "kda_tcgen05.cuh"
 
@@ -169,33 +171,34 @@ __device__ __forceinline__ uint4 pack8_in(const float (&f)[8]) {
   return u;
 }
 
-// All threads wait for a barrier phase; false (and a recorded timeout) if any
-// thread gave up.  Also acts as a CTA-wide barrier.
-__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *status) {
-  const bool ok = mbar_wait(bar, parity);
-  if (__syncthreads_or(!ok)) {
-    if (threadIdx.x == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
-    return false;
-  }
-  return true;
-}
-
-// kFused = false: q, k, v tiles come from HBM as given (already unit-normalised).
-// kFused = true:  the three tiles are the raw projections x (parts q, k, v of
-// head h); the prologue (causal width-4 conv with history, SiLU, L2 on q and
-// k) runs in fp32 in shared memory and overwrites them with q, k, v.
+// Modes.
+//   kSingle: one CTA per (sequence, head) walks its chunks in order and carries
+//            the state: the whole chunk update in one kernel.  q, k, v tiles
+//            come from HBM as given (already unit-normalised).
+//   kFused:  as kSingle, but the three tiles are the raw projections x (parts
+//            q, k, v of head h); the prologue (causal width-4 conv with
+//            history, SiLU, L2 on q and k) runs in fp32 in shared memory and
+//            overwrites them with q, k, v.
+//   kPrep:   the state-independent half only: persistent CTAs take the
+//            (chunk, head) items blockIdx.x, blockIdx.x + gridDim.x, ... and
+//            write one record per item (kda_chunk_record.cuh); the state pass
+//            (kda_chunk_state.cu) applies the records in order.
 //
 // Thread layout (512 threads, 16 warps): warp w reads TMEM lanes
 // 32*(w%4).. (its "quad") and handles column group w/4 of every accumulator it
 // reads; element-wise phases walk (row, 8-channel chunk) pairs.
-template <typename Tin, bool kFused>
+constexpr int kSingle = 0, kFusedMode = 1, kPrep = 2;
+
+template <typename Tin, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                 const float *__restrict__ beta, float scale, const float *s0,
                 const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
                 int *status, const float *__restrict__ conv_w, const Tin *cache_in,
-                Tin *cache_out) {
+                Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N) {
+  constexpr bool kFused = kMode == kFusedMode;
+  constexpr bool kPrepM = kMode == kPrep;
   // Element type of the q/k/v tiles the chunk phases read: the inputs as given,
   // or fp16 written by the fused prologue (q, k are unit vectors; v is guarded).
   using Tact = typename std::conditional<kFused, __half, Tin>::type;
@@ -204,7 +207,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, grp = warp >> 2;
-  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  const int n = blockIdx.x / H, hb = blockIdx.x % H;  // kSingle / kFused
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);
   uint64_t *bar_mma = bar_tma + 1;
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SM_SLOT);
@@ -221,9 +224,53 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   float *fegc = reinterpret_cast<float *>(sm + F_EGC);
   float *XS = reinterpret_cast<float *>(sm + SM_XS);
 
-  int bos, eos;
-  seq_bounds(cu, n, T, status, bos, eos);
-  const int nchunks = (eos - bos + 63) / 64;
+  // The work walk: (t0, Lc, head, chunk number) of step `it`.
+  struct Work {
+    int t0, Lc, h, ci;
+    bool ok;
+  };
+  int bos = 0, eos = 0, nchunks = 0;
+  long long items = 0;
+  int total_chunks = 0;
+  if constexpr (kPrepM) {
+    const long long cap = rec::chunk_capacity(N, T);
+    total_chunks = cu ? (int)min((long long)cprefix[N], cap) : (T + 63) / 64;
+    items = (long long)total_chunks * H;
+  } else {
+    seq_bounds(cu, n, T, status, bos, eos);
+    nchunks = (eos - bos + 63) / 64;
+  }
+  auto work_of = [&](int it) -> Work {
+    Work w;
+    if constexpr (kPrepM) {
+      const long long item = (long long)blockIdx.x + (long long)it * gridDim.x;
+      w.ok = item < items;
+      if (!w.ok) return w;
+      w.ci = (int)(item / H);
+      w.h = (int)(item % H);
+      int sb = 0, se = T, c0 = 0;
+      if (cu) {  // sequence of chunk ci: the last n with cprefix[n] <= ci
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (cprefix[mid] <= w.ci) lo = mid; else hi = mid - 1;
+        }
+        sb = min(max(cu[lo], 0), T);  // well-formed here: the index pass checked cu
+        se = min(max(cu[lo + 1], sb), T);
+        c0 = cprefix[lo];
+      }
+      w.t0 = sb + 64 * (w.ci - c0);
+      w.Lc = min(64, se - w.t0);
+      w.ok = w.Lc > 0;
+    } else {
+      w.ok = it < nchunks;
+      w.ci = it;
+      w.h = hb;
+      w.t0 = bos + 64 * it;
+      w.Lc = min(64, eos - w.t0);
+    }
+    return w;
+  };
 
   if (warp == 0) tmem_alloc(slot, TM_COLS);
   if (tid == 0) {
@@ -241,7 +288,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int dk0 = 32 * grp;
   float S[32];
   {
-    const float *src = s0 ? s0 + (((size_t)n * H + h) * 128 + j) * 128 + dk0 : nullptr;
+    const float *src = (s0 && !kPrepM) ? s0 + (((size_t)n * H + hb) * 128 + j) * 128 + dk0 : nullptr;
 #pragma unroll
     for (int x = 0; x < 32; x += 4) {
       float4 f = src ? *reinterpret_cast<const float4 *>(src + x) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -257,27 +304,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // The next chunk's tiles are requested as soon as each buffer is dead: q and k
   // after the Gram read-out, g after the inverse, v after the U read-out; one
   // mbarrier phase counts all four.
-  auto issue_tma_qk = [&](int t) {
+  auto issue_tma_qk = [&](const Work &w) {
     mbar_arrive_expect_tx(bar_tma, kTmaBytes);
     if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
-      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
-      tma_load_3d(sm + SM_K, &tm_q, bar_tma, 0, H + h, t);
+      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, w.h, w.t0);
+      tma_load_3d(sm + SM_K, &tm_q, bar_tma, 0, H + w.h, w.t0);
     } else {
-      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, h, t);
-      tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, h, t);
+      tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, w.h, w.t0);
+      tma_load_3d(sm + SM_K, &tm_k, bar_tma, 0, w.h, w.t0);
     }
   };
-  auto issue_tma_g = [&](int t) { tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, h, t); };
-  auto issue_tma_v = [&](int t) {
+  auto issue_tma_g = [&](const Work &w) { tma_load_3d(sm + SM_G, &tm_g, bar_tma, 0, w.h, w.t0); };
+  auto issue_tma_v = [&](const Work &w) {
     if constexpr (kFused)
-      tma_load_3d(sm + SM_V, &tm_q, bar_tma, 0, 2 * H + h, t);
+      tma_load_3d(sm + SM_V, &tm_q, bar_tma, 0, 2 * H + w.h, w.t0);
     else
-      tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, h, t);
+      tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, w.h, w.t0);
   };
-  auto issue_tma = [&](int t) {
-    issue_tma_qk(t);
-    issue_tma_g(t);
-    issue_tma_v(t);
+  auto issue_tma = [&](const Work &w) {
+    issue_tma_qk(w);
+    issue_tma_g(w);
+    issue_tma_v(w);
   };
   Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
   __nv_bfloat16 *corr = reinterpret_cast<__nv_bfloat16 *>(sm + SM_CORR);
@@ -286,7 +333,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if constexpr (kFused) {
     for (int idx = tid; idx < 3 * 128; idx += kThreads) {  // tap-major: lanes read consecutive channels
       const int p = idx >> 7, ch = idx & 127;
-      const float4 w = __ldg(reinterpret_cast<const float4 *>(conv_w + ((size_t)p * HD + h * 128 + ch) * 4));
+      const float4 w = __ldg(reinterpret_cast<const float4 *>(conv_w + ((size_t)p * HD + hb * 128 + ch) * 4));
       wconv[(p * 4 + 0) * 128 + ch] = w.x;
       wconv[(p * 4 + 1) * 128 + ch] = w.y;
       wconv[(p * 4 + 2) * 128 + ch] = w.z;
@@ -295,17 +342,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // conv history before the sequence: the cache rows (oldest first) or zero
     for (int idx = tid; idx < 9 * 128; idx += kThreads) {
       const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
-      hist[idx] = cache_in ? cache_in[((size_t)n * 3 + row) * 3 * HD + p * HD + h * 128 + ch]
+      hist[idx] = cache_in ? cache_in[((size_t)n * 3 + row) * 3 * HD + p * HD + hb * 128 + ch]
                            : from_f32<Tin>(0.f);
     }
     __syncthreads();
   }
-  if (tid == 0 && nchunks > 0) issue_tma(bos);
+  Work cur = work_of(0);
+  if (tid == 0 && cur.ok) issue_tma(cur);
 
   uint32_t tma_par = 0, mma_par = 0;
-  for (int c = 0; c < nchunks; ++c) {
-    const int t0 = bos + c * 64;
-    const int Lc = min(64, eos - t0);
+  int c = 0;
+  for (; cur.ok; ++c) {
+    const Work nxt = work_of(c + 1);
+    const int t0 = cur.t0, Lc = cur.Lc, h = cur.h;
 
     // ---- P0: raw tiles of this chunk ---------------------------------------------
     if (!wait_all(bar_tma, tma_par, status)) break;
@@ -450,6 +499,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       __syncthreads();
       if (tid < 128) fegc[d] = __expf(fegc[d]);  // every reader of gamma_63 is past the barrier
+    }
+    if constexpr (kPrepM) {
+      if (tid == 0) bulk_wait_read_all();  // the previous record's tiles have left shared memory
     }
     __syncthreads();
 
@@ -604,7 +656,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && c + 1 < nchunks) issue_tma_qk(t0 + 64);  // q, k tiles are dead
+    if (tid == 0 && nxt.ok) issue_tma_qk(nxt);  // q, k tiles are dead
 
     // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ------------------------------------
     // (i) the four diagonal 16x16 blocks by forward substitution, one column per
@@ -715,7 +767,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0 && c + 1 < nchunks) issue_tma_g(t0 + 64);  // A^T / T (the g tile) are dead
+    if (tid == 0 && nxt.ok) issue_tma_g(nxt);  // A^T / T (the g tile) are dead
 
     // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> fp16 operand ------------------------------
     if (tid == 0) {
@@ -731,7 +783,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_bf16(tmem + TM_U, desc_mnmajor(bv, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
       mma_commit(bar_mma);
     }
-    {
+    if constexpr (!kPrepM) {
       float amax = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -749,6 +801,54 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (!wait_all(bar_mma, mma_par, status)) break;
     mma_par ^= 1;
     tc_fence_after();
+
+    if constexpr (kPrepM) {
+      // ---- record: W (K-major, over the dead beta K G tile), Ut + fp32 remainder,
+      //      exp(gamma_63), <q_r, k_r>; then the tiles leave by bulk copies -------------
+      uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)cur.ci * H + h) * rec::BYTES;
+      {
+        float w[16];
+        tmem_ld16(tmem + lane_addr + TM_W + 16 * grp, w);  // W[16 grp + i][j]
+        __half *wt = reinterpret_cast<__half *>(sm + SM_BKG);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wt[(kmaj_off(64, 16 * grp + i, j >> 3) >> 1) + (j & 7)] = __float2half_rn(w[i]);
+      }
+      {
+        float u[16];
+        tmem_ld16(tmem + lane_addr + TM_U + 16 * grp, u);  // Ut[16 grp + i][j]
+        const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
+        float *ut = reinterpret_cast<float *>(rp + rec::UT);
+        float bvmax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = 16 * grp + i;
+          const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
+          const float bvv = beta_s[r] * vv;
+          bvmax = fmaxf(bvmax, fabsf(bvv));
+          ut[r * 128 + j] = u[i] + (bvv - __half2float(__float2half_rn(bvv)));
+        }
+        if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+      }
+      if (tid < 128) reinterpret_cast<float *>(rp + rec::GL)[tid] = fegc[tid];
+      if (tid < 64) reinterpret_cast<float *>(rp + rec::PD)[tid] = pdiag[tid];
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        if (nxt.ok) issue_tma_v(nxt);  // the v tile is dead
+        // A1 = [W ; Q G]: each k-atom holds the 64 W rows, then the 64 Q G rows
+        bulk_store(rp + rec::A1, sm + SM_BKG, 8192);
+        bulk_store(rp + rec::A1 + 8192, sm + SM_QG, 8192);
+        bulk_store(rp + rec::A1 + 16384, sm + SM_BKG + 8192, 8192);
+        bulk_store(rp + rec::A1 + 24576, sm + SM_QG + 8192, 8192);
+        bulk_store(rp + rec::KP, sm + SM_KP, 16384);
+        bulk_store(rp + rec::P, sm + SM_POP, 8192);
+        bulk_commit();
+      }
+      cur = nxt;
+      continue;
+    }
 
     // ---- P7: W^T read-out -> -W operand (MN-major, over beta K G) --------------------------
     {
@@ -823,7 +923,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && c + 1 < nchunks) issue_tma_v(t0 + 64);  // the v tile is dead
+    if (tid == 0 && nxt.ok) issue_tma_v(nxt);  // the v tile is dead
 
     // ---- P10: O^T += U^T P^T ; delta S^T = U^T K' ----------------------------------------
     if (tid == 0) {
@@ -860,6 +960,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
+    cur = nxt;
   }
 
   if constexpr (kFused) {
@@ -867,12 +968,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const Tin *hfin = hist + (nchunks & 1) * 1152;
       for (int idx = tid; idx < 9 * 128; idx += kThreads) {
         const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
-        cache_out[((size_t)n * 3 + row) * 3 * HD + p * HD + h * 128 + ch] = hfin[idx];
+        cache_out[((size_t)n * 3 + row) * 3 * HD + p * HD + hb * 128 + ch] = hfin[idx];
       }
     }
   }
-  if (sN) {
-    float *dst = sN + (((size_t)n * H + h) * 128 + j) * 128 + dk0;
+  if constexpr (kPrepM) {
+    if (tid == 0) bulk_wait_all();
+  }
+  if (sN && !kPrepM) {
+    float *dst = sN + (((size_t)n * H + hb) * 128 + j) * 128 + dk0;
 #pragma unroll
     for (int x = 0; x < 32; x += 4)
       *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
@@ -924,21 +1028,61 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
   const long long blocks = (long long)N * H;
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
   if (dt == KDA_BF16) {
-    auto kern = chunk_tc_kernel<__nv_bfloat16, false>;
+    auto kern = chunk_tc_kernel<__nv_bfloat16, kSingle>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
-                                                      sN, status, nullptr, nullptr, nullptr);
+                                                      sN, status, nullptr, nullptr, nullptr,
+                                                      nullptr, nullptr, N);
   } else {
-    auto kern = chunk_tc_kernel<__half, false>;
+    auto kern = chunk_tc_kernel<__half, kSingle>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
-                                                      sN, status, nullptr, nullptr, nullptr);
+                                                      sN, status, nullptr, nullptr, nullptr,
+                                                      nullptr, nullptr, N);
   }
   return cudaGetLastError();
+}
+
+namespace {
+template <typename Tin>
+cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                              const CUtensorMap &tg, const float *beta, const int32_t *cu, int N,
+                              int T, int H, uint8_t *ws, int *status, cudaStream_t s) {
+  auto kern = chunk_tc_kernel<Tin, kPrep>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SM_ALLOC);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  // Persistent: one CTA per SM (the kernel takes a whole SM's shared memory).
+  const long long items = rec::chunk_capacity(N, T) * H;
+  const unsigned grid = (unsigned)std::min<long long>(items, sms);
+  kern<<<grid, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, 1.f, nullptr, cu, T, H, nullptr,
+                                        nullptr, status, nullptr, nullptr, nullptr, ws,
+                                        reinterpret_cast<const int32_t *>(ws), N);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *cu, int N, int T, int H,
+                              kda_dtype dt, void *ws, int *status, cudaStream_t s) {
+  const CUtensorMapDataType act =
+      dt == KDA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tq, tk, tv, tg;
+  if (!make_map(&tq, q, act, 2, H, T) || !make_map(&tk, k, act, 2, H, T) ||
+      !make_map(&tv, v, act, 2, H, T) ||
+      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+    return cudaErrorInvalidValue;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  if (dt == KDA_BF16) return launch_prep_typed<__nv_bfloat16>(tq, tk, tv, tg, beta, cu, N, T, H, w, status, s);
+  return launch_prep_typed<__half>(tq, tk, tv, tg, beta, cu, N, T, H, w, status, s);
 }
 
 namespace {
@@ -954,13 +1098,13 @@ cudaError_t launch_fused_typed(const void *x, const float *conv_w, const void *c
     return cudaErrorInvalidValue;
   const long long blocks = (long long)N * H;
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
-  auto kern = chunk_tc_kernel<Tin, true>;
+  auto kern = chunk_tc_kernel<Tin, kFusedMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SM_ALLOC_FUSED);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)blocks, kThreads, SM_ALLOC_FUSED, s>>>(
       tx, tx, tx, tg, beta, scale, s0, cu, T, H, o, sN, status, conv_w,
-      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out));
+      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), nullptr, nullptr, N);
   return cudaGetLastError();
 }
 }  // namespace

@@ -192,6 +192,16 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             const float *beta, float scale, const float *s0, const int32_t *cu,
                             int N, int T, int H, kda_dtype dt, float *o, float *sN, int *status,
                             cudaStream_t s);
+// Two-pass tensor-core prefill (kda_chunk_record.cuh): the prep pass over all
+// (chunk, head) items, then the state pass over (sequence, head, value slice).
+cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *cu, int N, int T, int H,
+                              kda_dtype dt, void *ws, int *status, cudaStream_t s);
+cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *status,
+                               cudaStream_t s);
+cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
+                               int N, int T, int H, float *o, float *sN, int *status,
+                               cudaStream_t s);
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,
                                      void *cache_out, const float *g, const float *beta,
                                      float scale, const float *s0, const int32_t *cu, int N,

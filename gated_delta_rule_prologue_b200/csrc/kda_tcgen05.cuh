@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "kda_common.cuh"
+
 namespace kda {
 namespace tc {
 
@@ -87,6 +89,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   }
 }
 
+// All threads of the CTA wait for a barrier phase; false (and a recorded
+// timeout) if any thread gave up.  Also acts as a CTA-wide barrier.
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *status) {
+  const bool ok = mbar_wait(bar, parity);
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
+    return false;
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor tile loads; no multicast)
 // ---------------------------------------------------------------------------
@@ -102,6 +115,35 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Untiled bulk copies (addresses 16-byte aligned, sizes multiples of 16 bytes).
+// Global -> shared, completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Shared -> global, tracked by bulk groups of the issuing thread.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The issuing thread's bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// The issuing thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

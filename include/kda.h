@@ -39,6 +39,7 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -119,6 +120,39 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
                          const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
                          int chunk, kda_dtype dt, float *o, float *final_state,
                          kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_workspace_bytes -- bytes of scratch kda_chunk_fwd_ws needs for
+ * these sizes: one 88.75 KiB record per (chunk, head) plus a 1 KiB-aligned
+ * chunk index, sized for the worst case of N sequences in T tokens
+ * (ceil(T/64) + N chunks per head).  0 when the arguments do not select the
+ * tensor-core path (dt == KDA_F32, Dk or Dv != 128, chunk != 64, T == 0).
+ */
+size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt);
+
+/*
+ * kda_chunk_fwd_ws -- kda_chunk_fwd with a caller-owned scratch buffer, which
+ * lets the tensor-core path run as two passes.  [W4 Figure 1]: inside a chunk
+ * everything except the read of the entry state is independent of the
+ * carried state, so the first pass computes it for all (chunk, head) pairs
+ * at once (in-chunk log-decay, Gram products, the WY solve of [W5 §10.3]) and
+ * the second carries the state through the chunks of each sequence in order,
+ * one CTA per (sequence, head, 32 value channels).  Same arguments and
+ * results as kda_chunk_fwd (equal up to rounding order), plus:
+ *   workspace        device buffer of >= kda_chunk_fwd_workspace_bytes(...)
+ *                    bytes, 16-byte aligned, owned by the caller; its contents
+ *                    on entry do not matter and are unspecified on return.  It
+ *                    must not overlap any other argument, and calls that may
+ *                    run concurrently must not share one.  NULL: the call is
+ *                    exactly kda_chunk_fwd.
+ *   workspace_bytes  its size; KDA_ERR_INVALID_ARG if too small
+ */
+kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *initial_state,
+                            const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                            int chunk, kda_dtype dt, float *o, float *final_state,
+                            void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * kda_prologue_chunk_fwd -- the prologue fused into the chunkwise prefill: the

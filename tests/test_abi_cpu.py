@@ -22,13 +22,15 @@ def kda():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:kda_status|const char \*)\s*(kda_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:kda_status|const char \*|size_t)\s*(kda_\w+)\s*\(",
+                                 text, re.M)))
 
 
 def test_header_declares_the_hot_path_entry_points():
     names = declared_functions()
     for n in ("kda_prologue", "kda_chunk_fwd", "kda_decode_step", "kda_prologue_chunk_fwd",
-              "kda_get_device_status", "kda_last_error", "kda_version"):
+              "kda_chunk_fwd_ws", "kda_chunk_fwd_workspace_bytes", "kda_get_device_status",
+              "kda_last_error", "kda_version"):
         assert n in names
 
 
@@ -134,3 +136,40 @@ def test_fused_prefill_rejects_bad_arguments(kda):
                                   _vp(6 * ALIGNED), 1.0, None, None, 1, 8, 2, 128, 1, a, None,
                                   None)
     assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
+
+
+def test_chunk_workspace_size(kda):
+    """Two-pass scratch: a 1 KiB-aligned int32 chunk index of N + 1 entries,
+    then one record per (chunk, head) for ceil(T/64) + N chunks per head;
+    nothing for calls that do not take the tensor-core path."""
+    import torch
+    f = kda.kda_chunk_fwd_workspace_bytes
+    rec = f(1, 64, 1, 128, 128, 64, torch.bfloat16) - 1024
+    assert rec > 0 and rec % 32 == 0   # two records (ceil(64/64) + N = 2), 16-byte multiples
+    for N, T, H in ((1, 32768, 96), (16, 93891, 32), (300, 1000, 2)):
+        header = ((N + 1) * 4 + 1023) // 1024 * 1024
+        expect = header + ((T + 63) // 64 + N) * H * (rec // 2)
+        assert f(N, T, H, 128, 128, 64, torch.float16) == expect
+    assert f(1, 64, 1, 128, 128, 64, torch.float32) == 0
+    assert f(1, 64, 1, 64, 64, 64, torch.bfloat16) == 0
+    assert f(1, 64, 1, 128, 128, 32, torch.bfloat16) == 0
+    assert f(1, 0, 1, 128, 128, 64, torch.bfloat16) == 0
+
+
+def test_chunk_fwd_ws_rejects_bad_workspace(kda):
+    import torch
+    L = kda.lib
+    T, H = 128, 2
+    need = kda.kda_chunk_fwd_workspace_bytes(1, T, H, 128, 128, 64, torch.bfloat16)
+    q, k, v = _vp(0x10000), _vp(0x20000), _vp(0x30000)   # 64 KiB each
+    g, beta, o = _vp(0x40000), _vp(0x60000), _vp(0x70000)  # 128 KiB, 1 KiB, 128 KiB
+    ws = _vp(0x100000)
+    st = L.kda_chunk_fwd_ws(q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o,
+                            None, ws, need - 16, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace holds" in L.kda_last_error()
+    st = L.kda_chunk_fwd_ws(q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o,
+                            None, _vp(0x100008), need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"aligned" in L.kda_last_error()
+    st = L.kda_chunk_fwd_ws(q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o,
+                            None, _vp(0x78000), need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace overlaps" in L.kda_last_error()

@@ -57,7 +57,12 @@ def check_rounded(got, ref, dtype):
         assert rel_max(f64(got), ref) <= 1e-5
 
 
-def run_chunk(kda, inp, *, chunk=None, in_place=False):
+# kda_chunk_fwd's two ways through the tensor-core path: the two-pass kernels
+# with a scratch workspace (the default) and the one-pass kernel.
+PASSES = {"two_pass": "auto", "one_pass": None}
+
+
+def run_chunk(kda, inp, *, chunk=None, in_place=False, workspace="auto"):
     dev = "cuda"
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     g, beta = inp.g.to(dev), inp.beta.to(dev)
@@ -67,7 +72,7 @@ def run_chunk(kda, inp, *, chunk=None, in_place=False):
     fs = s0 if (in_place and s0 is not None) else torch.empty((N, H, D, D), device=dev)
     o = torch.empty(v.shape, dtype=torch.float32, device=dev)
     kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, initial_state=s0, final_state=fs,
-                      cu_seqlens=cu, chunk=chunk or inp.chunk)
+                      cu_seqlens=cu, chunk=chunk or inp.chunk, workspace=workspace)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     return f64(o), f64(fs)
@@ -90,9 +95,10 @@ def test_tiny_f32_parity(kda):
     assert rel_fro(S, S_ref) <= 1e-5
 
 
-def test_seq4k_bf16_parity(kda):
+@pytest.mark.parametrize("passes", list(PASSES))
+def test_seq4k_bf16_parity(kda, passes):
     inp = W.seq4k_bf16()
-    o, S = run_chunk(kda, inp)
+    o, S = run_chunk(kda, inp, workspace=PASSES[passes])
     o_ref, S_ref = oracle_chunk(inp)
     assert rel_max(o, o_ref) <= TOL_BF16
     assert rel_fro(S, S_ref) <= TOL_STATE
@@ -113,24 +119,28 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("passes", list(PASSES))
 @pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
-def test_chunk_edge_cases(kda, case):
+def test_chunk_edge_cases(kda, case, passes):
     name, D, chunk, bf16, lengths, g_shift, s0_std, g_fn = case
+    if passes == "one_pass" and not (bf16 and D == 128 and chunk == 64):
+        pytest.skip("only the tensor-core path has two variants")
     inp = W.random_prefill(100 + EDGE.index(case), sum(lengths), 3, D, bf16=bf16,
                            g_shift=g_shift, s0_std=s0_std, lengths=lengths, chunk=chunk,
                            g_fn=g_fn)
     inp.scale = 0.5
-    o, S = run_chunk(kda, inp)
+    o, S = run_chunk(kda, inp, workspace=PASSES[passes])
     o_ref, S_ref = oracle_chunk(inp)
     tol = TOL_BF16 if bf16 else TOL_F32
     assert rel_max(o, o_ref) <= tol
     assert rel_fro(S, S_ref) <= (TOL_STATE if bf16 else 1e-5)
 
 
-def test_chunk_final_state_in_place(kda):
+@pytest.mark.parametrize("passes", list(PASSES))
+def test_chunk_final_state_in_place(kda, passes):
     inp = W.random_prefill(5, 150, 2, 128, s0_std=0.1, lengths=[90, 60],
                            g_fn=lambda z: -5.0 * torch.sigmoid(z - 5.0))
-    o, S = run_chunk(kda, inp, in_place=True)
+    o, S = run_chunk(kda, inp, in_place=True, workspace=PASSES[passes])
     o_ref, S_ref = oracle_chunk(inp)
     assert rel_max(o, o_ref) <= TOL_BF16
     assert rel_fro(S, S_ref) <= TOL_STATE
@@ -146,14 +156,51 @@ def test_chunk_size_does_not_change_results(kda):
 
 
 def test_tensor_core_and_cuda_core_paths_agree(kda):
-    """bf16, d=128: chunk 64 runs the tcgen05 kernel, chunk 32 the fp32
-    CUDA-core kernel; both within the bf16 bound of each other."""
+    """bf16, d=128: chunk 64 runs the tcgen05 kernels (two-pass and one-pass),
+    chunk 32 the fp32 CUDA-core kernel; all within the bf16 bound of each
+    other, and the two tensor-core variants, which round the same operands,
+    much closer than that."""
     inp = W.random_prefill(9, 333, 2, 128, s0_std=0.1, lengths=[200, 133],
                            g_fn=lambda z: -5.0 * torch.sigmoid(z - 1.0))
     o_tc, S_tc = run_chunk(kda, inp, chunk=64)
+    o_1p, S_1p = run_chunk(kda, inp, chunk=64, workspace=None)
     o_cc, S_cc = run_chunk(kda, inp, chunk=32)
     assert rel_max(o_tc, o_cc) <= TOL_BF16
     assert rel_fro(S_tc, S_cc) <= TOL_STATE
+    assert rel_max(o_1p, o_cc) <= TOL_BF16
+    assert rel_max(o_tc, o_1p) <= 0.25 * TOL_BF16
+    assert rel_fro(S_tc, S_1p) <= 0.1 * TOL_STATE
+
+
+def test_two_pass_workspace_reuse_is_deterministic(kda):
+    """The same caller-owned workspace twice in a row, dirty from the first
+    call: bit-identical results."""
+    inp = W.random_prefill(12, 500, 4, 128, s0_std=0.05, lengths=[129, 0, 64, 307],
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 3.0))
+    N, T, H = inp.N, inp.T, inp.H
+    nbytes = kda.kda_chunk_fwd_workspace_bytes(N, T, H, 128, 128, 64, torch.bfloat16)
+    assert nbytes > 0
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device="cuda")
+    o1, S1 = run_chunk(kda, inp, workspace=ws)
+    o2, S2 = run_chunk(kda, inp, workspace=ws)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert rel_max(o1, o_ref) <= TOL_BF16
+    assert rel_fro(S1, S_ref) <= TOL_STATE
+
+
+def test_two_pass_malformed_cu_seqlens_sets_status_without_fault(kda):
+    inp = W.random_prefill(13, 256, 2, 128, lengths=[100, 156])
+    dev = "cuda"
+    bad = torch.tensor([0, 300, 20], dtype=torch.int32, device=dev)  # past T, then decreasing
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    o = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    kda.kda_chunk_fwd(q, k, v, inp.g.to(dev), inp.beta.to(dev), o, cu_seqlens=bad)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == kda.KDA_ERR_DEVICE_BOUNDS
+    o2, _ = run_chunk(kda, inp)
+    assert np.all(np.isfinite(o2))
 
 
 def test_malformed_cu_seqlens_sets_status_without_fault(kda):
