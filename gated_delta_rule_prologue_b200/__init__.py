@@ -74,13 +74,16 @@ lib.kda_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                               _i, _vp, _vp, _vp]
 lib.kda_chunk_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                  _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.kda_chunk_fwd_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i,
+                                     _i, _i, _vp, _vp, _vp]
 lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
-for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_decode_step,
+for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
+            lib.kda_decode_step,
             lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
@@ -195,6 +198,33 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
                                 _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
                                 _dtype(q), _ptr(o), _ptr(final_state), _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
+
+
+# Size of the library's fixed scratch buffer (one per device) used by
+# kda_chunk_fwd_static; equals KDA_CHUNK_STATIC_SCRATCH_BYTES in kda.h.
+KDA_CHUNK_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def kda_chunk_fwd_static(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None,
+                         final_state=None, cu_seqlens=None, chunk: int = 64, stream=None):
+    """The two-pass prefill with the library's fixed scratch buffer instead of
+    a workspace: allocates nothing.  Sizes needing more scratch than
+    KDA_CHUNK_STATIC_SCRATCH_BYTES raise KdaError (KDA_ERR_UNSUPPORTED).  All
+    calls on a device share the buffer, so calls that may overlap in time
+    (different streams) race; calls in order on one stream are safe."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.kda_chunk_fwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                    _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv,
+                                    chunk, _dtype(q), _ptr(o), _ptr(final_state),
+                                    _stream(stream)))
 
 
 def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: float = 1.0,

@@ -53,6 +53,29 @@ kda_status device_status_word(int **out) {
   return KDA_OK;
 }
 
+// Scratch of kda_chunk_fwd_static: a module global, one per device, never
+// allocated or freed by a call.  Its device address is looked up once per
+// device and cached.
+__device__ __align__(256) uint8_t g_static_scratch[KDA_CHUNK_STATIC_SCRATCH_BYTES];
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxDevices] = {nullptr};
+
+kda_status static_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return KDA_OK;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -285,6 +308,41 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
     e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
                                 final_state, status, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_ws launch");
+  return KDA_OK;
+}
+
+kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float scale, const float *initial_state,
+                                const int32_t *cu_seqlens, int N, int T, int H, int Dk,
+                                int Dv, int chunk, kda_dtype dt, float *o, float *final_state,
+                                kda_stream_t stream) {
+  kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                                   chunk, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, dt);
+  if (need == 0)
+    return kda_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                         chunk, dt, o, final_state, stream);
+  if (need > KDA_CHUNK_STATIC_SCRATCH_BYTES)
+    return fail(KDA_ERR_UNSUPPORTED,
+                "kda_chunk_fwd_static: N=%d T=%d H=%d needs %zu bytes of scratch, the static "
+                "buffer holds %zu (use kda_chunk_fwd_ws with a caller workspace)",
+                N, T, H, need, (size_t)KDA_CHUNK_STATIC_SCRATCH_BYTES);
+  void *scratch = nullptr;
+  st = static_scratch(&scratch);
+  if (st != KDA_OK) return st;
+  int *status = nullptr;
+  st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, scratch, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, scratch, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(scratch, cu_seqlens, initial_state, scale, N, T, H, o,
+                                final_state, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_static launch");
   return KDA_OK;
 }
 

@@ -155,6 +155,33 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
                             void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_static -- kda_chunk_fwd_ws without a caller workspace: the
+ * scratch is a fixed device buffer inside the library, and the call
+ * allocates and frees nothing.  The pages have no counterpart of this entry
+ * point; it is an engineering variant for callers that must not allocate, and
+ * it computes exactly what kda_chunk_fwd_ws computes (same kernels).
+ *   Buffer    one file-scope device array of KDA_CHUNK_STATIC_SCRATCH_BYTES
+ *             (64 MiB), 256-byte aligned, per device; its address is looked
+ *             up once per device (cudaGetSymbolAddress) on first use.
+ *   Sizes     if kda_chunk_fwd_workspace_bytes(...) exceeds the buffer the
+ *             call returns KDA_ERR_UNSUPPORTED before launching anything
+ *             (e.g. T=4096, H=8 needs 47.3 MB and fits; T=32768, H=96 needs
+ *             4.5 GB and does not); if it is 0 the call is kda_chunk_fwd.
+ *   Zeroing   nothing in the buffer has to start at zero: every byte a call
+ *             reads was written earlier in the same call.
+ *   Overlap   all calls on a device share the one buffer.  Calls that may run
+ *             at the same time (different streams, or host threads without
+ *             ordering between their streams) race on it and give undefined
+ *             results; calls issued in order on one stream are safe.
+ */
+#define KDA_CHUNK_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float scale, const float *initial_state,
+                                const int32_t *cu_seqlens, int N, int T, int H, int Dk,
+                                int Dv, int chunk, kda_dtype dt, float *o, float *final_state,
+                                kda_stream_t stream);
+
+/*
  * kda_prologue_chunk_fwd -- the prologue fused into the chunkwise prefill: the
  * same result as kda_prologue followed by kda_chunk_fwd (chunk 64), with q, k
  * and v never written to memory.  Each chunk's projections are convolved

@@ -173,3 +173,24 @@ def test_chunk_fwd_ws_rejects_bad_workspace(kda):
     st = L.kda_chunk_fwd_ws(q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o,
                             None, _vp(0x78000), need, None)
     assert st == kda.KDA_ERR_INVALID_ARG and b"workspace overlaps" in L.kda_last_error()
+
+
+def test_chunk_fwd_static_rejects_sizes_beyond_its_buffer(kda):
+    """Checked on the host before anything is launched (fake pointers are never
+    touched): T=32768, H=8 needs more than the fixed 64 MiB scratch."""
+    import torch
+    L = kda.lib
+    T, H = 32768, 8
+    assert kda.kda_chunk_fwd_workspace_bytes(1, T, H, 128, 128, 64, torch.bfloat16) > \
+        kda.KDA_CHUNK_STATIC_SCRATCH_BYTES
+    step = 0x10000000  # 256 MiB apart: no two fake arrays overlap
+    q, k, v, g, beta, o = (_vp(step * i) for i in range(1, 7))
+    st = L.kda_chunk_fwd_static(q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o,
+                                None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED and b"static buffer holds" in L.kda_last_error()
+
+
+def test_static_scratch_constant_matches_header(kda):
+    text = open(HEADER).read()
+    m = re.search(r"#define KDA_CHUNK_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == kda.KDA_CHUNK_STATIC_SCRATCH_BYTES
