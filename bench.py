@@ -4,8 +4,11 @@
 A *step* is one pass of the prefill hot path over the K3-layer-shaped
 workload: ``kda_prologue`` (short conv + SiLU + L2 over 32768 tokens x 96
 heads x 128 channels of q/k/v projections, fp16 q/k/v out) followed by
-``kda_chunk_fwd`` (tensor-core chunkwise prefill, chunk 64, fp32 state).  The
-fused variant ``kda_prologue_chunk_fwd`` is timed beside it.  ``value`` is prefill tokens/s
+``kda_chunk_fwd`` (tensor-core chunkwise prefill, chunk 64, fp32 state) with a
+preallocated workspace: its two-pass form, a parallel prep pass over every
+(chunk, head) and a state pass over (sequence, head, value slice).  The
+one-pass chunk kernel and the fused variant ``kda_prologue_chunk_fwd`` are
+timed beside it.  ``value`` is prefill tokens/s
 (a token is one position through all 96 heads) with inputs resident in HBM.
 The batched decode step (256 sequences x 96 heads, 100 consecutive steps,
 state updated in place) is timed in the same run and reported under
@@ -49,11 +52,13 @@ CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 # decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
 DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
 
+_CSRC = "gated_delta_rule_prologue_b200/csrc/"
 KERNEL_SOURCES = {
-    "kda_prologue_chunk_fwd": "gated_delta_rule_prologue_b200/csrc/kda_chunk_tc.cu",
-    "kda_prologue": "gated_delta_rule_prologue_b200/csrc/kda_prologue.cu",
-    "kda_chunk_fwd": "gated_delta_rule_prologue_b200/csrc/kda_chunk_tc.cu",
-    "kda_decode_step": "gated_delta_rule_prologue_b200/csrc/kda_decode.cu",
+    "kda_prologue_chunk_fwd": [_CSRC + "kda_chunk_tc.cu"],
+    "kda_prologue": [_CSRC + "kda_prologue.cu"],
+    "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
+    "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
+    "kda_decode_step": [_CSRC + "kda_decode.cu"],
 }
 
 
@@ -68,14 +73,18 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def src_sha(rel):
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_sha(rels):
+    """sha256 (first 16 hex digits) of the concatenated sources of one call."""
+    h = hashlib.sha256()
+    for rel in rels:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of the kernel (else None)."""
+    """DRAM bytes per call from the committed ncu summary (summed over the
+    call's launches), if it was taken on the current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -278,12 +287,14 @@ def run_ours(args, world, rank, local):
     fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
     q = torch.empty((T, H, D), dtype=torch.float16, device=dev)
     k, v = torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_bytes(1, T, H, D, D, inp.chunk, q.dtype),
+                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
         kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
-                          chunk=inp.chunk, stream=stream)
+                          chunk=inp.chunk, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -301,7 +312,7 @@ def run_ours(args, world, rank, local):
         kda.kda_prologue(x, w, q, k, v, H=H, D=D, stream=stream)
         ev[i][1].record(stream)
         kda.kda_chunk_fwd(q, k, v, g, beta, o, scale=inp.scale, final_state=fs,
-                          chunk=inp.chunk, stream=stream)
+                          chunk=inp.chunk, workspace=ws, stream=stream)
         ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -310,34 +321,44 @@ def run_ours(args, world, rank, local):
     pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     chk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     assert kda.kda_get_device_status() == 0
-    launches = 2 * args.steps
+    launches = 3 * args.steps  # prologue, chunk prep pass, chunk state pass
 
-    # the fused variant (prologue inside the chunk kernel), timed beside the step
+    # the fused variant (prologue inside the one-pass chunk kernel) and the
+    # one-pass chunk kernel, timed beside the step
     o2 = torch.empty_like(o)
-    side = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    side = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(3)]
     for i in range(3):
         side[i][0].record(stream)
         kda.kda_prologue_chunk_fwd(x, w, g, beta, o2, H=H, D=D, scale=inp.scale, stream=stream)
         side[i][1].record(stream)
+        side[i][2].record(stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o2, scale=inp.scale, chunk=inp.chunk,
+                          workspace=None, stream=stream)
+        side[i][3].record(stream)
     torch.cuda.synchronize(dev)
     fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in side[1:])
+    one_pass_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in side[1:])
     del o2
 
     th = T * H
+    step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
     kernels = {
         "kda_prologue_chunk_fwd": dict(ms=round(fused_ms, 4), **roofline(
             "hbm", FUSED_BYTES_PER_TH * th, fused_ms, hbm, "GB/s",
             recorded_traffic("kda_prologue_chunk_fwd"))),
         "kda_prologue": dict(ms=round(pro_ms, 4), **roofline(
             "hbm", PROLOGUE_BYTES_PER_TH * th, pro_ms, hbm, "GB/s", recorded_traffic("kda_prologue"))),
-        "kda_chunk_fwd": dict(ms=round(chk_ms, 4), **roofline(
+        "kda_chunk_fwd": dict(ms=round(chk_ms, 4), launches=2, **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, chk_ms, hbm, "GB/s", recorded_traffic("kda_chunk_fwd"))),
+        "kda_chunk_fwd_one_pass": dict(ms=round(one_pass_ms, 4), **roofline(
+            "hbm", CHUNK_BYTES_PER_TH * th, one_pass_ms, hbm, "GB/s",
+            recorded_traffic("kda_chunk_fwd_one_pass"))),
     }
     kernels["kda_chunk_fwd"]["tensor_tflops"] = round(
         CHUNK_FLOPS_PER_TH * th / (chk_ms * 1e-3) / 1e12, 2)
     dominant = "kda_chunk_fwd"
     roof = {k_: kernels[dominant][k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
-    roof["kernel"] = dominant
+    roof["kernel"] = dominant + " (one call: prep pass + state pass)"
     roof["peak_source"] = f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
     fused_floor_ms = 1e3 * FUSED_BYTES_PER_TH * th / (hbm * 1e9)
 
@@ -358,7 +379,7 @@ def run_ours(args, world, rank, local):
     e2e_value, e2e_ms = job_throughput(world, T, e0.elapsed_time(e1) / e2e_steps)
     h2d = inp.x.numel() * 2 + inp.g.numel() * 4 + inp.beta.numel() * 4
     d2h = out_host.numel() * 4
-    del x, o, g, beta, inp
+    del x, o, g, beta, inp, ws
     torch.cuda.empty_cache()
 
     # ---- batched decode: 256 sequences x 96 heads, consecutive steps ----
@@ -410,12 +431,12 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": "k3_prefill: kda_prologue (fp16 q/k/v out) + kda_chunk_fwd over "
-                        "T=32768 tokens, H=96, d_k=d_v=128, chunk 64, bf16 q/k/v projections, "
-                        "fp32 g/beta/state/o",
+            "workload": "k3_prefill: kda_prologue (fp16 q/k/v out) + kda_chunk_fwd (two-pass, "
+                        "preallocated workspace) over T=32768 tokens, H=96, d_k=d_v=128, "
+                        "chunk 64, bf16 q/k/v projections, fp32 g/beta/state/o",
             "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
             "parallelism": f"replicas x{world} (independent problems, no collective)",
-            "l2": "inputs larger than L2 (10.5 GB touched per step, no flush needed)",
+            "l2": f"inputs larger than L2 ({step_gb:.1f} GB touched per step, no flush needed)",
         },
         "roofline": roof,
         "kernels": kernels,
@@ -462,6 +483,9 @@ def run_ncu_case(args):
                 kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D)
             elif args.ncu_case == "prologue":
                 kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+            elif args.ncu_case == "chunk_one_pass":
+                kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+                kda.kda_chunk_fwd(q, k, v, g, beta, o, workspace=None)
             else:
                 kda.kda_prologue(x, w, q, k, v, H=H, D=D)
                 kda.kda_chunk_fwd(q, k, v, g, beta, o)
@@ -479,7 +503,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "decode"),
+    ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode"),
                     help="profiling mode: launch one kernel twice on a workload slice and exit")
     ap.add_argument("--ncu-tokens", type=int, default=4096)
     args = ap.parse_args()
