@@ -124,24 +124,32 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     load_kp(0);
   }
 
-  uint32_t pa = 0, pk = 0, pm = 0;
-  for (int c = 0; c < nch; ++c) {
-    const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
-    const uint8_t *rp = rec_of(c);
-    // record values read by threads, fetched before the MMA waits
-    float ut[32];
-    float pd = 0.f;
-    if (warp < 2) {  // token tid: its Ut slice and <q, k>
+  // Record values read by threads (Ut slice and <q_r, k_r> of token tid for
+  // warps 0-1, exp(gamma_last) of key t for all) are fetched one chunk ahead.
+  float ut[32];
+  float pd = 0.f, gl = 0.f;
+  auto fetch_u = [&](int c) {
+    if (warp < 2) {
+      const uint8_t *rp = rec_of(c);
       const float4 *src =
           reinterpret_cast<const float4 *>(rp + rec::UT + ((size_t)tid * 128 + slice * 32) * 4);
 #pragma unroll
       for (int x = 0; x < 8; ++x) {
-        const float4 f = src[x];
+        const float4 f = __ldcs(src + x);
         ut[4 * x] = f.x; ut[4 * x + 1] = f.y; ut[4 * x + 2] = f.z; ut[4 * x + 3] = f.w;
       }
-      pd = reinterpret_cast<const float *>(rp + rec::PD)[tid];
+      pd = __ldcs(reinterpret_cast<const float *>(rp + rec::PD) + tid);
     }
-    const float gl = reinterpret_cast<const float *>(rp + rec::GL)[t];
+  };
+  auto fetch_gl = [&](int c) { gl = __ldg(reinterpret_cast<const float *>(rec_of(c) + rec::GL) + t); };
+  if (nch > 0) {
+    fetch_u(0);
+    fetch_gl(0);
+  }
+
+  uint32_t pa = 0, pk = 0, pm = 0;
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
 
     // ---- D1 = [W ; Q G] S ----------------------------------------------------------
     if (!wait_all(bar_a1, pa, status)) break;
@@ -174,6 +182,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
         exch[i * 64 + r] = pd * u;  // the S operand is dead until the next chunk
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+      if (c + 1 < nch) fetch_u(c + 1);
     }
     fence_async_smem();
     tc_fence_before();
@@ -186,13 +195,12 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       const uint32_t a2 = smem_u32(sm + SB_A2), uop = smem_u32(sm + SB_U);
       const uint32_t kp = smem_u32(sm + SB_KP);
       constexpr uint32_t idO = idesc_fp16(128, 32, false, false);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_kmajor(uop, 32, ks), idO, 1);
       constexpr uint32_t idS = idesc_fp16(128, 32, true, false);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
+      for (int ks = 0; ks < 4; ++ks) {  // the two accumulators' steps interleaved
+        mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_kmajor(uop, 32, ks), idO, 1);
         mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_kmajor(uop, 32, ks), idS, ks > 0);
+      }
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, pm, status)) break;
@@ -206,6 +214,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       tmem_ld32(tmem + lane_addr + TB_D2, ds);
 #pragma unroll
       for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], gl, ds[i]);
+      if (c + 1 < nch) fetch_gl(c + 1);
     }
     if (warp >= 2) {
       float ov[32];

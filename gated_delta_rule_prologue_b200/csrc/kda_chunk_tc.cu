@@ -98,12 +98,16 @@ constexpr uint32_t SM_HIST = SM_CORR + 16384;
 constexpr uint32_t SM_WCONV = SM_HIST + 2 * 3 * 3 * 128 * 2;  // conv weights of head h [3][4 taps][128] f32
 constexpr uint32_t SM_TOTAL_FUSED = SM_WCONV + 3 * 128 * 4 * 4;
 constexpr uint32_t SM_ALLOC = SM_TOTAL + 1024;  // slack for 1024-byte alignment
+constexpr uint32_t SM_ALLOC_PREP = SM_CORR + 16384 + 1024;  // plus the remainder tile
 constexpr uint32_t SM_ALLOC_FUSED = SM_TOTAL_FUSED + 1024;
 static_assert(SM_ALLOC_FUSED <= 232448, "shared memory budget");
+static_assert(SM_ALLOC_PREP <= SM_ALLOC_FUSED, "the prep plan is a prefix of the fused one");
 static_assert(SM_GBL + 24576 <= SM_ST + 32768, "Gram tiles stay inside X, TOP, POP and ST");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
-constexpr uint32_t TM_G = 0;     // Gram, 96 columns
+constexpr uint32_t TM_G = 0;     // Gram, 96 columns (first of two partial sums)
+constexpr uint32_t TM_G2 = 288;  // second partial sum of the Gram, 96 columns; it lives
+                                 // over O and delta S, which are written only later
 constexpr uint32_t TM_W = 160;   // W^T, 64
 constexpr uint32_t TM_U = 224;   // U^T, 64
 constexpr uint32_t TM_O = 288;   // O^T, 64
@@ -304,8 +308,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // The next chunk's tiles are requested as soon as each buffer is dead: q and k
   // after the Gram read-out, g after the inverse, v after the U read-out; one
   // mbarrier phase counts all four.
+  // One mbarrier phase counts the four tiles of a work item; it is armed with
+  // their total at the item's first issue (the tiles go out as buffers die).
+  auto arm_tma = [&]() { mbar_arrive_expect_tx(bar_tma, kTmaBytes); };
   auto issue_tma_qk = [&](const Work &w) {
-    mbar_arrive_expect_tx(bar_tma, kTmaBytes);
     if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
       tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, w.h, w.t0);
       tma_load_3d(sm + SM_K, &tm_q, bar_tma, 0, H + w.h, w.t0);
@@ -322,6 +328,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, w.h, w.t0);
   };
   auto issue_tma = [&](const Work &w) {
+    arm_tma();
     issue_tma_qk(w);
     issue_tma_g(w);
     issue_tma_v(w);
@@ -349,6 +356,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   Work cur = work_of(0);
   if (tid == 0 && cur.ok) issue_tma(cur);
+  // beta of the current work item's tokens, fetched one item ahead
+  float beta_next = (cur.ok && tid < cur.Lc) ? __ldg(beta + (size_t)(cur.t0 + tid) * H + cur.h) : 0.f;
 
   uint32_t tma_par = 0, mma_par = 0;
   int c = 0;
@@ -361,7 +370,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tma_par ^= 1;
 
     // ---- P1: beta, in-chunk cumulative log-decay, per-channel factors, E ------------
-    if (tid < 64) beta_s[tid] = tid < Lc ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    if (tid < 64) {
+      beta_s[tid] = beta_next;
+      beta_next = (nxt.ok && tid < nxt.Lc) ? __ldg(beta + (size_t)(nxt.t0 + tid) * H + nxt.h) : 0.f;
+    }
     if constexpr (kFused) {
       // ---- Pc: prologue in place on the x tiles (fp32 arithmetic) ----------------------
       // thread: 8 channels (c8) of two consecutive rows r0, r0+1 of all three parts;
@@ -551,15 +563,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
       const uint32_t gal = smem_u32(sm + SM_GAL), gbl = smem_u32(sm + SM_GBL);
       constexpr uint32_t id = idesc_bf16(128, 96, false, false);
+      // two independent accumulation chains of 12 steps each, interleaved:
+      // G = hi.hi + (lo.hi over k < 64),  G2 = hi.lo + (lo.hi over k >= 64)
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 8; ++ks) {
         mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
+        mma_bf16(tmem + TM_G2, desc_kmajor(ga, 128, ks), desc_kmajor(gbl, 96, ks), id, ks > 0);
+      }
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gbl, 96, ks), id, 1);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 4; ++ks) {
         mma_bf16(tmem + TM_G, desc_kmajor(gal, 128, ks), desc_kmajor(gb, 96, ks), id, 1);
+        mma_bf16(tmem + TM_G2, desc_kmajor(gal, 128, ks + 4), desc_kmajor(gb, 96, ks + 4), id, 1);
+      }
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, mma_par, status)) break;
@@ -595,12 +610,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
       st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
       st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
+      if constexpr (kPrepM) {  // fp32 remainder beta v - f16(beta v), kept as bf16
+        float cr[8], bvmax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cr[e] = bv[e] - __half2float(__float2half_rn(bv[e]));
+          bvmax = fmaxf(bvmax, fabsf(bv[e]));
+        }
+        st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
+        if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+      }
     }
     __syncthreads();
+    if constexpr (kPrepM) {
+      if (tid == 0 && nxt.ok) {  // the v and g (E) tiles are dead: the next item's tiles start
+        arm_tma();
+        issue_tma_v(nxt);
+        issue_tma_g(nxt);
+      }
+    }
 
     // ---- P4b: <q_r, k_r> in fp32; Gram read-out -> A^T (fp32), strict P operand ---------
-    float *AT = Gf;           // AT[i*64 + r] = A[r][i]
-    float *TT = Gf + 4096;    // TT[r*64 + c] = T[r][c]
+    // AT[i*64 + r] = A[r][i], TT[r*64 + c] = T[r][c]: over the g tile, or (prep,
+    // which has no S^T operand) over the S^T tile so the next g tile can load now
+    float *AT = kPrepM ? reinterpret_cast<float *>(sm + SM_ST) : Gf;
+    float *TT = AT + 4096;
     for (int idx = tid; idx < 4096 / 4; idx += kThreads)
       reinterpret_cast<float4 *>(AT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     reinterpret_cast<uint4 *>(sm + SM_POP)[tid] = make_uint4(0u, 0u, 0u, 0u);  // 8 KB
@@ -630,13 +664,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float v[16];
       int i0s;
       if (quad & 1) {
-        tmem_ld16(tmem + lane_addr + TM_G + 32 + 16 * grp, v);
+        float w[16];
+        tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * grp, v);
+        tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * grp, w);
+        tmem_wait_ld(v, w);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] += w[e];
         i0s = 16 * grp;
       } else {
-        float v8[8];
-        tmem_ld8(tmem + lane_addr + TM_G + 8 * grp, v8);
+        float v8[8], w8[8];
+        tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * grp, v8);
+        tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * grp, w8);
+        tmem_wait_ld(v8, w8);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = v8[e];
+        for (int e = 0; e < 8; ++e) v[e] = v8[e] + w8[e];
         i0s = 8 * grp;
       }
       const int nch = (quad & 1) ? 2 : 1;
@@ -656,7 +697,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && nxt.ok) issue_tma_qk(nxt);  // q, k tiles are dead
+    if (tid == 0 && nxt.ok) {  // q, k tiles are dead
+      if constexpr (!kPrepM) arm_tma();
+      issue_tma_qk(nxt);
+    }
 
     // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ------------------------------------
     // (i) the four diagonal 16x16 blocks by forward substitution, one column per
@@ -767,7 +811,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0 && nxt.ok) issue_tma_g(nxt);  // A^T / T (the g tile) are dead
+    if constexpr (!kPrepM) {
+      if (tid == 0 && nxt.ok) issue_tma_g(nxt);  // A^T / T (the g tile) are dead
+    }
 
     // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> fp16 operand ------------------------------
     if (tid == 0) {
@@ -776,11 +822,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t bv = smem_u32(sm + SM_BV);
       constexpr uint32_t id = idesc_fp16(128, 64, true, false);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
+      for (int ks = 0; ks < 4; ++ks) {  // two independent chains, interleaved
         mma_bf16(tmem + TM_W, desc_mnmajor(bkg, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
         mma_bf16(tmem + TM_U, desc_mnmajor(bv, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
+      }
       mma_commit(bar_mma);
     }
     if constexpr (!kPrepM) {
@@ -817,18 +862,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       {
         float u[16];
         tmem_ld16(tmem + lane_addr + TM_U + 16 * grp, u);  // Ut[16 grp + i][j]
-        const Tact *Vr = reinterpret_cast<const Tact *>(sm + SM_V);
         float *ut = reinterpret_cast<float *>(rp + rec::UT);
-        float bvmax = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int r = 16 * grp + i;
-          const float vv = r < Lc ? to_f32(Vr[r * 128 + j]) : 0.f;
-          const float bvv = beta_s[r] * vv;
-          bvmax = fmaxf(bvmax, fabsf(bvv));
-          ut[r * 128 + j] = u[i] + (bvv - __half2float(__float2half_rn(bvv)));
+          ut[r * 128 + j] = u[i] + __bfloat162float(corr[r * 128 + j]);
         }
-        if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
       }
       if (tid < 128) reinterpret_cast<float *>(rp + rec::GL)[tid] = fegc[tid];
       if (tid < 64) reinterpret_cast<float *>(rp + rec::PD)[tid] = pdiag[tid];
@@ -836,7 +875,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       __syncthreads();
       if (tid == 0) {
-        if (nxt.ok) issue_tma_v(nxt);  // the v tile is dead
         // A1 = [W ; Q G]: each k-atom holds the 64 W rows, then the 64 Q G rows
         bulk_store(rp + rec::A1, sm + SM_BKG, 8192);
         bulk_store(rp + rec::A1 + 8192, sm + SM_QG, 8192);
@@ -1054,7 +1092,7 @@ cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, cons
                               int T, int H, uint8_t *ws, int *status, cudaStream_t s) {
   auto kern = chunk_tc_kernel<Tin, kPrep>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SM_ALLOC);
+                                       (int)SM_ALLOC_PREP);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -1063,7 +1101,7 @@ cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, cons
   // Persistent: one CTA per SM (the kernel takes a whole SM's shared memory).
   const long long items = rec::chunk_capacity(N, T) * H;
   const unsigned grid = (unsigned)std::min<long long>(items, sms);
-  kern<<<grid, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, 1.f, nullptr, cu, T, H, nullptr,
+  kern<<<grid, kThreads, SM_ALLOC_PREP, s>>>(tq, tk, tv, tg, beta, 1.f, nullptr, cu, T, H, nullptr,
                                         nullptr, status, nullptr, nullptr, nullptr, ws,
                                         reinterpret_cast<const int32_t *>(ws), N);
   return cudaGetLastError();

@@ -172,6 +172,21 @@ def test_tensor_core_and_cuda_core_paths_agree(kda):
     assert rel_fro(S_tc, S_1p) <= 0.1 * TOL_STATE
 
 
+def test_two_pass_many_ragged_sequences(kda):
+    """20 sequences x 4 heads through the two-pass path: empty sequences,
+    shorter than a chunk, exact multiples of 64, several chunks; the chunk
+    index, the record walk and the per-sequence state hand-off."""
+    lengths = [0, 1, 63, 64, 65, 128, 200, 7, 300, 129, 64, 0, 31, 190, 256, 2, 77, 140, 95, 33]
+    inp = W.random_prefill(14, sum(lengths), 4, 128, s0_std=0.1, lengths=lengths,
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 4.0))
+    o, S = run_chunk(kda, inp)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert rel_max(o, o_ref) <= TOL_BF16
+    assert rel_fro(S, S_ref) <= TOL_STATE
+    o1, S1 = run_chunk(kda, inp, workspace=None)
+    assert rel_max(o, o1) <= 0.25 * TOL_BF16
+
+
 def test_two_pass_workspace_reuse_is_deterministic(kda):
     """The same caller-owned workspace twice in a row, dirty from the first
     call: bit-identical results."""
