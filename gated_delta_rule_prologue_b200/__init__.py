@@ -76,6 +76,8 @@ lib.kda_chunk_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, 
                                  _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.kda_chunk_fwd_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i,
                                      _i, _i, _vp, _vp, _vp]
+lib.kda_prologue_chunk_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i,
+                                          _i, _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
@@ -83,7 +85,7 @@ lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _v
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
-            lib.kda_decode_step,
+            lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step,
             lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
@@ -229,9 +231,13 @@ def kda_chunk_fwd_static(q, k, v, g, beta, o, *, scale: float = 1.0, initial_sta
 
 def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: float = 1.0,
                            cache_in=None, cache_out=None, initial_state=None, final_state=None,
-                           cu_seqlens=None, stream=None):
+                           cu_seqlens=None, workspace="auto", stream=None):
     """Prologue fused into the chunkwise prefill (chunk 64): ``x`` [T, 3*H*D]
-    bf16/fp16 projections in, ``o`` [T, H, D] float32 out; q, k, v stay on chip."""
+    bf16/fp16 projections in, ``o`` [T, H, D] float32 out; q, k, v stay on chip.
+
+    ``workspace`` as in :func:`kda_chunk_fwd`: ``"auto"`` (two passes, scratch
+    from torch's caching allocator), a uint8 CUDA tensor, or ``None`` (the
+    one-pass kernel)."""
     for t, n in ((x, "x"), (cache_in, "cache_in"), (cache_out, "cache_out")):
         _need(t, n, x.dtype)
     for t, n in ((conv_w, "conv_w"), (o, "o"), (g, "g"), (beta, "beta"),
@@ -240,10 +246,23 @@ def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: floa
     _need(cu_seqlens, "cu_seqlens", torch.int32)
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     T = x.shape[0]
-    _check(lib.kda_prologue_chunk_fwd(_ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out),
-                                      _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
-                                      _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
-                                      _ptr(final_state), _stream(stream)))
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto', None or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, x.dtype)
+        workspace = (torch.empty(nbytes, dtype=torch.uint8, device=x.device) if nbytes else None)
+    if workspace is None:
+        _check(lib.kda_prologue_chunk_fwd(_ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out),
+                                          _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                                          _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
+                                          _ptr(final_state), _stream(stream)))
+        return
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_prologue_chunk_fwd_ws(_ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out),
+                                         _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                                         _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
+                                         _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)))
 
 
 def kda_decode_step(x, conv_w, conv_cache, g, beta, state, o, *, H: int, D: int,

@@ -346,12 +346,14 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
   return KDA_OK;
 }
 
-kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void *cache_in,
-                                  void *cache_out, const float *g, const float *beta,
-                                  float scale, const float *initial_state,
-                                  const int32_t *cu_seqlens, int N, int T, int H, int D,
-                                  kda_dtype dt, float *o, float *final_state,
-                                  kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+kda_status check_fused_args(const void *x, const float *conv_w, const void *cache_in,
+                            void *cache_out, const float *g, const float *beta,
+                            const float *initial_state, const int32_t *cu_seqlens, int N, int T,
+                            int H, int D, kda_dtype dt, float *o, float *final_state) {
   KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
   KDA_REQUIRE(N >= 1 && T >= 1 && H >= 1 && D >= 1, "bad sizes N=%d T=%d H=%d D=%d", N, T, H, D);
   KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
@@ -381,13 +383,78 @@ kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void
   KDA_REQUIRE(final_state == initial_state ||
                   !overlaps(final_state, sbytes, initial_state, sbytes),
               "final_state partially overlaps initial_state");
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void *cache_in,
+                                  void *cache_out, const float *g, const float *beta,
+                                  float scale, const float *initial_state,
+                                  const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                  kda_dtype dt, float *o, float *final_state,
+                                  kda_stream_t stream) {
+  kda_status st = check_fused_args(x, conv_w, cache_in, cache_out, g, beta, initial_state,
+                                   cu_seqlens, N, T, H, D, dt, o, final_state);
+  if (st != KDA_OK) return st;
   int *status = nullptr;
-  kda_status st = device_status_word(&status);
+  st = device_status_word(&status);
   if (st != KDA_OK) return st;
   cudaError_t e = kda::launch_prologue_chunk_tc(x, conv_w, cache_in, cache_out, g, beta, scale,
                                                 initial_state, cu_seqlens, N, T, H, dt, o,
                                                 final_state, status, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kda_prologue_chunk_fwd launch");
+  return KDA_OK;
+}
+
+kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const void *cache_in,
+                                     void *cache_out, const float *g, const float *beta,
+                                     float scale, const float *initial_state,
+                                     const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                     kda_dtype dt, float *o, float *final_state,
+                                     void *workspace, size_t workspace_bytes,
+                                     kda_stream_t stream) {
+  if (workspace == nullptr)
+    return kda_prologue_chunk_fwd(x, conv_w, cache_in, cache_out, g, beta, scale, initial_state,
+                                  cu_seqlens, N, T, H, D, dt, o, final_state, stream);
+  kda_status st = check_fused_args(x, conv_w, cache_in, cache_out, g, beta, initial_state,
+                                   cu_seqlens, N, T, H, D, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt);
+  KDA_OPT_PTR(workspace, "workspace");
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {
+    const size_t C = (size_t)3 * H * D, es = esize(dt);
+    const size_t sbytes = (size_t)N * H * D * D * sizeof(float);
+    const void *others[9] = {x, conv_w, cache_in, cache_out, g, beta, o, initial_state,
+                             final_state};
+    const size_t osz[9] = {(size_t)T * C * es, C * 4 * 4, (size_t)N * 3 * C * es,
+                           (size_t)N * 3 * C * es, (size_t)T * H * D * 4, (size_t)T * H * 4,
+                           (size_t)T * H * D * 4, sbytes, sbytes};
+    for (int i = 0; i < 9; ++i)
+      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
+                  "workspace overlaps another argument");
+    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
+                "workspace overlaps cu_seqlens");
+  }
+  int *status = nullptr;
+  st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N, T,
+                                        H, dt, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+                                final_state, status, s);
+  if (e == cudaSuccess && cu_seqlens && cache_out)
+    e = kda::launch_cache_pass(workspace, N, H, cache_in, cache_out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_prologue_chunk_fwd_ws launch");
   return KDA_OK;
 }
 

@@ -299,7 +299,29 @@ chunk_index_kernel(const int32_t *__restrict__ cu, int N, int T, int32_t *cprefi
   if (tid == 0) cprefix[N] = carry;
 }
 
+// Fused two-pass prefill: a sequence without chunks (empty, or every sequence
+// when the index pass rejected cu_seqlens) has no prep item to write its conv
+// cache, so it is passed through here: cache_out[n] = cache_in[n], or zero.
+// Elements are 16-bit (bf16 or fp16; +0.0 is all-zero bits in both).
+__global__ void __launch_bounds__(256)
+cache_pass_kernel(const int32_t *__restrict__ cprefix, const uint16_t *__restrict__ cache_in,
+                  uint16_t *__restrict__ cache_out, long long per_seq) {
+  const int n = blockIdx.x;
+  if (cprefix[n + 1] != cprefix[n]) return;
+  const size_t base = (size_t)n * per_seq;
+  for (long long i = threadIdx.x; i < per_seq; i += blockDim.x)
+    cache_out[base + i] = cache_in ? cache_in[base + i] : (uint16_t)0;
+}
+
 }  // namespace
+
+cudaError_t launch_cache_pass(const void *ws, int N, int H, const void *cache_in,
+                              void *cache_out, cudaStream_t s) {
+  cache_pass_kernel<<<N, 256, 0, s>>>(static_cast<const int32_t *>(ws),
+                                      static_cast<const uint16_t *>(cache_in),
+                                      static_cast<uint16_t *>(cache_out), 3LL * 3 * H * 128);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *status,
                                cudaStream_t s) {

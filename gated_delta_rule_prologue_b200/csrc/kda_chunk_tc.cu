@@ -115,6 +115,7 @@ constexpr uint32_t TM_S = 352;   // delta S^T, 128
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t kTmaBytes = 3 * 16384 + 32768;
+constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
 
 // Eight 16-bit values packed in a uint4, widened to floats.
@@ -187,11 +188,15 @@ __device__ __forceinline__ uint4 pack8_in(const float (&f)[8]) {
 //            (chunk, head) items blockIdx.x, blockIdx.x + gridDim.x, ... and
 //            write one record per item (kda_chunk_record.cuh); the state pass
 //            (kda_chunk_state.cu) applies the records in order.
+//   kPrepFused: kPrep on raw projections with the prologue of kFused; each
+//            item brings its own conv history (the three rows before the
+//            chunk, or the cache at a sequence start), and the item holding a
+//            sequence's last chunk writes that sequence's cache.
 //
 // Thread layout (512 threads, 16 warps): warp w reads TMEM lanes
 // 32*(w%4).. (its "quad") and handles column group w/4 of every accumulator it
 // reads; element-wise phases walk (row, 8-channel chunk) pairs.
-constexpr int kSingle = 0, kFusedMode = 1, kPrep = 2;
+constexpr int kSingle = 0, kFusedMode = 1, kPrep = 2, kPrepFused = 3;
 
 template <typename Tin, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -201,8 +206,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
                 int *status, const float *__restrict__ conv_w, const Tin *cache_in,
                 Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N) {
-  constexpr bool kFused = kMode == kFusedMode;
-  constexpr bool kPrepM = kMode == kPrep;
+  constexpr bool kFused = kMode == kFusedMode || kMode == kPrepFused;
+  constexpr bool kPrepM = kMode == kPrep || kMode == kPrepFused;
   // Element type of the q/k/v tiles the chunk phases read: the inputs as given,
   // or fp16 written by the fused prologue (q, k are unit vectors; v is guarded).
   using Tact = typename std::conditional<kFused, __half, Tin>::type;
@@ -231,6 +236,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // The work walk: (t0, Lc, head, chunk number) of step `it`.
   struct Work {
     int t0, Lc, h, ci;
+    int n, bos, eos;  // the chunk's sequence
     bool ok;
   };
   int bos = 0, eos = 0, nchunks = 0;
@@ -252,9 +258,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!w.ok) return w;
       w.ci = (int)(item / H);
       w.h = (int)(item % H);
-      int sb = 0, se = T, c0 = 0;
+      int sb = 0, se = T, c0 = 0, lo = 0;
       if (cu) {  // sequence of chunk ci: the last n with cprefix[n] <= ci
-        int lo = 0, hi = N - 1;
+        int hi = N - 1;
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
           if (cprefix[mid] <= w.ci) lo = mid; else hi = mid - 1;
@@ -265,6 +271,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       w.t0 = sb + 64 * (w.ci - c0);
       w.Lc = min(64, se - w.t0);
+      w.n = lo;
+      w.bos = sb;
+      w.eos = se;
       w.ok = w.Lc > 0;
     } else {
       w.ok = it < nchunks;
@@ -272,6 +281,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       w.h = hb;
       w.t0 = bos + 64 * it;
       w.Lc = min(64, eos - w.t0);
+      w.n = n;
+      w.bos = bos;
+      w.eos = eos;
     }
     return w;
   };
@@ -310,7 +322,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // mbarrier phase counts all four.
   // One mbarrier phase counts the four tiles of a work item; it is armed with
   // their total at the item's first issue (the tiles go out as buffers die).
-  auto arm_tma = [&]() { mbar_arrive_expect_tx(bar_tma, kTmaBytes); };
+  // kPrepFused: a chunk that does not start its sequence also brings the three
+  // raw rows before it (its conv history) into history slot 0.
+  auto has_halo = [&](const Work &w) { return kMode == kPrepFused && w.t0 > w.bos; };
+  auto arm_tma = [&](const Work &w) {
+    mbar_arrive_expect_tx(bar_tma, kTmaBytes + (has_halo(w) ? kHaloBytes : 0u));
+  };
   auto issue_tma_qk = [&](const Work &w) {
     if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
       tma_load_3d(sm + SM_Q, &tm_q, bar_tma, 0, w.h, w.t0);
@@ -327,17 +344,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     else
       tma_load_3d(sm + SM_V, &tm_v, bar_tma, 0, w.h, w.t0);
   };
+  Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
+  auto issue_tma_halo = [&](const Work &w) {  // tm_k maps x with a 3-row box
+    if (has_halo(w))
+      for (int p = 0; p < 3; ++p)
+        tma_load_3d(hist + p * 384, &tm_k, bar_tma, 0, p * H + w.h, w.t0 - 3);
+  };
   auto issue_tma = [&](const Work &w) {
-    arm_tma();
+    arm_tma(w);
     issue_tma_qk(w);
     issue_tma_g(w);
     issue_tma_v(w);
+    issue_tma_halo(w);
   };
-  Tin *hist = reinterpret_cast<Tin *>(sm + SM_HIST);  // [2][3 parts][3 rows][128]
   __nv_bfloat16 *corr = reinterpret_cast<__nv_bfloat16 *>(sm + SM_CORR);
   const int HD = H * 128;
   float *wconv = reinterpret_cast<float *>(sm + SM_WCONV);
-  if constexpr (kFused) {
+  if constexpr (kMode == kFusedMode) {
     for (int idx = tid; idx < 3 * 128; idx += kThreads) {  // tap-major: lanes read consecutive channels
       const int p = idx >> 7, ch = idx & 127;
       const float4 w = __ldg(reinterpret_cast<const float4 *>(conv_w + ((size_t)p * HD + hb * 128 + ch) * 4));
@@ -358,6 +381,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (tid == 0 && cur.ok) issue_tma(cur);
   // beta of the current work item's tokens, fetched one item ahead
   float beta_next = (cur.ok && tid < cur.Lc) ? __ldg(beta + (size_t)(cur.t0 + tid) * H + cur.h) : 0.f;
+  // kPrepFused: the item's conv weights [3 parts][128 channels][4 taps] (three
+  // per thread), fetched one item ahead and stored tap-major at the item start
+  float wnext[3] = {0.f, 0.f, 0.f};
+  auto fetch_w = [&](const Work &w) {
+    if constexpr (kMode == kPrepFused) {
+#pragma unroll
+      for (int m = 0; m < 3; ++m)
+        wnext[m] = __ldg(conv_w + (size_t)m * HD * 4 + (size_t)w.h * 512 + tid);
+    }
+  };
+  if (cur.ok) fetch_w(cur);
 
   uint32_t tma_par = 0, mma_par = 0;
   int c = 0;
@@ -368,6 +402,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ---- P0: raw tiles of this chunk ---------------------------------------------
     if (!wait_all(bar_tma, tma_par, status)) break;
     tma_par ^= 1;
+    if constexpr (kMode == kPrepFused) {
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {  // element tid + 512 m of the head's [part][channel][tap]
+        const int rem = tid, ch = rem >> 2, tap = rem & 3;
+        wconv[(m * 4 + tap) * 128 + ch] = wnext[m];
+      }
+      if (nxt.ok) fetch_w(nxt);
+      if (!has_halo(cur)) {  // sequence start: history from the cache rows or zero
+        for (int idx = tid; idx < 9 * 128; idx += kThreads) {
+          const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
+          hist[idx] = cache_in ? cache_in[((size_t)cur.n * 3 + row) * 3 * HD + p * HD + h * 128 + ch]
+                               : from_f32<Tin>(0.f);
+        }
+      }
+    }
 
     // ---- P1: beta, in-chunk cumulative log-decay, per-channel factors, E ------------
     if (tid < 64) {
@@ -379,8 +428,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // thread: 8 channels (c8) of two consecutive rows r0, r0+1 of all three parts;
       // all raw values are read before any tile is overwritten.
       __syncthreads();  // beta_s visible
-      const Tin *hcur = hist + (c & 1) * 1152;
-      Tin *hnxt = hist + ((c + 1) & 1) * 1152;
+      // history slots: alternate along the sequence (one pass), or slot 0 in,
+      // slot 1 out (each prep item brings its own history)
+      const Tin *hcur = hist + (kPrepM ? 0 : (c & 1) * 1152);
+      Tin *hnxt = hist + (kPrepM ? 1152 : ((c + 1) & 1) * 1152);
       const int c8 = tid & 15, d0 = c8 * 8, r0 = 2 * (tid >> 4);
       uint4 packed[3][2];      // q, k, v of rows r0, r0+1 as fp16, written after the barrier
       uint4 corr_pk[2];        // beta*v - f16(beta*f16(v)) as bf16
@@ -474,6 +525,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         st_shared_16(sm + SM_V, r * 256 + c8 * 16, packed[2][q2]);
         st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, corr_pk[q2]);
         if (c8 == 0) pdiag[r] = qk[q2];  // <q_r, k_r> of the fp32 prologue outputs
+      }
+      if constexpr (kMode == kPrepFused) {
+        if (cache_out && t0 + Lc == cur.eos) {  // the sequence's last three raw inputs
+          for (int idx = tid; idx < 9 * 128; idx += kThreads) {
+            const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
+            cache_out[((size_t)cur.n * 3 + row) * 3 * HD + p * HD + h * 128 + ch] = hnxt[idx];
+          }
+        }
       }
       __syncthreads();
     }
@@ -610,7 +669,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
       st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
       st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
-      if constexpr (kPrepM) {  // fp32 remainder beta v - f16(beta v), kept as bf16
+      if constexpr (kPrepM && !kFused) {  // fp32 remainder beta v - f16(beta v), kept as bf16
         float cr[8], bvmax = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -623,10 +682,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncthreads();
     if constexpr (kPrepM) {
-      if (tid == 0 && nxt.ok) {  // the v and g (E) tiles are dead: the next item's tiles start
-        arm_tma();
+      if (tid == 0 && nxt.ok) {  // the v and g (E) tiles and history slot 0 are dead:
+        arm_tma(nxt);            // the next item's tiles start
         issue_tma_v(nxt);
         issue_tma_g(nxt);
+        issue_tma_halo(nxt);
       }
     }
 
@@ -698,7 +758,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && nxt.ok) {  // q, k tiles are dead
-      if constexpr (!kPrepM) arm_tma();
+      if constexpr (!kPrepM) arm_tma(nxt);
       issue_tma_qk(nxt);
     }
 
@@ -1001,7 +1061,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     cur = nxt;
   }
 
-  if constexpr (kFused) {
+  if constexpr (kMode == kFusedMode) {
     if (cache_out) {  // the last three raw inputs of the sequence (oldest first)
       const Tin *hfin = hist + (nchunks & 1) * 1152;
       for (int idx = tid; idx < 9 * 128; idx += kThreads) {
@@ -1037,13 +1097,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over a [T, H, 128] tensor: box = 64 tokens x 1 head x 128 channels.
-bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esz, int H, int T) {
+// 3-D map over a [T, H, 128] tensor: box = `rows` tokens x 1 head x 128 channels.
+bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esz, int H, int T,
+              unsigned rows = 64) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
   cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)H * 128 * esz};
-  cuuint32_t box[3] = {128, 1, 64};
+  cuuint32_t box[3] = {128, 1, rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1146,6 +1207,48 @@ cudaError_t launch_fused_typed(const void *x, const float *conv_w, const void *c
   return cudaGetLastError();
 }
 }  // namespace
+
+namespace {
+template <typename Tin>
+cudaError_t launch_prep_fused_typed(const void *x, const float *conv_w, const void *cache_in,
+                                    void *cache_out, const float *g, const float *beta,
+                                    const int32_t *cu, int N, int T, int H,
+                                    CUtensorMapDataType act, void *ws, int *status,
+                                    cudaStream_t s) {
+  CUtensorMap tx, th, tg;
+  if (!make_map(&tx, x, act, 2, 3 * H, T) || !make_map(&th, x, act, 2, 3 * H, T, 3) ||
+      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+    return cudaErrorInvalidValue;
+  auto kern = chunk_tc_kernel<Tin, kPrepFused>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SM_ALLOC_FUSED);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const long long items = rec::chunk_capacity(N, T) * H;
+  const unsigned grid = (unsigned)std::min<long long>(items, sms);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  kern<<<grid, kThreads, SM_ALLOC_FUSED, s>>>(
+      tx, th, tx, tg, beta, 1.f, nullptr, cu, T, H, nullptr, nullptr, status, conv_w,
+      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), w,
+      reinterpret_cast<const int32_t *>(w), N);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
+                                       void *cache_out, const float *g, const float *beta,
+                                       const int32_t *cu, int N, int T, int H, kda_dtype dt,
+                                       void *ws, int *status, cudaStream_t s) {
+  if (dt == KDA_BF16)
+    return launch_prep_fused_typed<__nv_bfloat16>(x, conv_w, cache_in, cache_out, g, beta, cu, N,
+                                                  T, H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws,
+                                                  status, s);
+  return launch_prep_fused_typed<__half>(x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H,
+                                         CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, status, s);
+}
 
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,
                                      void *cache_out, const float *g, const float *beta,

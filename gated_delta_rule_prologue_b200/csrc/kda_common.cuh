@@ -202,6 +202,12 @@ cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *s
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, float *o, float *sN, int *status,
                                cudaStream_t s);
+cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
+                                       void *cache_out, const float *g, const float *beta,
+                                       const int32_t *cu, int N, int T, int H, kda_dtype dt,
+                                       void *ws, int *status, cudaStream_t s);
+cudaError_t launch_cache_pass(const void *ws, int N, int H, const void *cache_in,
+                              void *cache_out, cudaStream_t s);
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,
                                      void *cache_out, const float *g, const float *beta,
                                      float scale, const float *s0, const int32_t *cu, int N,

@@ -204,6 +204,26 @@ kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void
                                   kda_stream_t stream);
 
 /*
+ * kda_prologue_chunk_fwd_ws -- kda_prologue_chunk_fwd with a caller-owned
+ * scratch buffer, run as two passes like kda_chunk_fwd_ws with the prologue
+ * inside the parallel pass: each (chunk, head) item convolves its own 64 rows
+ * ([W1 第二站], [W4 ShortConv paragraph]), taking the three raw rows before the
+ * chunk, or cache_in at a sequence start, as the conv history; the state pass
+ * then carries the state through the chunks ([W4 Figure 1]).  Same arguments
+ * and results as kda_prologue_chunk_fwd (equal up to rounding order), plus
+ * workspace / workspace_bytes exactly as in kda_chunk_fwd_ws, sized by
+ * kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt).  NULL workspace: the
+ * call is kda_prologue_chunk_fwd.
+ */
+kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const void *cache_in,
+                                     void *cache_out, const float *g, const float *beta,
+                                     float scale, const float *initial_state,
+                                     const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                     kda_dtype dt, float *o, float *final_state,
+                                     void *workspace, size_t workspace_bytes,
+                                     kda_stream_t stream);
+
+/*
  * kda_decode_step -- one new token for each of N independent sequences: the
  * prologue on that token with the conv cache as history, then one step of
  * the recurrence on the state in place (the recurrent mode used for

@@ -265,28 +265,34 @@ def test_prologue_parity_varlen_with_cache(kda, dtype, out_dtype, D):
 # --- full-size workloads, sampled ------------------------------------------------
 
 def test_k3_prefill_full_size_sampled_heads(kda):
-    """Fused prologue + chunkwise prefill over 32768 tokens x 96 heads (the
-    benchmark's launch); heads 0, 53 and 95 recomputed by the oracle over all
-    tokens."""
+    """Fused prologue + chunkwise prefill over 32768 tokens x 96 heads, both the
+    two-pass launch (the benchmark's) and the one-pass kernel; heads 0, 53 and
+    95 recomputed by the oracle over all tokens."""
     inp = W.k3_prefill()
     T, H, D = inp.T, inp.H, inp.D
     dev = "cuda"
-    x = inp.x.to(dev)
-    o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
-    fs = torch.empty((1, H, D, D), device=dev)
-    cache = torch.empty((1, 3, 3 * H * D), dtype=torch.bfloat16, device=dev)
-    kda.kda_prologue_chunk_fwd(x, inp.conv_w.to(dev), inp.g.to(dev), inp.beta.to(dev), o, H=H,
-                               D=D, scale=inp.scale, final_state=fs, cache_out=cache)
-    torch.cuda.synchronize()
-    assert kda.kda_get_device_status() == 0
-    np.testing.assert_array_equal(f64(cache[0]), f64(inp.x[-3:]))
-    del x
+    x, w, g, beta = inp.x.to(dev), inp.conv_w.to(dev), inp.g.to(dev), inp.beta.to(dev)
+    runs = {}
+    for passes, ws in PASSES.items():
+        o = torch.empty((T, H, D), dtype=torch.float32, device=dev)
+        fs = torch.empty((1, H, D, D), device=dev)
+        cache = torch.empty((1, 3, 3 * H * D), dtype=torch.bfloat16, device=dev)
+        kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D, scale=inp.scale, final_state=fs,
+                                   cache_out=cache, workspace=ws)
+        torch.cuda.synchronize()
+        assert kda.kda_get_device_status() == 0
+        np.testing.assert_array_equal(f64(cache[0]), f64(inp.x[-3:]))
+        runs[passes] = (o.cpu(), fs.cpu())
+        del o
+        torch.cuda.empty_cache()
+    del x, g, beta
     for h in (0, 53, 95):
         xh, wh, gh, bh = W.k3_prefill_head(h)
         qr, kr, vr, _ = o_prologue(xh.reshape(T, 3 * D), wh.reshape(3 * D, 4), 1, D)
         o_ref, S_ref = kda_recurrent(qr, kr, vr, gh[:, None, :], bh[:, None], inp.scale)
-        assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16
-        assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE
+        for passes, (o, fs) in runs.items():
+            assert rel_max(f64(o[:, h]), o_ref[:, 0]) <= TOL_BF16, passes
+            assert rel_fro(f64(fs[0, h]), state_to_abi(S_ref)[0, 0]) <= TOL_STATE, passes
 
 
 def test_k3_unfused_full_size_sampled_heads(kda):
@@ -330,15 +336,19 @@ def test_k3_prologue_kernel_full_size_sampled_heads(kda):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_fused_prefill_varlen_with_cache_and_resume(kda, dtype):
+@pytest.mark.parametrize("passes", list(PASSES))
+@pytest.mark.parametrize("lengths", [([70, 1, 130, 64], [5, 100, 2, 66]),
+                                     ([70, 0, 130, 1, 200], [0, 100, 2, 66, 3])],
+                         ids=["nonempty", "with_empty"])
+def test_fused_prefill_varlen_with_cache_and_resume(kda, dtype, passes, lengths):
     """Fused path over packed sequences with conv cache and initial state in,
     cache and final state out; then a second call continuing every sequence
     from the first call's cache and state.  Both calls match the oracle run
-    over the concatenated tokens."""
+    over the concatenated tokens; a sequence that is empty in a call passes
+    its cache and state through."""
     dev = "cuda"
     H, D = 2, 128
-    l1 = [70, 1, 130, 64]
-    l2 = [5, 100, 2, 66]
+    l1, l2 = lengths
     N, C = len(l1), 3 * H * D
     r = torch.Generator().manual_seed(31)
     xs = [torch.randn((a + b, C), generator=r).to(dtype) for a, b in zip(l1, l2)]
@@ -362,7 +372,7 @@ def test_fused_prefill_varlen_with_cache_and_resume(kda, dtype):
         kda.kda_prologue_chunk_fwd(pack(xs, part).to(dev), w.to(dev), pack(gs, part).to(dev),
                                    pack(bs, part).to(dev), o, H=H, D=D, cache_in=cache_in,
                                    cache_out=cache_out, initial_state=state, final_state=fs,
-                                   cu_seqlens=cu)
+                                   cu_seqlens=cu, workspace=PASSES[passes])
         outs.append((o, cu))
         cache_in, state = cache_out, fs
     torch.cuda.synchronize()
