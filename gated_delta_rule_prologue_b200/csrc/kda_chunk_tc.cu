@@ -56,6 +56,10 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 512;
+constexpr int kHalf = kThreads / 2;
+
+// Barrier of the first half of the CTA (warps 0-7) only.
+__device__ __forceinline__ void bar_half() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // ---- shared memory plan (byte offsets from a 1024-aligned base) ----------------
 constexpr uint32_t SM_Q = 0;                // raw q tile [64][128] bf16
@@ -640,239 +644,249 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mma_par ^= 1;
     tc_fence_after();
 
-    // ---- P4a: WY / output operands (the Gram operands are dead) -------------------------
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const int p = tid + kThreads * m;
-      const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
-      const bool valid = r < Lc;
-      const float bt = beta_s[r];
-      const float *fec = r < 32 ? feca : fecb;
-      const float *fel = r < 32 ? fela : felb;
-      float k8[8], q8[8], v8[8], e8[8];
-      ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
-      ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
-      ld8_in<Tact>(sm + SM_V + r * 256 + c8 * 16, v8);
-      ld8_f32(Gf + r * 128 + d0, e8);
-      float bkg[8], bv[8], qg[8], kp[8], ec8[8], el8[8];
-      ld8_f32(fec + d0, ec8);
-      ld8_f32(fel + d0, el8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f, vv = valid ? v8[e] : 0.f;
-        bkg[e] = bt * kk * e8[e] * ec8[e];
-        bv[e] = bt * vv;
-        qg[e] = qq * e8[e] * ec8[e];
-        kp[e] = __fdividef(kk, e8[e]) * el8[e];
-      }
-      st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
-      st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
-      st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
-      st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
-      if constexpr (kPrepM && !kFused) {  // fp32 remainder beta v - f16(beta v), kept as bf16
-        float cr[8], bvmax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          cr[e] = bv[e] - __half2float(__float2half_rn(bv[e]));
-          bvmax = fmaxf(bvmax, fabsf(bv[e]));
-        }
-        st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
-        if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
-      }
-    }
-    __syncthreads();
-    if constexpr (kPrepM) {
-      if (tid == 0 && nxt.ok) {  // the v and g (E) tiles and history slot 0 are dead:
-        arm_tma(nxt);            // the next item's tiles start
-        issue_tma_v(nxt);
-        issue_tma_g(nxt);
-        issue_tma_halo(nxt);
-      }
-    }
-
-    // ---- P4b: <q_r, k_r> in fp32; Gram read-out -> A^T (fp32), strict P operand ---------
-    // AT[i*64 + r] = A[r][i], TT[r*64 + c] = T[r][c]: over the g tile, or (prep,
-    // which has no S^T operand) over the S^T tile so the next g tile can load now
-    float *AT = kPrepM ? reinterpret_cast<float *>(sm + SM_ST) : Gf;
-    float *TT = AT + 4096;
-    for (int idx = tid; idx < 4096 / 4; idx += kThreads)
-      reinterpret_cast<float4 *>(AT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-    reinterpret_cast<uint4 *>(sm + SM_POP)[tid] = make_uint4(0u, 0u, 0u, 0u);  // 8 KB
-    if constexpr (!kFused) {
-      const int r = tid >> 3, part = tid & 7;
-      float acc = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        float q8[8], k8[8];
-        ld8_in<Tact>(sm + SM_Q + r * 256 + (part * 2 + cc) * 16, q8);
-        ld8_in<Tact>(sm + SM_K + r * 256 + (part * 2 + cc) * 16, k8);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc = fmaf(q8[e], k8[e], acc);
-      }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      if (part == 0) pdiag[r] = r < Lc ? acc : 0.f;
-    }
-    __syncthreads();
-    {
+    // ---- P4: two warp groups ---------------------------------------------------------------
+    //   warps 0-7:  P4b (Gram read-out -> A^T, strict P), P5 (T = (I + A)^-1)
+    //   warps 8-15: P4a (the W / Ut / output operands; <q_r, k_r>), which needs neither
+    // A^T and T live over the S^T tile (dead from the Gram MMA to P6), so P4a can
+    // still read E from the g tile.
+    float *AT = reinterpret_cast<float *>(sm + SM_ST);  // AT[i*64 + r] = A[r][i]
+    float *TT = AT + 4096;                              // TT[r*64 + c] = T[r][c]
+    if (tid < kHalf) {
+      // ---- P4b: Gram read-out -> A^T (fp32, strictly lower part only: nothing else of
+      //      it is read), strict P operand ------------------------------------------------
+      // warp w reads TMEM lanes 32 (w % 4).. and column groups 2 (w / 4) + {0, 1}: the
+      // first half of the columns ([0, 32), i = col) in groups of 8, the second
+      // ([32, 96), i = col - 32) in groups of 16
       const bool isP = quad >= 2;
       const int r = 32 * (quad & 1) + lane;
       const float br = beta_s[r];
-      // first half: columns [0, 32), i = col, 8 per column group;
-      // second half: columns [32, 96), i = col - 32, 16 per column group
-      float v[16];
-      int i0s;
+      float v[2][16];
       if (quad & 1) {
-        float w[16];
-        tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * grp, v);
-        tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * grp, w);
-        tmem_wait_ld(v, w);
+        float w[2][16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] += w[e];
-        i0s = 16 * grp;
+        for (int gs = 0; gs < 2; ++gs) {
+          const int cg = 2 * (warp >> 2) + gs;
+          tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * cg, v[gs]);
+          tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * cg, w[gs]);
+        }
+        tmem_wait_ld(v[0], v[1]);
+        tmem_wait_ld(w[0], w[1]);
+#pragma unroll
+        for (int gs = 0; gs < 2; ++gs)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[gs][e] += w[gs][e];
       } else {
-        float v8[8], w8[8];
-        tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * grp, v8);
-        tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * grp, w8);
-        tmem_wait_ld(v8, w8);
+        float a8[2][8], b8[2][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = v8[e] + w8[e];
-        i0s = 8 * grp;
+        for (int gs = 0; gs < 2; ++gs) {
+          const int cg = 2 * (warp >> 2) + gs;
+          tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * cg, a8[gs]);
+          tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * cg, b8[gs]);
+        }
+        tmem_wait_ld(a8[0], a8[1]);
+        tmem_wait_ld(b8[0], b8[1]);
+#pragma unroll
+        for (int gs = 0; gs < 2; ++gs)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[gs][e] = a8[gs][e] + b8[gs][e];
       }
-      const int nch = (quad & 1) ? 2 : 1;
-      for (int g8 = 0; g8 < nch; ++g8) {
-        const int i0 = i0s + 8 * g8;
-        if (!isP) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
-        } else if (i0 < r) {
-          float p8[8];
+      for (int gs = 0; gs < 2; ++gs) {
+        const int cg = 2 * (warp >> 2) + gs;
+        const int i0s = (quad & 1) ? 16 * cg : 8 * cg;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
-          st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
+        for (int g8 = 0; g8 < 2; ++g8) {
+          if (g8 == 1 && !(quad & 1)) break;
+          const int i0 = i0s + 8 * g8;
+          if (!isP) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[gs][8 * g8 + e];
+          } else {  // every chunk of the strict P tile this thread reads is written
+            float p8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[gs][8 * g8 + e] : 0.f;
+            st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
+          }
         }
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && nxt.ok) {  // q, k tiles are dead
-      if constexpr (!kPrepM) arm_tma(nxt);
-      issue_tma_qk(nxt);
-    }
+      if (tid < 128) {  // P rows 0..31, columns 32..63: above the diagonal, not read out
+        const int rz = tid >> 2, cz = 4 + (tid & 3);
+        st_shared_16(sm + SM_POP, kmaj_off(64, rz, cz), make_uint4(0u, 0u, 0u, 0u));
+      }
+      bar_half();
 
-    // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ------------------------------------
-    // (i) the four diagonal 16x16 blocks by forward substitution, one column per
-    //     thread; (ii) the two 16x16 blocks under them inside each 32x32 half,
-    //     T_{s+1,s} = -T_{s+1,s+1} A_{s+1,s} T_{s,s}; (iii) the lower-left 32x32
-    //     block T_BL = -T_BR (A_BL T_TL).
-    if (tid < 64) {  // column jj of a diagonal block, swept row by row, stored at the end
-      const int base = 16 * (tid >> 4), jj = tid & 15;
-      float acc[16];
+      // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ----------------------------------
+      // (i) the four diagonal 16x16 blocks by forward substitution, one column per
+      //     thread; (ii) the two 16x16 blocks under them inside each 32x32 half,
+      //     T_{s+1,s} = -T_{s+1,s+1} A_{s+1,s} T_{s,s}; (iii) the lower-left 32x32
+      //     block T_BL = -T_BR (A_BL T_TL).
+      if (tid < 64) {  // column jj of a diagonal block, swept row by row, stored at the end
+        const int base = 16 * (tid >> 4), jj = tid & 15;
+        float acc[16];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
+        for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) {
-        acc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -acc[ii]);
-        const float *arow = AT + (base + ii) * 64 + base;  // A[base+rr][base+ii], rr > ii
+        for (int ii = 0; ii < 16; ++ii) {
+          acc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -acc[ii]);
+          const float *arow = AT + (base + ii) * 64 + base;  // A[base+rr][base+ii], rr > ii
 #pragma unroll
-        for (int rr = ii + 1; rr < 16; ++rr) acc[rr] = fmaf(arow[rr], acc[ii], acc[rr]);
-      }
-#pragma unroll
-      for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = acc[rr];
-    }
-    __syncthreads();
-    // Blocks below the diagonal, 2x2 output tiles per thread.  A is read through
-    // its transpose (columns of A are contiguous), T and Y by rows, so the
-    // operands of one k-step are float2 loads.
-    if (tid < 128) {  // (ii) X = A_{s+1,s} T_{s,s} for s = 0, 2
-      const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
-      float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const float2 av = *reinterpret_cast<const float2 *>(AT + (s0b + t) * 64 + s0b + 16 + a);
-        const float2 tv = *reinterpret_cast<const float2 *>(TT + (s0b + t) * 64 + s0b + b);
-        x00 = fmaf(av.x, tv.x, x00); x01 = fmaf(av.x, tv.y, x01);
-        x10 = fmaf(av.y, tv.x, x10); x11 = fmaf(av.y, tv.y, x11);
-      }
-      *reinterpret_cast<float2 *>(XS + blk * 256 + a * 16 + b) = make_float2(x00, x01);
-      *reinterpret_cast<float2 *>(XS + blk * 256 + (a + 1) * 16 + b) = make_float2(x10, x11);
-    }
-    __syncthreads();
-    if (tid < 128) {  // T_{s+1,s} = -T_{s+1,s+1} X
-      const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
-      const float *t0r = TT + (s0b + 16 + a) * 64 + s0b + 16;  // row a of T_{s+1,s+1}
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-      for (int t4 = 0; t4 < 16; t4 += 4) {  // diagonal blocks were stored with their zeros
-        const float4 ra = *reinterpret_cast<const float4 *>(t0r + t4);
-        const float4 rb = *reinterpret_cast<const float4 *>(t0r + 64 + t4);
-        const float ta[4] = {ra.x, ra.y, ra.z, ra.w}, tb[4] = {rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 xv = *reinterpret_cast<const float2 *>(XS + blk * 256 + (t4 + e) * 16 + b);
-          y00 = fmaf(ta[e], xv.x, y00); y01 = fmaf(ta[e], xv.y, y01);
-          y10 = fmaf(tb[e], xv.x, y10); y11 = fmaf(tb[e], xv.y, y11);
+          for (int rr = ii + 1; rr < 16; ++rr) acc[rr] = fmaf(arow[rr], acc[ii], acc[rr]);
         }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = acc[rr];
       }
-      *reinterpret_cast<float2 *>(TT + (s0b + 16 + a) * 64 + s0b + b) = make_float2(-y00, -y01);
-      *reinterpret_cast<float2 *>(TT + (s0b + 17 + a) * 64 + s0b + b) = make_float2(-y10, -y11);
-    }
-    __syncthreads();
-    if (tid < 256) {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31)
-      const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+      bar_half();
+      // Blocks below the diagonal, 2x2 output tiles per thread.  A is read through
+      // its transpose (columns of A are contiguous), T and Y by rows, so the
+      // operands of one k-step are float2 loads.
+      if (tid < 128) {  // (ii) X = A_{s+1,s} T_{s,s} for s = 0, 2
+        const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
+        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const float2 av = *reinterpret_cast<const float2 *>(AT + (s0b + t) * 64 + s0b + 16 + a);
+          const float2 tv = *reinterpret_cast<const float2 *>(TT + (s0b + t) * 64 + s0b + b);
+          x00 = fmaf(av.x, tv.x, x00); x01 = fmaf(av.x, tv.y, x01);
+          x10 = fmaf(av.y, tv.x, x10); x11 = fmaf(av.y, tv.y, x11);
+        }
+        *reinterpret_cast<float2 *>(XS + blk * 256 + a * 16 + b) = make_float2(x00, x01);
+        *reinterpret_cast<float2 *>(XS + blk * 256 + (a + 1) * 16 + b) = make_float2(x10, x11);
+      }
+      bar_half();
+      if (tid < 128) {  // T_{s+1,s} = -T_{s+1,s+1} X
+        const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
+        const float *t0r = TT + (s0b + 16 + a) * 64 + s0b + 16;  // row a of T_{s+1,s+1}
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+        for (int t4 = 0; t4 < 16; t4 += 4) {  // diagonal blocks were stored with their zeros
+          const float4 ra = *reinterpret_cast<const float4 *>(t0r + t4);
+          const float4 rb = *reinterpret_cast<const float4 *>(t0r + 64 + t4);
+          const float ta[4] = {ra.x, ra.y, ra.z, ra.w}, tb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xv = *reinterpret_cast<const float2 *>(XS + blk * 256 + (t4 + e) * 16 + b);
+            y00 = fmaf(ta[e], xv.x, y00); y01 = fmaf(ta[e], xv.y, y01);
+            y10 = fmaf(tb[e], xv.x, y10); y11 = fmaf(tb[e], xv.y, y11);
+          }
+        }
+        *reinterpret_cast<float2 *>(TT + (s0b + 16 + a) * 64 + s0b + b) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(TT + (s0b + 17 + a) * 64 + s0b + b) = make_float2(-y10, -y11);
+      }
+      bar_half();
+      {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31)
+        const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float2 av = *reinterpret_cast<const float2 *>(AT + m * 64 + 32 + a);
-        float2 tv = *reinterpret_cast<const float2 *>(TT + m * 64 + cc);  // T_TL[m][cc..cc+1]
-        tv.x = m >= cc ? tv.x : 0.f;                                      // upper blocks unwritten
-        tv.y = m >= cc + 1 ? tv.y : 0.f;
-        y00 = fmaf(av.x, tv.x, y00); y01 = fmaf(av.x, tv.y, y01);
-        y10 = fmaf(av.y, tv.x, y10); y11 = fmaf(av.y, tv.y, y11);
+        for (int m = 0; m < 32; ++m) {
+          const float2 av = *reinterpret_cast<const float2 *>(AT + m * 64 + 32 + a);
+          float2 tv = *reinterpret_cast<const float2 *>(TT + m * 64 + cc);  // T_TL[m][cc..cc+1]
+          tv.x = m >= cc ? tv.x : 0.f;                                      // upper blocks unwritten
+          tv.y = m >= cc + 1 ? tv.y : 0.f;
+          y00 = fmaf(av.x, tv.x, y00); y01 = fmaf(av.x, tv.y, y01);
+          y10 = fmaf(av.y, tv.x, y10); y11 = fmaf(av.y, tv.y, y11);
+        }
+        *reinterpret_cast<float2 *>(XS + a * 32 + cc) = make_float2(y00, y01);
+        *reinterpret_cast<float2 *>(XS + (a + 1) * 32 + cc) = make_float2(y10, y11);
       }
-      *reinterpret_cast<float2 *>(XS + a * 32 + cc) = make_float2(y00, y01);
-      *reinterpret_cast<float2 *>(XS + (a + 1) * 32 + cc) = make_float2(y10, y11);
-    }
-    __syncthreads();
-    if (tid < 256) {  // T_BL = -T_BR Y
-      const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
-      const float *tr = TT + (32 + a) * 64 + 32;  // row a of T_BR
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+      bar_half();
+      {  // T_BL = -T_BR Y
+        const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
+        const float *tr = TT + (32 + a) * 64 + 32;  // row a of T_BR
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 2
-      for (int m4 = 0; m4 < 32; m4 += 4) {
-        const float4 ra = *reinterpret_cast<const float4 *>(tr + m4);
-        const float4 rb = *reinterpret_cast<const float4 *>(tr + 64 + m4);
-        const float ta4[4] = {ra.x, ra.y, ra.z, ra.w}, tb4[4] = {rb.x, rb.y, rb.z, rb.w};
+        for (int m4 = 0; m4 < 32; m4 += 4) {
+          const float4 ra = *reinterpret_cast<const float4 *>(tr + m4);
+          const float4 rb = *reinterpret_cast<const float4 *>(tr + 64 + m4);
+          const float ta4[4] = {ra.x, ra.y, ra.z, ra.w}, tb4[4] = {rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {  // T_BR's upper-right 16x16 block was never written
-          const int m = m4 + e;
-          const float ta = m <= a ? ta4[e] : 0.f, tb = m <= a + 1 ? tb4[e] : 0.f;
-          const float2 yv = *reinterpret_cast<const float2 *>(XS + m * 32 + cc);
-          y00 = fmaf(ta, yv.x, y00); y01 = fmaf(ta, yv.y, y01);
-          y10 = fmaf(tb, yv.x, y10); y11 = fmaf(tb, yv.y, y11);
+          for (int e = 0; e < 4; ++e) {  // T_BR's upper-right 16x16 block was never written
+            const int m = m4 + e;
+            const float ta = m <= a ? ta4[e] : 0.f, tb = m <= a + 1 ? tb4[e] : 0.f;
+            const float2 yv = *reinterpret_cast<const float2 *>(XS + m * 32 + cc);
+            y00 = fmaf(ta, yv.x, y00); y01 = fmaf(ta, yv.y, y01);
+            y10 = fmaf(tb, yv.x, y10); y11 = fmaf(tb, yv.y, y11);
+          }
+        }
+        *reinterpret_cast<float2 *>(TT + (32 + a) * 64 + cc) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(TT + (33 + a) * 64 + cc) = make_float2(-y10, -y11);
+      }
+      bar_half();
+#pragma unroll
+      for (int task = tid; task < 512; task += kHalf) {  // T as the fp16 operand
+        const int r8 = task >> 3, c8 = task & 7;
+        float f[8];
+        ld8_f32(TT + r8 * 64 + 8 * c8, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int cc = 8 * c8 + e;
+          f[e] = cc < r8 ? f[e] : (cc == r8 ? 1.f : 0.f);
+        }
+        st_shared_16(sm + SM_TOP, kmaj_off(64, r8, c8), pack8_f16(f));
+      }
+    } else {
+      // ---- P4a: WY / output operands (the Gram operands are dead) -------------------------
+#pragma unroll 2
+      for (int m = 0; m < 4; ++m) {
+        const int p = (tid - kHalf) + kHalf * m;
+        const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
+        const bool valid = r < Lc;
+        const float bt = beta_s[r];
+        const float *fec = r < 32 ? feca : fecb;
+        const float *fel = r < 32 ? fela : felb;
+        float k8[8], q8[8], v8[8], e8[8];
+        ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
+        ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
+        ld8_in<Tact>(sm + SM_V + r * 256 + c8 * 16, v8);
+        ld8_f32(Gf + r * 128 + d0, e8);
+        float bkg[8], bv[8], qg[8], kp[8], ec8[8], el8[8];
+        ld8_f32(fec + d0, ec8);
+        ld8_f32(fel + d0, el8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f, vv = valid ? v8[e] : 0.f;
+          bkg[e] = bt * kk * e8[e] * ec8[e];
+          bv[e] = bt * vv;
+          qg[e] = qq * e8[e] * ec8[e];
+          kp[e] = __fdividef(kk, e8[e]) * el8[e];
+        }
+        st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
+        st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
+        st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
+        st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
+        if constexpr (!kFused) {  // <q_r, k_r> in fp32 over the row's 16 lanes
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc = fmaf(q8[e], k8[e], acc);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+          if (c8 == 0) pdiag[r] = valid ? acc : 0.f;
+        }
+        if constexpr (kPrepM && !kFused) {  // fp32 remainder beta v - f16(beta v), kept as bf16
+          float cr[8], bvmax = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            cr[e] = bv[e] - __half2float(__float2half_rn(bv[e]));
+            bvmax = fmaxf(bvmax, fabsf(bv[e]));
+          }
+          st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
+          if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
         }
       }
-      *reinterpret_cast<float2 *>(TT + (32 + a) * 64 + cc) = make_float2(-y00, -y01);
-      *reinterpret_cast<float2 *>(TT + (33 + a) * 64 + cc) = make_float2(-y10, -y11);
-    }
-    __syncthreads();
-    {
-      const int r = tid >> 3, c8 = tid & 7;
-      float f[8];
-      ld8_f32(TT + r * 64 + 8 * c8, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int cc = 8 * c8 + e;
-        f[e] = cc < r ? f[e] : (cc == r ? 1.f : 0.f);
-      }
-      st_shared_16(sm + SM_TOP, kmaj_off(64, r, c8), pack8_f16(f));
     }
     fence_async_smem();
+    tc_fence_before();
     __syncthreads();
-    if constexpr (!kPrepM) {
-      if (tid == 0 && nxt.ok) issue_tma_g(nxt);  // A^T / T (the g tile) are dead
+    if (tid == 0 && nxt.ok) {  // q, k, g (and in prep v and the history) are dead
+      arm_tma(nxt);
+      issue_tma_qk(nxt);
+      issue_tma_g(nxt);
+      if constexpr (kPrepM) {
+        issue_tma_v(nxt);
+        issue_tma_halo(nxt);
+      }
     }
 
     // ---- P6: W^T and Ut^T MMAs; meanwhile S^T -> fp16 operand ------------------------------
