@@ -54,7 +54,8 @@ DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4
 
 _CSRC = "gated_delta_rule_prologue_b200/csrc/"
 KERNEL_SOURCES = {
-    "kda_prologue_chunk_fwd": [_CSRC + "kda_chunk_tc.cu"],
+    "kda_prologue_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
+    "kda_prologue_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
     "kda_prologue": [_CSRC + "kda_prologue.cu"],
     "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
     "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
@@ -323,29 +324,37 @@ def run_ours(args, world, rank, local):
     assert kda.kda_get_device_status() == 0
     launches = 3 * args.steps  # prologue, chunk prep pass, chunk state pass
 
-    # the fused variant (prologue inside the one-pass chunk kernel) and the
-    # one-pass chunk kernel, timed beside the step
+    # timed beside the step: the prologue fused into the two-pass chunk call, the
+    # fused one-pass kernel, and the one-pass chunk kernel
     o2 = torch.empty_like(o)
-    side = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(3)]
+    side = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(3)]
     for i in range(3):
         side[i][0].record(stream)
-        kda.kda_prologue_chunk_fwd(x, w, g, beta, o2, H=H, D=D, scale=inp.scale, stream=stream)
+        kda.kda_prologue_chunk_fwd(x, w, g, beta, o2, H=H, D=D, scale=inp.scale, workspace=ws,
+                                   stream=stream)
         side[i][1].record(stream)
+        kda.kda_prologue_chunk_fwd(x, w, g, beta, o2, H=H, D=D, scale=inp.scale, workspace=None,
+                                   stream=stream)
         side[i][2].record(stream)
+        side[i][3].record(stream)
         kda.kda_chunk_fwd(q, k, v, g, beta, o2, scale=inp.scale, chunk=inp.chunk,
                           workspace=None, stream=stream)
-        side[i][3].record(stream)
+        side[i][4].record(stream)
     torch.cuda.synchronize(dev)
     fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in side[1:])
-    one_pass_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in side[1:])
+    fused_one_pass_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in side[1:])
+    one_pass_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in side[1:])
     del o2
 
     th = T * H
     step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
     kernels = {
-        "kda_prologue_chunk_fwd": dict(ms=round(fused_ms, 4), **roofline(
+        "kda_prologue_chunk_fwd": dict(ms=round(fused_ms, 4), launches=2, **roofline(
             "hbm", FUSED_BYTES_PER_TH * th, fused_ms, hbm, "GB/s",
             recorded_traffic("kda_prologue_chunk_fwd"))),
+        "kda_prologue_chunk_fwd_one_pass": dict(ms=round(fused_one_pass_ms, 4), **roofline(
+            "hbm", FUSED_BYTES_PER_TH * th, fused_one_pass_ms, hbm, "GB/s",
+            recorded_traffic("kda_prologue_chunk_fwd_one_pass"))),
         "kda_prologue": dict(ms=round(pro_ms, 4), **roofline(
             "hbm", PROLOGUE_BYTES_PER_TH * th, pro_ms, hbm, "GB/s", recorded_traffic("kda_prologue"))),
         "kda_chunk_fwd": dict(ms=round(chk_ms, 4), launches=2, **roofline(

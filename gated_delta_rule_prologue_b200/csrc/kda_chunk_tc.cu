@@ -660,39 +660,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const bool isP = quad >= 2;
       const int r = 32 * (quad & 1) + lane;
       const float br = beta_s[r];
-      float v[2][16];
-      if (quad & 1) {
-        float w[2][16];
-#pragma unroll
-        for (int gs = 0; gs < 2; ++gs) {
-          const int cg = 2 * (warp >> 2) + gs;
-          tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * cg, v[gs]);
-          tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * cg, w[gs]);
-        }
-        tmem_wait_ld(v[0], v[1]);
-        tmem_wait_ld(w[0], w[1]);
-#pragma unroll
-        for (int gs = 0; gs < 2; ++gs)
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[gs][e] += w[gs][e];
-      } else {
-        float a8[2][8], b8[2][8];
-#pragma unroll
-        for (int gs = 0; gs < 2; ++gs) {
-          const int cg = 2 * (warp >> 2) + gs;
-          tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * cg, a8[gs]);
-          tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * cg, b8[gs]);
-        }
-        tmem_wait_ld(a8[0], a8[1]);
-        tmem_wait_ld(b8[0], b8[1]);
-#pragma unroll
-        for (int gs = 0; gs < 2; ++gs)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[gs][e] = a8[gs][e] + b8[gs][e];
-      }
-#pragma unroll
-      for (int gs = 0; gs < 2; ++gs) {
-        const int cg = 2 * (warp >> 2) + gs;
+      // one column group: v holds the summed partial Grams of its 8 or 16 columns
+      auto emit = [&](int cg, const float (&v)[16]) {
         const int i0s = (quad & 1) ? 16 * cg : 8 * cg;
 #pragma unroll
         for (int g8 = 0; g8 < 2; ++g8) {
@@ -701,13 +670,46 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!isP) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[gs][8 * g8 + e];
+              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
           } else {  // every chunk of the strict P tile this thread reads is written
             float p8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[gs][8 * g8 + e] : 0.f;
+            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
             st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
           }
+        }
+      };
+      auto load_group = [&](int cg, float (&v)[16], float (&w)[16]) {
+        if (quad & 1) {
+          tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * cg, v);
+          tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * cg, w);
+        } else {
+          tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * cg, *reinterpret_cast<float(*)[8]>(v));
+          tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * cg, *reinterpret_cast<float(*)[8]>(w));
+        }
+      };
+      const int cg0 = 2 * (warp >> 2);
+      if constexpr (kMode == kPrep) {  // both groups in flight at once (registers allow it)
+        float v[2][16], w[2][16];
+        load_group(cg0, v[0], w[0]);
+        load_group(cg0 + 1, v[1], w[1]);
+        tmem_wait_ld(v[0], v[1]);
+        tmem_wait_ld(w[0], w[1]);
+#pragma unroll
+        for (int gs = 0; gs < 2; ++gs) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[gs][e] += w[gs][e];
+          emit(cg0 + gs, v[gs]);
+        }
+      } else {
+#pragma unroll 1
+        for (int gs = 0; gs < 2; ++gs) {
+          float v[16], w[16];
+          load_group(cg0 + gs, v, w);
+          tmem_wait_ld(v, w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] += w[e];
+          emit(cg0 + gs, v);
         }
       }
       if (tid < 128) {  // P rows 0..31, columns 32..63: above the diagonal, not read out
