@@ -15,7 +15,7 @@
 // c_A = gamma_15 for tokens 0..31 and c_B = gamma_47 for tokens 32..63.  With
 // g >= -5 a half spans at most 16 tokens on either side of its reference, so
 // E_r = exp(gamma_r - c(r)) lies in [e^-80, e^75] and every factor below fits
-// fp32/bf16:
+// the fp32 exponent range:
 //   Gram  D_G = [K*E ; Q*E] . [ver_A ; ver_B]^T          (M=128, N=96, K=128)
 //         ver_A_i = k_i / E_i                     (i < 32, reference c_A)
 //         ver_B_i = k_i / E_i * exp(c_B - c(i))   (i < 64, reference c_B; for i < 32
@@ -24,14 +24,14 @@
 //         rows of the first half read ver_A, rows of the second half ver_B.
 //         A[r,i] = beta_r D_G[r, i] (i < r);  P[r,i] = D_G[64+r, i] (i < r)
 //         P[r,r] = <q_r, k_r> is taken in fp32 from the unscaled tiles.
-//         Each Gram operand x is split as hi = bf16(x), lo = bf16(x - hi) and the
-//         Gram is hi.hi + hi.lo + lo.hi (three MMAs into one accumulator): the
-//         read-out's error is dominated by P, which this makes nearly exact.
+//         The Gram operands are fp32 rounded to tf32 (10-bit significand, fp32
+//         range; MMA kind::tf32), over two accumulators (key channels 0..63 and
+//         64..127) summed at read-out.
 //   WY    T = (I + A)^{-1} (fp32, blocked over 16x16 blocks)
 //         W^T = (beta K G)^T T^T,  Ut^T = (beta V)^T T^T           (G_r = exp(gamma_r))
 //   state U^T = Ut^T - S^T W^T,   O^T = S^T (Q G)^T + U^T P_strict^T
 //         S <- diag(G_last) S + U^T (K * G_last / G)    (value-major registers)
-//   Operand types: the Gram operands are bf16 (they need the e^+-80 range);
+//   Operand types: the Gram operands are tf32 (they need the e^+-80 range);
 //   every other operand (T, beta K G, beta V, S^T, W, Q G, U^T, P, K') has a
 //   modest range and is fp16, whose 11-bit significand keeps the read-out
 //   within the parity bound when the decay is slow.  A value that would not
@@ -39,8 +39,10 @@
 //   fp32 diagonal terms: u_r gets beta_r v_r - f16(beta_r v_r) back, and
 //   o_r gets <q_r, k_r> u_r in fp32, so a token's own (dominant) contribution
 //   to its read-out is never rounded to bf16.
-// One CTA (512 threads) per (sequence, head); the chunks of a sequence run in
-// order, the next chunk's tiles stream in by TMA during the current one.
+// One-pass modes: one CTA (512 threads) per (sequence, head); the chunks of a
+// sequence run in order, the next chunk's tiles stream in by TMA during the
+// current one.  Prep modes: the state-independent half per (chunk, head) item
+// (see the mode list at the kernel).
 #include <cuda.h>
 #include <algorithm>
 #include <cstring>
@@ -58,8 +60,9 @@ using namespace tc;
 constexpr int kThreads = 512;
 constexpr int kHalf = kThreads / 2;
 
-// Barrier of the first half of the CTA (warps 0-7) only.
+// Barriers of the first half of the CTA (warps 0-7) or of the second (warps 8-15) only.
 __device__ __forceinline__ void bar_half() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void bar_second_half() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
 // ---- shared memory plan (byte offsets from a 1024-aligned base) ----------------
 constexpr uint32_t SM_Q = 0;                // raw q tile [64][128] bf16
@@ -67,11 +70,9 @@ constexpr uint32_t SM_K = SM_Q + 16384;     // raw k tile
 constexpr uint32_t SM_V = SM_K + 16384;     // raw v tile
 constexpr uint32_t SM_G = SM_V + 16384;     // raw g [64][128] f32 -> gamma -> E -> (A^T, T)
 constexpr uint32_t SM_X = SM_G + 32768;     // 64 KB, reused within a chunk (the Gram's
-                                            // four tiles also use TOP, POP and ST, 112 KB):
-constexpr uint32_t SM_GA = SM_X;            //   Gram A operand, high bf16 part (K-major 128 x 128)
-constexpr uint32_t SM_GB = SM_X + 32768;    //   Gram B operand, high part (K-major 96 x 128)
-constexpr uint32_t SM_GAL = SM_X + 57344;   //   Gram A operand, low part x - bf16(x)
-constexpr uint32_t SM_GBL = SM_X + 90112;   //   Gram B operand, low part
+                                            // two tiles also use TOP, POP and ST, 112 KB):
+constexpr uint32_t SM_GA = SM_X;            //   Gram A operand, tf32 (K-major 128 x 128, 64 KB)
+constexpr uint32_t SM_GB = SM_X + 65536;    //   Gram B operand, tf32 (K-major 96 x 128, 48 KB)
 constexpr uint32_t SM_BKG = SM_X;           //   beta K G (MN-major, 64 k-rows)     16 KB; then W op
 constexpr uint32_t SM_BV = SM_X + 16384;    //   beta V   (MN-major)                16 KB
 constexpr uint32_t SM_QG = SM_X + 32768;    //   Q G      (K-major 64 x 128)        16 KB
@@ -106,7 +107,7 @@ constexpr uint32_t SM_ALLOC_PREP = SM_CORR + 16384 + 1024;  // plus the remainde
 constexpr uint32_t SM_ALLOC_FUSED = SM_TOTAL_FUSED + 1024;
 static_assert(SM_ALLOC_FUSED <= 232448, "shared memory budget");
 static_assert(SM_ALLOC_PREP <= SM_ALLOC_FUSED, "the prep plan is a prefix of the fused one");
-static_assert(SM_GBL + 24576 <= SM_ST + 32768, "Gram tiles stay inside X, TOP, POP and ST");
+static_assert(SM_GB + 49152 <= SM_ST + 32768, "Gram tiles stay inside X, TOP, POP and ST");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
 constexpr uint32_t TM_G = 0;     // Gram, 96 columns (first of two partial sums)
@@ -159,16 +160,14 @@ __device__ __forceinline__ void ld8_f32(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-// Split 8 floats into bf16 high parts and bf16 residuals.
-__device__ __forceinline__ void pack8_hilo(const float (&f)[8], uint4 &hi, uint4 &lo) {
-  float l[8];
-  __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[i] = __float2bfloat16_rn(f[i]);
-    l[i] = f[i] - __bfloat162float(h[i]);
-  }
-  lo = pack8_bf16(l);
+// 8 consecutive K-elements [8*c8, 8*c8+8) of `row` of a K-major fp32 tile of `rows`
+// rows, rounded to tf32: two 16-byte chunks.
+__device__ __forceinline__ void st_tf32x8(uint8_t *tile, int rows, int row, int c8,
+                                          const float (&f)[8]) {
+  const uint4 lo = make_uint4(tf32_rna(f[0]), tf32_rna(f[1]), tf32_rna(f[2]), tf32_rna(f[3]));
+  const uint4 hi = make_uint4(tf32_rna(f[4]), tf32_rna(f[5]), tf32_rna(f[6]), tf32_rna(f[7]));
+  st_shared_16(tile, kmaj_off(rows, row, 2 * c8), lo);
+  st_shared_16(tile, kmaj_off(rows, row, 2 * c8 + 1), hi);
 }
 
 template <typename Tin>
@@ -580,7 +579,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncthreads();
 
-    // ---- P2: Gram operands -------------------------------------------------------------
+    // ---- P2: Gram operands (fp32, rounded to tf32) -----------------------------------------
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int p = tid + kThreads * m;
@@ -590,7 +589,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
       ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
       ld8_f32(Gf + r * 128 + d0, e8);
-      float a[8], b[8], ki[8], hf[8];
+      float a[8], b[8], ki[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f;
@@ -598,24 +597,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         b[e] = qq * e8[e];
         ki[e] = __fdividef(kk, e8[e]);  // E in [e^-80, e^75]: inside the intrinsic's range
       }
-      uint4 hi, lo;
-      pack8_hilo(a, hi, lo);
-      st_shared_16(sm + SM_GA, kmaj_off(128, r, c8), hi);
-      st_shared_16(sm + SM_GAL, kmaj_off(128, r, c8), lo);
-      pack8_hilo(b, hi, lo);
-      st_shared_16(sm + SM_GA, kmaj_off(128, 64 + r, c8), hi);
-      st_shared_16(sm + SM_GAL, kmaj_off(128, 64 + r, c8), lo);
+      st_tf32x8(sm + SM_GA, 128, r, c8, a);
+      st_tf32x8(sm + SM_GA, 128, 64 + r, c8, b);
       if (r < 32) {
-        pack8_hilo(ki, hi, lo);
-        st_shared_16(sm + SM_GB, kmaj_off(96, r, c8), hi);
-        st_shared_16(sm + SM_GBL, kmaj_off(96, r, c8), lo);
+        st_tf32x8(sm + SM_GB, 96, r, c8, ki);
+        float hf[8];
         ld8_f32(feba + d0, hf);
 #pragma unroll
         for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * hf[e]) * hf[e];
       }
-      pack8_hilo(ki, hi, lo);
-      st_shared_16(sm + SM_GB, kmaj_off(96, 32 + r, c8), hi);
-      st_shared_16(sm + SM_GBL, kmaj_off(96, 32 + r, c8), lo);
+      st_tf32x8(sm + SM_GB, 96, 32 + r, c8, ki);
     }
     fence_async_smem();
     __syncthreads();
@@ -624,19 +615,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
-      const uint32_t gal = smem_u32(sm + SM_GAL), gbl = smem_u32(sm + SM_GBL);
-      constexpr uint32_t id = idesc_bf16(128, 96, false, false);
-      // two independent accumulation chains of 12 steps each, interleaved:
-      // G = hi.hi + (lo.hi over k < 64),  G2 = hi.lo + (lo.hi over k >= 64)
+      constexpr uint32_t id = idesc_tf32(128, 96, false, false);
+      // 16 K=8 steps in two independent accumulation chains, interleaved:
+      // G over key channels [0, 64), G2 over [64, 128)
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        mma_bf16(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
-        mma_bf16(tmem + TM_G2, desc_kmajor(ga, 128, ks), desc_kmajor(gbl, 96, ks), id, ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        mma_bf16(tmem + TM_G, desc_kmajor(gal, 128, ks), desc_kmajor(gb, 96, ks), id, 1);
-        mma_bf16(tmem + TM_G2, desc_kmajor(gal, 128, ks + 4), desc_kmajor(gb, 96, ks + 4), id, 1);
+        mma_tf32(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
+        mma_tf32(tmem + TM_G2, desc_kmajor(ga, 128, ks + 8), desc_kmajor(gb, 96, ks + 8), id,
+                 ks > 0);
       }
       mma_commit(bar_mma);
     }
@@ -877,17 +863,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
         }
       }
+      if constexpr (kPrepM) {
+        // the raw tiles (q, k, v, g; history slot 0) have no reader left in this item:
+        // the next item's tiles start now, while the other warps finish the inverse
+        bar_second_half();
+        if (tid == kHalf && nxt.ok) {
+          arm_tma(nxt);
+          issue_tma_qk(nxt);
+          issue_tma_g(nxt);
+          issue_tma_v(nxt);
+          issue_tma_halo(nxt);
+        }
+      }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && nxt.ok) {  // q, k, g (and in prep v and the history) are dead
-      arm_tma(nxt);
-      issue_tma_qk(nxt);
-      issue_tma_g(nxt);
-      if constexpr (kPrepM) {
-        issue_tma_v(nxt);
-        issue_tma_halo(nxt);
+    if constexpr (!kPrepM) {
+      if (tid == 0 && nxt.ok) {  // q, k and g are dead (v is read until the U read-out)
+        arm_tma(nxt);
+        issue_tma_qk(nxt);
+        issue_tma_g(nxt);
       }
     }
 

@@ -282,6 +282,17 @@ __host__ __device__ constexpr uint32_t idesc_fp16(int M, int N, bool a_mn_major,
   return idesc_f16kind(M, N, a_mn_major, b_mn_major, false);
 }
 
+// Instruction descriptor: kind::tf32 (fp32 operands read as tf32), fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                 // D format: f32
+         | (2u << 7)                               // A format: tf32
+         | (2u << 10)                              // B format: tf32
+         | ((a_mn_major ? 1u : 0u) << 15)          // A major
+         | ((b_mn_major ? 1u : 0u) << 16)          // B major
+         | ((uint32_t)(N >> 3) << 17)              // N / 8
+         | ((uint32_t)(M >> 4) << 24);             // M / 16
+}
+
 // Shared-memory matrix descriptor for a SWIZZLE_128B operand.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -314,6 +325,25 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// One thread: D[tmem] (+)= A * B^T for one K=8 step of tf32 operands (32 bytes of K, the
+// same byte step as a K=16 step of 16-bit operands).
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// fp32 rounded to the nearest tf32 (10-bit significand), as the fp32 bit pattern.
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
 // One thread: arrive once on `bar` when all previously issued MMAs complete.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile(
@@ -326,7 +356,8 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // Operand tile addressing (byte offsets inside a tile)
 // ---------------------------------------------------------------------------
 
-// K-major: 16-byte chunk holding columns [8*c8, 8*c8+8) of `row`.
+// K-major: 16-byte chunk c8 of `row` (columns [8*c8, 8*c8+8) of a 16-bit tile, or
+// [4*c8, 4*c8+4) of a 32-bit one).
 __device__ __forceinline__ uint32_t kmaj_off(int rows, int row, int c8) {
   return (uint32_t)((c8 >> 3) * rows * 128 + row * 128 + (((c8 & 7) ^ (row & 7)) << 4));
 }
