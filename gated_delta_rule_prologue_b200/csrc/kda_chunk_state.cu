@@ -40,17 +40,16 @@ constexpr uint32_t SB_P = 49152;
 constexpr uint32_t SB_A2 = SB_P - 8192;  // A operand [* ; P]: rows 0..63 overlay the tail of
                                          // K' (finite fp16 values whose products land in
                                          // accumulator rows that are never read again)
-constexpr uint32_t SB_S = 57344;         // S slice operand (K-major 32 x 128) 8 KB; between the
-                                         // two MMA groups: <q_r, k_r> U exchange [32][64] f32
-constexpr uint32_t SB_U = 65536;         // U operand (K-major 32 x 64)             4 KB
+constexpr uint32_t SB_S = 57344;         // S slice operand (value-contiguous, 128 key rows x 64 B,
+                                         // 64-byte swizzle) 8 KB; between the two MMA groups:
+                                         // <q_r, k_r> U exchange [32][64] f32
+constexpr uint32_t SB_U = 65536;         // U operand (value-contiguous, 64 token rows x 64 B) 4 KB
 constexpr uint32_t SB_BAR = 69632;       // three mbarriers, TMEM slot
 constexpr uint32_t SB_ALLOC = SB_BAR + 64 + 1024;
-constexpr uint32_t TB_D1 = 0, TB_D2 = 32, TB_COLS = 64;
+// D1 is accumulated as two halves over the key channels (two independent MMA
+// chains), summed at read-out; D2 = K'^T U.
+constexpr uint32_t TB_D1 = 0, TB_D1B = 32, TB_D2 = 64, TB_COLS = 128;
 static_assert(SB_KP + 24576 == SB_S, "K' and P are adjacent");
-
-__device__ __forceinline__ void st_half(uint8_t *tile, uint32_t chunk_off, int e, float x) {
-  reinterpret_cast<__half *>(tile + chunk_off)[e] = __float2half_rn(x);
-}
 
 __global__ void __launch_bounds__(kBT, 3)
 chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
@@ -91,12 +90,17 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 #pragma unroll
   for (int i = 0; i < 32; ++i) S[i] = s0 ? s0[sbase + (size_t)i * 128] : 0.f;
 
-  auto write_s_operand = [&]() {  // S slice as the K-major B operand: row = value, col = key
+  auto write_s_operand = [&]() {  // S slice as the B operand: key row t, 32 values
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      amax = fmaxf(amax, fabsf(S[i]));
-      st_half(sm + SB_S, kmaj_off(32, i, t >> 3), t & 7, S[i]);
+    for (int x = 0; x < 4; ++x) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        f[e] = S[8 * x + e];
+        amax = fmaxf(amax, fabsf(f[e]));
+      }
+      st_shared_16(sm + SB_S, mn32_sw64_off(t, x), pack8_f16(f));
     }
     if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
   };
@@ -157,10 +161,13 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     if (tid == 0) {
       tc_fence_after();
       const uint32_t a1 = smem_u32(sm + SB_A1), sop = smem_u32(sm + SB_S);
-      constexpr uint32_t id = idesc_fp16(128, 32, false, false);
+      constexpr uint32_t id = idesc_fp16(128, 32, false, true);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_bf16(tmem + TB_D1, desc_kmajor(a1, 128, ks), desc_kmajor(sop, 32, ks), id, ks > 0);
+      for (int ks = 0; ks < 4; ++ks) {  // key channels [0, 64) into D1, [64, 128) into D1B
+        mma_bf16(tmem + TB_D1, desc_kmajor(a1, 128, ks), desc_mn32_sw64(sop, ks), id, ks > 0);
+        mma_bf16(tmem + TB_D1B, desc_kmajor(a1, 128, ks + 4), desc_mn32_sw64(sop, ks + 4), id,
+                 ks > 0);
+      }
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, pm, status)) break;
@@ -170,16 +177,24 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 
     // ---- U = Ut - W S (warps 0-1: TMEM lanes 0..63 are the chunk's tokens) -------------
     if (warp < 2) {
-      float y[32];
-      tmem_ld32(tmem + lane_addr + TB_D1, y);
+      float y[32], y2[32];
+      tmem_ld32_nowait(tmem + lane_addr + TB_D1, y);
+      tmem_ld32_nowait(tmem + lane_addr + TB_D1B, y2);
+      tmem_wait_ld(y, y2);
       const int r = tid;
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float u = ut[i] - y[i];
-        amax = fmaxf(amax, fabsf(u));
-        st_half(sm + SB_U, kmaj_off(32, i, r >> 3), r & 7, u);
-        exch[i * 64 + r] = pd * u;  // the S operand is dead until the next chunk
+        y[i] = ut[i] - (y[i] + y2[i]);  // U
+        amax = fmaxf(amax, fabsf(y[i]));
+        exch[i * 64 + r] = pd * y[i];  // the S operand is dead until the next chunk
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = y[8 * x + e];
+        st_shared_16(sm + SB_U, mn32_sw64_off(r, x), pack8_f16(f));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
       if (c + 1 < nch) fetch_u(c + 1);
@@ -194,12 +209,12 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       tc_fence_after();
       const uint32_t a2 = smem_u32(sm + SB_A2), uop = smem_u32(sm + SB_U);
       const uint32_t kp = smem_u32(sm + SB_KP);
-      constexpr uint32_t idO = idesc_fp16(128, 32, false, false);
-      constexpr uint32_t idS = idesc_fp16(128, 32, true, false);
+      constexpr uint32_t idO = idesc_fp16(128, 32, false, true);
+      constexpr uint32_t idS = idesc_fp16(128, 32, true, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {  // the two accumulators' steps interleaved
-        mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_kmajor(uop, 32, ks), idO, 1);
-        mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_kmajor(uop, 32, ks), idS, ks > 0);
+        mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_mn32_sw64(uop, ks), idO, 1);
+        mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_mn32_sw64(uop, ks), idS, ks > 0);
       }
       mma_commit(bar_mma);
     }
@@ -217,8 +232,12 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       if (c + 1 < nch) fetch_gl(c + 1);
     }
     if (warp >= 2) {
-      float ov[32];
-      tmem_ld32(tmem + lane_addr + TB_D1, ov);
+      float ov[32], ov2[32];
+      tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
+      tmem_ld32_nowait(tmem + lane_addr + TB_D1B, ov2);
+      tmem_wait_ld(ov, ov2);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ov[i] += ov2[i];
       const int r = tid - 64;
       if (r < Lc) {
         float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * 128 + slice * 32);

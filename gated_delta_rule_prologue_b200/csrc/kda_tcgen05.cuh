@@ -304,6 +304,29 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
   return d;
 }
 
+// Shared-memory matrix descriptor for a SWIZZLE_64B MN-major operand of 32
+// 16-bit MN-elements (one 64-byte swizzle atom wide): K-row stride 64 B,
+// 8-row group stride (SBO) 512 B.  Element (mn, k) lives at
+//   k*64 + (((mn/8) ^ ((k/2) % 4)) * 16) + (mn%8)*2
+// (the XOR of byte-address bits [4,6) with [7,9), on 512-byte aligned tiles).
+// Descriptor of K-step ks (16 K-rows).
+__device__ __forceinline__ uint64_t desc_mn32_sw64(uint32_t tile, int ks) {
+  const uint32_t saddr = tile + (uint32_t)(ks * 1024);
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((512u >> 4) & 0x3FFFu) << 16;   // LBO: next 32-element atom; unused at N=32
+                                                   // (kept small so the tile's reads stay inside it)
+  d |= (uint64_t)((512u >> 4) & 0x3FFFu) << 32;   // SBO: 8 K-rows
+  d |= (uint64_t)1 << 46;                          // descriptor version (sm_100)
+  d |= (uint64_t)4 << 61;                          // SWIZZLE_64B
+  return d;
+}
+
+// Byte offset of the 16-byte chunk c (MN-elements [8c, 8c+8)) of K-row k in such a tile.
+__device__ __forceinline__ uint32_t mn32_sw64_off(int k, int c) {
+  return (uint32_t)(k * 64 + ((c ^ ((k >> 1) & 3)) << 4));
+}
+
 // K-major tile of `rows` rows: descriptor of K-step ks (16 bf16 columns).
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int rows, int ks) {
   return sdesc(tile + (uint32_t)((ks >> 2) * rows * 128 + (ks & 3) * 32), 16, 1024);
