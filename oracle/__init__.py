@@ -10,6 +10,7 @@ chunkwise evaluator is pinned against the recurrence.
 """
 from .kda_oracle import (  # noqa: F401
     L2_EPS,
+    gate,
     kda_chunkwise,
     kda_decode_step,
     kda_recurrent,

@@ -10,7 +10,8 @@ Sources (web pages; cited as [Wn section]):
   [W1] "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆" (yeyulingfeng.com) --
        the stations 第二站 (short conv, SiLU, L2), 第三站 (per-channel decay),
        第四站 (delta-rule write; naive_recurrent_kda excerpt), 第五站 (read
-       after write; query scale), 彩蛋 (chunked execution; bounded gate).
+       after write; query scale), 彩蛋 (chunked execution; bounded gate, the
+       gate.py excerpt).
   [W3] "Kimi K3 记忆架构总览：KDA、MLA、AttnRes 各管什么" (moonzj.com),
        section "KDA 谱系速查" (delta-rule pseudocode, reparameterisation).
   [W4] "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解"
@@ -125,6 +126,30 @@ def prologue(x, w, H, D, cu_seqlens=None, cache_in=None):
 # ---------------------------------------------------------------------------
 # The recurrence (definition)
 # ---------------------------------------------------------------------------
+
+def gate(g_raw, A_log=None, dt_bias=None, lower_bound=-5.0):
+    """Bounded log-decay from the gate pre-activations ([W1 彩蛋], the excerpt of
+    FLA's gate.py): add the per-(head, channel) bias, multiply by exp(A_log) of
+    the head, squash with a sigmoid and scale by the lower bound (-5 in K3):
+
+        g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h, :]))
+
+    so g lies in (lower_bound, 0) and alpha = exp(g) in (exp(lower_bound), 1).
+    Either parameter may be None (the excerpt skips it then).
+
+    g_raw [..., H, D]; A_log [H]; dt_bias [H, D].  Returns float64 g of g_raw's
+    shape.
+    """
+    z = _f64(g_raw)
+    if dt_bias is not None:
+        z = z + _f64(dt_bias)
+    if A_log is not None:
+        z = np.exp(_f64(A_log))[:, None] * z
+    # sigmoid in the form that never overflows: exp of a non-positive number only
+    e = np.exp(-np.abs(z))
+    sig = np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return float(lower_bound) * sig
+
 
 def kda_recurrent(q, k, v, g, beta, scale=1.0, initial_state=None, cu_seqlens=None):
     """Token-by-token KDA recurrence, all heads at once.
