@@ -78,6 +78,14 @@ lib.kda_chunk_fwd_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, 
                                      _i, _i, _vp, _vp, _vp]
 lib.kda_prologue_chunk_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i,
                                           _i, _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.kda_chunk_fwd_gated_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _f, _vp, _vp, _i,
+                                       _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, ctypes.c_size_t,
+                                       _vp]
+lib.kda_prologue_chunk_fwd_gated_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _f,
+                                                _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                                ctypes.c_size_t, _vp]
+lib.kda_decode_step_gated.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _f, _vp, _i, _i, _i,
+                                      _i, _vp, _vp]
 lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
@@ -85,7 +93,8 @@ lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _v
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
-            lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step,
+            lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
+            lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
@@ -276,3 +285,78 @@ def kda_decode_step(x, conv_w, conv_cache, g, beta, state, o, *, H: int, D: int,
     _check(lib.kda_decode_step(_ptr(x), _ptr(conv_w), _ptr(conv_cache), _ptr(g), _ptr(beta),
                                float(scale), _ptr(state), N, H, D, _dtype(x), _ptr(o),
                                _stream(stream)))
+
+
+def _auto_workspace(workspace, N, T, H, D, dtype, device):
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dtype)
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8)
+    return workspace
+
+
+def kda_chunk_fwd_gated(q, k, v, g_raw, beta, o, *, A_log=None, dt_bias=None,
+                        lower_bound: float = -5.0, scale: float = 1.0, initial_state=None,
+                        final_state=None, cu_seqlens=None, chunk: int = 64, workspace="auto",
+                        stream=None):
+    """Two-pass prefill with the log-decay computed in the kernel from the gate
+    pre-activations ``g_raw`` [T, H, Dk] (q's dtype):
+    g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h, :]))."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g_raw, "g_raw")):
+        _need(t, n, q.dtype)
+    for t, n in ((o, "o"), (beta, "beta"), (A_log, "A_log"), (dt_bias, "dt_bias"),
+                 (initial_state, "initial_state"), (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    workspace = _auto_workspace(workspace, N, T, H, Dk, q.dtype, q.device)
+    _check(lib.kda_chunk_fwd_gated_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(A_log),
+                                      _ptr(dt_bias), float(lower_bound), _ptr(beta), float(scale),
+                                      _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv,
+                                      chunk, _dtype(q), _ptr(o), _ptr(final_state),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def kda_prologue_chunk_fwd_gated(x, conv_w, g_raw, beta, o, *, H: int, D: int, A_log=None,
+                                 dt_bias=None, lower_bound: float = -5.0, scale: float = 1.0,
+                                 cache_in=None, cache_out=None, initial_state=None,
+                                 final_state=None, cu_seqlens=None, workspace="auto",
+                                 stream=None):
+    """Fused two-pass prefill (prologue in the prep pass) with the in-kernel gate."""
+    for t, n in ((x, "x"), (g_raw, "g_raw"), (cache_in, "cache_in"), (cache_out, "cache_out")):
+        _need(t, n, x.dtype)
+    for t, n in ((conv_w, "conv_w"), (o, "o"), (beta, "beta"), (A_log, "A_log"),
+                 (dt_bias, "dt_bias"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    T = x.shape[0]
+    workspace = _auto_workspace(workspace, N, T, H, D, x.dtype, x.device)
+    _check(lib.kda_prologue_chunk_fwd_gated_ws(_ptr(x), _ptr(conv_w), _ptr(cache_in),
+                                               _ptr(cache_out), _ptr(g_raw), _ptr(A_log),
+                                               _ptr(dt_bias), float(lower_bound), _ptr(beta),
+                                               float(scale), _ptr(initial_state),
+                                               _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
+                                               _ptr(final_state), _ptr(workspace),
+                                               workspace.numel(), _stream(stream)))
+
+
+def kda_decode_step_gated(x, conv_w, conv_cache, g_raw, beta, state, o, *, H: int, D: int,
+                          A_log=None, dt_bias=None, lower_bound: float = -5.0,
+                          scale: float = 1.0, stream=None):
+    """Decode step with the in-kernel gate; ``g_raw`` [N, H, D] of x's dtype."""
+    for t, n in ((x, "x"), (conv_cache, "conv_cache"), (g_raw, "g_raw")):
+        _need(t, n, x.dtype)
+    for t, n in ((o, "o"), (conv_w, "conv_w"), (beta, "beta"), (state, "state"),
+                 (A_log, "A_log"), (dt_bias, "dt_bias")):
+        _need(t, n, torch.float32)
+    N = x.shape[0]
+    _check(lib.kda_decode_step_gated(_ptr(x), _ptr(conv_w), _ptr(conv_cache), _ptr(g_raw),
+                                     _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(beta),
+                                     float(scale), _ptr(state), N, H, D, _dtype(x), _ptr(o),
+                                     _stream(stream)))

@@ -193,10 +193,11 @@ bool chunk_tc_path(int T, int Dk, int Dv, int chunk, kda_dtype dt) {
 }
 
 // Argument checks shared by kda_chunk_fwd and kda_chunk_fwd_ws.
-kda_status check_chunk_args(const void *q, const void *k, const void *v, const float *g,
+kda_status check_chunk_args(const void *q, const void *k, const void *v, const void *g,
                             const float *beta, const float *initial_state,
                             const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
-                            int chunk, kda_dtype dt, float *o, float *final_state) {
+                            int chunk, kda_dtype dt, float *o, float *final_state,
+                            size_t g_elem_bytes = 4) {
   KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
   KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1 && Dk >= 1 && Dv >= 1,
               "bad sizes N=%d T=%d H=%d Dk=%d Dv=%d", N, T, H, Dk, Dv);
@@ -221,7 +222,7 @@ kda_status check_chunk_args(const void *q, const void *k, const void *v, const f
   const size_t act = (size_t)T * H * Dk * es, obytes = (size_t)T * H * Dv * sizeof(float);
   const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
   const void *ins[5] = {q, k, v, g, beta};
-  const size_t insz[5] = {act, act, (size_t)T * H * Dv * es, (size_t)T * H * Dk * 4,
+  const size_t insz[5] = {act, act, (size_t)T * H * Dv * es, (size_t)T * H * Dk * g_elem_bytes,
                           (size_t)T * H * 4};
   for (int i = 0; i < 5; ++i)
     KDA_REQUIRE(!overlaps(o, obytes, ins[i], insz[i]), "o overlaps an input");
@@ -229,6 +230,21 @@ kda_status check_chunk_args(const void *q, const void *k, const void *v, const f
   KDA_REQUIRE(final_state == initial_state ||
                   !overlaps(final_state, sbytes, initial_state, sbytes),
               "final_state partially overlaps initial_state");
+  return KDA_OK;
+}
+
+// Gate parameters of the *_gated entry points.  The chunk kernels need
+// g >= -5 (their decay-range argument), so their lower bound is in [-5, 0).
+kda_status check_gate_args(const float *A_log, const float *dt_bias, float lower_bound,
+                           bool chunk_path) {
+  KDA_REQUIRE(lower_bound == lower_bound && lower_bound < 0.f && lower_bound > -1e30f,
+              "lower_bound must be finite and negative (got %g)", (double)lower_bound);
+  if (chunk_path && lower_bound < -5.f)
+    return fail(KDA_ERR_UNSUPPORTED,
+                "gated chunk path: lower_bound %g < -5 is outside the decay range the tensor-core "
+                "kernels are built for", (double)lower_bound);
+  KDA_OPT_PTR4(A_log, "A_log");
+  KDA_OPT_PTR(dt_bias, "dt_bias");
   return KDA_OK;
 }
 
@@ -266,6 +282,56 @@ size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int ch
   return kda::rec::workspace_bytes(N, T, H);
 }
 
+}  // extern "C"
+
+namespace {
+
+// The two-pass tensor-core prefill on a caller workspace, with g either the
+// fp32 log-decay or (gated) 16-bit gate pre-activations.  Arguments other than
+// the workspace have been checked.
+kda_status chunk_two_pass(const void *q, const void *k, const void *v, const void *g,
+                          size_t g_elem_bytes, const float *A_log, const float *dt_bias,
+                          float lower_bound, bool gated, const float *beta, float scale,
+                          const float *initial_state, const int32_t *cu_seqlens, int N, int T,
+                          int H, int Dk, int Dv, kda_dtype dt, float *o, float *final_state,
+                          void *workspace, size_t workspace_bytes, cudaStream_t s,
+                          const char *what) {
+  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, 64, dt);
+  KDA_OPT_PTR(workspace, "workspace");
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {
+    const size_t es = esize(dt), act = (size_t)T * H * Dk * es;
+    const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
+    const void *others[10] = {q, k, v, g, beta, o, initial_state, final_state, A_log, dt_bias};
+    const size_t osz[10] = {act, act, act, (size_t)T * H * Dk * g_elem_bytes, (size_t)T * H * 4,
+                            (size_t)T * H * Dv * 4, sbytes, sbytes, (size_t)H * 4,
+                            (size_t)H * Dk * 4};
+    for (int i = 0; i < 10; ++i)
+      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
+                  "workspace overlaps another argument");
+    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
+                "workspace overlaps cu_seqlens");
+  }
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, A_log,
+                               dt_bias, lower_bound, gated, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+                                final_state, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, float scale, const float *initial_state,
                             const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
@@ -277,38 +343,34 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
   kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
                                    chunk, dt, o, final_state);
   if (st != KDA_OK) return st;
-  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, dt);
-  if (need == 0)
+  if (kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, dt) == 0)
     return kda_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk, Dv,
                          chunk, dt, o, final_state, stream);
-  KDA_OPT_PTR(workspace, "workspace");
-  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
-              workspace_bytes, need);
-  {
-    const size_t es = esize(dt), act = (size_t)T * H * Dk * es;
-    const size_t sbytes = (size_t)N * H * Dv * Dk * sizeof(float);
-    const void *others[8] = {q, k, v, g, beta, o, initial_state, final_state};
-    const size_t osz[8] = {act, act, act, (size_t)T * H * Dk * 4, (size_t)T * H * 4,
-                           (size_t)T * H * Dv * 4, sbytes, sbytes};
-    for (int i = 0; i < 8; ++i)
-      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
-                  "workspace overlaps another argument");
-    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
-                "workspace overlaps cu_seqlens");
-  }
-  int *status = nullptr;
-  st = device_status_word(&status);
+  return chunk_two_pass(q, k, v, g, 4, nullptr, nullptr, 0.f, false, beta, scale, initial_state,
+                        cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, workspace,
+                        workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_ws launch");
+}
+
+kda_status kda_chunk_fwd_gated_ws(const void *q, const void *k, const void *v, const void *g_raw,
+                                  const float *A_log, const float *dt_bias, float lower_bound,
+                                  const float *beta, float scale, const float *initial_state,
+                                  const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                                  int chunk, kda_dtype dt, float *o, float *final_state,
+                                  void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_chunk_args(q, k, v, g_raw, beta, initial_state, cu_seqlens, N, T, H, Dk,
+                                   Dv, chunk, dt, o, final_state, esize(dt));
   if (st != KDA_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaSuccess;
-  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
-                                final_state, status, s);
-  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_ws launch");
-  return KDA_OK;
+  if (!chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_fwd_gated: needs bf16/f16, Dk == Dv == 128, chunk 64 "
+                                     "and T > 0 (got dt=%d Dk=%d chunk=%d T=%d)",
+                (int)dt, Dk, chunk, T);
+  st = check_gate_args(A_log, dt_bias, lower_bound, true);
+  if (st != KDA_OK) return st;
+  KDA_REQUIRE(workspace != nullptr, "chunk_fwd_gated: workspace is NULL");
+  return chunk_two_pass(q, k, v, g_raw, esize(dt), A_log, dt_bias, lower_bound, true, beta, scale,
+                        initial_state, cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state,
+                        workspace, workspace_bytes, (cudaStream_t)stream,
+                        "kda_chunk_fwd_gated_ws launch");
 }
 
 kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, const float *g,
@@ -338,7 +400,8 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
   cudaError_t e = cudaSuccess;
   if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, scratch, status, s);
   if (e == cudaSuccess)
-    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, scratch, status, s);
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, scratch, nullptr,
+                               nullptr, 0.f, false, status, s);
   if (e == cudaSuccess)
     e = kda::launch_chunk_state(scratch, cu_seqlens, initial_state, scale, N, T, H, o,
                                 final_state, status, s);
@@ -351,9 +414,10 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
 namespace {
 
 kda_status check_fused_args(const void *x, const float *conv_w, const void *cache_in,
-                            void *cache_out, const float *g, const float *beta,
+                            void *cache_out, const void *g, const float *beta,
                             const float *initial_state, const int32_t *cu_seqlens, int N, int T,
-                            int H, int D, kda_dtype dt, float *o, float *final_state) {
+                            int H, int D, kda_dtype dt, float *o, float *final_state,
+                            size_t g_elem_bytes = 4) {
   KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
   KDA_REQUIRE(N >= 1 && T >= 1 && H >= 1 && D >= 1, "bad sizes N=%d T=%d H=%d D=%d", N, T, H, D);
   KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
@@ -375,7 +439,7 @@ kda_status check_fused_args(const void *x, const float *conv_w, const void *cach
   const size_t sbytes = (size_t)N * H * D * D * sizeof(float);
   const size_t cache_bytes = (size_t)N * 3 * C * es;
   KDA_REQUIRE(!overlaps(o, obytes, x, (size_t)T * C * es), "o overlaps x");
-  KDA_REQUIRE(!overlaps(o, obytes, g, (size_t)T * H * D * 4), "o overlaps g");
+  KDA_REQUIRE(!overlaps(o, obytes, g, (size_t)T * H * D * g_elem_bytes), "o overlaps g");
   KDA_REQUIRE(!overlaps(o, obytes, beta, (size_t)T * H * 4), "o overlaps beta");
   KDA_REQUIRE(!overlaps(o, obytes, final_state, sbytes), "o overlaps final_state");
   KDA_REQUIRE(!overlaps(cache_in, cache_bytes, cache_out, cache_bytes),
@@ -409,6 +473,59 @@ kda_status kda_prologue_chunk_fwd(const void *x, const float *conv_w, const void
   return KDA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The two-pass prefill with the prologue in the prep pass (see chunk_two_pass).
+kda_status fused_two_pass(const void *x, const float *conv_w, const void *cache_in,
+                          void *cache_out, const void *g, size_t g_elem_bytes,
+                          const float *A_log, const float *dt_bias, float lower_bound, bool gated,
+                          const float *beta, float scale, const float *initial_state,
+                          const int32_t *cu_seqlens, int N, int T, int H, int D, kda_dtype dt,
+                          float *o, float *final_state, void *workspace, size_t workspace_bytes,
+                          cudaStream_t s, const char *what) {
+  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt);
+  KDA_OPT_PTR(workspace, "workspace");
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {
+    const size_t C = (size_t)3 * H * D, es = esize(dt);
+    const size_t sbytes = (size_t)N * H * D * D * sizeof(float);
+    const void *others[11] = {x, conv_w, cache_in, cache_out, g, beta, o, initial_state,
+                              final_state, A_log, dt_bias};
+    const size_t osz[11] = {(size_t)T * C * es, C * 4 * 4, (size_t)N * 3 * C * es,
+                            (size_t)N * 3 * C * es, (size_t)T * H * D * g_elem_bytes,
+                            (size_t)T * H * 4, (size_t)T * H * D * 4, sbytes, sbytes,
+                            (size_t)H * 4, (size_t)H * D * 4};
+    for (int i = 0; i < 11; ++i)
+      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
+                  "workspace overlaps another argument");
+    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
+                "workspace overlaps cu_seqlens");
+  }
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N, T,
+                                        H, dt, workspace, A_log, dt_bias, lower_bound, gated,
+                                        status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+                                final_state, status, s);
+  if (e == cudaSuccess && cu_seqlens && cache_out)
+    e = kda::launch_cache_pass(workspace, N, H, cache_in, cache_out, s);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const void *cache_in,
                                      void *cache_out, const float *g, const float *beta,
                                      float scale, const float *initial_state,
@@ -422,45 +539,43 @@ kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const v
   kda_status st = check_fused_args(x, conv_w, cache_in, cache_out, g, beta, initial_state,
                                    cu_seqlens, N, T, H, D, dt, o, final_state);
   if (st != KDA_OK) return st;
-  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt);
-  KDA_OPT_PTR(workspace, "workspace");
-  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
-              workspace_bytes, need);
-  {
-    const size_t C = (size_t)3 * H * D, es = esize(dt);
-    const size_t sbytes = (size_t)N * H * D * D * sizeof(float);
-    const void *others[9] = {x, conv_w, cache_in, cache_out, g, beta, o, initial_state,
-                             final_state};
-    const size_t osz[9] = {(size_t)T * C * es, C * 4 * 4, (size_t)N * 3 * C * es,
-                           (size_t)N * 3 * C * es, (size_t)T * H * D * 4, (size_t)T * H * 4,
-                           (size_t)T * H * D * 4, sbytes, sbytes};
-    for (int i = 0; i < 9; ++i)
-      KDA_REQUIRE(!overlaps(workspace, need, others[i], osz[i]),
-                  "workspace overlaps another argument");
-    KDA_REQUIRE(!overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * 4),
-                "workspace overlaps cu_seqlens");
-  }
-  int *status = nullptr;
-  st = device_status_word(&status);
-  if (st != KDA_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaSuccess;
-  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N, T,
-                                        H, dt, workspace, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
-                                final_state, status, s);
-  if (e == cudaSuccess && cu_seqlens && cache_out)
-    e = kda::launch_cache_pass(workspace, N, H, cache_in, cache_out, s);
-  if (e != cudaSuccess) return cuda_fail(e, "kda_prologue_chunk_fwd_ws launch");
-  return KDA_OK;
+  return fused_two_pass(x, conv_w, cache_in, cache_out, g, 4, nullptr, nullptr, 0.f, false, beta,
+                        scale, initial_state, cu_seqlens, N, T, H, D, dt, o, final_state,
+                        workspace, workspace_bytes, (cudaStream_t)stream,
+                        "kda_prologue_chunk_fwd_ws launch");
 }
 
-kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache, const float *g,
-                           const float *beta, float scale, float *state, int N, int H, int D,
-                           kda_dtype dt, float *o, kda_stream_t stream) {
+kda_status kda_prologue_chunk_fwd_gated_ws(const void *x, const float *conv_w,
+                                           const void *cache_in, void *cache_out,
+                                           const void *g_raw, const float *A_log,
+                                           const float *dt_bias, float lower_bound,
+                                           const float *beta, float scale,
+                                           const float *initial_state,
+                                           const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                           kda_dtype dt, float *o, float *final_state,
+                                           void *workspace, size_t workspace_bytes,
+                                           kda_stream_t stream) {
+  kda_status st = check_fused_args(x, conv_w, cache_in, cache_out, g_raw, beta, initial_state,
+                                   cu_seqlens, N, T, H, D, dt, o, final_state, esize(dt));
+  if (st != KDA_OK) return st;
+  st = check_gate_args(A_log, dt_bias, lower_bound, true);
+  if (st != KDA_OK) return st;
+  KDA_REQUIRE(workspace != nullptr, "prologue_chunk_fwd_gated: workspace is NULL");
+  return fused_two_pass(x, conv_w, cache_in, cache_out, g_raw, esize(dt), A_log, dt_bias,
+                        lower_bound, true, beta, scale, initial_state, cu_seqlens, N, T, H, D, dt,
+                        o, final_state, workspace, workspace_bytes, (cudaStream_t)stream,
+                        "kda_prologue_chunk_fwd_gated_ws launch");
+}
+
+}  // extern "C"
+
+namespace {
+
+kda_status decode_step(const void *x, const float *conv_w, void *conv_cache, const void *g,
+                       size_t g_elem_bytes, const float *A_log, const float *dt_bias,
+                       float lower_bound, bool gated, const float *beta, float scale,
+                       float *state, int N, int H, int D, kda_dtype dt, float *o,
+                       kda_stream_t stream, const char *what) {
   KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
   KDA_REQUIRE(N >= 0 && H >= 1 && D >= 1, "bad sizes N=%d H=%d D=%d", N, H, D);
   if (!supported_d(D)) return fail(KDA_ERR_UNSUPPORTED, "decode: D=%d not in {16,32,64,128}", D);
@@ -472,20 +587,47 @@ kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache,
   KDA_REQUIRE_PTR4(beta, "beta");
   KDA_REQUIRE_PTR(state, "state");
   KDA_REQUIRE_PTR(o, "o");
+  if (gated && g_elem_bytes == 2)  // 4 pre-activations per lane: 8-byte loads
+    KDA_REQUIRE((reinterpret_cast<uintptr_t>(g) & 7u) == 0, "g is not 8-byte aligned");
   const size_t es = esize(dt), C = (size_t)3 * H * D;
   const size_t obytes = (size_t)N * H * D * sizeof(float), sbytes = (size_t)N * H * D * D * 4;
   KDA_REQUIRE(!overlaps(o, obytes, state, sbytes), "o overlaps state");
   KDA_REQUIRE(!overlaps(o, obytes, conv_cache, (size_t)N * 3 * C * es), "o overlaps conv_cache");
   KDA_REQUIRE(!overlaps(o, obytes, x, (size_t)N * C * es), "o overlaps x");
+  KDA_REQUIRE(!overlaps(o, obytes, g, (size_t)N * H * D * g_elem_bytes), "o overlaps g");
   KDA_REQUIRE(!overlaps(state, sbytes, conv_cache, (size_t)N * 3 * C * es),
               "state overlaps conv_cache");
   int *status = nullptr;
   kda_status st = device_status_word(&status);
   if (st != KDA_OK) return st;
   cudaError_t e = kda::launch_decode(x, conv_w, conv_cache, g, beta, scale, state, N, H, D, dt, o,
-                                     status, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
+                                     A_log, dt_bias, lower_bound, gated, status,
+                                     (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, what);
   return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache, const float *g,
+                           const float *beta, float scale, float *state, int N, int H, int D,
+                           kda_dtype dt, float *o, kda_stream_t stream) {
+  return decode_step(x, conv_w, conv_cache, g, 4, nullptr, nullptr, 0.f, false, beta, scale,
+                     state, N, H, D, dt, o, stream, "kda_decode_step launch");
+}
+
+kda_status kda_decode_step_gated(const void *x, const float *conv_w, void *conv_cache,
+                                 const void *g_raw, const float *A_log, const float *dt_bias,
+                                 float lower_bound, const float *beta, float scale, float *state,
+                                 int N, int H, int D, kda_dtype dt, float *o,
+                                 kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  kda_status st = check_gate_args(A_log, dt_bias, lower_bound, false);
+  if (st != KDA_OK) return st;
+  return decode_step(x, conv_w, conv_cache, g_raw, esize(dt), A_log, dt_bias, lower_bound, true,
+                     beta, scale, state, N, H, D, dt, o, stream, "kda_decode_step_gated launch");
 }
 
 }  // extern "C"

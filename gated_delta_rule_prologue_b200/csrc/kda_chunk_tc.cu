@@ -119,7 +119,6 @@ constexpr uint32_t TM_O = 288;   // O^T, 64
 constexpr uint32_t TM_S = 352;   // delta S^T, 128
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t kTmaBytes = 3 * 16384 + 32768;
 constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
 
@@ -195,11 +194,24 @@ __device__ __forceinline__ uint4 pack8_in(const float (&f)[8]) {
 //            item brings its own conv history (the three rows before the
 //            chunk, or the cache at a sequence start), and the item holding a
 //            sequence's last chunk writes that sequence's cache.
+//   kPrepGated, kPrepFusedGated: kPrep / kPrepFused with the log-decay
+//            computed from gate pre-activations in the cumsum phase (GateArgs).
 //
 // Thread layout (512 threads, 16 warps): warp w reads TMEM lanes
 // 32*(w%4).. (its "quad") and handles column group w/4 of every accumulator it
 // reads; element-wise phases walk (row, 8-channel chunk) pairs.
-constexpr int kSingle = 0, kFusedMode = 1, kPrep = 2, kPrepFused = 3;
+constexpr int kSingle = 0, kFusedMode = 1, kPrep = 2, kPrepFused = 3, kPrepGated = 4,
+              kPrepFusedGated = 5;
+
+// Parameters of the in-kernel bounded gate (the gated prep modes): the g tile
+// holds the gate pre-activations (16-bit, like q/k/v or x) and
+// g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h, :])); either
+// pointer may be null (exp(A_log) = 1, dt_bias = 0).
+struct GateArgs {
+  const float *A_log;
+  const float *dt_bias;
+  float lower_bound;
+};
 
 template <typename Tin, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -208,9 +220,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float *__restrict__ beta, float scale, const float *s0,
                 const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
                 int *status, const float *__restrict__ conv_w, const Tin *cache_in,
-                Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N) {
-  constexpr bool kFused = kMode == kFusedMode || kMode == kPrepFused;
-  constexpr bool kPrepM = kMode == kPrep || kMode == kPrepFused;
+                Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N, GateArgs gate) {
+  constexpr bool kFused = kMode == kFusedMode || kMode == kPrepFused || kMode == kPrepFusedGated;
+  constexpr bool kGated = kMode == kPrepGated || kMode == kPrepFusedGated;
+  constexpr bool kPrepM = kMode == kPrep || kMode == kPrepFused || kGated;
+  // bytes of one work item's q, k, v (or x) tiles and its g tile (fp32 log-decay,
+  // or 16-bit gate pre-activations)
+  constexpr uint32_t kTileBytes = 3 * 16384 + (kGated ? 16384u : 32768u);
   // Element type of the q/k/v tiles the chunk phases read: the inputs as given,
   // or fp16 written by the fused prologue (q, k are unit vectors; v is guarded).
   using Tact = typename std::conditional<kFused, __half, Tin>::type;
@@ -327,9 +343,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // their total at the item's first issue (the tiles go out as buffers die).
   // kPrepFused: a chunk that does not start its sequence also brings the three
   // raw rows before it (its conv history) into history slot 0.
-  auto has_halo = [&](const Work &w) { return kMode == kPrepFused && w.t0 > w.bos; };
+  auto has_halo = [&](const Work &w) {
+    return (kMode == kPrepFused || kMode == kPrepFusedGated) && w.t0 > w.bos;
+  };
   auto arm_tma = [&](const Work &w) {
-    mbar_arrive_expect_tx(bar_tma, kTmaBytes + (has_halo(w) ? kHaloBytes : 0u));
+    mbar_arrive_expect_tx(bar_tma, kTileBytes + (has_halo(w) ? kHaloBytes : 0u));
   };
   auto issue_tma_qk = [&](const Work &w) {
     if constexpr (kFused) {  // x viewed as [T, 3H, 128]: part p of head h is row p*H + h
@@ -388,13 +406,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // per thread), fetched one item ahead and stored tap-major at the item start
   float wnext[3] = {0.f, 0.f, 0.f};
   auto fetch_w = [&](const Work &w) {
-    if constexpr (kMode == kPrepFused) {
+    if constexpr (kPrepM && kFused) {
 #pragma unroll
       for (int m = 0; m < 3; ++m)
         wnext[m] = __ldg(conv_w + (size_t)m * HD * 4 + (size_t)w.h * 512 + tid);
     }
   };
   if (cur.ok) fetch_w(cur);
+  // gated modes: the item's exp(A_log[h]) and dt_bias[h][tid % 128], one item ahead
+  float ga_next = 1.f, gb_next = 0.f, ga = 1.f, gb = 0.f;
+  auto fetch_gate = [&](const Work &w) {
+    if constexpr (kGated) {
+      ga_next = gate.A_log ? __expf(__ldg(gate.A_log + w.h)) : 1.f;
+      gb_next = gate.dt_bias ? __ldg(gate.dt_bias + (size_t)w.h * 128 + (tid & 127)) : 0.f;
+    }
+  };
+  if (cur.ok) fetch_gate(cur);
 
   uint32_t tma_par = 0, mma_par = 0;
   int c = 0;
@@ -405,7 +432,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ---- P0: raw tiles of this chunk ---------------------------------------------
     if (!wait_all(bar_tma, tma_par, status)) break;
     tma_par ^= 1;
-    if constexpr (kMode == kPrepFused) {
+    if constexpr (kGated) {
+      ga = ga_next;
+      gb = gb_next;
+      if (nxt.ok) fetch_gate(nxt);
+    }
+    if constexpr (kPrepM && kFused) {
 #pragma unroll
       for (int m = 0; m < 3; ++m) {  // element tid + 512 m of the head's [part][channel][tap]
         const int rem = tid, ch = rem >> 2, tap = rem & 3;
@@ -529,7 +561,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, corr_pk[q2]);
         if (c8 == 0) pdiag[r] = qk[q2];  // <q_r, k_r> of the fp32 prologue outputs
       }
-      if constexpr (kMode == kPrepFused) {
+      if constexpr (kPrepM) {
         if (cache_out && t0 + Lc == cur.eos) {  // the sequence's last three raw inputs
           for (int idx = tid; idx < 9 * 128; idx += kThreads) {
             const int pr = idx >> 7, ch = idx & 127, p = pr / 3, row = pr % 3;
@@ -546,7 +578,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         const int rr = 16 * part + r;
-        const float gv = Gf[rr * 128 + d];
+        float gv;
+        if constexpr (kGated)  // the 16-bit pre-activation tile, read before E overwrites it
+          gv = bounded_gate(to_f32(reinterpret_cast<const Tin *>(Gf)[rr * 128 + d]), ga, gb,
+                            gate.lower_bound);
+        else
+          gv = Gf[rr * 128 + d];
         acc += rr < Lc ? gv : 0.f;
         vals[r] = acc;
       }
@@ -1145,7 +1182,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
                                                       sN, status, nullptr, nullptr, nullptr,
-                                                      nullptr, nullptr, N);
+                                                      nullptr, nullptr, N, GateArgs{});
   } else {
     auto kern = chunk_tc_kernel<__half, kSingle>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1153,47 +1190,64 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
                                                       sN, status, nullptr, nullptr, nullptr,
-                                                      nullptr, nullptr, N);
+                                                      nullptr, nullptr, N, GateArgs{});
   }
   return cudaGetLastError();
 }
 
 namespace {
-template <typename Tin>
+// Grid of a persistent prep launch: one CTA per SM (each takes a whole SM's
+// shared memory), at most one per work item.
+cudaError_t prep_grid(int N, int T, int H, unsigned *grid) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  *grid = (unsigned)std::min<long long>(rec::chunk_capacity(N, T) * H, sms);
+  return cudaSuccess;
+}
+
+template <typename Tin, int kMode>
 cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                               const CUtensorMap &tg, const float *beta, const int32_t *cu, int N,
-                              int T, int H, uint8_t *ws, int *status, cudaStream_t s) {
-  auto kern = chunk_tc_kernel<Tin, kPrep>;
+                              int T, int H, uint8_t *ws, const GateArgs &gate, int *status,
+                              cudaStream_t s) {
+  auto kern = chunk_tc_kernel<Tin, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SM_ALLOC_PREP);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return e;
-  // Persistent: one CTA per SM (the kernel takes a whole SM's shared memory).
-  const long long items = rec::chunk_capacity(N, T) * H;
-  const unsigned grid = (unsigned)std::min<long long>(items, sms);
+  unsigned grid = 0;
+  if ((e = prep_grid(N, T, H, &grid)) != cudaSuccess) return e;
   kern<<<grid, kThreads, SM_ALLOC_PREP, s>>>(tq, tk, tv, tg, beta, 1.f, nullptr, cu, T, H, nullptr,
-                                        nullptr, status, nullptr, nullptr, nullptr, ws,
-                                        reinterpret_cast<const int32_t *>(ws), N);
+                                             nullptr, status, nullptr, nullptr, nullptr, ws,
+                                             reinterpret_cast<const int32_t *>(ws), N, gate);
   return cudaGetLastError();
 }
 }  // namespace
 
-cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
+cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const void *g,
                               const float *beta, const int32_t *cu, int N, int T, int H,
-                              kda_dtype dt, void *ws, int *status, cudaStream_t s) {
+                              kda_dtype dt, void *ws, const float *A_log, const float *dt_bias,
+                              float lower_bound, bool gated, int *status, cudaStream_t s) {
   const CUtensorMapDataType act =
       dt == KDA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv, tg;
   if (!make_map(&tq, q, act, 2, H, T) || !make_map(&tk, k, act, 2, H, T) ||
       !make_map(&tv, v, act, 2, H, T) ||
-      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+      !(gated ? make_map(&tg, g, act, 2, H, T)
+              : make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T)))
     return cudaErrorInvalidValue;
   uint8_t *w = static_cast<uint8_t *>(ws);
-  if (dt == KDA_BF16) return launch_prep_typed<__nv_bfloat16>(tq, tk, tv, tg, beta, cu, N, T, H, w, status, s);
-  return launch_prep_typed<__half>(tq, tk, tv, tg, beta, cu, N, T, H, w, status, s);
+  const GateArgs gate{A_log, dt_bias, lower_bound};
+  if (dt == KDA_BF16)
+    return gated ? launch_prep_typed<__nv_bfloat16, kPrepGated>(tq, tk, tv, tg, beta, cu, N, T, H,
+                                                                 w, gate, status, s)
+                 : launch_prep_typed<__nv_bfloat16, kPrep>(tq, tk, tv, tg, beta, cu, N, T, H, w,
+                                                            gate, status, s);
+  return gated ? launch_prep_typed<__half, kPrepGated>(tq, tk, tv, tg, beta, cu, N, T, H, w, gate,
+                                                        status, s)
+               : launch_prep_typed<__half, kPrep>(tq, tk, tv, tg, beta, cu, N, T, H, w, gate,
+                                                   status, s);
 }
 
 namespace {
@@ -1215,51 +1269,59 @@ cudaError_t launch_fused_typed(const void *x, const float *conv_w, const void *c
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)blocks, kThreads, SM_ALLOC_FUSED, s>>>(
       tx, tx, tx, tg, beta, scale, s0, cu, T, H, o, sN, status, conv_w,
-      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), nullptr, nullptr, N);
+      static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), nullptr, nullptr, N,
+      GateArgs{});
   return cudaGetLastError();
 }
 }  // namespace
 
 namespace {
-template <typename Tin>
+template <typename Tin, int kMode>
 cudaError_t launch_prep_fused_typed(const void *x, const float *conv_w, const void *cache_in,
-                                    void *cache_out, const float *g, const float *beta,
+                                    void *cache_out, const void *g, const float *beta,
                                     const int32_t *cu, int N, int T, int H,
-                                    CUtensorMapDataType act, void *ws, int *status,
-                                    cudaStream_t s) {
+                                    CUtensorMapDataType act, void *ws, const GateArgs &gate,
+                                    int *status, cudaStream_t s) {
+  constexpr bool kGatedM = kMode == kPrepFusedGated;
   CUtensorMap tx, th, tg;
   if (!make_map(&tx, x, act, 2, 3 * H, T) || !make_map(&th, x, act, 2, 3 * H, T, 3) ||
-      !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T))
+      !(kGatedM ? make_map(&tg, g, act, 2, H, T)
+                : make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T)))
     return cudaErrorInvalidValue;
-  auto kern = chunk_tc_kernel<Tin, kPrepFused>;
+  auto kern = chunk_tc_kernel<Tin, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SM_ALLOC_FUSED);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return e;
-  const long long items = rec::chunk_capacity(N, T) * H;
-  const unsigned grid = (unsigned)std::min<long long>(items, sms);
+  unsigned grid = 0;
+  if ((e = prep_grid(N, T, H, &grid)) != cudaSuccess) return e;
   uint8_t *w = static_cast<uint8_t *>(ws);
   kern<<<grid, kThreads, SM_ALLOC_FUSED, s>>>(
       tx, th, tx, tg, beta, 1.f, nullptr, cu, T, H, nullptr, nullptr, status, conv_w,
       static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), w,
-      reinterpret_cast<const int32_t *>(w), N);
+      reinterpret_cast<const int32_t *>(w), N, gate);
   return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
-                                       void *cache_out, const float *g, const float *beta,
+                                       void *cache_out, const void *g, const float *beta,
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,
-                                       void *ws, int *status, cudaStream_t s) {
-  if (dt == KDA_BF16)
-    return launch_prep_fused_typed<__nv_bfloat16>(x, conv_w, cache_in, cache_out, g, beta, cu, N,
-                                                  T, H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws,
-                                                  status, s);
-  return launch_prep_fused_typed<__half>(x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H,
-                                         CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, status, s);
+                                       void *ws, const float *A_log, const float *dt_bias,
+                                       float lower_bound, bool gated, int *status,
+                                       cudaStream_t s) {
+  const GateArgs gate{A_log, dt_bias, lower_bound};
+  if (dt == KDA_BF16) {
+    constexpr auto act = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return gated ? launch_prep_fused_typed<__nv_bfloat16, kPrepFusedGated>(
+                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s)
+                 : launch_prep_fused_typed<__nv_bfloat16, kPrepFused>(
+                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s);
+  }
+  constexpr auto act = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return gated ? launch_prep_fused_typed<__half, kPrepFusedGated>(
+                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s)
+               : launch_prep_fused_typed<__half, kPrepFused>(
+                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s);
 }
 
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,

@@ -134,6 +134,14 @@ __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __e
 // ---------------------------------------------------------------------------
 
 // Record the first fault code; later faults keep the first one.
+// Bounded log-decay gate ("Kimi K3的线性注意力：从源码看懂KDA如何更新记忆", 彩蛋, the
+// gate.py excerpt): g = lb * sigmoid(a * (graw + bias)) with a = exp(A_log[h]),
+// bias = dt_bias[h][channel] and lb the lower bound (-5 in K3), in fp32.
+__device__ __forceinline__ float bounded_gate(float graw, float a, float bias, float lb) {
+  const float z = a * (graw + bias);
+  return lb * __fdividef(1.f, 1.f + __expf(-z));  // 1/(1 + inf) = 0 for very negative z
+}
+
 __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
@@ -181,9 +189,10 @@ cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in,
                             const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
                             kda_dtype out_dt, void *q, void *k, void *v, int *status,
                             cudaStream_t s);
-cudaError_t launch_decode(const void *x, const float *w, void *cache, const float *g,
+cudaError_t launch_decode(const void *x, const float *w, void *cache, const void *g,
                           const float *beta, float scale, float *state, int N, int H, int D,
-                          kda_dtype dt, float *o, int *status, cudaStream_t s);
+                          kda_dtype dt, float *o, const float *A_log, const float *dt_bias,
+                          float lower_bound, bool gated, int *status, cudaStream_t s);
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, float scale, const float *s0,
                               const int32_t *cu, int N, int T, int H, int D, int chunk,
@@ -194,18 +203,23 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             cudaStream_t s);
 // Two-pass tensor-core prefill (kda_chunk_record.cuh): the prep pass over all
 // (chunk, head) items, then the state pass over (sequence, head, value slice).
-cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
+// g: fp32 log-decay, or (gated) 16-bit gate pre-activations of type dt turned
+// into the log-decay in the kernel (A_log, dt_bias may be null).
+cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const void *g,
                               const float *beta, const int32_t *cu, int N, int T, int H,
-                              kda_dtype dt, void *ws, int *status, cudaStream_t s);
+                              kda_dtype dt, void *ws, const float *A_log, const float *dt_bias,
+                              float lower_bound, bool gated, int *status, cudaStream_t s);
 cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *status,
                                cudaStream_t s);
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, float *o, float *sN, int *status,
                                cudaStream_t s);
 cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
-                                       void *cache_out, const float *g, const float *beta,
+                                       void *cache_out, const void *g, const float *beta,
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,
-                                       void *ws, int *status, cudaStream_t s);
+                                       void *ws, const float *A_log, const float *dt_bias,
+                                       float lower_bound, bool gated, int *status,
+                                       cudaStream_t s);
 cudaError_t launch_cache_pass(const void *ws, int N, int H, const void *cache_in,
                               void *cache_out, cudaStream_t s);
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,

@@ -31,11 +31,15 @@ struct DecodeShape {
   static_assert(kIters >= 1 && kIters * kRowsPerInstr * kWarps == D, "row split");
 };
 
-template <typename Tin, int D>
+// kGated: g holds gate pre-activations of type Tin and the log-decay is
+// lower_bound * sigmoid(exp(A_log[h]) * (g + dt_bias[h, :])) (pointers may be null).
+template <typename Tin, int D, bool kGated>
 __global__ void __launch_bounds__(DecodeShape<D>::kThreads)
 decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__restrict__ cache,
-              const float *__restrict__ g, const float *__restrict__ beta, float scale,
-              float *__restrict__ state, int N, int H, float *__restrict__ o) {
+              const void *__restrict__ g, const float *__restrict__ beta, float scale,
+              float *__restrict__ state, int N, int H, float *__restrict__ o,
+              const float *__restrict__ A_log, const float *__restrict__ dt_bias,
+              float lower_bound) {
   using Sh = DecodeShape<D>;
   constexpr int LPR = Sh::kLanesPerRow;
   __shared__ float qkv[3 * D];
@@ -57,7 +61,19 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
     const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
     s[it] = __ldcs(reinterpret_cast<const float4 *>(base + (size_t)j * D + dk0));
   }
-  const float4 g4 = __ldg(reinterpret_cast<const float4 *>(g + (size_t)nh * D + dk0));
+  float4 g4;
+  if constexpr (kGated) {
+    const Tin *gr = static_cast<const Tin *>(g) + (size_t)nh * D + dk0;
+    const float a = A_log ? __expf(__ldg(A_log + h)) : 1.f;
+    const float4 b4 = dt_bias ? __ldg(reinterpret_cast<const float4 *>(dt_bias + (size_t)h * D + dk0))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    g4 = make_float4(bounded_gate(to_f32(gr[0]), a, b4.x, lower_bound),
+                     bounded_gate(to_f32(gr[1]), a, b4.y, lower_bound),
+                     bounded_gate(to_f32(gr[2]), a, b4.z, lower_bound),
+                     bounded_gate(to_f32(gr[3]), a, b4.w, lower_bound));
+  } else {
+    g4 = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(g) + (size_t)nh * D + dk0));
+  }
   const float b = __ldg(beta + nh);
 
   // 2. Prologue for this head's 3*D channels; the conv cache is shifted in place.
@@ -138,40 +154,52 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
   for (int j = tid; j < D; j += Sh::kThreads) o[(size_t)nh * D + j] = o_s[j];
 }
 
+// Gate of the gated step (null A_log / dt_bias: neutral; unused when not gated).
+struct DecodeGate {
+  const float *A_log;
+  const float *dt_bias;
+  float lower_bound;
+  bool on;
+};
+
 template <typename Tin, int D>
-cudaError_t launch_typed(const void *x, const float *w, void *cache, const float *g,
+cudaError_t launch_typed(const void *x, const float *w, void *cache, const void *g,
                          const float *beta, float scale, float *state, int N, int H, float *o,
-                         cudaStream_t s) {
-  decode_kernel<Tin, D><<<N * H, DecodeShape<D>::kThreads, 0, s>>>(
-      static_cast<const Tin *>(x), w, static_cast<Tin *>(cache), g, beta, scale, state, N, H,
-      o);
+                         const DecodeGate &gt, cudaStream_t s) {
+  auto kern = gt.on ? decode_kernel<Tin, D, true> : decode_kernel<Tin, D, false>;
+  kern<<<N * H, DecodeShape<D>::kThreads, 0, s>>>(static_cast<const Tin *>(x), w,
+                                                  static_cast<Tin *>(cache), g, beta, scale,
+                                                  state, N, H, o, gt.A_log, gt.dt_bias,
+                                                  gt.lower_bound);
   return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t launch_d(int D, const void *x, const float *w, void *cache, const float *g,
+cudaError_t launch_d(int D, const void *x, const float *w, void *cache, const void *g,
                      const float *beta, float scale, float *state, int N, int H, float *o,
-                     cudaStream_t s) {
+                     const DecodeGate &gt, cudaStream_t s) {
   switch (D) {
-    case 16: return launch_typed<Tin, 16>(x, w, cache, g, beta, scale, state, N, H, o, s);
-    case 32: return launch_typed<Tin, 32>(x, w, cache, g, beta, scale, state, N, H, o, s);
-    case 64: return launch_typed<Tin, 64>(x, w, cache, g, beta, scale, state, N, H, o, s);
-    case 128: return launch_typed<Tin, 128>(x, w, cache, g, beta, scale, state, N, H, o, s);
+    case 16: return launch_typed<Tin, 16>(x, w, cache, g, beta, scale, state, N, H, o, gt, s);
+    case 32: return launch_typed<Tin, 32>(x, w, cache, g, beta, scale, state, N, H, o, gt, s);
+    case 64: return launch_typed<Tin, 64>(x, w, cache, g, beta, scale, state, N, H, o, gt, s);
+    case 128: return launch_typed<Tin, 128>(x, w, cache, g, beta, scale, state, N, H, o, gt, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const void *x, const float *w, void *cache, const float *g,
+cudaError_t launch_decode(const void *x, const float *w, void *cache, const void *g,
                           const float *beta, float scale, float *state, int N, int H, int D,
-                          kda_dtype dt, float *o, int *status, cudaStream_t s) {
+                          kda_dtype dt, float *o, const float *A_log, const float *dt_bias,
+                          float lower_bound, bool gated, int *status, cudaStream_t s) {
   (void)status;  // the decode kernel has no waits or data-dependent indices
   if ((long long)N * H >= (1LL << 31)) return cudaErrorInvalidValue;
+  const DecodeGate gt{A_log, dt_bias, lower_bound, gated};
   if (dt == KDA_BF16)
-    return launch_d<__nv_bfloat16>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
-  if (dt == KDA_F16) return launch_d<__half>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
-  return launch_d<float>(D, x, w, cache, g, beta, scale, state, N, H, o, s);
+    return launch_d<__nv_bfloat16>(D, x, w, cache, g, beta, scale, state, N, H, o, gt, s);
+  if (dt == KDA_F16) return launch_d<__half>(D, x, w, cache, g, beta, scale, state, N, H, o, gt, s);
+  return launch_d<float>(D, x, w, cache, g, beta, scale, state, N, H, o, gt, s);
 }
 
 }  // namespace kda

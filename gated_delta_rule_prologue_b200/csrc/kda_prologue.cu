@@ -24,7 +24,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTokensPerThread = 32;  // TT
 // tokens whose loads are in flight together (fewer for 32-byte float rows)
-template <typename Tin> __host__ __device__ constexpr int batch_of() { return sizeof(Tin) == 2 ? 8 : 4; }
+template <typename Tin> __host__ __device__ constexpr int batch_of() { return sizeof(Tin) == 2 ? 6 : 3; }
 
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -79,8 +79,10 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
     seq_bounds(cu, n, T, status, bos, eos);
   }
 
-  // History of t0: tokens t0-3, t0-2, t0-1 (from the cache before bos), packed.
+  // History of t0: tokens t0-3, t0-2, t0-1 (from the cache before bos), packed
+  // for the cache write-out and widened once for the convolution.
   Raw8<Tin> hm3, hm2, hm1;
+  float fm3[8], fm2[8], fm1[8];
   {
     Raw8<Tin> hv[3];
 #pragma unroll
@@ -97,6 +99,9 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
     hm3 = hv[0];
     hm2 = hv[1];
     hm1 = hv[2];
+    widen8(hm3, fm3);
+    widen8(hm2, fm2);
+    widen8(hm1, fm1);
   }
 
   constexpr int kBatch = batch_of<Tin>();
@@ -120,17 +125,13 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
         hm3 = load_or_zero(cr, ok);
         hm2 = load_or_zero(cr + C, ok);
         hm1 = load_or_zero(cr + 2 * C, ok);
+        widen8(hm3, fm3);
+        widen8(hm2, fm2);
+        widen8(hm1, fm1);
       }
       float y[8], f[8];
-      widen8(hm3, f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = wt[e][0] * f[e];
-      widen8(hm2, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][1], f[e], y[e]);
-      widen8(hm1, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][2], f[e], y[e]);
+      for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][2], fm1[e], fmaf(wt[e][1], fm2[e], wt[e][0] * fm3[e]));
       widen8(xr[i], f);
       float ss = 0.f;
 #pragma unroll
@@ -156,6 +157,12 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
       hm3 = hm2;
       hm2 = hm1;
       hm1 = xr[i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        fm3[e] = fm2[e];
+        fm2[e] = fm1[e];
+        fm1[e] = f[e];
+      }
     }
   }
 }

@@ -155,6 +155,33 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
                             void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * The *_gated entry points take the gate pre-activations instead of the
+ * log-decay and apply the bounded gate inside the kernels ([W1 彩蛋], the
+ * gate.py excerpt):
+ *     g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h, :]))
+ * with lower_bound -5 in K3, so the fp32 log-decay is never stored.
+ *   g_raw        [T, H, D] (prefill) or [N, H, D] (decode), element type dt
+ *   A_log        [H] f32, 4-byte aligned, or NULL (exp(A_log) taken as 1)
+ *   dt_bias      [H, D] f32, 16-byte aligned, or NULL (zero)
+ *   lower_bound  finite and negative; the prefill entry points need it in
+ *                [-5, 0) (their decay-range argument), else KDA_ERR_UNSUPPORTED
+ */
+
+/*
+ * kda_chunk_fwd_gated_ws -- kda_chunk_fwd_ws with the in-kernel gate: the
+ * two-pass tensor-core path only (dt KDA_BF16 or KDA_F16, Dk == Dv == 128,
+ * chunk 64, T > 0, a workspace of kda_chunk_fwd_workspace_bytes(...) bytes),
+ * else KDA_ERR_UNSUPPORTED / KDA_ERR_INVALID_ARG.  Other arguments as in
+ * kda_chunk_fwd_ws.
+ */
+kda_status kda_chunk_fwd_gated_ws(const void *q, const void *k, const void *v, const void *g_raw,
+                                  const float *A_log, const float *dt_bias, float lower_bound,
+                                  const float *beta, float scale, const float *initial_state,
+                                  const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                                  int chunk, kda_dtype dt, float *o, float *final_state,
+                                  void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_static -- kda_chunk_fwd_ws without a caller workspace: the
  * scratch is a fixed device buffer inside the library, and the call
  * allocates and frees nothing.  The pages have no counterpart of this entry
@@ -224,6 +251,21 @@ kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const v
                                      kda_stream_t stream);
 
 /*
+ * kda_prologue_chunk_fwd_gated_ws -- kda_prologue_chunk_fwd_ws with the
+ * in-kernel gate (see above; a workspace is required).
+ */
+kda_status kda_prologue_chunk_fwd_gated_ws(const void *x, const float *conv_w,
+                                           const void *cache_in, void *cache_out,
+                                           const void *g_raw, const float *A_log,
+                                           const float *dt_bias, float lower_bound,
+                                           const float *beta, float scale,
+                                           const float *initial_state,
+                                           const int32_t *cu_seqlens, int N, int T, int H, int D,
+                                           kda_dtype dt, float *o, float *final_state,
+                                           void *workspace, size_t workspace_bytes,
+                                           kda_stream_t stream);
+
+/*
  * kda_decode_step -- one new token for each of N independent sequences: the
  * prologue on that token with the conv cache as history, then one step of
  * the recurrence on the state in place (the recurrent mode used for
@@ -242,6 +284,17 @@ kda_status kda_decode_step(const void *x, const float *conv_w, void *conv_cache,
                            const float *g, const float *beta, float scale, float *state,
                            int N, int H, int D, kda_dtype dt, float *o,
                            kda_stream_t stream);
+
+/*
+ * kda_decode_step_gated -- kda_decode_step with the in-kernel gate: g_raw
+ * [N, H, D] of type dt (16-byte aligned) replaces g; any finite negative
+ * lower_bound.
+ */
+kda_status kda_decode_step_gated(const void *x, const float *conv_w, void *conv_cache,
+                                 const void *g_raw, const float *A_log, const float *dt_bias,
+                                 float lower_bound, const float *beta, float scale, float *state,
+                                 int N, int H, int D, kda_dtype dt, float *o,
+                                 kda_stream_t stream);
 
 /*
  * kda_get_device_status -- read and clear the current device's status word

@@ -194,3 +194,32 @@ def test_static_scratch_constant_matches_header(kda):
     text = open(HEADER).read()
     m = re.search(r"#define KDA_CHUNK_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == kda.KDA_CHUNK_STATIC_SCRATCH_BYTES
+
+
+def test_gated_entry_points_reject_bad_gate_arguments(kda):
+    L = kda.lib
+    T, H = 128, 2
+    need = kda.kda_chunk_fwd_workspace_bytes(1, T, H, 128, 128, 64, __import__("torch").bfloat16)
+    q, k, v = _vp(0x10000), _vp(0x20000), _vp(0x30000)   # 64 KiB each
+    g_raw, beta, o = _vp(0x40000), _vp(0x60000), _vp(0x70000)
+    ws = _vp(0x100000)
+    # lower bound below the chunk kernels' decay range
+    st = L.kda_chunk_fwd_gated_ws(q, k, v, g_raw, None, None, -6.0, beta, 1.0, None, None, 1, T, H,
+                                  128, 128, 64, 1, o, None, ws, need, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED and b"lower_bound" in L.kda_last_error()
+    # non-negative lower bound
+    st = L.kda_chunk_fwd_gated_ws(q, k, v, g_raw, None, None, 0.0, beta, 1.0, None, None, 1, T, H,
+                                  128, 128, 64, 1, o, None, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    # one-pass shapes are not supported by the gated path
+    st = L.kda_chunk_fwd_gated_ws(q, k, v, g_raw, None, None, -5.0, beta, 1.0, None, None, 1, T, H,
+                                  128, 128, 32, 1, o, None, ws, need, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    # a workspace is required
+    st = L.kda_chunk_fwd_gated_ws(q, k, v, g_raw, None, None, -5.0, beta, 1.0, None, None, 1, T, H,
+                                  128, 128, 64, 1, o, None, None, 0, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace" in L.kda_last_error()
+    # misaligned dt_bias
+    st = L.kda_decode_step_gated(q, _vp(0x200000), _vp(0x300000), g_raw, None, _vp(0x400008), -5.0,
+                                 beta, 1.0, _vp(0x500000), 1, H, 128, 1, o, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"dt_bias" in L.kda_last_error()
