@@ -48,6 +48,7 @@ QKV_DT = 2                                          # q/k/v handed from prologue
 PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/k/v      = 1536
 CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 1796
 FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
+GATED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 2 + 4 + D_ * 4  # bf16 q,k,v + bf16 g_raw + beta + o = 1540
 CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 # decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
 DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
@@ -59,6 +60,7 @@ KERNEL_SOURCES = {
     "kda_prologue": [_CSRC + "kda_prologue.cu"],
     "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
     "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
+    "kda_chunk_fwd_gated": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
     "kda_decode_step": [_CSRC + "kda_decode.cu"],
 }
 
@@ -344,7 +346,22 @@ def run_ours(args, world, rank, local):
     fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in side[1:])
     fused_one_pass_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in side[1:])
     one_pass_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in side[1:])
-    del o2
+    # the in-kernel gate: 16-bit gate pre-activations instead of the fp32 log-decay
+    gen = torch.Generator().manual_seed(7)
+    g_raw = torch.randn((T, H, D), generator=gen).to(torch.bfloat16).to(dev)
+    A_log = (0.5 * torch.randn((H,), generator=gen)).to(dev)
+    dt_bias = torch.randn((H, D), generator=gen).to(dev)
+    gq = q.to(torch.bfloat16)
+    gk, gv = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    for i in range(3):
+        gev[i][0].record(stream)
+        kda.kda_chunk_fwd_gated(gq, gk, gv, g_raw, beta, o2, A_log=A_log, dt_bias=dt_bias,
+                                scale=inp.scale, workspace=ws, stream=stream)
+        gev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    gated_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in gev[1:])
+    del o2, g_raw, gq, gk, gv
 
     th = T * H
     step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
@@ -359,6 +376,9 @@ def run_ours(args, world, rank, local):
             "hbm", PROLOGUE_BYTES_PER_TH * th, pro_ms, hbm, "GB/s", recorded_traffic("kda_prologue"))),
         "kda_chunk_fwd": dict(ms=round(chk_ms, 4), launches=2, **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, chk_ms, hbm, "GB/s", recorded_traffic("kda_chunk_fwd"))),
+        "kda_chunk_fwd_gated": dict(ms=round(gated_ms, 4), launches=2, **roofline(
+            "hbm", GATED_BYTES_PER_TH * th, gated_ms, hbm, "GB/s",
+            recorded_traffic("kda_chunk_fwd_gated"))),
         "kda_chunk_fwd_one_pass": dict(ms=round(one_pass_ms, 4), **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, one_pass_ms, hbm, "GB/s",
             recorded_traffic("kda_chunk_fwd_one_pass"))),
