@@ -49,6 +49,7 @@ PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/
 CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 1796
 FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
 GATED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 2 + 4 + D_ * 4  # bf16 q,k,v + bf16 g_raw + beta + o = 1540
+EPILOGUE_BYTES_PER_TH = D_ * 4 + 2 * D_ * 2             # o (f32) + gate, out (bf16) = 1024
 CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 # decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
 DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
@@ -61,6 +62,7 @@ KERNEL_SOURCES = {
     "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
     "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
     "kda_chunk_fwd_gated": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
+    "kda_output_epilogue": [_CSRC + "kda_epilogue.cu"],
     "kda_decode_step": [_CSRC + "kda_decode.cu"],
 }
 
@@ -361,7 +363,17 @@ def run_ours(args, world, rank, local):
         gev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     gated_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in gev[1:])
-    del o2, g_raw, gq, gk, gv
+    # the output epilogue on the step's read-out (RMSNorm x sigmoid gate, bf16 out)
+    ep_out = gq  # reuse a bf16 [T, H, D] buffer
+    ep_w = (0.5 + torch.rand((D,), generator=gen)).to(dev)
+    eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    for i in range(3):
+        eev[i][0].record(stream)
+        kda.kda_output_epilogue(o, g_raw, ep_w, ep_out, stream=stream)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    epi_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in eev[1:])
+    del o2, g_raw, gq, gk, gv, ep_out
 
     th = T * H
     step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
@@ -379,6 +391,9 @@ def run_ours(args, world, rank, local):
         "kda_chunk_fwd_gated": dict(ms=round(gated_ms, 4), launches=2, **roofline(
             "hbm", GATED_BYTES_PER_TH * th, gated_ms, hbm, "GB/s",
             recorded_traffic("kda_chunk_fwd_gated"))),
+        "kda_output_epilogue": dict(ms=round(epi_ms, 4), **roofline(
+            "hbm", EPILOGUE_BYTES_PER_TH * th, epi_ms, hbm, "GB/s",
+            recorded_traffic("kda_output_epilogue"))),
         "kda_chunk_fwd_one_pass": dict(ms=round(one_pass_ms, 4), **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, one_pass_ms, hbm, "GB/s",
             recorded_traffic("kda_chunk_fwd_one_pass"))),

@@ -86,6 +86,7 @@ lib.kda_prologue_chunk_fwd_gated_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _v
                                                 ctypes.c_size_t, _vp]
 lib.kda_decode_step_gated.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _f, _vp, _i, _i, _i,
                                       _i, _vp, _vp]
+lib.kda_output_epilogue.argtypes = [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp]
 lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
@@ -95,6 +96,7 @@ lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
+            lib.kda_output_epilogue,
             lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
@@ -360,3 +362,16 @@ def kda_decode_step_gated(x, conv_w, conv_cache, g_raw, beta, state, o, *, H: in
                                      _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(beta),
                                      float(scale), _ptr(state), N, H, D, _dtype(x), _ptr(o),
                                      _stream(stream)))
+
+
+def kda_output_epilogue(o, gate, weight, out, *, eps: float = 1e-5, stream=None):
+    """Per-head RMSNorm of the read-out ``o`` [T, H, D] (f32) times the output
+    gate: out = o / sqrt(mean(o^2) + eps) * weight * sigmoid(gate); ``gate`` and
+    ``out`` share a dtype."""
+    _need(o, "o", torch.float32)
+    _need(weight, "weight", torch.float32)
+    _need(gate, "gate", out.dtype)
+    _need(out, "out", out.dtype)
+    T, H, D = o.shape
+    _check(lib.kda_output_epilogue(_ptr(o), _ptr(gate), _ptr(weight), float(eps), T, H, D,
+                                   _dtype(out), _ptr(out), _stream(stream)))

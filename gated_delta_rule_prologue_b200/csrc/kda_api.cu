@@ -129,6 +129,28 @@ const char *kda_last_error(void) { return g_last_error.c_str(); }
 
 const char *kda_version(void) { return "libkda 0.1 (sm_100a)"; }
 
+kda_status kda_output_epilogue(const float *o, const void *gate, const float *weight, float eps,
+                               int T, int H, int D, kda_dtype dt, void *out,
+                               kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(T >= 0 && H >= 1 && D >= 1, "bad sizes T=%d H=%d D=%d", T, H, D);
+  if (!supported_d(D)) return fail(KDA_ERR_UNSUPPORTED, "epilogue: D=%d not in {16,32,64,128}", D);
+  KDA_REQUIRE(eps >= 0.f && eps < 1e30f, "eps must be finite and non-negative");
+  KDA_REQUIRE_PTR(weight, "weight");
+  if (T == 0) return KDA_OK;
+  KDA_REQUIRE_PTR(o, "o");
+  KDA_REQUIRE_PTR(gate, "gate");
+  KDA_REQUIRE_PTR(out, "out");
+  const size_t n = (size_t)T * H * D, es = esize(dt);
+  KDA_REQUIRE(!overlaps(out, n * es, o, n * 4), "out overlaps o");
+  KDA_REQUIRE(!overlaps(out, n * es, gate, n * es), "out overlaps gate");
+  KDA_REQUIRE(!overlaps(out, n * es, weight, (size_t)D * 4), "out overlaps weight");
+  cudaError_t e = kda::launch_epilogue(o, gate, weight, eps, (long long)T * H, D, dt, out,
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_output_epilogue launch");
+  return KDA_OK;
+}
+
 kda_status kda_get_device_status(int *code) {
   KDA_REQUIRE(code != nullptr, "code is NULL");
   int *word = nullptr;

@@ -193,6 +193,8 @@ cudaError_t launch_decode(const void *x, const float *w, void *cache, const void
                           const float *beta, float scale, float *state, int N, int H, int D,
                           kda_dtype dt, float *o, const float *A_log, const float *dt_bias,
                           float lower_bound, bool gated, int *status, cudaStream_t s);
+cudaError_t launch_epilogue(const float *o, const void *gate, const float *weight, float eps,
+                            long long rows, int D, kda_dtype dt, void *out, cudaStream_t s);
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, float scale, const float *s0,
                               const int32_t *cu, int N, int T, int H, int D, int chunk,

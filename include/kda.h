@@ -297,6 +297,23 @@ kda_status kda_decode_step_gated(const void *x, const float *conv_w, void *conv_
                                  kda_stream_t stream);
 
 /*
+ * kda_output_epilogue -- the output path after the read ([W1 第六站]): per-head
+ * RMSNorm of the read-out, then the per-channel output gate:
+ *     out[t, h, :] = o[t, h, :] / sqrt(mean_d o^2 + eps) * weight * sigmoid(gate[t, h, :])
+ * The page's formula is lost in the extraction; the sigmoid gate (a
+ * per-channel proportion) and the caller's eps are readings.  The gate
+ * pre-activations come from the output-gate projection of x_t, which is not
+ * part of this library.
+ *   o       [T, H, D] f32 (a read-out of kda_chunk_fwd & co.)
+ *   gate    [T, H, D] dt;  weight [D] f32 (shared by the heads);  eps >= 0
+ *   out     [T, H, D] dt, must not overlap o, gate or weight
+ * Supported: D in {16, 32, 64, 128}.
+ */
+kda_status kda_output_epilogue(const float *o, const void *gate, const float *weight, float eps,
+                               int T, int H, int D, kda_dtype dt, void *out,
+                               kda_stream_t stream);
+
+/*
  * kda_get_device_status -- read and clear the current device's status word
  * (KDA_OK if no kernel recorded a fault).  Synchronises the device.
  */

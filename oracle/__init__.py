@@ -15,6 +15,7 @@ from .kda_oracle import (  # noqa: F401
     kda_decode_step,
     kda_recurrent,
     l2_normalize,
+    output_epilogue,
     prologue,
     short_conv,
     silu,

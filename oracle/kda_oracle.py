@@ -10,8 +10,8 @@ Sources (web pages; cited as [Wn section]):
   [W1] "Kimi K3的线性注意力：从源码看懂KDA如何更新记忆" (yeyulingfeng.com) --
        the stations 第二站 (short conv, SiLU, L2), 第三站 (per-channel decay),
        第四站 (delta-rule write; naive_recurrent_kda excerpt), 第五站 (read
-       after write; query scale), 彩蛋 (chunked execution; bounded gate, the
-       gate.py excerpt).
+       after write; query scale), 第六站 (per-head RMSNorm and output gate),
+       彩蛋 (chunked execution; bounded gate, the gate.py excerpt).
   [W3] "Kimi K3 记忆架构总览：KDA、MLA、AttnRes 各管什么" (moonzj.com),
        section "KDA 谱系速查" (delta-rule pseudocode, reparameterisation).
   [W4] "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解"
@@ -149,6 +149,24 @@ def gate(g_raw, A_log=None, dt_bias=None, lower_bound=-5.0):
     e = np.exp(-np.abs(z))
     sig = np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
     return float(lower_bound) * sig
+
+
+def output_epilogue(o, gate_preact, weight, eps=1e-5):
+    """Output path after the read ([W1 第六站]): per-head RMSNorm of the read-out,
+    then the output gate scales each channel.  Reading of the garbled formula:
+    the gate is a sigmoid of its pre-activation (a per-channel proportion in
+    (0, 1)), the norm's epsilon is a parameter:
+
+        out = o / sqrt(mean_d(o^2) + eps) * weight * sigmoid(gate_preact)
+
+    o, gate_preact [..., D]; weight [D] (shared by the heads).  float64.
+    """
+    o = _f64(o)
+    z = _f64(gate_preact)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + float(eps))
+    e = np.exp(-np.abs(z))
+    sig = np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return o / rms * _f64(weight) * sig
 
 
 def kda_recurrent(q, k, v, g, beta, scale=1.0, initial_state=None, cu_seqlens=None):

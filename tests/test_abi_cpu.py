@@ -223,3 +223,16 @@ def test_gated_entry_points_reject_bad_gate_arguments(kda):
     st = L.kda_decode_step_gated(q, _vp(0x200000), _vp(0x300000), g_raw, None, _vp(0x400008), -5.0,
                                  beta, 1.0, _vp(0x500000), 1, H, 128, 1, o, None)
     assert st == kda.KDA_ERR_INVALID_ARG and b"dt_bias" in L.kda_last_error()
+
+
+def test_output_epilogue_rejects_bad_arguments(kda):
+    L = kda.lib
+    o, g, w, out = _vp(0x100000), _vp(0x200000), _vp(0x300000), _vp(0x400000)
+    st = L.kda_output_epilogue(o, g, w, 1e-5, 10, 2, 48, 1, out, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_output_epilogue(o, g, w, -1.0, 10, 2, 128, 1, out, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    st = L.kda_output_epilogue(o, g, None, 1e-5, 10, 2, 128, 1, out, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"weight" in L.kda_last_error()
+    st = L.kda_output_epilogue(o, g, w, 1e-5, 10, 2, 128, 1, _vp(0x100010), None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
