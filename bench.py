@@ -275,6 +275,51 @@ def run_reference(args, world, rank):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def seq4k_side(kda, dev, stream, hbm):
+    """The single-sequence bf16 prefill (T=4096, H=8, d=128, initial state):
+    its 32 (head, value slice) chains fill a fifth of the GPU, so the library
+    splits the sequence into segments (sequence-parallel state pass).  Timed
+    split and whole, L2 flushed before every call (the inputs fit in L2)."""
+    sinp = W.seq4k_bf16()
+    T4, H4, D4 = sinp.T, sinp.H, sinp.q.shape[2]
+    q4, k4, v4 = sinp.q.to(dev), sinp.k.to(dev), sinp.v.to(dev)
+    g4, b4, s04 = sinp.g.to(dev), sinp.beta.to(dev), sinp.initial_state.to(dev)
+    o4 = torch.empty((T4, H4, D4), dtype=torch.float32, device=dev)
+    f4 = torch.empty_like(s04)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = kda.kda_chunk_fwd_segment_chunks(1, T4, H4)
+    out = {"workload": "seq4k_bf16: T=4096, H=8, d_k=d_v=128, chunk 64, bf16 q/k/v, "
+                       "initial state, one sequence", "segment_chunks": L,
+           "l2": "256 MiB written before every timed call"}
+    for name, seg in (("split", None), ("whole", 0)):
+        nb = (kda.kda_chunk_fwd_workspace_bytes(1, T4, H4, D4, D4, 64, q4.dtype) if seg is None
+              else kda.kda_chunk_fwd_segmented_workspace_bytes(1, T4, H4, D4, D4, 64, q4.dtype,
+                                                               seg))
+        ws4 = torch.empty(nb, dtype=torch.uint8, device=dev)
+        call = lambda: kda.kda_chunk_fwd(q4, k4, v4, g4, b4, o4, scale=sinp.scale,
+                                         initial_state=s04, final_state=f4, workspace=ws4,
+                                         segment_chunks=seg, stream=stream)
+        for _ in range(3):
+            call()
+        times = []
+        for _ in range(10):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        out[name] = dict(ms=round(ms, 4), tokens_per_s=round(T4 / (ms * 1e-3), 1),
+                         **roofline("hbm", CHUNK_BYTES_PER_TH * T4 * H4, ms, hbm, "GB/s", None))
+        del ws4
+    assert kda.kda_get_device_status() == 0
+    out["speedup"] = round(out["whole"]["ms"] / out["split"]["ms"], 3)
+    del q4, k4, v4, g4, b4, s04, o4, f4, flush
+    return out
+
+
 def run_ours(args, world, rank, local):
     import gated_delta_rule_prologue_b200 as kda
     dev = torch.device("cuda", local)
@@ -374,6 +419,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     epi_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in eev[1:])
     del o2, g_raw, gq, gk, gv, ep_out
+    seq4k = seq4k_side(kda, dev, stream, hbm)
 
     th = T * H
     step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
@@ -486,6 +532,7 @@ def run_ours(args, world, rank, local):
         "kernels": kernels,
         "fused_hbm_floor_ms": round(fused_floor_ms, 4),
         "decode": decode,
+        "seq4k": seq4k,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

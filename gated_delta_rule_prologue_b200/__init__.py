@@ -89,11 +89,18 @@ lib.kda_decode_step_gated.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _f,
 lib.kda_output_epilogue.argtypes = [_vp, _vp, _vp, _f, _i, _i, _i, _i, _vp, _vp]
 lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
+lib.kda_chunk_fwd_segmented_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+lib.kda_chunk_fwd_segmented_workspace_bytes.restype = ctypes.c_size_t
+lib.kda_chunk_fwd_segment_chunks.argtypes = [_i, _i, _i]
+lib.kda_chunk_fwd_segment_chunks.restype = ctypes.c_int
+lib.kda_chunk_fwd_segmented_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
+                                           _i, _i, _i, _vp, _vp, _i, _vp, ctypes.c_size_t, _vp]
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
+            lib.kda_chunk_fwd_segmented_ws,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_output_epilogue,
@@ -178,15 +185,34 @@ def kda_chunk_fwd_workspace_bytes(N: int, T: int, H: int, Dk: int, Dv: int, chun
     return int(lib.kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, chunk, _DTYPES[dtype]))
 
 
+def kda_chunk_fwd_segment_chunks(N: int, T: int, H: int) -> int:
+    """Segment length (in 64-token chunks) of the sequence-parallel state pass
+    that the workspace entry points pick for these sizes (0: whole sequences)."""
+    return int(lib.kda_chunk_fwd_segment_chunks(N, T, H))
+
+
+def kda_chunk_fwd_segmented_workspace_bytes(N: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
+                                            dtype: torch.dtype, segment_chunks: int) -> int:
+    """Scratch bytes of the two-pass prefill at an explicit segment length."""
+    return int(lib.kda_chunk_fwd_segmented_workspace_bytes(N, T, H, Dk, Dv, chunk,
+                                                           _DTYPES[dtype], segment_chunks))
+
+
 def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None,
                   final_state=None, cu_seqlens=None, chunk: int = 64, workspace="auto",
-                  stream=None):
+                  segment_chunks=None, stream=None):
     """Chunkwise prefill: writes ``o`` [T, H, Dv] and optionally ``final_state``.
 
     ``workspace``: ``"auto"`` allocates the two-pass path's scratch from
     torch's caching allocator; a uint8 CUDA tensor is used as given (at least
     :func:`kda_chunk_fwd_workspace_bytes`); ``None`` runs the one-pass kernels.
+    ``segment_chunks``: ``None`` lets the library pick the state pass's segment
+    length; an int (0: whole sequences) calls ``kda_chunk_fwd_segmented_ws``
+    with it (workspace sized by :func:`kda_chunk_fwd_segmented_workspace_bytes`).
     """
+    if segment_chunks is not None:
+        return _chunk_fwd_segmented(q, k, v, g, beta, o, scale, initial_state, final_state,
+                                    cu_seqlens, chunk, workspace, int(segment_chunks), stream)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
     for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
@@ -211,6 +237,31 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
                                 _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
                                 _dtype(q), _ptr(o), _ptr(final_state), _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
+
+
+def _chunk_fwd_segmented(q, k, v, g, beta, o, scale, initial_state, final_state, cu_seqlens,
+                         chunk, workspace, segment_chunks, stream):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_fwd_segmented_workspace_bytes(N, T, H, Dk, Dv, chunk, q.dtype,
+                                                         segment_chunks)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_chunk_fwd_segmented_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                          float(scale), _ptr(initial_state), _ptr(cu_seqlens), N,
+                                          T, H, Dk, Dv, chunk, _dtype(q), _ptr(o),
+                                          _ptr(final_state), segment_chunks, _ptr(workspace),
+                                          workspace.numel(), _stream(stream)))
 
 
 # Size of the library's fixed scratch buffer (one per device) used by

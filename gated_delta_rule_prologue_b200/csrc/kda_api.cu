@@ -301,7 +301,19 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
 size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
                                      kda_dtype dt) {
   if (N < 1 || T < 0 || H < 1 || !chunk_tc_path(T, Dk, Dv, chunk, dt)) return 0;
-  return kda::rec::workspace_bytes(N, T, H);
+  return kda::rec::workspace_bytes(N, T, H, kda::rec::segment_chunks(N, T, H));
+}
+
+size_t kda_chunk_fwd_segmented_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                               kda_dtype dt, int segment_chunks) {
+  if (N < 1 || T < 0 || H < 1 || segment_chunks < 0 || !chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return 0;
+  return kda::rec::workspace_bytes(N, T, H, segment_chunks);
+}
+
+int kda_chunk_fwd_segment_chunks(int N, int T, int H) {
+  if (N < 1 || T < 0 || H < 1) return 0;
+  return kda::rec::segment_chunks(N, T, H);
 }
 
 }  // extern "C"
@@ -317,8 +329,8 @@ kda_status chunk_two_pass(const void *q, const void *k, const void *v, const voi
                           const float *initial_state, const int32_t *cu_seqlens, int N, int T,
                           int H, int Dk, int Dv, kda_dtype dt, float *o, float *final_state,
                           void *workspace, size_t workspace_bytes, cudaStream_t s,
-                          const char *what) {
-  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, Dk, Dv, 64, dt);
+                          const char *what, int L) {
+  const size_t need = kda::rec::workspace_bytes(N, T, H, L);
   KDA_OPT_PTR(workspace, "workspace");
   KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
               workspace_bytes, need);
@@ -339,12 +351,13 @@ kda_status chunk_two_pass(const void *q, const void *k, const void *v, const voi
   kda_status st = device_status_word(&status);
   if (st != KDA_OK) return st;
   cudaError_t e = cudaSuccess;
-  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  if (cu_seqlens || L > 0)
+    e = kda::launch_chunk_index(cu_seqlens, N, T, L, workspace, status, s);
   if (e == cudaSuccess)
     e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, A_log,
                                dt_bias, lower_bound, gated, status, s);
   if (e == cudaSuccess)
-    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, L, o,
                                 final_state, status, s);
   if (e != cudaSuccess) return cuda_fail(e, what);
   return KDA_OK;
@@ -370,7 +383,30 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
                          chunk, dt, o, final_state, stream);
   return chunk_two_pass(q, k, v, g, 4, nullptr, nullptr, 0.f, false, beta, scale, initial_state,
                         cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, workspace,
-                        workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_ws launch");
+                        workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_ws launch",
+                        kda::rec::segment_chunks(N, T, H));
+}
+
+kda_status kda_chunk_fwd_segmented_ws(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, float scale,
+                                      const float *initial_state, const int32_t *cu_seqlens,
+                                      int N, int T, int H, int Dk, int Dv, int chunk,
+                                      kda_dtype dt, float *o, float *final_state,
+                                      int segment_chunks, void *workspace,
+                                      size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                                   chunk, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  if (!chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_fwd_segmented: needs bf16/f16, Dk == Dv == 128, "
+                                     "chunk 64 and T > 0 (got dt=%d Dk=%d chunk=%d T=%d)",
+                (int)dt, Dk, chunk, T);
+  KDA_REQUIRE(segment_chunks >= 0, "segment_chunks=%d is negative", segment_chunks);
+  KDA_REQUIRE(workspace != nullptr, "chunk_fwd_segmented: workspace is NULL");
+  return chunk_two_pass(q, k, v, g, 4, nullptr, nullptr, 0.f, false, beta, scale, initial_state,
+                        cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, workspace,
+                        workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_segmented_ws launch",
+                        segment_chunks);
 }
 
 kda_status kda_chunk_fwd_gated_ws(const void *q, const void *k, const void *v, const void *g_raw,
@@ -392,7 +428,7 @@ kda_status kda_chunk_fwd_gated_ws(const void *q, const void *k, const void *v, c
   return chunk_two_pass(q, k, v, g_raw, esize(dt), A_log, dt_bias, lower_bound, true, beta, scale,
                         initial_state, cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state,
                         workspace, workspace_bytes, (cudaStream_t)stream,
-                        "kda_chunk_fwd_gated_ws launch");
+                        "kda_chunk_fwd_gated_ws launch", kda::rec::segment_chunks(N, T, H));
 }
 
 kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, const float *g,
@@ -420,12 +456,13 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
   if (st != KDA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
-  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, scratch, status, s);
+  const int L = kda::rec::segment_chunks(N, T, H);
+  if (cu_seqlens || L > 0) e = kda::launch_chunk_index(cu_seqlens, N, T, L, scratch, status, s);
   if (e == cudaSuccess)
     e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, scratch, nullptr,
                                nullptr, 0.f, false, status, s);
   if (e == cudaSuccess)
-    e = kda::launch_chunk_state(scratch, cu_seqlens, initial_state, scale, N, T, H, o,
+    e = kda::launch_chunk_state(scratch, cu_seqlens, initial_state, scale, N, T, H, L, o,
                                 final_state, status, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_static launch");
   return KDA_OK;
@@ -530,13 +567,15 @@ kda_status fused_two_pass(const void *x, const float *conv_w, const void *cache_
   kda_status st = device_status_word(&status);
   if (st != KDA_OK) return st;
   cudaError_t e = cudaSuccess;
-  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, workspace, status, s);
+  const int L = kda::rec::segment_chunks(N, T, H);
+  if (cu_seqlens || L > 0)
+    e = kda::launch_chunk_index(cu_seqlens, N, T, L, workspace, status, s);
   if (e == cudaSuccess)
     e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N, T,
                                         H, dt, workspace, A_log, dt_bias, lower_bound, gated,
                                         status, s);
   if (e == cudaSuccess)
-    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, o,
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, L, o,
                                 final_state, status, s);
   if (e == cudaSuccess && cu_seqlens && cache_out)
     e = kda::launch_cache_pass(workspace, N, H, cache_in, cache_out, s);

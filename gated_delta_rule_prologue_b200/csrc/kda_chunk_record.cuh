@@ -26,9 +26,25 @@
 //                     remainder beta v - f16(beta v) already added
 //   GL  exp(gamma_63) fp32 [128]
 //   PD  <q_r, k_r>    fp32 [64]
-// The workspace is [cprefix: int32 [N + 1], padded to 1 KB][records], record
-// (ci, h) at index ci * H + h, where ci numbers the chunks of all sequences
-// in order (cprefix[n] = first chunk of sequence n).
+// The workspace is [cprefix: int32 [N + 1], sprefix: int32 [N + 1], padded to
+// 1 KB][records][segment maps], record (ci, h) at index ci * H + h, where ci
+// numbers the chunks of all sequences in order (cprefix[n] = first chunk of
+// sequence n).
+//
+// Sequence-parallel state pass ("KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与
+// 状态压缩机制详解", Figure 1 and Figure 3: the chunk map S -> M S + B is affine,
+// so maps compose).  With a segment length of L chunks, sequence n is cut into
+// G_n = max(1, ceil(nch_n / L)) segments of balanced length; sprefix[n] numbers
+// the first segment of sequence n.  For every segment s that is not the last
+// of its sequence the segment area holds, per head, three fp32 128 x 128
+// blocks, each stored like a state (column-major: element (row r, column j)
+// at j * 128 + r):
+//   M  the segment's transition, end state = M * entry state + B (unused for
+//      the first segment of a sequence)
+//   B  the end state from a zero entry state
+//   E  the entry state of segment s (for the first segment of a split
+//      sequence, a copy of the caller's initial state)
+// With L = 0 every sequence is one segment and there is no segment area.
 #pragma once
 
 #include <stddef.h>
@@ -54,11 +70,72 @@ __host__ __device__ inline long long chunk_capacity(int N, int T) {
 }
 
 __host__ __device__ inline size_t header_bytes(int N) {
-  return ((size_t)(N + 1) * 4 + 1023) & ~(size_t)1023;
+  return ((size_t)(N + 1) * 8 + 1023) & ~(size_t)1023;
 }
 
-__host__ __device__ inline size_t workspace_bytes(int N, int T, int H) {
+// Bound on sum_n ceil(len_n / 64) for lengths summing to at most T:
+// sum floor((len_n + 63) / 64) <= floor((T + 63 N) / 64).
+__host__ __device__ inline long long chunk_sum_bound(int N, int T) {
+  return ((long long)T + 63LL * N) / 64;
+}
+
+// Bound on the number of segments: sum_n max(1, ceil(nch_n / L)) <= N + floor(sum nch_n / L).
+__host__ __device__ inline long long segment_capacity(int N, int T, int L) {
+  return L > 0 ? N + chunk_sum_bound(N, T) / L : N;
+}
+
+constexpr int kStateSlots = 444;   // resident state-pass CTAs: 148 SMs x 3
+
+// Model of the state pass's time (microseconds) for `ctas` CTAs that each walk
+// L chunks: waves of at most kStateSlots CTAs; a chunk step takes 2.9 us with
+// up to one CTA per SM, rising to 4.1 us at 2.5 CTAs per SM (the CTAs of an SM
+// share its tensor and memory pipes).  Fitted to B200 measurements of the
+// state kernel.
+inline double state_pass_us(long long ctas, long long L) {
+  if (ctas <= 0 || L <= 0) return 0.0;
+  const long long waves = (ctas + kStateSlots - 1) / kStateSlots;
+  const double occ = (double)((ctas + waves - 1) / waves) / 148.0;
+  double f = (occ - 1.0) / 1.5;
+  f = f < 0.0 ? 0.0 : f > 1.0 ? 1.0 : f;
+  return (double)waves * (double)L * (2.9 + 1.2 * f);
+}
+
+// Segment length of the state pass for a batch (0: one segment per sequence).
+// A batch whose (sequence, head, value slice) CTAs already fill two per SM
+// keeps whole sequences.  Otherwise the search assumes the worst chain, one
+// sequence holding all chunks: whole
+// sequences cost one chain of them; G >= 3 segments cost the transition pass
+// (8 CTAs per (segment, head) but 4 for the first segment), an entry-state
+// scan of G - 2 steps (2.6 us each) and the output pass, plus two launches.
+// The cheapest G wins if it saves at least 10%.
+inline int segment_chunks(int N, int T, int H) {
+  if (N < 1 || T < 1 || H < 1 || (long long)N * H * 4 >= 2 * 148) return 0;
+  const long long cb = chunk_sum_bound(N, T);
+  const double whole = state_pass_us((long long)N * H * 4, cb);
+  double best = 0.9 * whole;
+  int bestL = 0;
+  for (long long G = 3; G <= cb && G <= 256; ++G) {
+    const long long L = (cb + G - 1) / G, Gs = (cb + L - 1) / L;
+    if (Gs < 3) continue;
+    const double cost = state_pass_us(((Gs - 1) * 8 - 4) * H, L) +
+                        state_pass_us((Gs + N - 1) * 4 * H, L) + 2.6 * (double)(Gs - 2) + 8.0;
+    if (cost < best) {
+      best = cost;
+      bestL = (int)L;
+    }
+  }
+  return bestL;
+}
+
+constexpr size_t SEG_BLOCK = 128 * 128 * sizeof(float);
+
+__host__ __device__ inline size_t segment_area_offset(int N, int T, int H) {
   return header_bytes(N) + (size_t)chunk_capacity(N, T) * H * BYTES;
+}
+
+__host__ __device__ inline size_t workspace_bytes(int N, int T, int H, int L) {
+  return segment_area_offset(N, T, H) +
+         (L > 0 ? (size_t)segment_capacity(N, T, L) * H * 3 * SEG_BLOCK : 0);
 }
 
 }  // namespace rec

@@ -20,6 +20,17 @@
 //   S  = diag(G_last) S + D2          (fp32 registers; thread = key channel)
 // Operand roundings are those of the one-pass kernel: fp16 S, W, Q G, U, P,
 // K' with fp32 accumulation and fp32 diagonal terms.
+//
+// Sequence-parallel form (segment length L > 0, layout in kda_chunk_record.cuh):
+// a chunk maps S to M_c S + B_c with M_c = diag(G_last) - K'^T W and
+// B_c = K'^T Ut, so the same kernel run over a segment from the identity with
+// Ut = 0 yields the segment's transition M (value slices of the identity are
+// its columns), and run from a zero state yields B.  The transition pass
+// (kRole = kTransition, 8 CTAs per (segment, head): 4 column slices of M, 4
+// value slices of B) writes them; state_scan_kernel composes the entry states
+// E_{g+1} = M_g E_g + B_g in fp32; the output pass then runs every segment
+// from its entry state at once.  The first segment of a sequence runs from
+// the caller's initial state in the transition pass, so its B is E_1.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -51,29 +62,107 @@ constexpr uint32_t SB_ALLOC = SB_BAR + 64 + 1024;
 constexpr uint32_t TB_D1 = 0, TB_D1B = 32, TB_D2 = 64, TB_COLS = 128;
 static_assert(SB_KP + 24576 == SB_S, "K' and P are adjacent");
 
+enum { kOutputs = 0, kTransition = 1 };
+
+// Segment s (or sequence s when L == 0) of the batch: its sequence n, its
+// index g among the G segments of n, and its chunk range [c_lo, c_hi) within n.
+struct Segment {
+  int n, g, G, c_lo, c_hi;
+};
+
+__device__ __forceinline__ bool segment_of(const int32_t *cprefix, const int32_t *sprefix,
+                                           int N, int L, int s, int nch_whole, Segment &sg) {
+  if (L == 0) {
+    sg.n = s;
+    sg.g = 0;
+    sg.G = 1;
+    sg.c_lo = 0;
+    sg.c_hi = nch_whole;
+    return true;
+  }
+  if (s >= sprefix[N]) return false;
+  int lo = 0, hi = N - 1;  // last n with sprefix[n] <= s
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sprefix[mid] <= s) lo = mid;
+    else hi = mid - 1;
+  }
+  const int nch = cprefix[lo + 1] - cprefix[lo];
+  sg.n = lo;
+  sg.g = s - sprefix[lo];
+  sg.G = sprefix[lo + 1] - sprefix[lo];
+  sg.c_lo = (int)((long long)sg.g * nch / sg.G);
+  sg.c_hi = (int)((long long)(sg.g + 1) * nch / sg.G);
+  return true;
+}
+
+template <int kRole>
 __global__ void __launch_bounds__(kBT, 3)
 chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
-                   const float *s0, float scale, int N, int T, int H, float *__restrict__ o,
+                   const float *s0, float scale, int N, int T, int H, int L, float *__restrict__ o,
                    float *sN, int *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int slice = blockIdx.x % kSlices;
-  const int nh = blockIdx.x / kSlices, h = nh % H, n = nh / H;
+  constexpr int kParts = kRole == kTransition ? 2 : 1;
+  const int sub = blockIdx.x % (kSlices * kParts);
+  const int slice = sub & 3, part = sub >> 2;  // part (transition pass): 0 = M, 1 = B
+  const int item = blockIdx.x / (kSlices * kParts), h = item % H, s = item / H;
   const int32_t *cprefix = reinterpret_cast<const int32_t *>(ws);
+  const int32_t *sprefix = cprefix + (N + 1);
   const uint8_t *recs = ws + rec::header_bytes(N);
+  float *segbuf = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) +
+                                            rec::segment_area_offset(N, T, H));
   uint64_t *bar_a1 = reinterpret_cast<uint64_t *>(sm + SB_BAR);
   uint64_t *bar_kp = bar_a1 + 1, *bar_mma = bar_a1 + 2;
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SB_BAR + 32);
   float *exch = reinterpret_cast<float *>(sm + SB_S);
 
+  Segment sg;
+  {
+    const int n0 = L == 0 ? s : 0;
+    int bos0, eos0;
+    seq_bounds(cu, n0, T, status, bos0, eos0);
+    if (!segment_of(cprefix, sprefix, N, L, s, (eos0 - bos0 + 63) / 64, sg)) return;
+  }
+  const int n = sg.n;
   int bos, eos;
   seq_bounds(cu, n, T, status, bos, eos);
-  int cbase = 0, nch = (eos - bos + 63) / 64;
-  if (cu) {  // zero chunks for every sequence when the index pass rejected cu
+  int cbase = 0;
+  int c_lo = sg.c_lo, c_hi = sg.c_hi;
+  if (cu || L > 0) {  // zero chunks for every sequence when the index pass rejected cu
     cbase = cprefix[n];
-    nch = cprefix[n + 1] - cbase;
+    if (L == 0) c_hi = cprefix[n + 1] - cbase;
+  }
+  // Where the state comes from and goes to.  Slot (s, h, kind) of the segment area.
+  auto seg_slot = [&](int seg, int kind) -> float * {
+    return segbuf + (((size_t)seg * H + h) * 3 + kind) * (128 * 128);
+  };
+  const size_t head_off = ((size_t)n * H + h) * 128 * 128;
+  const float *s_in = nullptr;
+  float *s_out = nullptr, *s_copy = nullptr;
+  bool identity = false, use_ut = true;
+  if (kRole == kTransition) {
+    if (sg.g == sg.G - 1) return;           // the last segment needs no map
+    if (sg.g == 0 && part == 0) return;     // the first runs from the initial state
+    if (part == 0) {
+      identity = true;
+      use_ut = false;
+      s_out = seg_slot(s, 0);
+    } else if (sg.g == 0) {
+      s_in = s0 ? s0 + head_off : nullptr;
+      s_copy = seg_slot(s, 2);
+      s_out = seg_slot(s + 1, 2);
+    } else {
+      s_out = seg_slot(s, 1);
+    }
+  } else {
+    // A split sequence reads its initial state from the copy the transition
+    // pass took (E of its first segment): the final state may be written over
+    // the initial state by the last segment while the first is still to run.
+    s_in = sg.G > 1 ? seg_slot(s, 2) : s0 ? s0 + head_off : nullptr;
+    s_out = sg.g == sg.G - 1 && sN ? sN + head_off : nullptr;
   }
 
   if (warp == 0) tmem_alloc(slot, TB_COLS);
@@ -85,10 +174,15 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   }
   // S[i] = S[key tid][value 32 slice + i]; the state is stored value-major [dv][dk].
   const int t = tid;
-  const size_t sbase = ((size_t)n * H + h) * 128 * 128 + (size_t)slice * 32 * 128 + t;
+  const size_t sbase = (size_t)slice * 32 * 128 + t;
   float S[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) S[i] = s0 ? s0[sbase + (size_t)i * 128] : 0.f;
+  for (int i = 0; i < 32; ++i)
+    S[i] = identity ? (t == 32 * slice + i ? 1.f : 0.f) : s_in ? s_in[sbase + (size_t)i * 128] : 0.f;
+  if (s_copy) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s_copy[sbase + (size_t)i * 128] = S[i];
+  }
 
   auto write_s_operand = [&]() {  // S slice as the B operand: key row t, 32 values
     float amax = 0.f;
@@ -123,17 +217,19 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     mbar_arrive_expect_tx(bar_kp, 24576);
     bulk_load(sm + SB_KP, rec_of(c) + rec::KP, 24576, bar_kp);
   };
-  if (tid == 0 && nch > 0) {
-    load_a1(0);
-    load_kp(0);
+  if (tid == 0 && c_lo < c_hi) {
+    load_a1(c_lo);
+    load_kp(c_lo);
   }
 
   // Record values read by threads (Ut slice and <q_r, k_r> of token tid for
   // warps 0-1, exp(gamma_last) of key t for all) are fetched one chunk ahead.
   float ut[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) ut[i] = 0.f;
   float pd = 0.f, gl = 0.f;
   auto fetch_u = [&](int c) {
-    if (warp < 2) {
+    if (warp < 2 && use_ut) {
       const uint8_t *rp = rec_of(c);
       const float4 *src =
           reinterpret_cast<const float4 *>(rp + rec::UT + ((size_t)tid * 128 + slice * 32) * 4);
@@ -146,13 +242,13 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     }
   };
   auto fetch_gl = [&](int c) { gl = __ldg(reinterpret_cast<const float *>(rec_of(c) + rec::GL) + t); };
-  if (nch > 0) {
-    fetch_u(0);
-    fetch_gl(0);
+  if (c_lo < c_hi) {
+    fetch_u(c_lo);
+    fetch_gl(c_lo);
   }
 
   uint32_t pa = 0, pk = 0, pm = 0;
-  for (int c = 0; c < nch; ++c) {
+  for (int c = c_lo; c < c_hi; ++c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
 
     // ---- D1 = [W ; Q G] S ----------------------------------------------------------
@@ -173,7 +269,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     if (!wait_all(bar_mma, pm, status)) break;
     pm ^= 1;
     tc_fence_after();
-    if (tid == 0 && c + 1 < nch) load_a1(c + 1);  // A1 has been read
+    if (tid == 0 && c + 1 < c_hi) load_a1(c + 1);  // A1 has been read
 
     // ---- U = Ut - W S (warps 0-1: TMEM lanes 0..63 are the chunk's tokens) -------------
     if (warp < 2) {
@@ -187,7 +283,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       for (int i = 0; i < 32; ++i) {
         y[i] = ut[i] - (y[i] + y2[i]);  // U
         amax = fmaxf(amax, fabsf(y[i]));
-        exch[i * 64 + r] = pd * y[i];  // the S operand is dead until the next chunk
+        if (kRole == kOutputs) exch[i * 64 + r] = pd * y[i];  // S operand is dead until the next chunk
       }
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
@@ -197,7 +293,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
         st_shared_16(sm + SB_U, mn32_sw64_off(r, x), pack8_f16(f));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
-      if (c + 1 < nch) fetch_u(c + 1);
+      if (c + 1 < c_hi) fetch_u(c + 1);
     }
     fence_async_smem();
     tc_fence_before();
@@ -221,7 +317,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     if (!wait_all(bar_mma, pm, status)) break;
     pm ^= 1;
     tc_fence_after();
-    if (tid == 0 && c + 1 < nch) load_kp(c + 1);  // K' and P have been read
+    if (tid == 0 && c + 1 < c_hi) load_kp(c + 1);  // K' and P have been read
 
     // ---- outputs (warps 2-3: TMEM lanes 64..127) and the state update ---------------------
     {
@@ -229,9 +325,9 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       tmem_ld32(tmem + lane_addr + TB_D2, ds);
 #pragma unroll
       for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], gl, ds[i]);
-      if (c + 1 < nch) fetch_gl(c + 1);
+      if (c + 1 < c_hi) fetch_gl(c + 1);
     }
-    if (warp >= 2) {
+    if (kRole == kOutputs && warp >= 2) {
       float ov[32], ov2[32];
       tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
       tmem_ld32_nowait(tmem + lane_addr + TB_D1B, ov2);
@@ -259,63 +355,220 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     __syncthreads();
   }
 
-  if (sN) {
+  if (s_out) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) sN[sbase + (size_t)i * 128] = S[i];
+    for (int i = 0; i < 32; ++i) s_out[sbase + (size_t)i * 128] = S[i];
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, TB_COLS);
 }
 
-// cprefix[n] = number of chunks of sequences 0..n-1 (cprefix[N] = total).  A
-// malformed cu_seqlens (decreasing, or outside [0, T]) is recorded and gives
-// every sequence zero chunks, so no pass reads or writes past the workspace.
+// Inclusive-to-exclusive block scan step over 1024 threads: returns the
+// exclusive prefix of x among the threads and adds the block total to carry.
+__device__ __forceinline__ int block_exclusive_scan(int x, int *wsum, int &carry) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int v = x;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, d);
+    if (lane >= d) v += y;
+  }
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += y;
+    }
+    wsum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int r = carry + (warp > 0 ? wsum[warp - 1] : 0) + v - x;
+  carry += wsum[31];
+  __syncthreads();
+  return r;
+}
+
+// cprefix[n] = number of chunks of sequences 0..n-1 (cprefix[N] = total); with
+// a segment length L > 0 also sprefix[n] = number of segments of sequences
+// 0..n-1, sequence n having max(1, ceil(nch_n / L)).  cu == NULL is one
+// sequence of T tokens.  A malformed cu_seqlens (decreasing, or outside
+// [0, T]) is recorded and gives every sequence zero chunks and one segment,
+// so no pass reads or writes past the workspace.  A segment total above
+// seg_cap (not reachable for valid cu) falls back to one segment per sequence.
 __global__ void __launch_bounds__(1024)
-chunk_index_kernel(const int32_t *__restrict__ cu, int N, int T, int32_t *cprefix, int *status) {
+chunk_index_kernel(const int32_t *__restrict__ cu, int N, int T, int L, long long seg_cap,
+                   int32_t *cprefix, int *status) {
   __shared__ int bad;
   __shared__ int wsum[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t *sprefix = cprefix + (N + 1);
+  const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
   __syncthreads();
-  for (int i = tid; i < N; i += 1024) {
+  for (int i = tid; i < N && cu; i += 1024) {
     const int a = cu[i], b = cu[i + 1];
     if (a < 0 || b < a || b > T) bad = 1;
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) report(status, KDA_ERR_DEVICE_BOUNDS);
-    for (int i = tid; i <= N; i += 1024) cprefix[i] = 0;
+    for (int i = tid; i <= N; i += 1024) {
+      cprefix[i] = 0;
+      if (L > 0) sprefix[i] = i;
+    }
     return;
   }
-  int carry = 0;
+  int carry = 0, scarry = 0;
   for (int base = 0; base < N; base += 1024) {
     const int i = base + tid;
-    const int cnt = i < N ? (cu[i + 1] - cu[i] + 63) / 64 : 0;
-    int x = cnt;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, d);
-      if (lane >= d) x += y;
+    const int len = i < N ? (cu ? cu[i + 1] - cu[i] : T) : 0;
+    const int cnt = (len + 63) / 64;
+    const int c = block_exclusive_scan(cnt, wsum, carry);
+    if (i < N) cprefix[i] = c;
+    if (L > 0) {
+      const int sc = block_exclusive_scan(i < N ? max(1, (cnt + L - 1) / L) : 0, wsum, scarry);
+      if (i < N) sprefix[i] = sc;
     }
-    if (lane == 31) wsum[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = wsum[lane];
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, d);
-        if (lane >= d) w += y;
-      }
-      wsum[lane] = w;  // inclusive over warps
-    }
-    __syncthreads();
-    const int before = warp > 0 ? wsum[warp - 1] : 0;
-    if (i < N) cprefix[i] = carry + before + x - cnt;
-    carry += wsum[31];
-    __syncthreads();
   }
-  if (tid == 0) cprefix[N] = carry;
+  if (tid == 0) {
+    cprefix[N] = carry;
+    if (L > 0) sprefix[N] = scarry;
+  }
+  if (L > 0 && scarry > seg_cap) {
+    __syncthreads();
+    for (int i = tid; i <= N; i += 1024) sprefix[i] = i;
+  }
+}
+
+// Entry states of the segments: E_1 (written by the transition pass) and
+// E_{g+1} = M_g E_g + B_g for g = 1 .. G-2, in fp32.  One CTA per (sequence,
+// head, 8 value columns).  E_g sits in shared memory; M_g (64 KB, stored
+// column by column) is brought into shared memory by a bulk copy,
+// double-buffered so that M_{g+1} arrives while step g computes.  Warp w sums
+// the key channels k in [32 w, 32 w + 32) and lane l rows l + 32 i (i < 4), so
+// each broadcast read of a row of E_g feeds four rows; the four warps' partial
+// sums meet in shared memory, where thread r adds up row r.
+constexpr int kScanCols = 8;
+constexpr uint32_t SC_M = 0;                                   // 2 x 64 KB
+constexpr uint32_t SC_E = 2 * 65536;                           // [128][kScanCols] fp32
+constexpr uint32_t SC_P = SC_E + 128 * kScanCols * 4;          // [4][128][kScanCols] fp32
+constexpr uint32_t SC_BAR = SC_P + 4 * 128 * kScanCols * 4;    // two mbarriers
+constexpr uint32_t SC_ALLOC = SC_BAR + 16 + 128;               // + alignment slack
+
+__global__ void __launch_bounds__(128)
+state_scan_kernel(const uint8_t *__restrict__ ws, int N, int T, int H, int *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                            ~static_cast<uintptr_t>(127));
+  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
+  const int cb = blockIdx.x % (128 / kScanCols), nh = blockIdx.x / (128 / kScanCols);
+  const int h = nh % H, n = nh / H;
+  const int32_t *sprefix = reinterpret_cast<const int32_t *>(ws) + (N + 1);
+  const int s0 = sprefix[n], G = sprefix[n + 1] - s0;
+  if (G <= 2) return;
+  float *segbuf = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) +
+                                            rec::segment_area_offset(N, T, H));
+  auto slot = [&](int seg, int kind) -> float * {
+    return segbuf + (((size_t)seg * H + h) * 3 + kind) * (128 * 128);
+  };
+  constexpr int kQ = kScanCols / 4;  // float4 per row
+  float4 *Es = reinterpret_cast<float4 *>(sm + SC_E);
+  float4 *Ps = reinterpret_cast<float4 *>(sm + SC_P);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SC_BAR);
+  if (r == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, 65536);
+    bulk_load(sm + SC_M, slot(s0 + 1, 0), 65536, bar);
+  }
+  const int j0 = cb * kScanCols;
+  {
+    const float *e = slot(s0 + 1, 2);
+    float v[kScanCols];
+#pragma unroll
+    for (int j = 0; j < kScanCols; ++j) v[j] = e[(size_t)(j0 + j) * 128 + r];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q)
+      Es[r * kQ + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+  __syncthreads();
+  // B_g (row r) is read one step ahead, so its latency hides behind the step before.
+  float bnext[kScanCols];
+  auto load_b = [&](int g) {
+    const float *B = slot(s0 + g, 1);
+#pragma unroll
+    for (int j = 0; j < kScanCols; ++j) bnext[j] = B[(size_t)(j0 + j) * 128 + r];
+  };
+  load_b(1);
+  uint32_t phase = 0;  // bit b: parity of buffer b
+  for (int g = 1; g + 1 < G; ++g) {
+    const int b = (g - 1) & 1;
+    if (r == 0 && g + 2 < G) {  // buffer b^1 was last read in step g - 1
+      mbar_arrive_expect_tx(bar + (b ^ 1), 65536);
+      bulk_load(sm + SC_M + (b ^ 1) * 65536, slot(s0 + g + 1, 0), 65536, bar + (b ^ 1));
+    }
+    float bcur[kScanCols];
+#pragma unroll
+    for (int j = 0; j < kScanCols; ++j) bcur[j] = bnext[j];
+    if (g + 2 < G) load_b(g + 1);
+    if (!wait_all(bar + b, (phase >> b) & 1, status)) return;
+    phase ^= 1u << b;
+    const float *Ms = reinterpret_cast<const float *>(sm + SC_M + b * 65536);
+    float acc[4][kScanCols];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < kScanCols; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < 32; ++kk) {
+      const int k = 32 * warp + kk;
+      float m[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[i] = Ms[k * 128 + lane + 32 * i];  // M_g[row][k]
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        const float4 e = Es[k * kQ + q];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i][4 * q] = fmaf(m[i], e.x, acc[i][4 * q]);
+          acc[i][4 * q + 1] = fmaf(m[i], e.y, acc[i][4 * q + 1]);
+          acc[i][4 * q + 2] = fmaf(m[i], e.z, acc[i][4 * q + 2]);
+          acc[i][4 * q + 3] = fmaf(m[i], e.w, acc[i][4 * q + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < kQ; ++q)
+        Ps[(warp * 128 + lane + 32 * i) * kQ + q] =
+            make_float4(acc[i][4 * q], acc[i][4 * q + 1], acc[i][4 * q + 2], acc[i][4 * q + 3]);
+    __syncthreads();  // partial sums written; every thread has read E_g and M_g
+    float out[kScanCols];
+#pragma unroll
+    for (int j = 0; j < kScanCols; ++j) out[j] = bcur[j];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        const float4 p = Ps[(w * 128 + r) * kQ + q];
+        out[4 * q] += p.x;
+        out[4 * q + 1] += p.y;
+        out[4 * q + 2] += p.z;
+        out[4 * q + 3] += p.w;
+      }
+    float *e = slot(s0 + g + 1, 2);
+#pragma unroll
+    for (int j = 0; j < kScanCols; ++j) e[(size_t)(j0 + j) * 128 + r] = out[j];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q)
+      Es[r * kQ + q] = make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+    __syncthreads();  // E_{g+1} in place; the partial sums have been read
+  }
 }
 
 // Fused two-pass prefill: a sequence without chunks (empty, or every sequence
@@ -342,23 +595,46 @@ cudaError_t launch_cache_pass(const void *ws, int N, int H, const void *cache_in
   return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *status,
+cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws, int *status,
                                cudaStream_t s) {
-  chunk_index_kernel<<<1, 1024, 0, s>>>(cu, N, T, static_cast<int32_t *>(ws), status);
+  chunk_index_kernel<<<1, 1024, 0, s>>>(cu, N, T, L, rec::segment_capacity(N, T, L),
+                                        static_cast<int32_t *>(ws), status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
-                               int N, int T, int H, float *o, float *sN, int *status,
-                               cudaStream_t s) {
-  const long long blocks = (long long)N * H * kSlices;
+namespace {
+template <int kRole>
+cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0, float scale,
+                              int N, int T, int H, int L, float *o, float *sN, int *status,
+                              cudaStream_t s) {
+  const long long items = L > 0 ? rec::segment_capacity(N, T, L) : N;
+  const long long blocks = items * H * kSlices * (kRole == kTransition ? 2 : 1);
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel,
+  cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<kRole>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB_ALLOC);
   if (e != cudaSuccess) return e;
-  chunk_state_kernel<<<(unsigned)blocks, kBT, SB_ALLOC, s>>>(
-      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, o, sN, status);
+  chunk_state_kernel<kRole><<<(unsigned)blocks, kBT, SB_ALLOC, s>>>(
+      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, status);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
+                               int N, int T, int H, int L, float *o, float *sN, int *status,
+                               cudaStream_t s) {
+  cudaError_t e;
+  if (L > 0) {
+    e = launch_state_role<kTransition>(ws, cu, s0, scale, N, T, H, L, o, sN, status, s);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SC_ALLOC);
+    if (e != cudaSuccess) return e;
+    state_scan_kernel<<<N * H * (128 / kScanCols), 128, SC_ALLOC, s>>>(
+        static_cast<const uint8_t *>(ws), N, T, H, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return launch_state_role<kOutputs>(ws, cu, s0, scale, N, T, H, L, o, sN, status, s);
 }
 
 }  // namespace kda

@@ -204,17 +204,20 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             int N, int T, int H, kda_dtype dt, float *o, float *sN, int *status,
                             cudaStream_t s);
 // Two-pass tensor-core prefill (kda_chunk_record.cuh): the prep pass over all
-// (chunk, head) items, then the state pass over (sequence, head, value slice).
+// (chunk, head) items, then the state pass over (segment, head, value slice);
+// L is the segment length in chunks (0: whole sequences), and with L > 0 the
+// index pass must run (for cu == NULL too) and the state pass is the
+// transition pass, the entry-state scan and the output pass.
 // g: fp32 log-decay, or (gated) 16-bit gate pre-activations of type dt turned
 // into the log-decay in the kernel (A_log, dt_bias may be null).
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const void *g,
                               const float *beta, const int32_t *cu, int N, int T, int H,
                               kda_dtype dt, void *ws, const float *A_log, const float *dt_bias,
                               float lower_bound, bool gated, int *status, cudaStream_t s);
-cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, void *ws, int *status,
+cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws, int *status,
                                cudaStream_t s);
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
-                               int N, int T, int H, float *o, float *sN, int *status,
+                               int N, int T, int H, int L, float *o, float *sN, int *status,
                                cudaStream_t s);
 cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
                                        void *cache_out, const void *g, const float *beta,

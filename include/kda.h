@@ -124,12 +124,34 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
 /*
  * kda_chunk_fwd_workspace_bytes -- bytes of scratch kda_chunk_fwd_ws needs for
  * these sizes: one 88.75 KiB record per (chunk, head) plus a 1 KiB-aligned
- * chunk index, sized for the worst case of N sequences in T tokens
- * (ceil(T/64) + N chunks per head).  0 when the arguments do not select the
- * tensor-core path (dt == KDA_F32, Dk or Dv != 128, chunk != 64, T == 0).
+ * chunk and segment index, sized for the worst case of N sequences in T
+ * tokens (ceil(T/64) + N chunks per head), plus, when these sizes split
+ * sequences into segments (kda_chunk_fwd_segment_chunks > 0), 192 KiB per
+ * (segment, head) for the segment maps.  0 when the arguments do not select
+ * the tensor-core path (dt == KDA_F32, Dk or Dv != 128, chunk != 64, T == 0).
  */
 size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
                                      kda_dtype dt);
+
+/*
+ * kda_chunk_fwd_segment_chunks -- the segment length, in 64-token chunks, that
+ * the workspace entry points (kda_chunk_fwd_ws, kda_chunk_fwd_gated_ws,
+ * kda_chunk_fwd_static and the two-pass prologue entry points) use for these
+ * sizes; 0 means every sequence is carried whole by one chain of CTAs.  A
+ * batch whose (sequence, head, 32 value channels) chains already fill two
+ * CTAs per SM is not split; otherwise sequences are cut into segments of at
+ * most this many chunks (at least 4) so that the segment maps fill the GPU.
+ * 0 for invalid sizes.
+ */
+int kda_chunk_fwd_segment_chunks(int N, int T, int H);
+
+/*
+ * kda_chunk_fwd_segmented_workspace_bytes -- kda_chunk_fwd_workspace_bytes
+ * for an explicit segment length (segment_chunks >= 0; 0: whole sequences).
+ * 0 for arguments off the tensor-core path or a negative segment_chunks.
+ */
+size_t kda_chunk_fwd_segmented_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                               kda_dtype dt, int segment_chunks);
 
 /*
  * kda_chunk_fwd_ws -- kda_chunk_fwd with a caller-owned scratch buffer, which
@@ -138,7 +160,9 @@ size_t kda_chunk_fwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int ch
  * carried state, so the first pass computes it for all (chunk, head) pairs
  * at once (in-chunk log-decay, Gram products, the WY solve of [W5 §10.3]) and
  * the second carries the state through the chunks of each sequence in order,
- * one CTA per (sequence, head, 32 value channels).  Same arguments and
+ * one CTA per (sequence, head, 32 value channels), or per (segment, head, 32
+ * value channels) when kda_chunk_fwd_segment_chunks splits the sequences (see
+ * kda_chunk_fwd_segmented_ws).  Same arguments and
  * results as kda_chunk_fwd (equal up to rounding order), plus:
  *   workspace        device buffer of >= kda_chunk_fwd_workspace_bytes(...)
  *                    bytes, 16-byte aligned, owned by the caller; its contents
@@ -153,6 +177,32 @@ kda_status kda_chunk_fwd_ws(const void *q, const void *k, const void *v, const f
                             const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
                             int chunk, kda_dtype dt, float *o, float *final_state,
                             void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_segmented_ws -- kda_chunk_fwd_ws with the sequence-parallel
+ * state pass at an explicit segment length.  [W4 Figure 1, Figure 3]: the
+ * chunk update is an affine map of the entry state, S -> M S + B with
+ * M = diag(exp(gamma_last)) - K'^T W and B = K'^T Ut, so maps compose.  Each
+ * sequence of nch chunks is cut into G = max(1, ceil(nch / segment_chunks))
+ * segments of balanced length; a transition pass computes, for every segment
+ * but the last, its map (M from the identity with Ut = 0, B from a zero
+ * state; the first segment runs from the initial state) with the same
+ * tensor-core chunk update; an fp32 scan composes the entry states; the output
+ * pass then runs all segments at once from their entry states.
+ * Same arguments and results as kda_chunk_fwd_ws (equal up to rounding), plus:
+ *   segment_chunks   >= 0 (KDA_ERR_INVALID_ARG if negative); 0: whole sequences
+ *   workspace        device buffer of >= kda_chunk_fwd_segmented_workspace_bytes
+ *                    (..., segment_chunks) bytes, 16-byte aligned, caller-owned,
+ *                    not NULL; the same overlap and concurrency rules
+ * Tensor-core path only (else KDA_ERR_UNSUPPORTED).
+ */
+kda_status kda_chunk_fwd_segmented_ws(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, float scale,
+                                      const float *initial_state, const int32_t *cu_seqlens,
+                                      int N, int T, int H, int Dk, int Dv, int chunk,
+                                      kda_dtype dt, float *o, float *final_state,
+                                      int segment_chunks, void *workspace,
+                                      size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * The *_gated entry points take the gate pre-activations instead of the

@@ -139,21 +139,74 @@ def test_fused_prefill_rejects_bad_arguments(kda):
 
 
 def test_chunk_workspace_size(kda):
-    """Two-pass scratch: a 1 KiB-aligned int32 chunk index of N + 1 entries,
-    then one record per (chunk, head) for ceil(T/64) + N chunks per head;
+    """Two-pass scratch: a 1 KiB-aligned int32 chunk index and segment index of
+    N + 1 entries each, then one record per (chunk, head) for ceil(T/64) + N
+    chunks per head, then (segment length L > 0) three 64 KiB fp32 blocks per
+    (segment, head) for at most N + floor((T + 63 N) / 64 / L) segments;
     nothing for calls that do not take the tensor-core path."""
     import torch
     f = kda.kda_chunk_fwd_workspace_bytes
-    rec = f(1, 64, 1, 128, 128, 64, torch.bfloat16) - 1024
+    fs = kda.kda_chunk_fwd_segmented_workspace_bytes
+    rec = fs(1, 64, 1, 128, 128, 64, torch.bfloat16, 0) - 1024
     assert rec > 0 and rec % 32 == 0   # two records (ceil(64/64) + N = 2), 16-byte multiples
-    for N, T, H in ((1, 32768, 96), (16, 93891, 32), (300, 1000, 2)):
-        header = ((N + 1) * 4 + 1023) // 1024 * 1024
-        expect = header + ((T + 63) // 64 + N) * H * (rec // 2)
-        assert f(N, T, H, 128, 128, 64, torch.float16) == expect
+    rec //= 2
+    for N, T, H in ((1, 32768, 96), (16, 93891, 32), (300, 1000, 2), (1, 4096, 8), (3, 999, 2)):
+        header = ((N + 1) * 8 + 1023) // 1024 * 1024
+        base = header + ((T + 63) // 64 + N) * H * rec
+        for L in (0, 1, 3, 10):
+            seg = 0 if L == 0 else (N + (T + 63 * N) // 64 // L) * H * 3 * 65536
+            assert fs(N, T, H, 128, 128, 64, torch.float16, L) == base + seg
+        L = kda.kda_chunk_fwd_segment_chunks(N, T, H)
+        assert f(N, T, H, 128, 128, 64, torch.float16) == fs(N, T, H, 128, 128, 64,
+                                                             torch.float16, L)
     assert f(1, 64, 1, 128, 128, 64, torch.float32) == 0
     assert f(1, 64, 1, 64, 64, 64, torch.bfloat16) == 0
     assert f(1, 64, 1, 128, 128, 32, torch.bfloat16) == 0
     assert f(1, 0, 1, 128, 128, 64, torch.bfloat16) == 0
+    assert fs(1, 64, 1, 128, 128, 64, torch.bfloat16, -1) == 0
+
+
+def test_segment_length_choice(kda):
+    """Sequences are split only when the (sequence, head, 32-value-channel)
+    chains fill fewer than two CTAs per SM of 148, and only into three or more
+    segments (with two, the transition and output passes walk as many chunks
+    one after the other as the whole sequence does)."""
+    sc = kda.kda_chunk_fwd_segment_chunks
+    assert sc(1, 32768, 96) == 0        # 384 chains: whole sequences
+    assert sc(16, 130000, 32) == 0      # varlen batch of 16 x 32 heads
+    assert sc(1, 4096, 32) == 0         # 128 chains of 64 chunks: no split pays
+    assert sc(1, 4096, 8) == 8          # 64 chunks, 8 heads: 8 segments of 8
+    assert sc(1, 256, 2) == 0           # 4 chunks
+    assert sc(2, 64, 1) == 0
+    assert sc(0, 64, 1) == 0 and sc(1, -1, 1) == 0 and sc(1, 64, 0) == 0
+    for T, H in ((1000, 2), (8192, 2), (16384, 8), (32768, 16), (131072, 1), (4096, 16)):
+        L = sc(1, T, H)
+        nch = (T + 63) // 64
+        assert L > 0 and (nch + L - 1) // L >= 3, (T, H, L)
+
+
+def test_chunk_fwd_segmented_rejects_bad_arguments(kda):
+    """Argument checks run before any device call: a negative segment length,
+    a NULL or short workspace, and sizes off the tensor-core path."""
+    import torch
+    L = kda.lib
+    T, H = 640, 2
+    need = kda.kda_chunk_fwd_segmented_workspace_bytes(1, T, H, 128, 128, 64, torch.bfloat16, 3)
+    assert need > kda.kda_chunk_fwd_segmented_workspace_bytes(1, T, H, 128, 128, 64,
+                                                              torch.bfloat16, 0)
+    q, k, v = _vp(0x100000), _vp(0x200000), _vp(0x300000)
+    g, beta, o = _vp(0x400000), _vp(0x800000), _vp(0x900000)
+    ws = _vp(0x1000000)
+    args = (q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o, None)
+    st = L.kda_chunk_fwd_segmented_ws(*args, -1, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"negative" in L.kda_last_error()
+    st = L.kda_chunk_fwd_segmented_ws(*args, 3, None, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace is NULL" in L.kda_last_error()
+    st = L.kda_chunk_fwd_segmented_ws(*args, 3, ws, need - 16, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace holds" in L.kda_last_error()
+    f32 = (q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 0, o, None)
+    st = L.kda_chunk_fwd_segmented_ws(*f32, 3, ws, need, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
 
 
 def test_chunk_fwd_ws_rejects_bad_workspace(kda):
