@@ -550,7 +550,17 @@ def run_ncu_case(args):
     of the workload, for profiling runs; prints nothing."""
     import gated_delta_rule_prologue_b200 as kda
     dev = torch.device("cuda", 0)
-    if args.ncu_case == "decode":
+    if args.ncu_case in ("seq4k", "seq4k_whole"):
+        sinp = W.seq4k_bf16()
+        args4 = [t.to(dev) for t in (sinp.q, sinp.k, sinp.v, sinp.g, sinp.beta)]
+        s04 = sinp.initial_state.to(dev)
+        o = torch.empty(sinp.q.shape, device=dev)
+        fs = torch.empty_like(s04)
+        seg = None if args.ncu_case == "seq4k" else 0
+        for _ in range(2):
+            kda.kda_chunk_fwd(*args4, o, scale=sinp.scale, initial_state=s04, final_state=fs,
+                              segment_chunks=seg)
+    elif args.ncu_case == "decode":
         d = W.decode256(steps=2)
         state, cache = d.state.to(dev), d.conv_cache.to(dev)
         w = d.conv_w.to(dev)
@@ -594,7 +604,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode"),
+    ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode",
+                                           "seq4k", "seq4k_whole"),
                     help="profiling mode: launch one kernel twice on a workload slice and exit")
     ap.add_argument("--ncu-tokens", type=int, default=4096)
     args = ap.parse_args()
