@@ -12,8 +12,10 @@ from .kda_oracle import (  # noqa: F401
     L2_EPS,
     gate,
     kda_chunkwise,
+    kda_chunkwise_backward,
     kda_decode_step,
     kda_recurrent,
+    kda_recurrent_backward,
     l2_normalize,
     output_epilogue,
     prologue,

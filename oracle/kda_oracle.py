@@ -203,6 +203,68 @@ def kda_recurrent(q, k, v, g, beta, scale=1.0, initial_state=None, cu_seqlens=No
     return o, final
 
 
+def kda_recurrent_backward(q, k, v, g, beta, do, d_final_state=None, scale=1.0,
+                           initial_state=None, cu_seqlens=None):
+    """Gradients of the token-by-token recurrence (reverse-mode, float64).
+
+    The loss is taken as L = sum(do * o) + sum(d_final_state * final_state),
+    with ``o`` and ``final_state`` those of :func:`kda_recurrent`; this is the
+    adjoint of each step of that recurrence, taken in reverse token order:
+
+        after the read  o_t = scale S_t^T q_t:
+            dS_t += scale q_t do_t^T;          dq_t = scale S_t do_t
+        after the write S_t = Sd + beta_t k_t e^T (Sd the decayed state):
+            dbeta_t = k_t^T dS_t e;            dk_t = beta_t dS_t e
+            de = beta_t dS_t^T k_t;            dSd = dS_t
+        after the error e = v_t - Sd^T k_t:
+            dv_t = de;  dSd -= k_t de^T;       dk_t -= Sd de
+        after the decay Sd = diag(exp(g_t)) S_{t-1}:
+            dg_t = rowsum(dSd * Sd);           dS_{t-1} = diag(exp(g_t)) dSd
+
+    Training is mentioned on [W1 彩蛋]; the pages give no backward, so this
+    is the plain chain rule through the forward definition.  Shapes as in
+    :func:`kda_recurrent`; ``do`` [T, H, Dv]; ``d_final_state`` [N, H, Dk,
+    Dv] (key-first) or None.  Returns dq, dk, dg [T, H, Dk], dv [T, H, Dv],
+    dbeta [T, H] and d_initial_state [N, H, Dk, Dv].
+    """
+    q, k, v, g, beta, do = (_f64(a) for a in (q, k, v, g, beta, do))
+    T, H, Dk = k.shape
+    Dv = v.shape[2]
+    segs = _segments(T, cu_seqlens)
+    s0 = None if initial_state is None else _f64(initial_state)
+    dsN = None if d_final_state is None else _f64(d_final_state)
+    dq, dk, dg = np.zeros((T, H, Dk)), np.zeros((T, H, Dk)), np.zeros((T, H, Dk))
+    dv, dbeta = np.zeros((T, H, Dv)), np.zeros((T, H))
+    ds0 = np.zeros((len(segs), H, Dk, Dv))
+    for n, (a, b) in enumerate(segs):
+        # forward, keeping the decayed state, the error and the state after each token
+        S = np.zeros((H, Dk, Dv)) if s0 is None else s0[n].copy()
+        Sd_hist, err_hist, S_hist = [], [], []
+        for t in range(a, b):
+            Sd = S * np.exp(g[t])[:, :, None]
+            err = v[t] - np.einsum("hkv,hk->hv", Sd, k[t])
+            S = Sd + beta[t][:, None, None] * k[t][:, :, None] * err[:, None, :]
+            Sd_hist.append(Sd)
+            err_hist.append(err)
+            S_hist.append(S)
+        dS = np.zeros((H, Dk, Dv)) if dsN is None else dsN[n].copy()
+        for t in range(b - 1, a - 1, -1):
+            i = t - a
+            Sd, err, St = Sd_hist[i], err_hist[i], S_hist[i]
+            dS = dS + scale * q[t][:, :, None] * do[t][:, None, :]
+            dq[t] = scale * np.einsum("hkv,hv->hk", St, do[t])
+            dSe = np.einsum("hkv,hv->hk", dS, err)           # dS_t e
+            dbeta[t] = np.einsum("hk,hk->h", k[t], dSe)
+            de = beta[t][:, None] * np.einsum("hkv,hk->hv", dS, k[t])
+            dv[t] = de
+            dk[t] = beta[t][:, None] * dSe - np.einsum("hkv,hv->hk", Sd, de)
+            dSd = dS - k[t][:, :, None] * de[:, None, :]
+            dg[t] = np.einsum("hkv,hkv->hk", dSd, Sd)
+            dS = dSd * np.exp(g[t])[:, :, None]
+        ds0[n] = dS
+    return dq, dk, dv, dg, dbeta, ds0
+
+
 # ---------------------------------------------------------------------------
 # Chunkwise evaluation (second oracle)
 # ---------------------------------------------------------------------------
@@ -267,6 +329,108 @@ def kda_chunkwise(q, k, v, g, beta, scale=1.0, initial_state=None, cu_seqlens=No
                 S[h] = G[-1][:, None] * S[h] + (Kc * (G[-1] / G)).T @ U
         final[n] = S
     return o, final
+
+
+def _solve_unit_upper_transposed(L, rhs):
+    """Solve ``L^T X = rhs`` for unit-lower-triangular ``L`` by back
+    substitution (row by row, last first)."""
+    n = L.shape[0]
+    X = np.zeros_like(rhs)
+    for r in range(n - 1, -1, -1):
+        X[r] = rhs[r] - L[r + 1:, r] @ X[r + 1:]
+    return X
+
+
+def kda_chunkwise_backward(q, k, v, g, beta, do, d_final_state=None, scale=1.0,
+                           initial_state=None, cu_seqlens=None, chunk=64):
+    """Gradients of :func:`kda_chunkwise`, chunk by chunk (second oracle).
+
+    The chain rule through the chunk algebra of :func:`kda_chunkwise`, in
+    float64, with the entry state of every chunk from a forward sweep and
+    the adjoint of its exit state dS' from the chunk after it (reverse sweep).
+    With R = diag(beta)(V - (K*G) S0) (so U = (I + A)^{-1} R), K' = K*G_last/G
+    and dO' = scale dO, per chunk:
+
+        dU  = P^T dO' + K' dS'               dP  = lower(dO' U^T)
+        dR  = (I + A)^{-T} dU                dA  = -strict_lower(dR U^T)
+        dV  = diag(beta) dR                  dK' = U dS'^T
+        dQG = dO' S0^T + dP (K/G)
+        dKG = -diag(beta) dR S0^T + diag(beta) dA (K/G)
+        dKD = (diag(beta) dA)^T (K*G) + dP^T (Q*G)
+        dbeta_r = <dR_r, V_r - ((K*G) S0)_r> + sum_i dA[r,i] ((K*G)(K/G)^T)[r,i]
+        dS0 = diag(G_last) dS' + (Q*G)^T dO' - (diag(beta) K*G)^T dR
+        dq = dQG*G;   dk = dKG*G + dKD/G + dK'*G_last/G
+        dgamma = dQG*(Q*G) + dKG*(K*G) - dKD*(K/G) - dK'*K', and on the last
+                 row also + G_last*rowsum(S0*dS') + sum_i dK'_i*K'_i
+        dg = reverse cumulative sum of dgamma over the chunk's rows
+
+    (the gradient of gamma_r = sum_{j<=r} g_j).  Must agree with
+    :func:`kda_recurrent_backward` up to rounding; same shapes and returns.
+    """
+    q, k, v, g, beta, do = (_f64(a) for a in (q, k, v, g, beta, do))
+    T, H, Dk = k.shape
+    Dv = v.shape[2]
+    segs = _segments(T, cu_seqlens)
+    s0 = None if initial_state is None else _f64(initial_state)
+    dsN = None if d_final_state is None else _f64(d_final_state)
+    dq, dk, dg = np.zeros((T, H, Dk)), np.zeros((T, H, Dk)), np.zeros((T, H, Dk))
+    dv, dbeta = np.zeros((T, H, Dv)), np.zeros((T, H))
+    ds0 = np.zeros((len(segs), H, Dk, Dv))
+    for n, (a, b) in enumerate(segs):
+        starts = list(range(a, b, chunk))
+        # forward sweep: entry state of every chunk
+        S = np.zeros((H, Dk, Dv)) if s0 is None else s0[n].copy()
+        entry = []
+        for c0 in starts:
+            entry.append(S.copy())
+            c1 = min(c0 + chunk, b)
+            for h in range(H):
+                Kc, Vc, bc = k[c0:c1, h], v[c0:c1, h], beta[c0:c1, h]
+                G = np.exp(np.cumsum(g[c0:c1, h], axis=0))
+                KG, KD = Kc * G, Kc / G
+                A = np.tril(bc[:, None] * (KG @ KD.T), k=-1)
+                R = bc[:, None] * (Vc - KG @ S[h])
+                U = _solve_unit_lower(np.eye(c1 - c0) + A, R)
+                S[h] = G[-1][:, None] * S[h] + (Kc * (G[-1] / G)).T @ U
+        # reverse sweep
+        dS = np.zeros((H, Dk, Dv)) if dsN is None else dsN[n].copy()
+        for ci in range(len(starts) - 1, -1, -1):
+            c0 = starts[ci]
+            c1 = min(c0 + chunk, b)
+            L = c1 - c0
+            for h in range(H):
+                S0c = entry[ci][h]
+                Kc, Qc, Vc = k[c0:c1, h], q[c0:c1, h], v[c0:c1, h]
+                bc = beta[c0:c1, h]
+                G = np.exp(np.cumsum(g[c0:c1, h], axis=0))
+                KG, KD, QG = Kc * G, Kc / G, Qc * G
+                KK = KG @ KD.T
+                A = np.tril(bc[:, None] * KK, k=-1)
+                P = np.tril(QG @ KD.T, k=0)
+                E = Vc - KG @ S0c
+                R = bc[:, None] * E
+                U = _solve_unit_lower(np.eye(L) + A, R)
+                Kp = Kc * (G[-1] / G)
+                dOp = scale * do[c0:c1, h]
+                dSp = dS[h]
+                dU = P.T @ dOp + Kp @ dSp
+                dP = np.tril(dOp @ U.T, k=0)
+                dR = _solve_unit_upper_transposed(np.eye(L) + A, dU)
+                dA = -np.tril(dR @ U.T, k=-1)
+                dKp = U @ dSp.T
+                dQG = dOp @ S0c.T + dP @ KD
+                dKG = -bc[:, None] * (dR @ S0c.T) + bc[:, None] * (dA @ KD)
+                dKD = (bc[:, None] * dA).T @ KG + dP.T @ QG
+                dv[c0:c1, h] = bc[:, None] * dR
+                dbeta[c0:c1, h] = np.sum(dR * E, axis=1) + np.sum(dA * KK, axis=1)
+                dq[c0:c1, h] = dQG * G
+                dk[c0:c1, h] = dKG * G + dKD / G + dKp * (G[-1] / G)
+                dgam = dQG * QG + dKG * KG - dKD * KD - dKp * Kp
+                dgam[-1] += G[-1] * np.sum(S0c * dSp, axis=1) + np.sum(dKp * Kp, axis=0)
+                dg[c0:c1, h] = np.cumsum(dgam[::-1], axis=0)[::-1]
+                dS[h] = G[-1][:, None] * dSp + QG.T @ dOp - (bc[:, None] * KG).T @ dR
+        ds0[n] = dS
+    return dq, dk, dv, dg, dbeta, ds0
 
 
 # ---------------------------------------------------------------------------
