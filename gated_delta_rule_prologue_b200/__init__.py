@@ -91,6 +91,11 @@ lib.kda_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_chunk_fwd_segmented_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 lib.kda_chunk_fwd_segmented_workspace_bytes.restype = ctypes.c_size_t
+lib.kda_chunk_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+lib.kda_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
+lib.kda_chunk_bwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                 _vp]
 lib.kda_chunk_fwd_segment_chunks.argtypes = [_i, _i, _i]
 lib.kda_chunk_fwd_segment_chunks.restype = ctypes.c_int
 lib.kda_chunk_fwd_segmented_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
@@ -100,7 +105,7 @@ lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _v
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
-            lib.kda_chunk_fwd_segmented_ws,
+            lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_output_epilogue,
@@ -262,6 +267,53 @@ def _chunk_fwd_segmented(q, k, v, g, beta, o, scale, initial_state, final_state,
                                           T, H, Dk, Dv, chunk, _dtype(q), _ptr(o),
                                           _ptr(final_state), segment_chunks, _ptr(workspace),
                                           workspace.numel(), _stream(stream)))
+
+
+def kda_chunk_bwd_workspace_bytes(N: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
+                                  dtype: torch.dtype) -> int:
+    """Scratch bytes of :func:`kda_chunk_bwd` (0 off the tensor-core shapes)."""
+    return int(lib.kda_chunk_bwd_workspace_bytes(N, T, H, Dk, Dv, chunk, _DTYPES[dtype]))
+
+
+def kda_chunk_bwd(q, k, v, g, beta, d_o, *, scale: float = 1.0, initial_state=None,
+                  d_final_state=None, cu_seqlens=None, chunk: int = 64, dq=None, dk=None,
+                  dv=None, dg=None, dbeta=None, d_initial_state=None, want_d_initial_state=True,
+                  workspace="auto", stream=None):
+    """Gradients of :func:`kda_chunk_fwd` for L = sum(d_o * o) + sum(d_final_state *
+    final_state).  Returns ``(dq, dk, dv, dg, dbeta, d_initial_state)`` (fp32; the
+    last is None unless wanted); output tensors not given are allocated."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((g, "g"), (beta, "beta"), (d_o, "d_o"), (initial_state, "initial_state"),
+                 (d_final_state, "d_final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    dev = q.device
+    dq = torch.empty((T, H, Dk), device=dev) if dq is None else dq
+    dk = torch.empty((T, H, Dk), device=dev) if dk is None else dk
+    dv = torch.empty((T, H, Dv), device=dev) if dv is None else dv
+    dg = torch.empty((T, H, Dk), device=dev) if dg is None else dg
+    dbeta = torch.empty((T, H), device=dev) if dbeta is None else dbeta
+    if d_initial_state is None and want_d_initial_state:
+        d_initial_state = torch.empty((N, H, Dv, Dk), device=dev)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dg, "dg"), (dbeta, "dbeta"),
+                 (d_initial_state, "d_initial_state")):
+        _need(t, n, torch.float32)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_bwd_workspace_bytes(N, T, H, Dk, Dv, chunk, q.dtype)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_chunk_bwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
+                                _dtype(q), _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk),
+                                _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(d_initial_state),
+                                _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv, dg, dbeta, d_initial_state
 
 
 # Size of the library's fixed scratch buffer (one per device) used by

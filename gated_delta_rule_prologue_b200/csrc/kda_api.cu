@@ -692,3 +692,94 @@ kda_status kda_decode_step_gated(const void *x, const float *conv_w, void *conv_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward of the two-pass prefill
+// ---------------------------------------------------------------------------
+
+extern "C" {
+
+size_t kda_chunk_bwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt) {
+  if (N < 1 || T < 0 || H < 1 || !chunk_tc_path(T, Dk, Dv, chunk, dt)) return 0;
+  return kda::rec::workspace_bytes(N, T, H, 0) +
+         2 * (size_t)kda::rec::chunk_capacity(N, T) * H * kda::rec::SEG_BLOCK;
+}
+
+kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *initial_state,
+                            const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                            int chunk, kda_dtype dt, const float *d_o,
+                            const float *d_final_state, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                            size_t workspace_bytes, kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1, "bad sizes N=%d T=%d H=%d", N, T, H);
+  KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
+  if (!chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_bwd: needs bf16/f16, Dk == Dv == 128, chunk 64 and "
+                                     "T > 0 (got dt=%d Dk=%d Dv=%d chunk=%d T=%d)",
+                (int)dt, Dk, Dv, chunk, T);
+  KDA_REQUIRE_PTR(q, "q");
+  KDA_REQUIRE_PTR(k, "k");
+  KDA_REQUIRE_PTR(v, "v");
+  KDA_REQUIRE_PTR(g, "g");
+  KDA_REQUIRE_PTR4(beta, "beta");
+  KDA_REQUIRE_PTR(d_o, "d_o");
+  KDA_REQUIRE_PTR(dq, "dq");
+  KDA_REQUIRE_PTR(dk, "dk");
+  KDA_REQUIRE_PTR(dv, "dv");
+  KDA_REQUIRE_PTR(dg, "dg");
+  KDA_REQUIRE_PTR4(dbeta, "dbeta");
+  KDA_OPT_PTR(initial_state, "initial_state");
+  KDA_OPT_PTR(d_final_state, "d_final_state");
+  KDA_OPT_PTR(d_initial_state, "d_initial_state");
+  KDA_OPT_PTR4(cu_seqlens, "cu_seqlens");
+  KDA_REQUIRE(workspace != nullptr, "chunk_bwd: workspace is NULL");
+  KDA_OPT_PTR(workspace, "workspace");
+  const size_t need = kda_chunk_bwd_workspace_bytes(N, T, H, Dk, Dv, chunk, dt);
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {  // outputs must not overlap the inputs, each other or the workspace
+    const size_t es = esize(dt), act = (size_t)T * H * 128 * es, f32 = (size_t)T * H * 128 * 4;
+    const size_t sbytes = (size_t)N * H * 128 * 128 * 4, bb = (size_t)T * H * 4;
+    const void *outs[6] = {dq, dk, dv, dg, dbeta, d_initial_state};
+    const size_t osz[6] = {f32, f32, f32, f32, bb, sbytes};
+    const void *ins[9] = {q, k, v, g, beta, d_o, initial_state, d_final_state, cu_seqlens};
+    const size_t isz[9] = {act, act, act, f32, bb, f32, sbytes, sbytes, (size_t)(N + 1) * 4};
+    for (int a = 0; a < 6; ++a) {
+      for (int b = 0; b < 9; ++b)
+        KDA_REQUIRE(!overlaps(outs[a], osz[a], ins[b], isz[b]), "an output overlaps an input");
+      for (int b = a + 1; b < 6; ++b)
+        KDA_REQUIRE(!overlaps(outs[a], osz[a], outs[b], osz[b]), "two outputs overlap");
+      KDA_REQUIRE(!overlaps(outs[a], osz[a], workspace, need), "an output overlaps the workspace");
+    }
+    for (int b = 0; b < 9; ++b)
+      KDA_REQUIRE(!overlaps(workspace, need, ins[b], isz[b]), "workspace overlaps an input");
+  }
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  float *ckpt = reinterpret_cast<float *>(wsb + kda::rec::workspace_bytes(N, T, H, 0));
+  float *dckpt = ckpt + (size_t)kda::rec::chunk_capacity(N, T) * H * 128 * 128;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, 0, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, nullptr,
+                               nullptr, 0.f, false, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, 0, nullptr,
+                                nullptr, status, s, ckpt);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_bwd_state(workspace, cu_seqlens, d_final_state, d_o, scale, N, T, H,
+                                    dckpt, d_initial_state, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_bwd_local(q, k, v, g, beta, d_o, scale, cu_seqlens, workspace, ckpt,
+                                    dckpt, N, T, H, dt, dq, dk, dv, dg, dbeta, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd_ws launch");
+  return KDA_OK;
+}
+
+}  // extern "C"

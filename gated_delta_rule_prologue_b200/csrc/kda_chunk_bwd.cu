@@ -1,0 +1,778 @@
+// Backward of the two-pass tensor-core prefill: gradients of o and of the final
+// state with respect to q, k, v, g, beta and the initial state.
+//
+// The pages mention training ("Kimi K3的线性注意力：从源码看懂KDA如何更新记忆",
+// 彩蛋) but give no backward; this is the chain rule through the chunk algebra
+// of the forward (kda_chunk_record.cuh).  With R = diag(beta)(V - (K G) S),
+// U = (I + A)^{-1} R, K' = K G_last / G, dO' = scale dO, and dS' the adjoint of a
+// chunk's exit state:
+//   dU  = P^T dO' + K' dS'                 dS = diag(G_last) dS' + (Q G)^T dO' - W^T dU
+// (W = (I + A)^{-1} diag(beta) K G), so the adjoint state runs backwards through
+// the chunks by the transpose of the forward's affine map ("KimiK3轻量化复刻实现KDA
+// 并行解析，Chunkwise并行与状态压缩机制详解", Figure 1).  Two passes:
+//
+// * chunk_bwd_state_kernel: one CTA (128 threads) per (sequence, head, 32 value
+//   channels), chunks in reverse order, on the forward's records.  Per chunk,
+//   tcgen05 MMAs with fp32 accumulators in TMEM:
+//     D_u = P^T (scale dO) + K' dS'        (M = 128 of which rows 0..63 are used;
+//                                           P^T is the record's P tile read
+//                                           MN-major, K' its K-major tile)
+//     dU  = D_u + <q_r, k_r> scale dO_r    (fp32 diagonal term)
+//     D_s = [W^T | (Q G)^T] [-dU ; scale dO]   (the record's [W; Q G] tile read
+//                                               MN-major, K = 128)
+//     dS  = diag(G_last) dS' + D_s         (fp32 registers; thread = key channel)
+//   It writes dS' (the adjoint of every chunk's exit state) and the gradient of
+//   the initial state.
+//
+// * chunk_bwd_local_kernel: one CTA (256 threads) per (chunk, head), fp32 on CUDA
+//   cores.  From the chunk's entry state (saved by the forward state pass) and
+//   dS', it walks the chunk in sub-chunks of 16 tokens: in a 16-token block the
+//   in-block log-decay is at least -80 when g >= -5, so exp(+-gamma) stay in fp32
+//   range and the chunk algebra applies with plain factors.  Sub-chunk sb is
+//   reached by recomputing the forward through sub-chunks 0..sb-1 from the entry
+//   state; its backward (the same relations as the float64 chunkwise backward
+//   oracle) gives dq, dk, dv, dg, dbeta and the adjoint entering the sub-chunk
+//   before it.
+#include <cuda_fp16.h>
+
+#include "kda_chunk_record.cuh"
+#include "kda_common.cuh"
+#include "kda_tcgen05.cuh"
+
+namespace kda {
+namespace {
+using namespace tc;
+
+// ----------------------------------------------------------------------------
+// Reverse state pass
+// ----------------------------------------------------------------------------
+
+constexpr int kBT = 128;
+constexpr int kSlices = 4;
+constexpr uint32_t BB_A1 = 0;       // [W ; Q G] (record), read MN-major            32 KB
+constexpr uint32_t BB_KP = 32768;   // K' (record, K-major 64 rows) then P          24 KB
+constexpr uint32_t BB_P = 49152;
+constexpr uint32_t BB_DS = 57344;   // dS' operand: 128 key rows x 32 values, 64-byte swizzle  8 KB
+constexpr uint32_t BB_B2 = 65536;   // [-dU ; scale dO]: 128 token rows x 32 values             8 KB
+constexpr uint32_t BB_BAR = 73728;  // three mbarriers, TMEM slot
+constexpr uint32_t BB_ALLOC = BB_BAR + 64 + 1024;
+constexpr uint32_t TB_DU = 0, TB_DS = 32, TB_COLS = 64;
+// P^T is an M = 128 MN-major operand whose second MN block (rows 64..127 of D_u,
+// never read back) lies over the dS' tile; K' as an M = 128 K-major operand reads
+// its rows 64..127 from the next k-atom and P: all inside the allocation.
+static_assert(BB_P + 8192 == BB_DS, "P^T's unused MN block overlays the dS' tile");
+
+__global__ void __launch_bounds__(kBT, 3)
+chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
+                       const float *dsN, const float *__restrict__ dout, float scale, int N,
+                       int T, int H, float *__restrict__ dckpt, float *ds0, int *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int slice = blockIdx.x % kSlices;
+  const int nh = blockIdx.x / kSlices, h = nh % H, n = nh / H;
+  const int32_t *cprefix = reinterpret_cast<const int32_t *>(ws);
+  const uint8_t *recs = ws + rec::header_bytes(N);
+  uint64_t *bar_a1 = reinterpret_cast<uint64_t *>(sm + BB_BAR);
+  uint64_t *bar_kp = bar_a1 + 1, *bar_mma = bar_a1 + 2;
+  uint32_t *slot = reinterpret_cast<uint32_t *>(sm + BB_BAR + 32);
+
+  int bos, eos;
+  seq_bounds(cu, n, T, status, bos, eos);
+  int cbase = 0, nch = (eos - bos + 63) / 64;
+  if (cu) {
+    cbase = cprefix[n];
+    nch = cprefix[n + 1] - cbase;
+  }
+  if (warp == 0) tmem_alloc(slot, TB_COLS);
+  if (tid == 0) {
+    mbar_init(bar_a1, 1);
+    mbar_init(bar_kp, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+  }
+  // dS[i] = dS'[key t][value 32 slice + i]; stored value-major [dv][dk] like the state.
+  const int t = tid;
+  const size_t head_off = ((size_t)n * H + h) * 128 * 128;
+  const size_t sbase = (size_t)slice * 32 * 128 + t;
+  float dS[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) dS[i] = dsN ? dsN[head_off + sbase + (size_t)i * 128] : 0.f;
+
+  auto write_ds_operand = [&]() {
+    float amax = 0.f;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        f[e] = dS[8 * x + e];
+        amax = fmaxf(amax, fabsf(f[e]));
+      }
+      st_shared_16(sm + BB_DS, mn32_sw64_off(t, x), pack8_f16(f));
+    }
+    if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+  };
+  write_ds_operand();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t lane_addr = static_cast<uint32_t>(32 * warp) << 16;
+
+  auto rec_of = [&](int c) -> const uint8_t * {
+    return recs + ((size_t)(cbase + c) * H + h) * rec::BYTES;
+  };
+  auto load_a1 = [&](int c) {
+    mbar_arrive_expect_tx(bar_a1, 32768);
+    bulk_load(sm + BB_A1, rec_of(c) + rec::A1, 32768, bar_a1);
+  };
+  auto load_kp = [&](int c) {
+    mbar_arrive_expect_tx(bar_kp, 24576);
+    bulk_load(sm + BB_KP, rec_of(c) + rec::KP, 24576, bar_kp);
+  };
+  if (tid == 0 && nch > 0) {
+    load_a1(nch - 1);
+    load_kp(nch - 1);
+  }
+
+  uint32_t pa = 0, pk = 0, pm = 0;
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
+    const uint8_t *rp = rec_of(c);
+    {  // the adjoint of this chunk's exit state, for the local pass
+      float *dst = dckpt + ((size_t)(cbase + c) * H + h) * (128 * 128) + sbase;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dst[(size_t)i * 128] = dS[i];
+    }
+    // scale dO of token r (warps 0-1: TMEM lanes 0..63 are the chunk's tokens)
+    float sdo[32];
+    float pd = 0.f;
+    if (warp < 2) {
+      const int r = tid;
+      if (r < Lc) {
+        const float4 *src = reinterpret_cast<const float4 *>(
+            dout + ((size_t)(t0 + r) * H + h) * 128 + slice * 32);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float4 f = __ldg(src + x);
+          sdo[4 * x] = scale * f.x;
+          sdo[4 * x + 1] = scale * f.y;
+          sdo[4 * x + 2] = scale * f.z;
+          sdo[4 * x + 3] = scale * f.w;
+        }
+        pd = __ldg(reinterpret_cast<const float *>(rp + rec::PD) + r);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sdo[i] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          f[e] = sdo[8 * x + e];
+          amax = fmaxf(amax, fabsf(f[e]));
+        }
+        st_shared_16(sm + BB_B2, mn32_sw64_off(64 + r, x), pack8_f16(f));
+      }
+      if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+    }
+    const float gl = __ldg(reinterpret_cast<const float *>(rp + rec::GL) + t);
+    fence_async_smem();
+    tc_fence_before();
+    if (!wait_all(bar_kp, pk, status)) break;  // K', P of this chunk; also a CTA barrier
+    pk ^= 1;
+
+    // ---- D_u = P^T (scale dO) + K' dS' -------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t p = smem_u32(sm + BB_P), kp = smem_u32(sm + BB_KP);
+      const uint32_t b2 = smem_u32(sm + BB_B2), dso = smem_u32(sm + BB_DS);
+      constexpr uint32_t idT = idesc_fp16(128, 32, true, true);
+      constexpr uint32_t idK = idesc_fp16(128, 32, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16(tmem + TB_DU, desc_mnmajor(p, 64, ks), desc_mn32_sw64(b2 + 4096, ks), idT,
+                 ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TB_DU, desc_kmajor(kp, 64, ks), desc_mn32_sw64(dso, ks), idK, 1);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, pm, status)) break;
+    pm ^= 1;
+    tc_fence_after();
+    if (tid == 0 && c > 0) load_kp(c - 1);  // K' and P have been read
+
+    // ---- dU (fp32), then -dU as the upper half of the second B operand ----------------------
+    if (warp < 2) {
+      const int r = tid;
+      float du[32];
+      tmem_ld32(tmem + lane_addr + TB_DU, du);
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        du[i] = r < Lc ? -fmaf(pd, sdo[i], du[i]) : 0.f;
+        amax = fmaxf(amax, fabsf(du[i]));
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = du[8 * x + e];
+        st_shared_16(sm + BB_B2, mn32_sw64_off(r, x), pack8_f16(f));
+      }
+      if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    if (!wait_all(bar_a1, pa, status)) break;  // [W; Q G] of this chunk; also a CTA barrier
+    pa ^= 1;
+
+    // ---- D_s = [W^T | (Q G)^T] [-dU ; scale dO] ----------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t a1 = smem_u32(sm + BB_A1), b2 = smem_u32(sm + BB_B2);
+      constexpr uint32_t idT = idesc_fp16(128, 32, true, true);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_bf16(tmem + TB_DS, desc_mnmajor(a1, 128, ks), desc_mn32_sw64(b2, ks), idT, ks > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, pm, status)) break;
+    pm ^= 1;
+    tc_fence_after();
+    if (tid == 0 && c > 0) load_a1(c - 1);  // [W; Q G] has been read
+    {
+      float ds[32];
+      tmem_ld32(tmem + lane_addr + TB_DS, ds);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dS[i] = fmaf(gl, dS[i], ds[i]);
+    }
+    __syncthreads();
+    write_ds_operand();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (ds0) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ds0[head_off + sbase + (size_t)i * 128] = dS[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, TB_COLS);
+}
+
+// ----------------------------------------------------------------------------
+// Local pass: fp32, 16-token sub-chunks
+// ----------------------------------------------------------------------------
+
+constexpr int kLT = 256;       // threads
+constexpr int kSub = 16;       // tokens per sub-chunk
+constexpr int RS = 132;        // row stride (floats) of the 128-wide shared matrices
+constexpr int SS = 17;         // row stride of the 16 x 16 matrices
+
+struct LocalSmem {
+  float S[128 * RS];    // entry state of the current sub-chunk, [key][value]
+  float dS[128 * RS];   // adjoint of the current sub-chunk's exit state, [key][value]
+  float G[kSub * RS];   // exp(gamma), gamma the in-sub-chunk inclusive cumsum of g
+  float KG[kSub * RS];  // k exp(gamma)
+  float KD[kSub * RS];  // k exp(-gamma)
+  float QG[kSub * RS];  // q exp(gamma)
+  float KP[kSub * RS];  // k exp(gamma_last - gamma)
+  float E[kSub * RS];   // v - (K G) S
+  float U[kSub * RS];   // (I + A)^{-1} diag(beta) E
+  float dO[kSub * RS];  // scale dO
+  float dU[kSub * RS];  // dU, then dR in place
+  float A[kSub * SS];   // strict lower beta_r <k_r G_r, k_i / G_i>
+  float KK[kSub * SS];  // <k_r G_r, k_i / G_i>
+  float P[kSub * SS];   // lower <q_r G_r, k_i / G_i> (diagonal included)
+  float dP[kSub * SS];
+  float dA[kSub * SS];
+  float beta[kSub];
+  float gc[128];        // exp(gamma_last)
+};
+
+template <typename Tin>
+__device__ __forceinline__ void load8(const Tin *p, float (&f)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) f[e] = to_f32(p[e]);
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kLT, 1)
+chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                       const Tin *__restrict__ v, const float *__restrict__ g,
+                       const float *__restrict__ beta, const float *__restrict__ dout,
+                       float scale, const int32_t *__restrict__ cu, const uint8_t *ws,
+                       const float *__restrict__ ckpt, const float *__restrict__ dckpt, int N,
+                       int T, int H, float *__restrict__ dq, float *__restrict__ dk,
+                       float *__restrict__ dv, float *__restrict__ dg,
+                       float *__restrict__ dbeta, int *status) {
+  extern __shared__ float4 smem_f4[];
+  LocalSmem &sm = *reinterpret_cast<LocalSmem *>(smem_f4);
+  const int tid = threadIdx.x;
+  const int h = blockIdx.x % H, ci = blockIdx.x / H;
+  const int32_t *cprefix = reinterpret_cast<const int32_t *>(ws);
+
+  // ---- which chunk ---------------------------------------------------------------------
+  int n = 0, c = ci;
+  if (cu) {
+    if (ci >= cprefix[N]) return;
+    int lo = 0, hi = N - 1;  // last n with cprefix[n] <= ci
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cprefix[mid] <= ci) lo = mid;
+      else hi = mid - 1;
+    }
+    n = lo;
+    c = ci - cprefix[n];
+  } else if (ci >= (T + 63) / 64) {
+    return;
+  }
+  int bos, eos;
+  seq_bounds(cu, n, T, status, bos, eos);
+  const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
+  if (Lc <= 0) return;
+  const int nsub = (Lc + kSub - 1) / kSub;
+  const size_t rec_idx = (size_t)ci * H + h;
+  const float *S0 = ckpt + rec_idx * (128 * 128);
+  const float *dS1 = dckpt + rec_idx * (128 * 128);
+
+  // thread roles
+  const int rr = tid >> 4, c8 = tid & 15;          // (row, 8 value columns) for 16 x 128 outputs
+  const int kt = tid >> 1, half = tid & 1;         // (key channel, half) for key-indexed work
+  // value columns of (rr, c8): {4 c8 .. 4 c8 + 3} and {64 + 4 c8 .. 64 + 4 c8 + 3}
+  const int ca = 4 * c8, cb = 64 + 4 * c8;
+
+  auto load_state = [&](float *dst, const float *src) {  // src [value][key] -> dst[key][value]
+    for (int idx = tid; idx < 128 * 128; idx += kLT) {
+      const int j = idx >> 7, key = idx & 127;
+      dst[key * RS + j] = src[idx];
+    }
+  };
+
+  // Inputs of sub-chunk sb: G, KG, KD, QG, KP, E (= v for now), dO (scaled), beta, gc.
+  auto load_sub = [&](int sb, bool with_grad) {
+    const int r0 = kSub * sb;
+    {  // g (raw) into G, q and k and v per (row, 8 channels)
+      const int r = rr, tok = t0 + r0 + r;
+      const bool ok = r0 + r < Lc;
+      const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int col = part ? cb : ca;
+        float gv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ok) {
+          const float4 f = __ldg(reinterpret_cast<const float4 *>(g + base + col));
+          gv[0] = f.x; gv[1] = f.y; gv[2] = f.z; gv[3] = f.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sm.G[r * RS + col + e] = gv[e];
+      }
+      if (c8 == 0) sm.beta[r] = ok ? __ldg(beta + (size_t)tok * H + h) : 0.f;
+    }
+    __syncthreads();
+    if (tid < 128) {  // inclusive cumsum over the rows, per key channel
+      float run = 0.f;
+#pragma unroll
+      for (int r = 0; r < kSub; ++r) {
+        run += sm.G[r * RS + tid];
+        sm.G[r * RS + tid] = run;
+      }
+      sm.gc[tid] = __expf(run);
+      // a 16-token block needs its log-decay within fp32's exp range (g >= -5 gives >= -80)
+      if (!(run >= -87.f)) report(status, KDA_ERR_DEVICE_RANGE);
+    }
+    __syncthreads();
+    {
+      const int r = rr, tok = t0 + r0 + r;
+      const bool ok = r0 + r < Lc;
+      const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int col = part ? cb : ca;
+        float kv[4] = {0.f, 0.f, 0.f, 0.f}, qv[4] = {0.f, 0.f, 0.f, 0.f};
+        float vv[4] = {0.f, 0.f, 0.f, 0.f}, dv4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ok) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kv[e] = to_f32(k[base + col + e]);
+            qv[e] = to_f32(q[base + col + e]);
+            vv[e] = to_f32(v[base + col + e]);
+          }
+          if (with_grad) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(dout + base + col));
+            dv4[0] = scale * f.x; dv4[1] = scale * f.y; dv4[2] = scale * f.z; dv4[3] = scale * f.w;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = col + e;
+          const float gam = sm.G[r * RS + j], glast = sm.G[(kSub - 1) * RS + j];
+          const float Gv = __expf(gam), Gi = __expf(-gam);
+          sm.KG[r * RS + j] = kv[e] * Gv;
+          sm.KD[r * RS + j] = kv[e] * Gi;
+          sm.QG[r * RS + j] = qv[e] * Gv;
+          sm.KP[r * RS + j] = kv[e] * __expf(glast - gam);
+          sm.E[r * RS + j] = vv[e];
+          sm.dO[r * RS + j] = dv4[e];
+        }
+      }
+    }
+    __syncthreads();
+    {  // G = exp(gamma) in place (every reader of gamma above is done)
+      const int r = rr;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int col = part ? cb : ca;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sm.G[r * RS + col + e] = __expf(sm.G[r * RS + col + e]);
+      }
+    }
+  };
+
+  // E = V - (K G) S;  KK, A, P;  U = (I + A)^{-1} diag(beta) E.
+  auto forward_local = [&](bool with_p) {
+    {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[e] = sm.E[rr * RS + ca + e];
+        acc[4 + e] = sm.E[rr * RS + cb + e];
+      }
+#pragma unroll 4
+      for (int key = 0; key < 128; ++key) {
+        const float a = sm.KG[rr * RS + key];
+        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + ca]);
+        const float4 s2 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + cb]);
+        acc[0] -= a * s1.x; acc[1] -= a * s1.y; acc[2] -= a * s1.z; acc[3] -= a * s1.w;
+        acc[4] -= a * s2.x; acc[5] -= a * s2.y; acc[6] -= a * s2.z; acc[7] -= a * s2.w;
+      }
+      __syncthreads();  // all reads of E (= v) done before it is overwritten
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sm.E[rr * RS + ca + e] = acc[e];
+        sm.E[rr * RS + cb + e] = acc[4 + e];
+      }
+    }
+    {  // 16 x 16 Grams: thread (r, i)
+      const int r = tid >> 4, i = tid & 15;
+      float kk = 0.f, pp = 0.f;
+#pragma unroll 8
+      for (int key = 0; key < 128; ++key) {
+        const float kd = sm.KD[i * RS + key];
+        kk = fmaf(sm.KG[r * RS + key], kd, kk);
+        if (with_p) pp = fmaf(sm.QG[r * RS + key], kd, pp);
+      }
+      sm.KK[r * SS + i] = kk;
+      sm.A[r * SS + i] = i < r ? sm.beta[r] * kk : 0.f;
+      sm.P[r * SS + i] = i <= r ? pp : 0.f;
+    }
+    __syncthreads();
+    if (tid < 128) {  // forward substitution, one value column per thread
+      const int j = tid;
+      float u[kSub];
+#pragma unroll
+      for (int r = 0; r < kSub; ++r) {
+        float x = sm.beta[r] * sm.E[r * RS + j];
+#pragma unroll
+        for (int i = 0; i < r; ++i) x = fmaf(-sm.A[r * SS + i], u[i], x);
+        u[r] = x;
+        sm.U[r * RS + j] = x;
+      }
+    }
+    __syncthreads();
+  };
+
+  // S <- diag(G_last) S + K'^T U   (thread (key, half of the values))
+  auto advance_state = [&]() {
+    const float gck = sm.gc[kt];
+    float *row = &sm.S[kt * RS + 64 * half];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      float4 s = *reinterpret_cast<float4 *>(row + 4 * x);
+      s.x *= gck; s.y *= gck; s.z *= gck; s.w *= gck;
+#pragma unroll
+      for (int r = 0; r < kSub; ++r) {
+        const float kp = sm.KP[r * RS + kt];
+        const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + 64 * half + 4 * x]);
+        s.x = fmaf(kp, u.x, s.x); s.y = fmaf(kp, u.y, s.y);
+        s.z = fmaf(kp, u.z, s.z); s.w = fmaf(kp, u.w, s.w);
+      }
+      *reinterpret_cast<float4 *>(row + 4 * x) = s;
+    }
+    __syncthreads();
+  };
+
+  load_state(sm.dS, dS1);
+  for (int sb = nsub - 1; sb >= 0; --sb) {
+    // ---- entry state of sub-chunk sb: the chunk's entry state, walked forward ---------------
+    load_state(sm.S, S0);
+    __syncthreads();
+    for (int j = 0; j < sb; ++j) {
+      load_sub(j, false);
+      __syncthreads();
+      forward_local(false);
+      advance_state();
+    }
+    load_sub(sb, true);
+    __syncthreads();
+    forward_local(true);
+    const int r0 = kSub * sb;
+
+    // ---- dU = P^T dO' + K' dS'  (thread (r, 8 value columns)) ------------------------------
+    {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kSub; ++i) {
+        const float p = sm.P[i * SS + rr];
+        const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + ca]);
+        const float4 d2 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + cb]);
+        acc[0] = fmaf(p, d1.x, acc[0]); acc[1] = fmaf(p, d1.y, acc[1]);
+        acc[2] = fmaf(p, d1.z, acc[2]); acc[3] = fmaf(p, d1.w, acc[3]);
+        acc[4] = fmaf(p, d2.x, acc[4]); acc[5] = fmaf(p, d2.y, acc[5]);
+        acc[6] = fmaf(p, d2.z, acc[6]); acc[7] = fmaf(p, d2.w, acc[7]);
+      }
+#pragma unroll 4
+      for (int key = 0; key < 128; ++key) {
+        const float a = sm.KP[rr * RS + key];
+        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + ca]);
+        const float4 s2 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + cb]);
+        acc[0] = fmaf(a, s1.x, acc[0]); acc[1] = fmaf(a, s1.y, acc[1]);
+        acc[2] = fmaf(a, s1.z, acc[2]); acc[3] = fmaf(a, s1.w, acc[3]);
+        acc[4] = fmaf(a, s2.x, acc[4]); acc[5] = fmaf(a, s2.y, acc[5]);
+        acc[6] = fmaf(a, s2.z, acc[6]); acc[7] = fmaf(a, s2.w, acc[7]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sm.dU[rr * RS + ca + e] = acc[e];
+        sm.dU[rr * RS + cb + e] = acc[4 + e];
+      }
+    }
+    {  // dP = lower(dO' U^T)   (thread (r, i))
+      const int r = tid >> 4, i = tid & 15;
+      float acc = 0.f;
+      if (i <= r) {
+#pragma unroll 8
+        for (int j = 0; j < 128; j += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
+          const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
+          acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
+          acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+        }
+      }
+      sm.dP[r * SS + i] = acc;
+    }
+    __syncthreads();
+    if (tid < 128) {  // dR = (I + A)^{-T} dU, back substitution in place
+      const int j = tid;
+      float x[kSub];
+#pragma unroll
+      for (int r = kSub - 1; r >= 0; --r) {
+        float y = sm.dU[r * RS + j];
+#pragma unroll
+        for (int i = r + 1; i < kSub; ++i) y = fmaf(-sm.A[i * SS + r], x[i], y);
+        x[r] = y;
+        sm.dU[r * RS + j] = y;
+      }
+    }
+    __syncthreads();
+    {  // dA = -strict_lower(dR U^T); dbeta; dv = beta dR
+      const int r = tid >> 4, i = tid & 15;
+      float acc = 0.f;
+      if (i < r) {
+#pragma unroll 8
+        for (int j = 0; j < 128; j += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
+          const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
+          acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
+          acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+        }
+      }
+      const float da = -acc;
+      sm.dA[r * SS + i] = da;
+      // dbeta_r = <dR_r, E_r> + sum_{i<r} dA[r,i] KK[r,i]; lanes (r, 0..15) share row r
+      float part = i < r ? da * sm.KK[r * SS + i] : 0.f;
+#pragma unroll
+      for (int jj = i; jj < 128; jj += 16) part = fmaf(sm.dU[r * RS + jj], sm.E[r * RS + jj], part);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (i == 0 && r0 + r < Lc) dbeta[(size_t)(t0 + r0 + r) * H + h] = part;
+    }
+    if (r0 + rr < Lc) {
+      const float b = sm.beta[rr];
+      float *dst = dv + ((size_t)(t0 + r0 + rr) * H + h) * 128;
+      float4 o1, o2;
+      o1.x = b * sm.dU[rr * RS + ca]; o1.y = b * sm.dU[rr * RS + ca + 1];
+      o1.z = b * sm.dU[rr * RS + ca + 2]; o1.w = b * sm.dU[rr * RS + ca + 3];
+      o2.x = b * sm.dU[rr * RS + cb]; o2.y = b * sm.dU[rr * RS + cb + 1];
+      o2.z = b * sm.dU[rr * RS + cb + 2]; o2.w = b * sm.dU[rr * RS + cb + 3];
+      *reinterpret_cast<float4 *>(dst + ca) = o1;
+      *reinterpret_cast<float4 *>(dst + cb) = o2;
+    }
+    __syncthreads();
+
+    // ---- key-indexed gradients: thread (key kt, rows 8 half .. 8 half + 7) -------------------
+    {
+      const int rb = 8 * half;
+      float dqg[8], dkg[8], dkp[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) dqg[x] = dkg[x] = dkp[x] = 0.f;
+      float sds = 0.f;  // rowsum(S * dS') of key kt
+      const float *srow = &sm.S[kt * RS], *dsrow = &sm.dS[kt * RS];
+#pragma unroll 2
+      for (int j = 0; j < 128; j += 4) {
+        const float4 s = *reinterpret_cast<const float4 *>(srow + j);
+        const float4 d = *reinterpret_cast<const float4 *>(dsrow + j);
+        sds = fmaf(s.x, d.x, sds); sds = fmaf(s.y, d.y, sds);
+        sds = fmaf(s.z, d.z, sds); sds = fmaf(s.w, d.w, sds);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const int r = rb + x;
+          const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
+          const float4 rr4 = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
+          const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + j]);
+          dqg[x] = fmaf(o.x, s.x, dqg[x]); dqg[x] = fmaf(o.y, s.y, dqg[x]);
+          dqg[x] = fmaf(o.z, s.z, dqg[x]); dqg[x] = fmaf(o.w, s.w, dqg[x]);
+          dkg[x] = fmaf(rr4.x, s.x, dkg[x]); dkg[x] = fmaf(rr4.y, s.y, dkg[x]);
+          dkg[x] = fmaf(rr4.z, s.z, dkg[x]); dkg[x] = fmaf(rr4.w, s.w, dkg[x]);
+          dkp[x] = fmaf(u.x, d.x, dkp[x]); dkp[x] = fmaf(u.y, d.y, dkp[x]);
+          dkp[x] = fmaf(u.z, d.z, dkp[x]); dkp[x] = fmaf(u.w, d.w, dkp[x]);
+        }
+      }
+      float dgam[8], dkd[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int r = rb + x;
+        float pq = 0.f, pa = 0.f, kd = 0.f;
+#pragma unroll
+        for (int i = 0; i < kSub; ++i) {
+          const float kdi = sm.KD[i * RS + kt];
+          pq = fmaf(sm.dP[r * SS + i], kdi, pq);   // (dP K/G)[r]
+          pa = fmaf(sm.dA[r * SS + i], kdi, pa);   // (dA K/G)[r]
+          // (diag(beta) dA)^T (K G) + dP^T (Q G), row r
+          kd = fmaf(sm.beta[i] * sm.dA[i * SS + r], sm.KG[i * RS + kt], kd);
+          kd = fmaf(sm.dP[i * SS + r], sm.QG[i * RS + kt], kd);
+        }
+        const float b = sm.beta[r];
+        dqg[x] += pq;
+        dkg[x] = b * (pa - dkg[x]);
+        dkd[x] = kd;
+        dgam[x] = dqg[x] * sm.QG[r * RS + kt] + dkg[x] * sm.KG[r * RS + kt] -
+                  dkd[x] * sm.KD[r * RS + kt] - dkp[x] * sm.KP[r * RS + kt];
+      }
+      // last row: + G_last rowsum(S * dS') + sum_i dK'_i K'_i (the rows of both halves)
+      float kpsum = 0.f;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) kpsum = fmaf(dkp[x], sm.KP[(rb + x) * RS + kt], kpsum);
+      kpsum += __shfl_xor_sync(0xffffffffu, kpsum, 1);
+      if (half == 1) dgam[7] += sm.gc[kt] * sds + kpsum;
+      // dg = reverse cumulative sum over the 16 rows (rows 8..15 live on the odd lane)
+      float suffix = 0.f;
+#pragma unroll
+      for (int x = 7; x >= 0; --x) {
+        suffix += dgam[x];
+        dgam[x] = suffix;
+      }
+      const float upper = __shfl_xor_sync(0xffffffffu, suffix, 1);
+      if (half == 0) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) dgam[x] += upper;
+      }
+      const float gck = sm.gc[kt];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int r = rb + x;
+        if (r0 + r < Lc) {
+          const float Gv = sm.G[r * RS + kt];
+          const size_t o = ((size_t)(t0 + r0 + r) * H + h) * 128 + kt;
+          dq[o] = dqg[x] * Gv;
+          dk[o] = dkg[x] * Gv + __fdividef(dkd[x] + dkp[x] * gck, Gv);
+          dg[o] = dgam[x];
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- dS <- diag(G_last) dS' + (Q G)^T dO' - (diag(beta) K G)^T dR  (thread (key, half)) --
+    {
+      const float gck = sm.gc[kt];
+      float *row = &sm.dS[kt * RS + 64 * half];
+#pragma unroll 2
+      for (int x = 0; x < 16; ++x) {
+        float4 s = *reinterpret_cast<float4 *>(row + 4 * x);
+        s.x *= gck; s.y *= gck; s.z *= gck; s.w *= gck;
+#pragma unroll
+        for (int r = 0; r < kSub; ++r) {
+          const float a = sm.QG[r * RS + kt], b = -sm.beta[r] * sm.KG[r * RS + kt];
+          const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + 64 * half + 4 * x]);
+          const float4 d = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + 64 * half + 4 * x]);
+          s.x = fmaf(a, o.x, fmaf(b, d.x, s.x)); s.y = fmaf(a, o.y, fmaf(b, d.y, s.y));
+          s.z = fmaf(a, o.z, fmaf(b, d.z, s.z)); s.w = fmaf(a, o.w, fmaf(b, d.w, s.w));
+        }
+        *reinterpret_cast<float4 *>(row + 4 * x) = s;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_bwd_state(const void *ws, const int32_t *cu, const float *dsN,
+                                   const float *dout, float scale, int N, int T, int H,
+                                   float *dckpt, float *ds0, int *status, cudaStream_t s) {
+  const long long blocks = (long long)N * H * kSlices;
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(chunk_bwd_state_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BB_ALLOC);
+  if (e != cudaSuccess) return e;
+  chunk_bwd_state_kernel<<<(unsigned)blocks, kBT, BB_ALLOC, s>>>(
+      static_cast<const uint8_t *>(ws), cu, dsN, dout, scale, N, T, H, dckpt, ds0, status);
+  return cudaGetLastError();
+}
+
+namespace {
+template <typename Tin>
+cudaError_t launch_local_typed(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *dout, float scale,
+                               const int32_t *cu, const void *ws, const float *ckpt,
+                               const float *dckpt, int N, int T, int H, float *dq, float *dk,
+                               float *dv, float *dg, float *dbeta, int *status, cudaStream_t s) {
+  const long long blocks = rec::chunk_capacity(N, T) * H;
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  const int bytes = (int)sizeof(LocalSmem);
+  cudaError_t e = cudaFuncSetAttribute(chunk_bwd_local_kernel<Tin>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  chunk_bwd_local_kernel<Tin><<<(unsigned)blocks, kLT, bytes, s>>>(
+      static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), g,
+      beta, dout, scale, cu, static_cast<const uint8_t *>(ws), ckpt, dckpt, N, T, H, dq, dk, dv,
+      dg, dbeta, status);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *dout, float scale,
+                                   const int32_t *cu, const void *ws, const float *ckpt,
+                                   const float *dckpt, int N, int T, int H, kda_dtype dt,
+                                   float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                   int *status, cudaStream_t s) {
+  if (dt == KDA_BF16)
+    return launch_local_typed<__nv_bfloat16>(q, k, v, g, beta, dout, scale, cu, ws, ckpt, dckpt,
+                                             N, T, H, dq, dk, dv, dg, dbeta, status, s);
+  if (dt == KDA_F16)
+    return launch_local_typed<__half>(q, k, v, g, beta, dout, scale, cu, ws, ckpt, dckpt, N, T,
+                                      H, dq, dk, dv, dg, dbeta, status, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -100,7 +100,7 @@ template <int kRole>
 __global__ void __launch_bounds__(kBT, 3)
 chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
                    const float *s0, float scale, int N, int T, int H, int L, float *__restrict__ o,
-                   float *sN, int *status) {
+                   float *sN, float *ckpt, int *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -250,6 +250,11 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   uint32_t pa = 0, pk = 0, pm = 0;
   for (int c = c_lo; c < c_hi; ++c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
+    if (ckpt) {  // entry state of the chunk, for the backward pass
+      float *dst = ckpt + ((size_t)(cbase + c) * H + h) * (128 * 128) + sbase;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dst[(size_t)i * 128] = S[i];
+    }
 
     // ---- D1 = [W ; Q G] S ----------------------------------------------------------
     if (!wait_all(bar_a1, pa, status)) break;
@@ -327,7 +332,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], gl, ds[i]);
       if (c + 1 < c_hi) fetch_gl(c + 1);
     }
-    if (kRole == kOutputs && warp >= 2) {
+    if (kRole == kOutputs && warp >= 2 && o) {
       float ov[32], ov2[32];
       tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
       tmem_ld32_nowait(tmem + lane_addr + TB_D1B, ov2);
@@ -605,8 +610,8 @@ cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws,
 namespace {
 template <int kRole>
 cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0, float scale,
-                              int N, int T, int H, int L, float *o, float *sN, int *status,
-                              cudaStream_t s) {
+                              int N, int T, int H, int L, float *o, float *sN, float *ckpt,
+                              int *status, cudaStream_t s) {
   const long long items = L > 0 ? rec::segment_capacity(N, T, L) : N;
   const long long blocks = items * H * kSlices * (kRole == kTransition ? 2 : 1);
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
@@ -614,17 +619,18 @@ cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB_ALLOC);
   if (e != cudaSuccess) return e;
   chunk_state_kernel<kRole><<<(unsigned)blocks, kBT, SB_ALLOC, s>>>(
-      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, status);
+      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, ckpt, status);
   return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,
-                               cudaStream_t s) {
+                               cudaStream_t s, float *ckpt) {
   cudaError_t e;
   if (L > 0) {
-    e = launch_state_role<kTransition>(ws, cu, s0, scale, N, T, H, L, o, sN, status, s);
+    e = launch_state_role<kTransition>(ws, cu, s0, scale, N, T, H, L, o, sN, nullptr, status,
+                                       s);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SC_ALLOC);
@@ -634,7 +640,7 @@ cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_state_role<kOutputs>(ws, cu, s0, scale, N, T, H, L, o, sN, status, s);
+  return launch_state_role<kOutputs>(ws, cu, s0, scale, N, T, H, L, o, sN, ckpt, status, s);
 }
 
 }  // namespace kda

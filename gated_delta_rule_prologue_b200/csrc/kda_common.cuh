@@ -216,9 +216,23 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
                               float lower_bound, bool gated, int *status, cudaStream_t s);
 cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws, int *status,
                                cudaStream_t s);
+// ckpt (optional, [chunks][H][Dv][Dk] fp32 in record order): the entry state of
+// every chunk, for the backward pass; o may then be NULL.
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,
-                               cudaStream_t s);
+                               cudaStream_t s, float *ckpt = nullptr);
+// Backward of the two-pass prefill (kda_chunk_bwd.cu): the reverse state pass over
+// (sequence, head, value slice) writing the adjoint of every chunk's exit state
+// (dckpt, record order) and d_s0, then the local pass over (chunk, head).
+cudaError_t launch_chunk_bwd_state(const void *ws, const int32_t *cu, const float *dsN,
+                                   const float *dout, float scale, int N, int T, int H,
+                                   float *dckpt, float *ds0, int *status, cudaStream_t s);
+cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *dout, float scale,
+                                   const int32_t *cu, const void *ws, const float *ckpt,
+                                   const float *dckpt, int N, int T, int H, kda_dtype dt,
+                                   float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                   int *status, cudaStream_t s);
 cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
                                        void *cache_out, const void *g, const float *beta,
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,

@@ -259,6 +259,54 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
                                 kda_stream_t stream);
 
 /*
+ * Backward of the chunkwise prefill.  The pages mention training ([W1 彩蛋])
+ * but print no backward; these are the gradients of the loss
+ *     L = sum(d_o * o) + sum(d_final_state * final_state)
+ * with o and final_state those of kda_chunk_fwd on the same inputs, i.e. the
+ * chain rule through the recurrence of [W1 第三站 - 第五站].  The adjoint of
+ * the state is carried backwards through the chunks by the transpose of the
+ * forward's affine chunk map [W4 Figure 1]; inside a chunk the gradients come
+ * from the chunk algebra, evaluated in fp32 on 16-token blocks.
+ *
+ * kda_chunk_bwd_workspace_bytes -- scratch bytes of kda_chunk_bwd_ws: the
+ * forward's records and chunk index (kda_chunk_fwd_segmented_workspace_bytes
+ * with segment length 0) plus two fp32 128 x 128 blocks per (chunk, head)
+ * (the entry state and the adjoint of the exit state of every chunk).  0 off
+ * the tensor-core path (dt == KDA_F32, Dk or Dv != 128, chunk != 64, T == 0).
+ */
+size_t kda_chunk_bwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt);
+
+/*
+ * kda_chunk_bwd_ws -- gradients of kda_chunk_fwd.  Inputs as in kda_chunk_fwd
+ * (q, k, v, g, beta, scale, initial_state, cu_seqlens, N, T, H, Dk, Dv, chunk,
+ * dt; the tensor-core shapes only: dt KDA_BF16 or KDA_F16, Dk == Dv == 128,
+ * chunk 64, T > 0, else KDA_ERR_UNSUPPORTED), plus:
+ *   d_o              [T, H, Dv] f32, 16-byte aligned: dL/do
+ *   d_final_state    [N, H, Dv, Dk] f32 or NULL (zero): dL/dfinal_state
+ *   dq, dk, dg       [T, H, Dk] f32 outputs (dk, dg w.r.t. the k and g given)
+ *   dv               [T, H, Dv] f32 output
+ *   dbeta            [T, H] f32 output
+ *   d_initial_state  [N, H, Dv, Dk] f32 output or NULL (not written)
+ *   workspace        >= kda_chunk_bwd_workspace_bytes(...) bytes, 16-byte
+ *                    aligned, caller-owned, not NULL; contents on entry do not
+ *                    matter and are unspecified on return
+ * The forward is recomputed inside the call (o is not needed).  Rows of tokens
+ * outside every sequence are not written.  Outputs must not overlap the
+ * inputs, each other or the workspace (KDA_ERR_INVALID_ARG).  g >= -5 is
+ * required, as on the forward's tensor-core path; a 16-token block whose
+ * log-decay falls below -87 is reported as KDA_ERR_DEVICE_RANGE.  Asynchronous
+ * on `stream`; calls that may run concurrently must not share a workspace.
+ */
+kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float scale, const float *initial_state,
+                            const int32_t *cu_seqlens, int N, int T, int H, int Dk, int Dv,
+                            int chunk, kda_dtype dt, const float *d_o,
+                            const float *d_final_state, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                            size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_prologue_chunk_fwd -- the prologue fused into the chunkwise prefill: the
  * same result as kda_prologue followed by kda_chunk_fwd (chunk 64), with q, k
  * and v never written to memory.  Each chunk's projections are convolved

@@ -1,0 +1,138 @@
+"""GPU parity of the prefill backward (kda_chunk_bwd_ws) against the float64
+adjoint of the recurrence (oracle.kda_recurrent_backward, itself pinned by
+central differences in test_oracle_backward.py).
+
+Loss L = sum(d_o * o) + sum(d_final_state * final_state).  Tolerance: every
+gradient within max|delta| / RMS(reference) <= 2e-2, the bound the workloads
+state for bf16-input outputs (the backward rounds the same fp16 state operands
+as the forward's tensor-core path, and recomputes the chunk algebra in fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import kda_recurrent_backward, state_from_abi, state_to_abi
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+DEV = "cuda"
+NAMES = ("dq", "dk", "dv", "dg", "dbeta", "d_initial_state")
+
+
+@pytest.fixture(scope="module")
+def kda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import gated_delta_rule_prologue_b200 as m
+    return m
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel_max(got, ref):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got))
+    return float(np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref * ref)))
+
+
+def grads_inputs(inp, seed, with_dsN=True):
+    r = torch.Generator().manual_seed(seed)
+    d_o = torch.randn((inp.T, inp.H, inp.v.shape[2]), generator=r)
+    dsN = (torch.randn((inp.N, inp.H, 128, 128), generator=r) if with_dsN else None)
+    return d_o, dsN
+
+
+def run_bwd(kda, inp, d_o, dsN, workspace="auto"):
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(DEV)
+    s0 = None if inp.initial_state is None else inp.initial_state.to(DEV).contiguous()
+    out = kda.kda_chunk_bwd(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.g.to(DEV),
+                            inp.beta.to(DEV), d_o.to(DEV), scale=inp.scale, initial_state=s0,
+                            d_final_state=None if dsN is None else dsN.to(DEV), cu_seqlens=cu,
+                            workspace=workspace)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    return [f64(t) for t in out]
+
+
+def oracle_bwd(inp, d_o, dsN):
+    s0 = None if inp.initial_state is None else state_from_abi(inp.initial_state)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    dq, dk, dv, dg, db, ds0 = kda_recurrent_backward(
+        inp.q, inp.k, inp.v, inp.g, inp.beta, d_o, None if dsN is None else state_from_abi(dsN),
+        inp.scale, s0, cu)
+    return [dq, dk, dv, dg, db, state_to_abi(ds0)]
+
+
+def check(got, ref, tol=TOL):
+    errs = {n: rel_max(a, b) for n, a, b in zip(NAMES, got, ref)}
+    assert all(e <= tol for e in errs.values()), errs
+    return errs
+
+
+LENGTHS = [200, 0, 1, 64, 63, 130, 17]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_backward_varlen_matches_oracle(kda, dtype):
+    """Seven sequences: several chunks with a ragged tail, empty, one token, an
+    exact chunk, a chunk minus one, two chunks plus two, a short one."""
+    inp = W.random_prefill(80, sum(LENGTHS), 2, 128, s0_std=0.2, lengths=LENGTHS,
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z - 2.0))
+    inp.scale = 0.5
+    if dtype == "f16":
+        inp.q, inp.k, inp.v = inp.q.half(), inp.k.half(), inp.v.half()
+    d_o, dsN = grads_inputs(inp, 81)
+    check(run_bwd(kda, inp, d_o, dsN), oracle_bwd(inp, d_o, dsN))
+
+
+@pytest.mark.parametrize("g_fn", [lambda z: -5.0 * torch.sigmoid(z),
+                                  lambda z: -5.0 * torch.sigmoid(z - 6.0),
+                                  lambda z: torch.full_like(z, -5.0),
+                                  lambda z: torch.zeros_like(z)],
+                         ids=["k3_decay", "slow_decay", "saturated_decay", "no_decay"])
+def test_backward_single_sequence_decays(kda, g_fn):
+    """cu_seqlens NULL, 333 tokens (6 chunks, the last ragged), across the decay
+    range the tensor-core path supports (g in [-5, 0])."""
+    inp = W.random_prefill(82, 333, 2, 128, s0_std=0.1, g_fn=g_fn)
+    d_o, dsN = grads_inputs(inp, 83)
+    check(run_bwd(kda, inp, d_o, dsN), oracle_bwd(inp, d_o, dsN))
+
+
+def test_backward_without_initial_or_final_state_gradient(kda):
+    inp = W.random_prefill(84, 250, 3, 128, s0_std=0.0, lengths=[120, 130])
+    inp.initial_state = None
+    d_o, _ = grads_inputs(inp, 85, with_dsN=False)
+    check(run_bwd(kda, inp, d_o, None), oracle_bwd(inp, d_o, None))
+
+
+def test_backward_dirty_workspace_is_deterministic(kda):
+    inp = W.random_prefill(86, 400, 2, 128, s0_std=0.1, lengths=[150, 250])
+    d_o, dsN = grads_inputs(inp, 87)
+    N, T, H = inp.N, inp.T, inp.H
+    nbytes = kda.kda_chunk_bwd_workspace_bytes(N, T, H, 128, 128, 64, torch.bfloat16)
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=DEV)
+    a = run_bwd(kda, inp, d_o, dsN, workspace=ws)
+    b = run_bwd(kda, inp, d_o, dsN, workspace=ws)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_backward_long_sequence_sampled_head(kda):
+    """2048 tokens x 8 heads (the single-sequence workload's head count, half
+    its length): the GPU runs all heads, the oracle recomputes head 5."""
+    inp = W.random_prefill(88, 2048, 8, 128, s0_std=0.02, lengths=[2048],
+                           g_fn=lambda z: -5.0 * torch.sigmoid(z + 2.0))
+    d_o, dsN = grads_inputs(inp, 89)
+    got = run_bwd(kda, inp, d_o, dsN)
+    h = 5
+    sub = W.PrefillInputs(inp.q[:, h:h + 1].contiguous(), inp.k[:, h:h + 1].contiguous(),
+                          inp.v[:, h:h + 1].contiguous(), inp.g[:, h:h + 1].contiguous(),
+                          inp.beta[:, h:h + 1].contiguous(),
+                          inp.initial_state[:, h:h + 1].contiguous(), inp.cu_seqlens,
+                          inp.chunk, inp.scale, inp.dtype)
+    ref = oracle_bwd(sub, d_o[:, h:h + 1], dsN[:, h:h + 1])
+    got_h = [x[:, h:h + 1] for x in got]
+    check(got_h, ref)
