@@ -703,7 +703,8 @@ size_t kda_chunk_bwd_workspace_bytes(int N, int T, int H, int Dk, int Dv, int ch
                                      kda_dtype dt) {
   if (N < 1 || T < 0 || H < 1 || !chunk_tc_path(T, Dk, Dv, chunk, dt)) return 0;
   return kda::rec::workspace_bytes(N, T, H, 0) +
-         2 * (size_t)kda::rec::chunk_capacity(N, T) * H * kda::rec::SEG_BLOCK;
+         2 * (size_t)kda::rec::chunk_capacity(N, T) * H * kda::rec::SEG_BLOCK +
+         kda::chunk_bwd_local_scratch_bytes();
 }
 
 kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const float *g,
@@ -764,6 +765,7 @@ kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const f
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
   float *ckpt = reinterpret_cast<float *>(wsb + kda::rec::workspace_bytes(N, T, H, 0));
   float *dckpt = ckpt + (size_t)kda::rec::chunk_capacity(N, T) * H * 128 * 128;
+  float *scratch = dckpt + (size_t)kda::rec::chunk_capacity(N, T) * H * 128 * 128;
   cudaError_t e = cudaSuccess;
   if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, 0, workspace, status, s);
   if (e == cudaSuccess)
@@ -777,7 +779,7 @@ kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const f
                                     dckpt, d_initial_state, status, s);
   if (e == cudaSuccess)
     e = kda::launch_chunk_bwd_local(q, k, v, g, beta, d_o, scale, cu_seqlens, workspace, ckpt,
-                                    dckpt, N, T, H, dt, dq, dk, dv, dg, dbeta, status, s);
+                                    dckpt, scratch, N, T, H, dt, dq, dk, dv, dg, dbeta, status, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd_ws launch");
   return KDA_OK;
 }

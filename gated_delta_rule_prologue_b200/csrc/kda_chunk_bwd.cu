@@ -275,7 +275,8 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
 
 constexpr int kLT = 256;       // threads
 constexpr int kSub = 16;       // tokens per sub-chunk
-constexpr int RS = 132;        // row stride (floats) of the 128-wide shared matrices
+constexpr int RS = 132;        // row stride (floats) of the 128-wide shared matrices: eight
+                               // consecutive rows start 4 banks apart
 constexpr int SS = 17;         // row stride of the 16 x 16 matrices
 
 struct LocalSmem {
@@ -297,13 +298,14 @@ struct LocalSmem {
   float dA[kSub * SS];
   float beta[kSub];
   float gc[128];        // exp(gamma_last)
+  float xch[2][128];    // per-key partial sums passed between the two row halves
 };
 
-template <typename Tin>
-__device__ __forceinline__ void load8(const Tin *p, float (&f)[8]) {
-#pragma unroll
-  for (int e = 0; e < 8; ++e) f[e] = to_f32(p[e]);
-}
+// Persistent grid: one CTA per SM, each with a scratch slot for the entry states of
+// sub-chunks 1..3 of its current chunk (written by the forward walk, read back by the
+// backward walk; 192 KB per CTA, resident in L2).
+constexpr int kLocalCTAs = 148;
+constexpr size_t kLocalSlotFloats = (size_t)3 * 128 * 128;
 
 template <typename Tin>
 __global__ void __launch_bounds__(kLT, 1)
@@ -311,416 +313,489 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                        const Tin *__restrict__ v, const float *__restrict__ g,
                        const float *__restrict__ beta, const float *__restrict__ dout,
                        float scale, const int32_t *__restrict__ cu, const uint8_t *ws,
-                       const float *__restrict__ ckpt, const float *__restrict__ dckpt, int N,
-                       int T, int H, float *__restrict__ dq, float *__restrict__ dk,
-                       float *__restrict__ dv, float *__restrict__ dg,
-                       float *__restrict__ dbeta, int *status) {
+                       const float *__restrict__ ckpt, const float *__restrict__ dckpt,
+                       float *__restrict__ scratch, long long items, int N, int T, int H,
+                       float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
+                       float *__restrict__ dg, float *__restrict__ dbeta, int *status) {
   extern __shared__ float4 smem_f4[];
   LocalSmem &sm = *reinterpret_cast<LocalSmem *>(smem_f4);
   const int tid = threadIdx.x;
-  const int h = blockIdx.x % H, ci = blockIdx.x / H;
   const int32_t *cprefix = reinterpret_cast<const int32_t *>(ws);
-
-  // ---- which chunk ---------------------------------------------------------------------
-  int n = 0, c = ci;
-  if (cu) {
-    if (ci >= cprefix[N]) return;
-    int lo = 0, hi = N - 1;  // last n with cprefix[n] <= ci
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cprefix[mid] <= ci) lo = mid;
-      else hi = mid - 1;
-    }
-    n = lo;
-    c = ci - cprefix[n];
-  } else if (ci >= (T + 63) / 64) {
-    return;
-  }
-  int bos, eos;
-  seq_bounds(cu, n, T, status, bos, eos);
-  const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
-  if (Lc <= 0) return;
-  const int nsub = (Lc + kSub - 1) / kSub;
-  const size_t rec_idx = (size_t)ci * H + h;
-  const float *S0 = ckpt + rec_idx * (128 * 128);
-  const float *dS1 = dckpt + rec_idx * (128 * 128);
+  float *slot = scratch + (size_t)blockIdx.x * kLocalSlotFloats;
 
   // thread roles
-  const int rr = tid >> 4, c8 = tid & 15;          // (row, 8 value columns) for 16 x 128 outputs
-  const int kt = tid >> 1, half = tid & 1;         // (key channel, half) for key-indexed work
-  // value columns of (rr, c8): {4 c8 .. 4 c8 + 3} and {64 + 4 c8 .. 64 + 4 c8 + 3}
-  const int ca = 4 * c8, cb = 64 + 4 * c8;
+  const int rr = tid >> 4, c8 = tid & 15;     // (row, 8 value columns) for 16 x 128 outputs
+  const int ca = 4 * c8, cb = 64 + 4 * c8;    // its columns: [ca, ca+4) and [cb, cb+4)
+  const int kt = tid & 127, rh = tid >> 7;    // (key, rows 8 rh .. 8 rh + 7): a warp holds 32 keys
+  const int kq = tid & 63, q4 = tid >> 6;     // (keys kq and kq + 64, value chunks 16 m + 4 q4)
 
-  auto load_state = [&](float *dst, const float *src) {  // src [value][key] -> dst[key][value]
+  // [value][key] in global <-> [key][value] in shared memory.  Lane l moves key
+  // base + l % 8 of value row j0 + l / 8: the 32 lanes hit 32 distinct banks, and
+  // the global side reads 32-byte runs of keys.
+  auto load_state = [&](float *dst, const float *src) {
     for (int idx = tid; idx < 128 * 128; idx += kLT) {
-      const int j = idx >> 7, key = idx & 127;
-      dst[key * RS + j] = src[idx];
+      const int w = idx >> 5, l = idx & 31;           // w: 512 groups of 32
+      const int key = 8 * (w & 15) + (l & 7), j = 4 * (w >> 4) + (l >> 3);
+      dst[key * RS + j] = src[(size_t)j * 128 + key];
+    }
+  };
+  auto store_state = [&](float *dst, const float *src) {
+    for (int idx = tid; idx < 128 * 128; idx += kLT) {
+      const int w = idx >> 5, l = idx & 31;
+      const int key = 8 * (w & 15) + (l & 7), j = 4 * (w >> 4) + (l >> 3);
+      dst[(size_t)j * 128 + key] = src[key * RS + j];
     }
   };
 
-  // Inputs of sub-chunk sb: G, KG, KD, QG, KP, E (= v for now), dO (scaled), beta, gc.
-  auto load_sub = [&](int sb, bool with_grad) {
-    const int r0 = kSub * sb;
-    {  // g (raw) into G, q and k and v per (row, 8 channels)
-      const int r = rr, tok = t0 + r0 + r;
-      const bool ok = r0 + r < Lc;
-      const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
+  for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+    const int h = (int)(it % H), ci = (int)(it / H);
+    // ---- which chunk (uniform over the CTA) ---------------------------------------------
+    int n = 0, c = ci;
+    if (cu) {
+      if (ci >= cprefix[N]) break;  // items are in chunk order: none left
+      int lo = 0, hi = N - 1;       // last n with cprefix[n] <= ci
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cprefix[mid] <= ci) lo = mid;
+        else hi = mid - 1;
+      }
+      n = lo;
+      c = ci - cprefix[n];
+    } else if (ci >= (T + 63) / 64) {
+      break;
+    }
+    int bos, eos;
+    seq_bounds(cu, n, T, status, bos, eos);
+    const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
+    if (Lc <= 0) continue;
+    const int nsub = (Lc + kSub - 1) / kSub;
+    const size_t rec_idx = (size_t)ci * H + h;
+    const float *S0 = ckpt + rec_idx * (128 * 128);
+    const float *dS1 = dckpt + rec_idx * (128 * 128);
+
+    // Inputs of sub-chunk sb: G, KG, KD, QG, KP, E (= v for now), dO (scaled), beta, gc.
+    auto load_sub = [&](int sb, bool with_grad) {
+      const int r0 = kSub * sb;
+      {  // g (raw) into G, beta
+        const int r = rr, tok = t0 + r0 + r;
+        const bool ok = r0 + r < Lc;
+        const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int col = part ? cb : ca;
-        float gv[4] = {0.f, 0.f, 0.f, 0.f};
-        if (ok) {
-          const float4 f = __ldg(reinterpret_cast<const float4 *>(g + base + col));
-          gv[0] = f.x; gv[1] = f.y; gv[2] = f.z; gv[3] = f.w;
+        for (int part = 0; part < 2; ++part) {
+          const int col = part ? cb : ca;
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ok) f = __ldg(reinterpret_cast<const float4 *>(g + base + col));
+          *reinterpret_cast<float4 *>(&sm.G[r * RS + col]) = f;
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sm.G[r * RS + col + e] = gv[e];
+        if (c8 == 0) sm.beta[r] = ok ? __ldg(beta + (size_t)tok * H + h) : 0.f;
       }
-      if (c8 == 0) sm.beta[r] = ok ? __ldg(beta + (size_t)tok * H + h) : 0.f;
-    }
-    __syncthreads();
-    if (tid < 128) {  // inclusive cumsum over the rows, per key channel
-      float run = 0.f;
+      __syncthreads();
+      if (tid < 128) {  // inclusive cumsum over the rows, per key channel
+        float run = 0.f;
 #pragma unroll
-      for (int r = 0; r < kSub; ++r) {
-        run += sm.G[r * RS + tid];
-        sm.G[r * RS + tid] = run;
+        for (int r = 0; r < kSub; ++r) {
+          run += sm.G[r * RS + tid];
+          sm.G[r * RS + tid] = run;
+        }
+        sm.gc[tid] = __expf(run);
+        // a 16-token block needs its log-decay within fp32's exp range (g >= -5 gives >= -80)
+        if (!(run >= -87.f)) report(status, KDA_ERR_DEVICE_RANGE);
       }
-      sm.gc[tid] = __expf(run);
-      // a 16-token block needs its log-decay within fp32's exp range (g >= -5 gives >= -80)
-      if (!(run >= -87.f)) report(status, KDA_ERR_DEVICE_RANGE);
-    }
-    __syncthreads();
-    {
-      const int r = rr, tok = t0 + r0 + r;
-      const bool ok = r0 + r < Lc;
-      const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
+      __syncthreads();
+      {
+        const int r = rr, tok = t0 + r0 + r;
+        const bool ok = r0 + r < Lc;
+        const size_t base = ((size_t)(ok ? tok : 0) * H + h) * 128;
+        float gm[8];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int col = part ? cb : ca;
-        float kv[4] = {0.f, 0.f, 0.f, 0.f}, qv[4] = {0.f, 0.f, 0.f, 0.f};
-        float vv[4] = {0.f, 0.f, 0.f, 0.f}, dv4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (ok) {
+        for (int part = 0; part < 2; ++part) {
+          const int col = part ? cb : ca;
+          float kv[4] = {0.f, 0.f, 0.f, 0.f}, qv[4] = {0.f, 0.f, 0.f, 0.f};
+          float vv[4] = {0.f, 0.f, 0.f, 0.f}, dv4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              kv[e] = to_f32(k[base + col + e]);
+              qv[e] = to_f32(q[base + col + e]);
+              vv[e] = to_f32(v[base + col + e]);
+            }
+            if (with_grad) {
+              const float4 f = __ldg(reinterpret_cast<const float4 *>(dout + base + col));
+              dv4[0] = scale * f.x; dv4[1] = scale * f.y; dv4[2] = scale * f.z; dv4[3] = scale * f.w;
+            }
+          }
+          const float4 gam4 = *reinterpret_cast<const float4 *>(&sm.G[r * RS + col]);
+          const float4 gl4 = *reinterpret_cast<const float4 *>(&sm.G[(kSub - 1) * RS + col]);
+          const float gam[4] = {gam4.x, gam4.y, gam4.z, gam4.w};
+          const float glast[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+          float kg[4], kd[4], qg[4], kpv[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            kv[e] = to_f32(k[base + col + e]);
-            qv[e] = to_f32(q[base + col + e]);
-            vv[e] = to_f32(v[base + col + e]);
+            const float Gv = __expf(gam[e]), Gi = __expf(-gam[e]);
+            gm[4 * part + e] = Gv;
+            kg[e] = kv[e] * Gv;
+            kd[e] = kv[e] * Gi;
+            qg[e] = qv[e] * Gv;
+            kpv[e] = kv[e] * __expf(glast[e] - gam[e]);
           }
-          if (with_grad) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(dout + base + col));
-            dv4[0] = scale * f.x; dv4[1] = scale * f.y; dv4[2] = scale * f.z; dv4[3] = scale * f.w;
-          }
+          const int o = r * RS + col;
+          *reinterpret_cast<float4 *>(&sm.KG[o]) = make_float4(kg[0], kg[1], kg[2], kg[3]);
+          *reinterpret_cast<float4 *>(&sm.KD[o]) = make_float4(kd[0], kd[1], kd[2], kd[3]);
+          *reinterpret_cast<float4 *>(&sm.QG[o]) = make_float4(qg[0], qg[1], qg[2], qg[3]);
+          *reinterpret_cast<float4 *>(&sm.KP[o]) = make_float4(kpv[0], kpv[1], kpv[2], kpv[3]);
+          *reinterpret_cast<float4 *>(&sm.E[o]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+          *reinterpret_cast<float4 *>(&sm.dO[o]) = make_float4(dv4[0], dv4[1], dv4[2], dv4[3]);
         }
+        __syncthreads();  // gamma of the last row has been read by every thread
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const int col = part ? cb : ca;
+          *reinterpret_cast<float4 *>(&sm.G[r * RS + col]) =
+              make_float4(gm[4 * part], gm[4 * part + 1], gm[4 * part + 2], gm[4 * part + 3]);
+        }
+      }
+      __syncthreads();
+    };
+
+    // E = V - (K G) S;  KK, A, P;  U = (I + A)^{-1} diag(beta) E.
+    auto forward_local = [&](bool with_p) {
+      {
+        float acc[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = col + e;
-          const float gam = sm.G[r * RS + j], glast = sm.G[(kSub - 1) * RS + j];
-          const float Gv = __expf(gam), Gi = __expf(-gam);
-          sm.KG[r * RS + j] = kv[e] * Gv;
-          sm.KD[r * RS + j] = kv[e] * Gi;
-          sm.QG[r * RS + j] = qv[e] * Gv;
-          sm.KP[r * RS + j] = kv[e] * __expf(glast - gam);
-          sm.E[r * RS + j] = vv[e];
-          sm.dO[r * RS + j] = dv4[e];
+          acc[e] = sm.E[rr * RS + ca + e];
+          acc[4 + e] = sm.E[rr * RS + cb + e];
+        }
+#pragma unroll 4
+        for (int key = 0; key < 128; ++key) {
+          const float a = sm.KG[rr * RS + key];
+          const float4 s1 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + ca]);
+          const float4 s2 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + cb]);
+          acc[0] -= a * s1.x; acc[1] -= a * s1.y; acc[2] -= a * s1.z; acc[3] -= a * s1.w;
+          acc[4] -= a * s2.x; acc[5] -= a * s2.y; acc[6] -= a * s2.z; acc[7] -= a * s2.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // each thread rewrites only the entries it read
+          sm.E[rr * RS + ca + e] = acc[e];
+          sm.E[rr * RS + cb + e] = acc[4 + e];
         }
       }
-    }
-    __syncthreads();
-    {  // G = exp(gamma) in place (every reader of gamma above is done)
-      const int r = rr;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int col = part ? cb : ca;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sm.G[r * RS + col + e] = __expf(sm.G[r * RS + col + e]);
-      }
-    }
-  };
-
-  // E = V - (K G) S;  KK, A, P;  U = (I + A)^{-1} diag(beta) E.
-  auto forward_local = [&](bool with_p) {
-    {
-      float acc[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[e] = sm.E[rr * RS + ca + e];
-        acc[4 + e] = sm.E[rr * RS + cb + e];
-      }
+      {  // 16 x 16 Grams: thread (r, i)
+        const int r = tid >> 4, i = tid & 15;
+        float kk = 0.f, pp = 0.f;
 #pragma unroll 4
-      for (int key = 0; key < 128; ++key) {
-        const float a = sm.KG[rr * RS + key];
-        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + ca]);
-        const float4 s2 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + cb]);
-        acc[0] -= a * s1.x; acc[1] -= a * s1.y; acc[2] -= a * s1.z; acc[3] -= a * s1.w;
-        acc[4] -= a * s2.x; acc[5] -= a * s2.y; acc[6] -= a * s2.z; acc[7] -= a * s2.w;
+        for (int key = 0; key < 128; key += 4) {
+          const float4 kd = *reinterpret_cast<const float4 *>(&sm.KD[i * RS + key]);
+          const float4 kg = *reinterpret_cast<const float4 *>(&sm.KG[r * RS + key]);
+          kk = fmaf(kg.x, kd.x, kk); kk = fmaf(kg.y, kd.y, kk);
+          kk = fmaf(kg.z, kd.z, kk); kk = fmaf(kg.w, kd.w, kk);
+          if (with_p) {
+            const float4 qg = *reinterpret_cast<const float4 *>(&sm.QG[r * RS + key]);
+            pp = fmaf(qg.x, kd.x, pp); pp = fmaf(qg.y, kd.y, pp);
+            pp = fmaf(qg.z, kd.z, pp); pp = fmaf(qg.w, kd.w, pp);
+          }
+        }
+        sm.KK[r * SS + i] = kk;
+        sm.A[r * SS + i] = i < r ? sm.beta[r] * kk : 0.f;
+        sm.P[r * SS + i] = i <= r ? pp : 0.f;
       }
-      __syncthreads();  // all reads of E (= v) done before it is overwritten
+      __syncthreads();
+      if (tid < 128) {  // forward substitution, one value column per thread
+        const int j = tid;
+        float u[kSub];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        sm.E[rr * RS + ca + e] = acc[e];
-        sm.E[rr * RS + cb + e] = acc[4 + e];
-      }
-    }
-    {  // 16 x 16 Grams: thread (r, i)
-      const int r = tid >> 4, i = tid & 15;
-      float kk = 0.f, pp = 0.f;
-#pragma unroll 8
-      for (int key = 0; key < 128; ++key) {
-        const float kd = sm.KD[i * RS + key];
-        kk = fmaf(sm.KG[r * RS + key], kd, kk);
-        if (with_p) pp = fmaf(sm.QG[r * RS + key], kd, pp);
-      }
-      sm.KK[r * SS + i] = kk;
-      sm.A[r * SS + i] = i < r ? sm.beta[r] * kk : 0.f;
-      sm.P[r * SS + i] = i <= r ? pp : 0.f;
-    }
-    __syncthreads();
-    if (tid < 128) {  // forward substitution, one value column per thread
-      const int j = tid;
-      float u[kSub];
+        for (int r = 0; r < kSub; ++r) {
+          float x = sm.beta[r] * sm.E[r * RS + j];
 #pragma unroll
-      for (int r = 0; r < kSub; ++r) {
-        float x = sm.beta[r] * sm.E[r * RS + j];
-#pragma unroll
-        for (int i = 0; i < r; ++i) x = fmaf(-sm.A[r * SS + i], u[i], x);
-        u[r] = x;
-        sm.U[r * RS + j] = x;
+          for (int i = 0; i < r; ++i) x = fmaf(-sm.A[r * SS + i], u[i], x);
+          u[r] = x;
+          sm.U[r * RS + j] = x;
+        }
       }
-    }
-    __syncthreads();
-  };
+      __syncthreads();
+    };
 
-  // S <- diag(G_last) S + K'^T U   (thread (key, half of the values))
-  auto advance_state = [&]() {
-    const float gck = sm.gc[kt];
-    float *row = &sm.S[kt * RS + 64 * half];
+    // S <- diag(G_last) S + K'^T U   (thread (keys kq, kq + 64; value chunks 16 m + 4 q4))
+    auto advance_state = [&]() {
+      float st[2][32];
 #pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      float4 s = *reinterpret_cast<float4 *>(row + 4 * x);
-      s.x *= gck; s.y *= gck; s.z *= gck; s.w *= gck;
+      for (int kk = 0; kk < 2; ++kk) {
+        const int key = kq + 64 * kk;
+        const float gck = sm.gc[key];
 #pragma unroll
-      for (int r = 0; r < kSub; ++r) {
-        const float kp = sm.KP[r * RS + kt];
-        const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + 64 * half + 4 * x]);
-        s.x = fmaf(kp, u.x, s.x); s.y = fmaf(kp, u.y, s.y);
-        s.z = fmaf(kp, u.z, s.z); s.w = fmaf(kp, u.w, s.w);
+        for (int m = 0; m < 8; ++m) {
+          const float4 x = *reinterpret_cast<const float4 *>(&sm.S[key * RS + 16 * m + 4 * q4]);
+          st[kk][4 * m] = gck * x.x; st[kk][4 * m + 1] = gck * x.y;
+          st[kk][4 * m + 2] = gck * x.z; st[kk][4 * m + 3] = gck * x.w;
+        }
       }
-      *reinterpret_cast<float4 *>(row + 4 * x) = s;
-    }
-    __syncthreads();
-  };
+#pragma unroll 2
+      for (int r = 0; r < kSub; ++r) {
+        const float kp0 = sm.KP[r * RS + kq], kp1 = sm.KP[r * RS + kq + 64];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + 16 * m + 4 * q4]);
+          st[0][4 * m] = fmaf(kp0, u.x, st[0][4 * m]); st[0][4 * m + 1] = fmaf(kp0, u.y, st[0][4 * m + 1]);
+          st[0][4 * m + 2] = fmaf(kp0, u.z, st[0][4 * m + 2]); st[0][4 * m + 3] = fmaf(kp0, u.w, st[0][4 * m + 3]);
+          st[1][4 * m] = fmaf(kp1, u.x, st[1][4 * m]); st[1][4 * m + 1] = fmaf(kp1, u.y, st[1][4 * m + 1]);
+          st[1][4 * m + 2] = fmaf(kp1, u.z, st[1][4 * m + 2]); st[1][4 * m + 3] = fmaf(kp1, u.w, st[1][4 * m + 3]);
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          *reinterpret_cast<float4 *>(&sm.S[(kq + 64 * kk) * RS + 16 * m + 4 * q4]) =
+              make_float4(st[kk][4 * m], st[kk][4 * m + 1], st[kk][4 * m + 2], st[kk][4 * m + 3]);
+      __syncthreads();
+    };
 
-  load_state(sm.dS, dS1);
-  for (int sb = nsub - 1; sb >= 0; --sb) {
-    // ---- entry state of sub-chunk sb: the chunk's entry state, walked forward ---------------
+    // ---- forward walk: entry states of sub-chunks 1 .. nsub-1 into the scratch slot -------
     load_state(sm.S, S0);
     __syncthreads();
-    for (int j = 0; j < sb; ++j) {
+    for (int j = 0; j + 1 < nsub; ++j) {
       load_sub(j, false);
-      __syncthreads();
       forward_local(false);
       advance_state();
+      store_state(slot + (size_t)j * 128 * 128, sm.S);
     }
-    load_sub(sb, true);
-    __syncthreads();
-    forward_local(true);
-    const int r0 = kSub * sb;
+    load_state(sm.dS, dS1);
 
-    // ---- dU = P^T dO' + K' dS'  (thread (r, 8 value columns)) ------------------------------
-    {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < kSub; ++i) {
-        const float p = sm.P[i * SS + rr];
-        const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + ca]);
-        const float4 d2 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + cb]);
-        acc[0] = fmaf(p, d1.x, acc[0]); acc[1] = fmaf(p, d1.y, acc[1]);
-        acc[2] = fmaf(p, d1.z, acc[2]); acc[3] = fmaf(p, d1.w, acc[3]);
-        acc[4] = fmaf(p, d2.x, acc[4]); acc[5] = fmaf(p, d2.y, acc[5]);
-        acc[6] = fmaf(p, d2.z, acc[6]); acc[7] = fmaf(p, d2.w, acc[7]);
+    // ---- backward walk -------------------------------------------------------------------
+    for (int sb = nsub - 1; sb >= 0; --sb) {
+      if (sb < nsub - 1) {  // the last sub-chunk's entry state is still in place
+        __syncthreads();    // every thread is done with the previous sub-chunk's state
+        load_state(sm.S, sb == 0 ? S0 : slot + (size_t)(sb - 1) * 128 * 128);
       }
+      __syncthreads();
+      load_sub(sb, true);
+      forward_local(true);
+      const int r0 = kSub * sb;
+
+      // ---- dU = P^T dO' + K' dS'  (thread (r, 8 value columns)) ----------------------------
+      {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < kSub; ++i) {
+          const float p = sm.P[i * SS + rr];
+          const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + ca]);
+          const float4 d2 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + cb]);
+          acc[0] = fmaf(p, d1.x, acc[0]); acc[1] = fmaf(p, d1.y, acc[1]);
+          acc[2] = fmaf(p, d1.z, acc[2]); acc[3] = fmaf(p, d1.w, acc[3]);
+          acc[4] = fmaf(p, d2.x, acc[4]); acc[5] = fmaf(p, d2.y, acc[5]);
+          acc[6] = fmaf(p, d2.z, acc[6]); acc[7] = fmaf(p, d2.w, acc[7]);
+        }
 #pragma unroll 4
-      for (int key = 0; key < 128; ++key) {
-        const float a = sm.KP[rr * RS + key];
-        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + ca]);
-        const float4 s2 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + cb]);
-        acc[0] = fmaf(a, s1.x, acc[0]); acc[1] = fmaf(a, s1.y, acc[1]);
-        acc[2] = fmaf(a, s1.z, acc[2]); acc[3] = fmaf(a, s1.w, acc[3]);
-        acc[4] = fmaf(a, s2.x, acc[4]); acc[5] = fmaf(a, s2.y, acc[5]);
-        acc[6] = fmaf(a, s2.z, acc[6]); acc[7] = fmaf(a, s2.w, acc[7]);
+        for (int key = 0; key < 128; ++key) {
+          const float a = sm.KP[rr * RS + key];
+          const float4 s1 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + ca]);
+          const float4 s2 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + cb]);
+          acc[0] = fmaf(a, s1.x, acc[0]); acc[1] = fmaf(a, s1.y, acc[1]);
+          acc[2] = fmaf(a, s1.z, acc[2]); acc[3] = fmaf(a, s1.w, acc[3]);
+          acc[4] = fmaf(a, s2.x, acc[4]); acc[5] = fmaf(a, s2.y, acc[5]);
+          acc[6] = fmaf(a, s2.z, acc[6]); acc[7] = fmaf(a, s2.w, acc[7]);
+        }
+        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + ca]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + cb]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        sm.dU[rr * RS + ca + e] = acc[e];
-        sm.dU[rr * RS + cb + e] = acc[4 + e];
-      }
-    }
-    {  // dP = lower(dO' U^T)   (thread (r, i))
-      const int r = tid >> 4, i = tid & 15;
-      float acc = 0.f;
-      if (i <= r) {
+      {  // dP = lower(dO' U^T)   (thread (r, i))
+        const int r = tid >> 4, i = tid & 15;
+        float acc = 0.f;
+        if (i <= r) {
 #pragma unroll 8
-        for (int j = 0; j < 128; j += 4) {
-          const float4 a = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
-          const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
-          acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
-          acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+          for (int j = 0; j < 128; j += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
+            const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
+            acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
+            acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+          }
+        }
+        sm.dP[r * SS + i] = acc;
+      }
+      __syncthreads();
+      if (tid < 128) {  // dR = (I + A)^{-T} dU, back substitution in place
+        const int j = tid;
+        float x[kSub];
+#pragma unroll
+        for (int r = kSub - 1; r >= 0; --r) {
+          float y = sm.dU[r * RS + j];
+#pragma unroll
+          for (int i = r + 1; i < kSub; ++i) y = fmaf(-sm.A[i * SS + r], x[i], y);
+          x[r] = y;
+          sm.dU[r * RS + j] = y;
         }
       }
-      sm.dP[r * SS + i] = acc;
-    }
-    __syncthreads();
-    if (tid < 128) {  // dR = (I + A)^{-T} dU, back substitution in place
-      const int j = tid;
-      float x[kSub];
-#pragma unroll
-      for (int r = kSub - 1; r >= 0; --r) {
-        float y = sm.dU[r * RS + j];
-#pragma unroll
-        for (int i = r + 1; i < kSub; ++i) y = fmaf(-sm.A[i * SS + r], x[i], y);
-        x[r] = y;
-        sm.dU[r * RS + j] = y;
-      }
-    }
-    __syncthreads();
-    {  // dA = -strict_lower(dR U^T); dbeta; dv = beta dR
-      const int r = tid >> 4, i = tid & 15;
-      float acc = 0.f;
-      if (i < r) {
+      __syncthreads();
+      {  // dA = -strict_lower(dR U^T); dbeta; dv = beta dR
+        const int r = tid >> 4, i = tid & 15;
+        float acc = 0.f;
+        if (i < r) {
 #pragma unroll 8
-        for (int j = 0; j < 128; j += 4) {
-          const float4 a = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
-          const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
-          acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
-          acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+          for (int j = 0; j < 128; j += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
+            const float4 b = *reinterpret_cast<const float4 *>(&sm.U[i * RS + j]);
+            acc = fmaf(a.x, b.x, acc); acc = fmaf(a.y, b.y, acc);
+            acc = fmaf(a.z, b.z, acc); acc = fmaf(a.w, b.w, acc);
+          }
         }
+        const float da = -acc;
+        sm.dA[r * SS + i] = da;
+        // dbeta_r = <dR_r, E_r> + sum_{i<r} dA[r,i] KK[r,i]; lanes (r, 0..15) share row r
+        float part = i < r ? da * sm.KK[r * SS + i] : 0.f;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const float4 a = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + 8 * i + 4 * x]);
+          const float4 b = *reinterpret_cast<const float4 *>(&sm.E[r * RS + 8 * i + 4 * x]);
+          part = fmaf(a.x, b.x, part); part = fmaf(a.y, b.y, part);
+          part = fmaf(a.z, b.z, part); part = fmaf(a.w, b.w, part);
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if (i == 0 && r0 + r < Lc) dbeta[(size_t)(t0 + r0 + r) * H + h] = part;
       }
-      const float da = -acc;
-      sm.dA[r * SS + i] = da;
-      // dbeta_r = <dR_r, E_r> + sum_{i<r} dA[r,i] KK[r,i]; lanes (r, 0..15) share row r
-      float part = i < r ? da * sm.KK[r * SS + i] : 0.f;
-#pragma unroll
-      for (int jj = i; jj < 128; jj += 16) part = fmaf(sm.dU[r * RS + jj], sm.E[r * RS + jj], part);
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (i == 0 && r0 + r < Lc) dbeta[(size_t)(t0 + r0 + r) * H + h] = part;
-    }
-    if (r0 + rr < Lc) {
-      const float b = sm.beta[rr];
-      float *dst = dv + ((size_t)(t0 + r0 + rr) * H + h) * 128;
-      float4 o1, o2;
-      o1.x = b * sm.dU[rr * RS + ca]; o1.y = b * sm.dU[rr * RS + ca + 1];
-      o1.z = b * sm.dU[rr * RS + ca + 2]; o1.w = b * sm.dU[rr * RS + ca + 3];
-      o2.x = b * sm.dU[rr * RS + cb]; o2.y = b * sm.dU[rr * RS + cb + 1];
-      o2.z = b * sm.dU[rr * RS + cb + 2]; o2.w = b * sm.dU[rr * RS + cb + 3];
-      *reinterpret_cast<float4 *>(dst + ca) = o1;
-      *reinterpret_cast<float4 *>(dst + cb) = o2;
-    }
-    __syncthreads();
+      if (r0 + rr < Lc) {
+        const float b = sm.beta[rr];
+        float *dst = dv + ((size_t)(t0 + r0 + rr) * H + h) * 128;
+        const float4 a1 = *reinterpret_cast<const float4 *>(&sm.dU[rr * RS + ca]);
+        const float4 a2 = *reinterpret_cast<const float4 *>(&sm.dU[rr * RS + cb]);
+        *reinterpret_cast<float4 *>(dst + ca) = make_float4(b * a1.x, b * a1.y, b * a1.z, b * a1.w);
+        *reinterpret_cast<float4 *>(dst + cb) = make_float4(b * a2.x, b * a2.y, b * a2.z, b * a2.w);
+      }
+      __syncthreads();
 
-    // ---- key-indexed gradients: thread (key kt, rows 8 half .. 8 half + 7) -------------------
-    {
-      const int rb = 8 * half;
-      float dqg[8], dkg[8], dkp[8];
+      // ---- key-indexed gradients: thread (key kt, rows 8 rh .. 8 rh + 7) -----------------------
+      {
+        const int rb = 8 * rh;
+        float dqg[8], dkg[8], dkp[8];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) dqg[x] = dkg[x] = dkp[x] = 0.f;
-      float sds = 0.f;  // rowsum(S * dS') of key kt
-      const float *srow = &sm.S[kt * RS], *dsrow = &sm.dS[kt * RS];
+        for (int x = 0; x < 8; ++x) dqg[x] = dkg[x] = dkp[x] = 0.f;
+        float sds = 0.f;  // rowsum(S * dS') of key kt
+        const float *srow = &sm.S[kt * RS], *dsrow = &sm.dS[kt * RS];
 #pragma unroll 2
-      for (int j = 0; j < 128; j += 4) {
-        const float4 s = *reinterpret_cast<const float4 *>(srow + j);
-        const float4 d = *reinterpret_cast<const float4 *>(dsrow + j);
-        sds = fmaf(s.x, d.x, sds); sds = fmaf(s.y, d.y, sds);
-        sds = fmaf(s.z, d.z, sds); sds = fmaf(s.w, d.w, sds);
+        for (int j = 0; j < 128; j += 4) {
+          const float4 sv = *reinterpret_cast<const float4 *>(srow + j);
+          const float4 dv4 = *reinterpret_cast<const float4 *>(dsrow + j);
+          sds = fmaf(sv.x, dv4.x, sds); sds = fmaf(sv.y, dv4.y, sds);
+          sds = fmaf(sv.z, dv4.z, sds); sds = fmaf(sv.w, dv4.w, sds);
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const int r = rb + x;  // the same row for the whole warp: broadcast reads
+            const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
+            const float4 rr4 = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
+            const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + j]);
+            dqg[x] = fmaf(o.x, sv.x, dqg[x]); dqg[x] = fmaf(o.y, sv.y, dqg[x]);
+            dqg[x] = fmaf(o.z, sv.z, dqg[x]); dqg[x] = fmaf(o.w, sv.w, dqg[x]);
+            dkg[x] = fmaf(rr4.x, sv.x, dkg[x]); dkg[x] = fmaf(rr4.y, sv.y, dkg[x]);
+            dkg[x] = fmaf(rr4.z, sv.z, dkg[x]); dkg[x] = fmaf(rr4.w, sv.w, dkg[x]);
+            dkp[x] = fmaf(u.x, dv4.x, dkp[x]); dkp[x] = fmaf(u.y, dv4.y, dkp[x]);
+            dkp[x] = fmaf(u.z, dv4.z, dkp[x]); dkp[x] = fmaf(u.w, dv4.w, dkp[x]);
+          }
+        }
+        float dgam[8], dkd[8];
+        float kps = 0.f;  // sum over this thread's rows of dK' K'
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           const int r = rb + x;
-          const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
-          const float4 rr4 = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
-          const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + j]);
-          dqg[x] = fmaf(o.x, s.x, dqg[x]); dqg[x] = fmaf(o.y, s.y, dqg[x]);
-          dqg[x] = fmaf(o.z, s.z, dqg[x]); dqg[x] = fmaf(o.w, s.w, dqg[x]);
-          dkg[x] = fmaf(rr4.x, s.x, dkg[x]); dkg[x] = fmaf(rr4.y, s.y, dkg[x]);
-          dkg[x] = fmaf(rr4.z, s.z, dkg[x]); dkg[x] = fmaf(rr4.w, s.w, dkg[x]);
-          dkp[x] = fmaf(u.x, d.x, dkp[x]); dkp[x] = fmaf(u.y, d.y, dkp[x]);
-          dkp[x] = fmaf(u.z, d.z, dkp[x]); dkp[x] = fmaf(u.w, d.w, dkp[x]);
+          float pq = 0.f, pa = 0.f, kd = 0.f;
+#pragma unroll
+          for (int i = 0; i < kSub; ++i) {
+            const float kdi = sm.KD[i * RS + kt];
+            pq = fmaf(sm.dP[r * SS + i], kdi, pq);   // (dP K/G)[r]
+            pa = fmaf(sm.dA[r * SS + i], kdi, pa);   // (dA K/G)[r]
+            // ((diag(beta) dA)^T (K G) + dP^T (Q G))[r]
+            kd = fmaf(sm.beta[i] * sm.dA[i * SS + r], sm.KG[i * RS + kt],
+                      fmaf(sm.dP[i * SS + r], sm.QG[i * RS + kt], kd));
+          }
+          const float b = sm.beta[r], kpr = sm.KP[r * RS + kt];
+          dqg[x] += pq;
+          dkg[x] = b * (pa - dkg[x]);
+          dkd[x] = kd;
+          dgam[x] = dqg[x] * sm.QG[r * RS + kt] + dkg[x] * sm.KG[r * RS + kt] -
+                    dkd[x] * sm.KD[r * RS + kt] - dkp[x] * kpr;
+          kps = fmaf(dkp[x], kpr, kps);
+        }
+        // reverse cumulative sum within this thread's 8 rows
+        float tot = 0.f;
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+          tot += dgam[x];
+          dgam[x] = tot;
+        }
+        sm.xch[rh][kt] = rh ? tot : kps;  // upper half: its dgamma total; lower: its dK' K' sum
+        __syncthreads();
+        const float other = sm.xch[rh ^ 1][kt];
+        __syncthreads();
+        // the last row (row 15, upper half) gains G_last rowsum(S dS') + sum over all 16 rows
+        // of dK' K'; every row at or above it sees that term in its suffix sum.
+        const float last = rh ? sm.gc[kt] * sds + kps + other : 0.f;
+        if (rh == 1) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) dgam[x] += last;
+          sm.xch[0][kt] = tot + last;   // the whole upper half, for the lower half's suffixes
+        }
+        __syncthreads();
+        if (rh == 0) {
+          const float upper = sm.xch[0][kt];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) dgam[x] += upper;
+        }
+        const float gck = sm.gc[kt];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const int r = rb + x;
+          if (r0 + r < Lc) {
+            const float Gv = sm.G[r * RS + kt];
+            const size_t o = ((size_t)(t0 + r0 + r) * H + h) * 128 + kt;
+            dq[o] = dqg[x] * Gv;
+            dk[o] = dkg[x] * Gv + __fdividef(dkd[x] + dkp[x] * gck, Gv);
+            dg[o] = dgam[x];
+          }
         }
       }
-      float dgam[8], dkd[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int r = rb + x;
-        float pq = 0.f, pa = 0.f, kd = 0.f;
-#pragma unroll
-        for (int i = 0; i < kSub; ++i) {
-          const float kdi = sm.KD[i * RS + kt];
-          pq = fmaf(sm.dP[r * SS + i], kdi, pq);   // (dP K/G)[r]
-          pa = fmaf(sm.dA[r * SS + i], kdi, pa);   // (dA K/G)[r]
-          // (diag(beta) dA)^T (K G) + dP^T (Q G), row r
-          kd = fmaf(sm.beta[i] * sm.dA[i * SS + r], sm.KG[i * RS + kt], kd);
-          kd = fmaf(sm.dP[i * SS + r], sm.QG[i * RS + kt], kd);
-        }
-        const float b = sm.beta[r];
-        dqg[x] += pq;
-        dkg[x] = b * (pa - dkg[x]);
-        dkd[x] = kd;
-        dgam[x] = dqg[x] * sm.QG[r * RS + kt] + dkg[x] * sm.KG[r * RS + kt] -
-                  dkd[x] * sm.KD[r * RS + kt] - dkp[x] * sm.KP[r * RS + kt];
-      }
-      // last row: + G_last rowsum(S * dS') + sum_i dK'_i K'_i (the rows of both halves)
-      float kpsum = 0.f;
-#pragma unroll
-      for (int x = 0; x < 8; ++x) kpsum = fmaf(dkp[x], sm.KP[(rb + x) * RS + kt], kpsum);
-      kpsum += __shfl_xor_sync(0xffffffffu, kpsum, 1);
-      if (half == 1) dgam[7] += sm.gc[kt] * sds + kpsum;
-      // dg = reverse cumulative sum over the 16 rows (rows 8..15 live on the odd lane)
-      float suffix = 0.f;
-#pragma unroll
-      for (int x = 7; x >= 0; --x) {
-        suffix += dgam[x];
-        dgam[x] = suffix;
-      }
-      const float upper = __shfl_xor_sync(0xffffffffu, suffix, 1);
-      if (half == 0) {
-#pragma unroll
-        for (int x = 0; x < 8; ++x) dgam[x] += upper;
-      }
-      const float gck = sm.gc[kt];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int r = rb + x;
-        if (r0 + r < Lc) {
-          const float Gv = sm.G[r * RS + kt];
-          const size_t o = ((size_t)(t0 + r0 + r) * H + h) * 128 + kt;
-          dq[o] = dqg[x] * Gv;
-          dk[o] = dkg[x] * Gv + __fdividef(dkd[x] + dkp[x] * gck, Gv);
-          dg[o] = dgam[x];
-        }
-      }
-    }
-    __syncthreads();
+      __syncthreads();
 
-    // ---- dS <- diag(G_last) dS' + (Q G)^T dO' - (diag(beta) K G)^T dR  (thread (key, half)) --
-    {
-      const float gck = sm.gc[kt];
-      float *row = &sm.dS[kt * RS + 64 * half];
-#pragma unroll 2
-      for (int x = 0; x < 16; ++x) {
-        float4 s = *reinterpret_cast<float4 *>(row + 4 * x);
-        s.x *= gck; s.y *= gck; s.z *= gck; s.w *= gck;
+      // ---- dS <- diag(G_last) dS' + (Q G)^T dO' - (diag(beta) K G)^T dR  (keys kq, kq + 64) --
+      {
+        float st[2][32];
 #pragma unroll
-        for (int r = 0; r < kSub; ++r) {
-          const float a = sm.QG[r * RS + kt], b = -sm.beta[r] * sm.KG[r * RS + kt];
-          const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + 64 * half + 4 * x]);
-          const float4 d = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + 64 * half + 4 * x]);
-          s.x = fmaf(a, o.x, fmaf(b, d.x, s.x)); s.y = fmaf(a, o.y, fmaf(b, d.y, s.y));
-          s.z = fmaf(a, o.z, fmaf(b, d.z, s.z)); s.w = fmaf(a, o.w, fmaf(b, d.w, s.w));
+        for (int kk = 0; kk < 2; ++kk) {
+          const int key = kq + 64 * kk;
+          const float gck = sm.gc[key];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 x = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + 16 * m + 4 * q4]);
+            st[kk][4 * m] = gck * x.x; st[kk][4 * m + 1] = gck * x.y;
+            st[kk][4 * m + 2] = gck * x.z; st[kk][4 * m + 3] = gck * x.w;
+          }
         }
-        *reinterpret_cast<float4 *>(row + 4 * x) = s;
+#pragma unroll 2
+        for (int r = 0; r < kSub; ++r) {
+          const float nb = -sm.beta[r];
+          const float a0 = sm.QG[r * RS + kq], a1 = sm.QG[r * RS + kq + 64];
+          const float b0 = nb * sm.KG[r * RS + kq], b1 = nb * sm.KG[r * RS + kq + 64];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + 16 * m + 4 * q4]);
+            const float4 d = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + 16 * m + 4 * q4]);
+            st[0][4 * m] = fmaf(a0, o.x, fmaf(b0, d.x, st[0][4 * m]));
+            st[0][4 * m + 1] = fmaf(a0, o.y, fmaf(b0, d.y, st[0][4 * m + 1]));
+            st[0][4 * m + 2] = fmaf(a0, o.z, fmaf(b0, d.z, st[0][4 * m + 2]));
+            st[0][4 * m + 3] = fmaf(a0, o.w, fmaf(b0, d.w, st[0][4 * m + 3]));
+            st[1][4 * m] = fmaf(a1, o.x, fmaf(b1, d.x, st[1][4 * m]));
+            st[1][4 * m + 1] = fmaf(a1, o.y, fmaf(b1, d.y, st[1][4 * m + 1]));
+            st[1][4 * m + 2] = fmaf(a1, o.z, fmaf(b1, d.z, st[1][4 * m + 2]));
+            st[1][4 * m + 3] = fmaf(a1, o.w, fmaf(b1, d.w, st[1][4 * m + 3]));
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            *reinterpret_cast<float4 *>(&sm.dS[(kq + 64 * kk) * RS + 16 * m + 4 * q4]) =
+                make_float4(st[kk][4 * m], st[kk][4 * m + 1], st[kk][4 * m + 2], st[kk][4 * m + 3]);
       }
     }
-    __syncthreads();
+    __syncthreads();  // before the next item overwrites the shared matrices
   }
 }
 
@@ -744,34 +819,37 @@ template <typename Tin>
 cudaError_t launch_local_typed(const void *q, const void *k, const void *v, const float *g,
                                const float *beta, const float *dout, float scale,
                                const int32_t *cu, const void *ws, const float *ckpt,
-                               const float *dckpt, int N, int T, int H, float *dq, float *dk,
-                               float *dv, float *dg, float *dbeta, int *status, cudaStream_t s) {
-  const long long blocks = rec::chunk_capacity(N, T) * H;
-  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+                               const float *dckpt, float *scratch, int N, int T, int H,
+                               float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                               int *status, cudaStream_t s) {
+  const long long items = rec::chunk_capacity(N, T) * H;
+  const int blocks = (int)(items < kLocalCTAs ? items : kLocalCTAs);
   const int bytes = (int)sizeof(LocalSmem);
   cudaError_t e = cudaFuncSetAttribute(chunk_bwd_local_kernel<Tin>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  chunk_bwd_local_kernel<Tin><<<(unsigned)blocks, kLT, bytes, s>>>(
+  chunk_bwd_local_kernel<Tin><<<blocks, kLT, bytes, s>>>(
       static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), g,
-      beta, dout, scale, cu, static_cast<const uint8_t *>(ws), ckpt, dckpt, N, T, H, dq, dk, dv,
-      dg, dbeta, status);
+      beta, dout, scale, cu, static_cast<const uint8_t *>(ws), ckpt, dckpt, scratch, items, N, T,
+      H, dq, dk, dv, dg, dbeta, status);
   return cudaGetLastError();
 }
 }  // namespace
 
+size_t chunk_bwd_local_scratch_bytes() { return (size_t)kLocalCTAs * kLocalSlotFloats * 4; }
+
 cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *dout, float scale,
                                    const int32_t *cu, const void *ws, const float *ckpt,
-                                   const float *dckpt, int N, int T, int H, kda_dtype dt,
-                                   float *dq, float *dk, float *dv, float *dg, float *dbeta,
-                                   int *status, cudaStream_t s) {
+                                   const float *dckpt, float *scratch, int N, int T, int H,
+                                   kda_dtype dt, float *dq, float *dk, float *dv, float *dg,
+                                   float *dbeta, int *status, cudaStream_t s) {
   if (dt == KDA_BF16)
     return launch_local_typed<__nv_bfloat16>(q, k, v, g, beta, dout, scale, cu, ws, ckpt, dckpt,
-                                             N, T, H, dq, dk, dv, dg, dbeta, status, s);
+                                             scratch, N, T, H, dq, dk, dv, dg, dbeta, status, s);
   if (dt == KDA_F16)
-    return launch_local_typed<__half>(q, k, v, g, beta, dout, scale, cu, ws, ckpt, dckpt, N, T,
-                                      H, dq, dk, dv, dg, dbeta, status, s);
+    return launch_local_typed<__half>(q, k, v, g, beta, dout, scale, cu, ws, ckpt, dckpt,
+                                      scratch, N, T, H, dq, dk, dv, dg, dbeta, status, s);
   return cudaErrorInvalidValue;
 }
 

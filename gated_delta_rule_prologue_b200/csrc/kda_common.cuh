@@ -227,12 +227,14 @@ cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s
 cudaError_t launch_chunk_bwd_state(const void *ws, const int32_t *cu, const float *dsN,
                                    const float *dout, float scale, int N, int T, int H,
                                    float *dckpt, float *ds0, int *status, cudaStream_t s);
+// scratch: chunk_bwd_local_scratch_bytes() (one slot per CTA of the persistent grid).
+size_t chunk_bwd_local_scratch_bytes();
 cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *dout, float scale,
                                    const int32_t *cu, const void *ws, const float *ckpt,
-                                   const float *dckpt, int N, int T, int H, kda_dtype dt,
-                                   float *dq, float *dk, float *dv, float *dg, float *dbeta,
-                                   int *status, cudaStream_t s);
+                                   const float *dckpt, float *scratch, int N, int T, int H,
+                                   kda_dtype dt, float *dq, float *dk, float *dv, float *dg,
+                                   float *dbeta, int *status, cudaStream_t s);
 cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const void *cache_in,
                                        void *cache_out, const void *g, const float *beta,
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,
