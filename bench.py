@@ -50,6 +50,8 @@ CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta +
 FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
 GATED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 2 + 4 + D_ * 4  # bf16 q,k,v + bf16 g_raw + beta + o = 1540
 EPILOGUE_BYTES_PER_TH = D_ * 4 + 2 * D_ * 2             # o (f32) + gate, out (bf16) = 1024
+# backward: q, k, v (fp16) + g + beta + dL/do in; dq, dk, dv, dg (f32) + dbeta out = 3848
+BWD_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4 + 4 * D_ * 4 + 4
 CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 # decode per (sequence, head): state read+write, x, conv cache read+write, g, beta, o (f32)
 DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
@@ -63,6 +65,8 @@ KERNEL_SOURCES = {
     "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
     "kda_chunk_fwd_gated": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
     "kda_output_epilogue": [_CSRC + "kda_epilogue.cu"],
+    "kda_chunk_bwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu",
+                      _CSRC + "kda_chunk_bwd.cu"],
     "kda_decode_step": [_CSRC + "kda_decode.cu"],
 }
 
@@ -419,6 +423,24 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     epi_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in eev[1:])
     del o2, g_raw, gq, gk, gv, ep_out
+    # the prefill backward on the step's q/k/v (fp16), g, beta: dL/do ~ N(0,1) fp32
+    d_o = torch.randn((T, H, D), generator=gen).to(dev)
+    bwd_out = [torch.empty((T, H, D), device=dev) for _ in range(4)]
+    d_beta = torch.empty((T, H), device=dev)
+    bws = torch.empty(kda.kda_chunk_bwd_workspace_bytes(1, T, H, D, D, inp.chunk, q.dtype),
+                      dtype=torch.uint8, device=dev)
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    for i in range(3):
+        bev[i][0].record(stream)
+        kda.kda_chunk_bwd(q, k, v, g, beta, d_o, scale=inp.scale, dq=bwd_out[0], dk=bwd_out[1],
+                          dv=bwd_out[2], dg=bwd_out[3], dbeta=d_beta, want_d_initial_state=False,
+                          workspace=bws, stream=stream)
+        bev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
+    bwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in bev[1:])
+    del d_o, bwd_out, d_beta, bws
+    torch.cuda.empty_cache()
     seq4k = seq4k_side(kda, dev, stream, hbm)
 
     th = T * H
@@ -440,6 +462,8 @@ def run_ours(args, world, rank, local):
         "kda_output_epilogue": dict(ms=round(epi_ms, 4), **roofline(
             "hbm", EPILOGUE_BYTES_PER_TH * th, epi_ms, hbm, "GB/s",
             recorded_traffic("kda_output_epilogue"))),
+        "kda_chunk_bwd": dict(ms=round(bwd_ms, 4), launches=4, **roofline(
+            "hbm", BWD_BYTES_PER_TH * th, bwd_ms, hbm, "GB/s", recorded_traffic("kda_chunk_bwd"))),
         "kda_chunk_fwd_one_pass": dict(ms=round(one_pass_ms, 4), **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, one_pass_ms, hbm, "GB/s",
             recorded_traffic("kda_chunk_fwd_one_pass"))),
@@ -584,6 +608,10 @@ def run_ncu_case(args):
                 kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D)
             elif args.ncu_case == "prologue":
                 kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+            elif args.ncu_case == "bwd":
+                kda.kda_prologue(x, w, q, k, v, H=H, D=D)
+                d_o = torch.randn((T, H, D), generator=torch.Generator().manual_seed(3)).to(dev)
+                kda.kda_chunk_bwd(q, k, v, g, beta, d_o, want_d_initial_state=False)
             elif args.ncu_case == "chunk_one_pass":
                 kda.kda_prologue(x, w, q, k, v, H=H, D=D)
                 kda.kda_chunk_fwd(q, k, v, g, beta, o, workspace=None)
@@ -605,7 +633,7 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode",
-                                           "seq4k", "seq4k_whole"),
+                                           "seq4k", "seq4k_whole", "bwd"),
                     help="profiling mode: launch one kernel twice on a workload slice and exit")
     ap.add_argument("--ncu-tokens", type=int, default=4096)
     args = ap.parse_args()
