@@ -299,26 +299,33 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
       if (c + 1 < c_hi) fetch_u(c + 1);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    if (!wait_all(bar_kp, pk, status)) break;  // K', P of this chunk; also a CTA barrier
-    pk ^= 1;
+      // Only warps 0-1 wrote the U operand and read D1: they alone meet before the
+      // issuing thread (warp 0) starts the MMAs that read U and accumulate into D1.
+      fence_async_smem();
+      tc_fence_before();
+      asm volatile("bar.sync 1, 64;" ::: "memory");
 
-    // ---- D1 += [* ; P] U ;  D2 = K'^T U ----------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t a2 = smem_u32(sm + SB_A2), uop = smem_u32(sm + SB_U);
-      const uint32_t kp = smem_u32(sm + SB_KP);
-      constexpr uint32_t idO = idesc_fp16(128, 32, false, true);
-      constexpr uint32_t idS = idesc_fp16(128, 32, true, true);
+      // ---- D1 += [* ; P] U ;  D2 = K'^T U ------------------------------------------
+      if (tid == 0) {
+        if (mbar_wait(bar_kp, pk)) {  // K', P of this chunk
+          tc_fence_after();
+          const uint32_t a2 = smem_u32(sm + SB_A2), uop = smem_u32(sm + SB_U);
+          const uint32_t kp = smem_u32(sm + SB_KP);
+          constexpr uint32_t idO = idesc_fp16(128, 32, false, true);
+          constexpr uint32_t idS = idesc_fp16(128, 32, true, true);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {  // the two accumulators' steps interleaved
-        mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_mn32_sw64(uop, ks), idO, 1);
-        mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_mn32_sw64(uop, ks), idS, ks > 0);
+          for (int ks = 0; ks < 4; ++ks) {  // the two accumulators' steps interleaved
+            mma_bf16(tmem + TB_D1, desc_kmajor(a2, 128, ks), desc_mn32_sw64(uop, ks), idO, 1);
+            mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_mn32_sw64(uop, ks), idS,
+                     ks > 0);
+          }
+          mma_commit(bar_mma);
+        } else {
+          report(status, KDA_ERR_DEVICE_TIMEOUT);  // no commit: the wait below times out too
+        }
       }
-      mma_commit(bar_mma);
     }
+    pk ^= 1;
     if (!wait_all(bar_mma, pm, status)) break;
     pm ^= 1;
     tc_fence_after();
@@ -357,7 +364,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     write_s_operand();
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    // the next chunk's wait on its [W; Q G] tile is the barrier before MMA1 reads S
   }
 
   if (s_out) {
