@@ -55,7 +55,7 @@ constexpr uint32_t SB_S = 57344;         // S slice operand (value-contiguous, 1
                                          // 64-byte swizzle) 8 KB; between the two MMA groups:
                                          // <q_r, k_r> U exchange [32][64] f32
 constexpr uint32_t SB_U = 65536;         // U operand (value-contiguous, 64 token rows x 64 B) 4 KB
-constexpr uint32_t SB_BAR = 69632;       // three mbarriers, TMEM slot
+constexpr uint32_t SB_BAR = 69632;       // four mbarriers, TMEM slot
 constexpr uint32_t SB_ALLOC = SB_BAR + 64 + 1024;
 // D1 is accumulated as two halves over the key channels (two independent MMA
 // chains), summed at read-out; D2 = K'^T U.
@@ -115,7 +115,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   float *segbuf = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) +
                                             rec::segment_area_offset(N, T, H));
   uint64_t *bar_a1 = reinterpret_cast<uint64_t *>(sm + SB_BAR);
-  uint64_t *bar_kp = bar_a1 + 1, *bar_mma = bar_a1 + 2;
+  uint64_t *bar_kp = bar_a1 + 1, *bar_mma = bar_a1 + 2, *bar_m2 = bar_a1 + 3;
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SB_BAR + 32);
   float *exch = reinterpret_cast<float *>(sm + SB_S);
 
@@ -170,6 +170,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     mbar_init(bar_a1, 1);
     mbar_init(bar_kp, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_m2, 1);
     fence_mbar_init();
   }
   // S[i] = S[key tid][value 32 slice + i]; the state is stored value-major [dv][dk].
@@ -247,7 +248,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     fetch_gl(c_lo);
   }
 
-  uint32_t pa = 0, pk = 0, pm = 0;
+  uint32_t pa = 0, pk = 0, pm = 0, pm2 = 0;
   for (int c = c_lo; c < c_hi; ++c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
     if (ckpt) {  // entry state of the chunk, for the backward pass
@@ -271,10 +272,17 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       }
       mma_commit(bar_mma);
     }
-    if (!wait_all(bar_mma, pm, status)) break;
+    // Only warps 0-1 read this group's result (W S, TMEM lanes 0..63); warps 2-3 go on
+    // to the second group's wait.  A failed wait stops the issuing thread from starting
+    // the second group, so every thread's wait on it then fails and the loop ends.
+    bool ok1 = true;
+    if (warp < 2) {
+      ok1 = mbar_wait(bar_mma, pm);
+      if (!ok1) report(status, KDA_ERR_DEVICE_TIMEOUT);
+      tc_fence_after();
+      if (tid == 0 && ok1 && c + 1 < c_hi) load_a1(c + 1);  // A1 has been read
+    }
     pm ^= 1;
-    tc_fence_after();
-    if (tid == 0 && c + 1 < c_hi) load_a1(c + 1);  // A1 has been read
 
     // ---- U = Ut - W S (warps 0-1: TMEM lanes 0..63 are the chunk's tokens) -------------
     if (warp < 2) {
@@ -307,7 +315,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 
       // ---- D1 += [* ; P] U ;  D2 = K'^T U ------------------------------------------
       if (tid == 0) {
-        if (mbar_wait(bar_kp, pk)) {  // K', P of this chunk
+        if (ok1 && mbar_wait(bar_kp, pk)) {  // K', P of this chunk
           tc_fence_after();
           const uint32_t a2 = smem_u32(sm + SB_A2), uop = smem_u32(sm + SB_U);
           const uint32_t kp = smem_u32(sm + SB_KP);
@@ -319,15 +327,15 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
             mma_bf16(tmem + TB_D2, desc_mnmajor(kp, 64, ks), desc_mn32_sw64(uop, ks), idS,
                      ks > 0);
           }
-          mma_commit(bar_mma);
+          mma_commit(bar_m2);
         } else {
           report(status, KDA_ERR_DEVICE_TIMEOUT);  // no commit: the wait below times out too
         }
       }
     }
     pk ^= 1;
-    if (!wait_all(bar_mma, pm, status)) break;
-    pm ^= 1;
+    if (!wait_all(bar_m2, pm2, status)) break;
+    pm2 ^= 1;
     tc_fence_after();
     if (tid == 0 && c + 1 < c_hi) load_kp(c + 1);  // K' and P have been read
 
