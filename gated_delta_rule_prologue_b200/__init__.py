@@ -96,6 +96,11 @@ lib.kda_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_chunk_bwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                  _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
                                  _vp]
+lib.kda_chunk_map_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+lib.kda_chunk_map_workspace_bytes.restype = ctypes.c_size_t
+lib.kda_chunk_map_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                 _vp, ctypes.c_size_t, _vp]
+lib.kda_state_compose.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]
 lib.kda_chunk_fwd_segment_chunks.argtypes = [_i, _i, _i]
 lib.kda_chunk_fwd_segment_chunks.restype = ctypes.c_int
 lib.kda_chunk_fwd_segmented_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
@@ -105,7 +110,8 @@ lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _v
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
-            lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws,
+            lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
+            lib.kda_state_compose,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_output_epilogue,
@@ -314,6 +320,46 @@ def kda_chunk_bwd(q, k, v, g, beta, d_o, *, scale: float = 1.0, initial_state=No
                                 _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(d_initial_state),
                                 _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv, dg, dbeta, d_initial_state
+
+
+def kda_chunk_map(q, k, v, g, beta, *, cu_seqlens=None, chunk: int = 64, M=None, B=None,
+                  workspace="auto", stream=None):
+    """Affine map of each sequence's prefill, final = M S0 + B: returns ``(M, B)``,
+    both [N, H, D, D] fp32 stored like a state (column-major)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((g, "g"), (beta, "beta")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    M = torch.empty((N, H, Dk, Dk), device=q.device) if M is None else M
+    B = torch.empty((N, H, Dv, Dk), device=q.device) if B is None else B
+    _need(M, "M", torch.float32)
+    _need(B, "B", torch.float32)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+        nbytes = int(lib.kda_chunk_map_workspace_bytes(N, T, H, Dk, Dv, chunk, _DTYPES[q.dtype]))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_chunk_map_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N,
+                                T, H, Dk, Dv, chunk, _dtype(q), _ptr(M), _ptr(B), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
+    return M, B
+
+
+def kda_state_compose(M, B, E_in, E_out=None, stream=None):
+    """E_out = M E_in + B per (sequence, head) (E_in None: zero); returns E_out."""
+    for t, n in ((M, "M"), (B, "B"), (E_in, "E_in")):
+        _need(t, n, torch.float32)
+    N, H, D = B.shape[0], B.shape[1], B.shape[2]
+    E_out = torch.empty_like(B) if E_out is None else E_out
+    _need(E_out, "E_out", torch.float32)
+    _check(lib.kda_state_compose(_ptr(M), _ptr(B), _ptr(E_in), _ptr(E_out), N, H, D,
+                                 _stream(stream)))
+    return E_out
 
 
 # Size of the library's fixed scratch buffer (one per device) used by

@@ -785,3 +785,84 @@ kda_status kda_chunk_bwd_ws(const void *q, const void *k, const void *v, const f
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Affine chunk maps across ranks (sequence split)
+// ---------------------------------------------------------------------------
+
+extern "C" {
+
+size_t kda_chunk_map_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt) {
+  return kda_chunk_fwd_segmented_workspace_bytes(N, T, H, Dk, Dv, chunk, dt, 0);
+}
+
+kda_status kda_chunk_map_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const int32_t *cu_seqlens, int N, int T, int H,
+                            int Dk, int Dv, int chunk, kda_dtype dt, float *M, float *B,
+                            void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+  KDA_REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  KDA_REQUIRE(N >= 1 && T >= 0 && H >= 1, "bad sizes N=%d T=%d H=%d", N, T, H);
+  KDA_REQUIRE(cu_seqlens != nullptr || N == 1, "cu_seqlens is NULL but N=%d", N);
+  if (!chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_map: needs bf16/f16, Dk == Dv == 128, chunk 64 and "
+                                     "T > 0 (got dt=%d Dk=%d Dv=%d chunk=%d T=%d)",
+                (int)dt, Dk, Dv, chunk, T);
+  KDA_REQUIRE_PTR(q, "q");
+  KDA_REQUIRE_PTR(k, "k");
+  KDA_REQUIRE_PTR(v, "v");
+  KDA_REQUIRE_PTR(g, "g");
+  KDA_REQUIRE_PTR4(beta, "beta");
+  KDA_REQUIRE_PTR(M, "M");
+  KDA_REQUIRE_PTR(B, "B");
+  KDA_OPT_PTR4(cu_seqlens, "cu_seqlens");
+  KDA_REQUIRE(workspace != nullptr, "chunk_map: workspace is NULL");
+  KDA_OPT_PTR(workspace, "workspace");
+  const size_t need = kda_chunk_map_workspace_bytes(N, T, H, Dk, Dv, chunk, dt);
+  KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
+              workspace_bytes, need);
+  {
+    const size_t es = esize(dt), act = (size_t)T * H * 128 * es, sbytes = (size_t)N * H * 128 * 128 * 4;
+    const void *ins[7] = {q, k, v, g, beta, cu_seqlens, workspace};
+    const size_t isz[7] = {act, act, act, (size_t)T * H * 128 * 4, (size_t)T * H * 4,
+                           (size_t)(N + 1) * 4, need};
+    for (int i = 0; i < 7; ++i) {
+      KDA_REQUIRE(!overlaps(M, sbytes, ins[i], isz[i]), "M overlaps an input or the workspace");
+      KDA_REQUIRE(!overlaps(B, sbytes, ins[i], isz[i]), "B overlaps an input or the workspace");
+    }
+    KDA_REQUIRE(!overlaps(M, sbytes, B, sbytes), "M overlaps B");
+    for (int i = 0; i < 6; ++i)
+      KDA_REQUIRE(!overlaps(workspace, need, ins[i], isz[i]), "workspace overlaps an input");
+  }
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (cu_seqlens) e = kda::launch_chunk_index(cu_seqlens, N, T, 0, workspace, status, s);
+  if (e == cudaSuccess)
+    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, nullptr,
+                               nullptr, 0.f, false, status, s);
+  if (e == cudaSuccess) e = kda::launch_chunk_map(workspace, cu_seqlens, N, T, H, M, B, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_map_ws launch");
+  return KDA_OK;
+}
+
+kda_status kda_state_compose(const float *M, const float *B, const float *E_in, float *E_out,
+                             int N, int H, int D, kda_stream_t stream) {
+  KDA_REQUIRE(N >= 1 && H >= 1, "bad sizes N=%d H=%d", N, H);
+  if (D != 128) return fail(KDA_ERR_UNSUPPORTED, "state_compose: D=%d (needs 128)", D);
+  KDA_REQUIRE_PTR(M, "M");
+  KDA_REQUIRE_PTR(B, "B");
+  KDA_REQUIRE_PTR(E_out, "E_out");
+  KDA_OPT_PTR(E_in, "E_in");
+  const size_t sbytes = (size_t)N * H * D * D * 4;
+  KDA_REQUIRE(!overlaps(E_out, sbytes, M, sbytes) && !overlaps(E_out, sbytes, B, sbytes) &&
+                  !overlaps(E_out, sbytes, E_in, sbytes),
+              "E_out overlaps an input");
+  cudaError_t e = kda::launch_state_compose(M, B, E_in, E_out, N * H, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_state_compose launch");
+  return KDA_OK;
+}
+
+}  // extern "C"

@@ -62,7 +62,7 @@ constexpr uint32_t SB_ALLOC = SB_BAR + 64 + 1024;
 constexpr uint32_t TB_D1 = 0, TB_D1B = 32, TB_D2 = 64, TB_COLS = 128;
 static_assert(SB_KP + 24576 == SB_S, "K' and P are adjacent");
 
-enum { kOutputs = 0, kTransition = 1 };
+enum { kOutputs = 0, kTransition = 1, kMap = 2 };
 
 // Segment s (or sequence s when L == 0) of the batch: its sequence n, its
 // index g among the G segments of n, and its chunk range [c_lo, c_hi) within n.
@@ -100,12 +100,12 @@ template <int kRole>
 __global__ void __launch_bounds__(kBT, 3)
 chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
                    const float *s0, float scale, int N, int T, int H, int L, float *__restrict__ o,
-                   float *sN, float *ckpt, int *status) {
+                   float *sN, float *ckpt, float *map_m, float *map_b, int *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr int kParts = kRole == kTransition ? 2 : 1;
+  constexpr int kParts = kRole == kOutputs ? 1 : 2;
   const int sub = blockIdx.x % (kSlices * kParts);
   const int slice = sub & 3, part = sub >> 2;  // part (transition pass): 0 = M, 1 = B
   const int item = blockIdx.x / (kSlices * kParts), h = item % H, s = item / H;
@@ -143,7 +143,15 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   const float *s_in = nullptr;
   float *s_out = nullptr, *s_copy = nullptr;
   bool identity = false, use_ut = true;
-  if (kRole == kTransition) {
+  if (kRole == kMap) {  // every sequence is one segment: its whole map, M and B
+    if (part == 0) {
+      identity = true;
+      use_ut = false;
+      s_out = map_m + head_off;
+    } else {
+      s_out = map_b + head_off;
+    }
+  } else if (kRole == kTransition) {
     if (sg.g == sg.G - 1) return;           // the last segment needs no map
     if (sg.g == 0 && part == 0) return;     // the first runs from the initial state
     if (part == 0) {
@@ -626,18 +634,65 @@ namespace {
 template <int kRole>
 cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0, float scale,
                               int N, int T, int H, int L, float *o, float *sN, float *ckpt,
-                              int *status, cudaStream_t s) {
+                              int *status, cudaStream_t s, float *map_m = nullptr,
+                              float *map_b = nullptr) {
   const long long items = L > 0 ? rec::segment_capacity(N, T, L) : N;
-  const long long blocks = items * H * kSlices * (kRole == kTransition ? 2 : 1);
+  const long long blocks = items * H * kSlices * (kRole == kOutputs ? 1 : 2);
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<kRole>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB_ALLOC);
   if (e != cudaSuccess) return e;
   chunk_state_kernel<kRole><<<(unsigned)blocks, kBT, SB_ALLOC, s>>>(
-      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, ckpt, status);
+      static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, ckpt, map_m, map_b,
+      status);
   return cudaGetLastError();
 }
 }  // namespace
+
+cudaError_t launch_chunk_map(const void *ws, const int32_t *cu, int N, int T, int H, float *map_m,
+                             float *map_b, int *status, cudaStream_t s) {
+  return launch_state_role<kMap>(ws, cu, nullptr, 1.f, N, T, H, 0, nullptr, nullptr, nullptr,
+                                 status, s, map_m, map_b);
+}
+
+namespace {
+// E_out = M E_in + B per (sequence, head), fp32: one CTA per (sequence, head, 8 value
+// columns), thread r owns row r (key channel); E_in's 8 columns sit in shared memory
+// and row r of M is read column by column (consecutive threads, consecutive words).
+__global__ void __launch_bounds__(128)
+state_compose_kernel(const float *__restrict__ M, const float *__restrict__ B,
+                     const float *__restrict__ E_in, float *__restrict__ E_out, int NH) {
+  __shared__ float Es[128][kScanCols];
+  const int r = threadIdx.x;
+  const int cb = blockIdx.x % (128 / kScanCols), nh = blockIdx.x / (128 / kScanCols);
+  const size_t off = (size_t)nh * 128 * 128;
+  const int j0 = cb * kScanCols;
+#pragma unroll
+  for (int j = 0; j < kScanCols; ++j) Es[r][j] = E_in ? E_in[off + (size_t)(j0 + j) * 128 + r] : 0.f;
+  __syncthreads();
+  float acc[kScanCols];
+#pragma unroll
+  for (int j = 0; j < kScanCols; ++j) acc[j] = B[off + (size_t)(j0 + j) * 128 + r];
+  if (E_in) {
+#pragma unroll 8
+    for (int k = 0; k < 128; ++k) {
+      const float m = M[off + (size_t)k * 128 + r];  // M[r][k]
+#pragma unroll
+      for (int j = 0; j < kScanCols; ++j) acc[j] = fmaf(m, Es[k][j], acc[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kScanCols; ++j) E_out[off + (size_t)(j0 + j) * 128 + r] = acc[j];
+}
+}  // namespace
+
+cudaError_t launch_state_compose(const float *M, const float *B, const float *E_in, float *E_out,
+                                 int NH, cudaStream_t s) {
+  const long long blocks = (long long)NH * (128 / kScanCols);
+  if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
+  state_compose_kernel<<<(unsigned)blocks, 128, 0, s>>>(M, B, E_in, E_out, NH);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,

@@ -221,6 +221,14 @@ cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws,
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,
                                cudaStream_t s, float *ckpt = nullptr);
+// Affine map of every sequence (one segment each; records from the prep pass):
+// map_m [N][H][Dk][Dk] with M[t][k] at k * Dk + t, map_b [N][H][Dv][Dk] like a state.
+cudaError_t launch_chunk_map(const void *ws, const int32_t *cu, int N, int T, int H, float *map_m,
+                             float *map_b, int *status, cudaStream_t s);
+// E_out = M E_in + B for NH (sequence, head) pairs (E_in NULL: zero); E_out must not
+// overlap the inputs.
+cudaError_t launch_state_compose(const float *M, const float *B, const float *E_in, float *E_out,
+                                 int NH, cudaStream_t s);
 // Backward of the two-pass prefill (kda_chunk_bwd.cu): the reverse state pass over
 // (sequence, head, value slice) writing the adjoint of every chunk's exit state
 // (dckpt, record order) and d_s0, then the local pass over (chunk, head).

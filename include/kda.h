@@ -259,6 +259,49 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
                                 kda_stream_t stream);
 
 /*
+ * Affine chunk maps, for splitting one sequence across ranks.  [W4 Figure 1,
+ * Figure 3]: the prefill maps its entry state affinely, final = M S0 + B, with
+ * M (d_k x d_k) depending on k, g, beta only and B the final state from a
+ * zero start.  A sequence cut into stretches held by different ranks is
+ * evaluated by computing every stretch's (M, B) where it lives, exchanging
+ * them, composing each stretch's entry state E_{r+1} = M_r E_r + B_r from the
+ * ones before it, and running kda_chunk_fwd on each stretch from its entry
+ * state (the Python package's kda_chunk_fwd_sequence_parallel does this over
+ * torch.distributed).  No counterpart in code on the pages.
+ *
+ * kda_chunk_map_workspace_bytes -- scratch of kda_chunk_map_ws (the two-pass
+ * records and chunk index); 0 off the tensor-core shapes.
+ */
+size_t kda_chunk_map_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt);
+
+/*
+ * kda_chunk_map_ws -- the affine map of each of the N sequences (cu_seqlens as
+ * in kda_chunk_fwd; tensor-core shapes only, else KDA_ERR_UNSUPPORTED):
+ *   M  [N, H, Dk, Dk] f32 output, 16-byte aligned; element (row t, column k) of
+ *      the map at M[n][h][k][t] (stored like a state, column-major)
+ *   B  [N, H, Dv, Dk] f32 output: the final state from a zero initial state
+ *   workspace >= kda_chunk_map_workspace_bytes(...) bytes, caller-owned
+ * Outputs must not overlap the inputs, each other or the workspace.  M is
+ * computed by the tensor-core state pass from the identity with the value
+ * term removed (one CTA per 32 of its columns), B from a zero state; the
+ * rounding is that of kda_chunk_fwd_ws.
+ */
+kda_status kda_chunk_map_ws(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const int32_t *cu_seqlens, int N, int T, int H,
+                            int Dk, int Dv, int chunk, kda_dtype dt, float *M, float *B,
+                            void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_state_compose -- E_out = M E_in + B for N sequences x H heads, in fp32
+ * (layouts as in kda_chunk_map_ws; E_in and E_out like a state [N, H, D, D]).
+ * E_in NULL means zero (E_out = B).  D must be 128.  E_out must not overlap
+ * M, B or E_in.
+ */
+kda_status kda_state_compose(const float *M, const float *B, const float *E_in, float *E_out,
+                             int N, int H, int D, kda_stream_t stream);
+
+/*
  * Backward of the chunkwise prefill.  The pages mention training ([W1 彩蛋])
  * but print no backward; these are the gradients of the loss
  *     L = sum(d_o * o) + sum(d_final_state * final_state)

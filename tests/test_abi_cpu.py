@@ -289,3 +289,31 @@ def test_output_epilogue_rejects_bad_arguments(kda):
     assert st == kda.KDA_ERR_INVALID_ARG and b"weight" in L.kda_last_error()
     st = L.kda_output_epilogue(o, g, w, 1e-5, 10, 2, 128, 1, _vp(0x100010), None)
     assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
+
+
+def test_chunk_map_and_compose_reject_bad_arguments(kda):
+    import torch
+    L = kda.lib
+    T, H = 200, 2
+    need = L.kda_chunk_map_workspace_bytes(1, T, H, 128, 128, 64, 1)
+    assert need == kda.kda_chunk_fwd_segmented_workspace_bytes(1, T, H, 128, 128, 64,
+                                                                torch.bfloat16, 0)
+    assert L.kda_chunk_map_workspace_bytes(1, T, H, 128, 128, 64, 0) == 0
+    q, k, v = _vp(0x100000), _vp(0x200000), _vp(0x300000)
+    g, beta = _vp(0x400000), _vp(0x800000)
+    M, B, ws = _vp(0x1000000), _vp(0x1100000), _vp(0x2000000)
+    args = (q, k, v, g, beta, None, 1, T, H, 128, 128, 64)
+    st = L.kda_chunk_map_ws(*args, 0, M, B, ws, need, None)           # f32: no tensor cores
+    assert st == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_chunk_map_ws(*args, 1, None, B, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"M is NULL" in L.kda_last_error()
+    st = L.kda_chunk_map_ws(*args, 1, M, M, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
+    st = L.kda_chunk_map_ws(*args, 1, M, B, ws, need - 16, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace holds" in L.kda_last_error()
+    E = _vp(0x1200000)
+    assert L.kda_state_compose(M, B, E, _vp(0x1300000), 1, 2, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    st = L.kda_state_compose(M, B, E, E, 1, 2, 128, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"E_out overlaps" in L.kda_last_error()
+    st = L.kda_state_compose(M, None, E, _vp(0x1300000), 1, 2, 128, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"B is NULL" in L.kda_last_error()
