@@ -477,23 +477,48 @@ def run_ours(args, world, rank, local):
     fused_floor_ms = 1e3 * FUSED_BYTES_PER_TH * th / (hbm * 1e9)
 
     # ---- end to end through the C ABI with host buffers ----
-    out_host = torch.empty((T, H, D), dtype=torch.float32, pin_memory=True)
-    e2e_steps = max(1, args.e2e_steps)
+    # Every step copies its inputs in from pinned host memory and its read-out back.
+    # Three streams with double-buffered inputs and outputs: step i+1's inputs
+    # travel host -> device while step i computes and its read-out travels
+    # device -> host (the two directions of the host link run at the same time).
+    e2e_steps = max(2, args.e2e_steps)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    xs, gs, bs = [x, torch.empty_like(x)], [g, torch.empty_like(g)], [beta, torch.empty_like(beta)]
+    outs = [o, torch.empty_like(o)]
+    out_host = [torch.empty((T, H, D), dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(inp.x, non_blocking=True)
-        g.copy_(inp.g, non_blocking=True)
-        beta.copy_(inp.beta, non_blocking=True)
-        step()
-        out_host.copy_(o, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        b = i % 2
+        if i >= 2:
+            s_in.wait_event(comp_done[b])   # step i-2 has read slot b
+        with torch.cuda.stream(s_in):
+            xs[b].copy_(inp.x, non_blocking=True)
+            gs[b].copy_(inp.g, non_blocking=True)
+            bs[b].copy_(inp.beta, non_blocking=True)
+        in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])  # step i-2's read-out has left slot b
+        kda.kda_prologue(xs[b], w, q, k, v, H=H, D=D, stream=stream)
+        kda.kda_chunk_fwd(q, k, v, gs[b], bs[b], outs[b], scale=inp.scale, final_state=fs,
+                          chunk=inp.chunk, workspace=ws, stream=stream)
+        comp_done[b].record(stream)
+        s_out.wait_event(comp_done[b])
+        with torch.cuda.stream(s_out):
+            out_host[b].copy_(outs[b], non_blocking=True)
+        out_done[b].record(s_out)
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
     e2e_value, e2e_ms = job_throughput(world, T, e0.elapsed_time(e1) / e2e_steps)
     h2d = inp.x.numel() * 2 + inp.g.numel() * 4 + inp.beta.numel() * 4
-    d2h = out_host.numel() * 4
-    del x, o, g, beta, inp, ws
+    d2h = out_host[0].numel() * 4
+    del x, o, g, beta, inp, ws, xs, gs, bs, outs, out_host
     torch.cuda.empty_cache()
 
     # ---- batched decode: 256 sequences x 96 heads, consecutive steps ----
@@ -559,7 +584,10 @@ def run_ours(args, world, rank, local):
         "seq4k": seq4k,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipeline": "three streams, inputs and outputs double-buffered: step i+1's "
+                            "inputs are copied in while step i computes and its o is "
+                            "copied out"},
         "gpu_launches": launches_total,
         "clocks": clk,
     }
@@ -629,7 +657,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode",
