@@ -245,6 +245,26 @@ def cpu_baseline(n_tokens=1024):
                       f"(prologue + token-by-token recurrence, float64 NumPy), {wall:.1f} s"}
 
 
+# Bytes of one record of the two-pass prefill and the workspace of one K3 call (the
+# library's layout: a 1 KiB index header, then (ceil(T/64) + 1) * H records).
+RECORD_BYTES = 90880
+
+
+def k3_config(world, T=32768, H=96, D=128):
+    """The benchmark's workload description, shared by both arms."""
+    th = T * H
+    ws_bytes = 1024 + ((T + 63) // 64 + 1) * H * RECORD_BYTES
+    step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws_bytes) / 1e9
+    return {
+        "workload": "k3_prefill: kda_prologue (fp16 q/k/v out) + kda_chunk_fwd (two-pass, "
+                    "preallocated workspace) over T=32768 tokens, H=96, d_k=d_v=128, "
+                    "chunk 64, bf16 q/k/v projections, fp32 g/beta/state/o",
+        "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
+        "parallelism": f"replicas x{world} (independent problems, no collective)",
+        "l2": f"inputs larger than L2 ({step_gb:.1f} GB touched per step, no flush needed)",
+    }
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -264,11 +284,11 @@ def run_reference(args, world, rank):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "k3_prefill sample: first %d tokens x 96 heads x d=128 "
-                               "(prologue + recurrence)" % n_tok},
+        "config": k3_config(world),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": f"first {n_tok} tokens of the K3-layer prefill per step"},
+                         "sample": f"first {n_tok} tokens x 96 heads of the K3-layer prefill "
+                                   "per step (prologue + recurrence, float64)"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -444,7 +464,8 @@ def run_ours(args, world, rank, local):
     seq4k = seq4k_side(kda, dev, stream, hbm)
 
     th = T * H
-    step_gb = (PROLOGUE_BYTES_PER_TH * th + CHUNK_BYTES_PER_TH * th + 2 * ws.numel()) / 1e9
+    # the shared workload description assumes the library's record layout
+    assert ws.numel() == 1024 + ((T + 63) // 64 + 1) * H * RECORD_BYTES
     kernels = {
         "kda_prologue_chunk_fwd": dict(ms=round(fused_ms, 4), launches=2, **roofline(
             "hbm", FUSED_BYTES_PER_TH * th, fused_ms, hbm, "GB/s",
@@ -569,14 +590,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": "k3_prefill: kda_prologue (fp16 q/k/v out) + kda_chunk_fwd (two-pass, "
-                        "preallocated workspace) over T=32768 tokens, H=96, d_k=d_v=128, "
-                        "chunk 64, bf16 q/k/v projections, fp32 g/beta/state/o",
-            "global_batch": world, "seq_len": T, "heads": H, "head_dim": D,
-            "parallelism": f"replicas x{world} (independent problems, no collective)",
-            "l2": f"inputs larger than L2 ({step_gb:.1f} GB touched per step, no flush needed)",
-        },
+        "config": k3_config(world, T, H, D),
         "roofline": roof,
         "kernels": kernels,
         "fused_hbm_floor_ms": round(fused_floor_ms, 4),
