@@ -14,8 +14,11 @@
 //     e_j = v_j - p_j
 //     S^T[j,:] = s' + beta e_j k
 //     o_j = scale * <S^T[j,:], q> = scale * (r_j + beta e_j <k, q>)
-// so both reductions are independent and <k, q> is computed once per head.
+// so both reductions are independent and <k, q> is one reduction per head, not per row.
 // HBM traffic is dominated by the state: 2 * 4 * D^2 bytes per (seq, head).
+// The block meets once, after the prologue: each warp then reduces the norms
+// of q and k itself and writes the read-out of its own rows, so no warp waits
+// for another while the state streams through.
 #include "kda_common.cuh"
 
 namespace kda {
@@ -43,8 +46,6 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
   using Sh = DecodeShape<D>;
   constexpr int LPR = Sh::kLanesPerRow;
   __shared__ float qkv[3 * D];
-  __shared__ float red[4];
-  __shared__ float o_s[D];
 
   const int nh = blockIdx.x;
   const int n = nh / H, h = nh % H;
@@ -95,29 +96,23 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
     cr[2 * C] = xin;
   }
   __syncthreads();
-  if (warp == 0) {
-    float sq = 0.f, sk = 0.f, skq = 0.f;
-    for (int d = lane; d < D; d += 32) {
-      const float qq = qkv[d], kk = qkv[D + d];
-      sq = fmaf(qq, qq, sq);
-      sk = fmaf(kk, kk, sk);
-      skq = fmaf(kk, qq, skq);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      sk += __shfl_xor_sync(0xffffffffu, sk, off);
-      skq += __shfl_xor_sync(0xffffffffu, skq, off);
-    }
-    if (lane == 0) {
-      const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
-      red[0] = rq;
-      red[1] = rk;
-      red[2] = skq * rq * rk;  // <k, q> of the normalised vectors
-    }
+  // Every warp reduces |q|^2, |k|^2 and <k, q> itself (the same operations in the
+  // same order, so the same values): no second block barrier.
+  float sq = 0.f, sk = 0.f, skq = 0.f;
+  for (int d = lane; d < D; d += 32) {
+    const float qq = qkv[d], kk = qkv[D + d];
+    sq = fmaf(qq, qq, sq);
+    sk = fmaf(kk, kk, sk);
+    skq = fmaf(kk, qq, skq);
   }
-  __syncthreads();
-  const float rq = red[0], rk = red[1], kq = red[2];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+    skq += __shfl_xor_sync(0xffffffffu, skq, off);
+  }
+  const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
+  const float kq = skq * rq * rk;  // <k, q> of the normalised vectors
   const float4 q4 = make_float4(qkv[dk0] * rq, qkv[dk0 + 1] * rq, qkv[dk0 + 2] * rq,
                                 qkv[dk0 + 3] * rq);
   const float4 k4 = make_float4(qkv[D + dk0] * rk, qkv[D + dk0 + 1] * rk,
@@ -148,10 +143,8 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
     sp.z = fmaf(be, k4.z, sp.z);
     sp.w = fmaf(be, k4.w, sp.w);
     __stcs(reinterpret_cast<float4 *>(base + (size_t)j * D + dk0), sp);
-    if (sub == 0) o_s[j] = scale * fmaf(be, kq, pq);
+    if (sub == 0) o[(size_t)nh * D + j] = scale * fmaf(be, kq, pq);
   }
-  __syncthreads();
-  for (int j = tid; j < D; j += Sh::kThreads) o[(size_t)nh * D + j] = o_s[j];
 }
 
 // Gate of the gated step (null A_log / dt_bias: neutral; unused when not gated).
