@@ -37,7 +37,7 @@ struct DecodeShape {
 // kGated: g holds gate pre-activations of type Tin and the log-decay is
 // lower_bound * sigmoid(exp(A_log[h]) * (g + dt_bias[h, :])) (pointers may be null).
 template <typename Tin, int D, bool kGated>
-__global__ void __launch_bounds__(DecodeShape<D>::kThreads)
+__global__ void __launch_bounds__(DecodeShape<D>::kThreads, 2)  // two CTAs per SM: at most 128 registers
 decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__restrict__ cache,
               const void *__restrict__ g, const float *__restrict__ beta, float scale,
               float *__restrict__ state, int N, int H, float *__restrict__ o,
@@ -78,22 +78,40 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
   const float b = __ldg(beta + nh);
 
   // 2. Prologue for this head's 3*D channels; the conv cache is shifted in place.
+  //    A thread's channels (two at most) have all their loads issued before any
+  //    is used, so the barrier waits for one round trip, not two.
   const int C = 3 * H * D;
-  for (int i = tid; i < 3 * D; i += Sh::kThreads) {
-    const int pidx = i / D, d = i % D;
-    const int c = pidx * H * D + h * D + d;
-    Tin *cr = cache + (size_t)n * 3 * C + c;
-    const float c0 = to_f32(cr[0]), c1 = to_f32(cr[C]), c2 = to_f32(cr[2 * C]);
-    const Tin xin = x[(size_t)n * C + c];
-    const float4 wc = __ldg(reinterpret_cast<const float4 *>(w + (size_t)c * 4));
-    float a = wc.x * c0;
-    a = fmaf(wc.y, c1, a);
-    a = fmaf(wc.z, c2, a);
-    a = fmaf(wc.w, to_f32(xin), a);
-    qkv[i] = silu(a);
-    cr[0] = cr[C];
-    cr[C] = cr[2 * C];
-    cr[2 * C] = xin;
+  constexpr int kCh = (3 * D + Sh::kThreads - 1) / Sh::kThreads;
+  Tin r0[kCh], r1[kCh], r2[kCh], xin[kCh];
+  float4 wc[kCh];
+#pragma unroll
+  for (int m = 0; m < kCh; ++m) {
+    const int i = tid + m * Sh::kThreads;
+    if (i < 3 * D) {
+      const int c = (i / D) * H * D + h * D + i % D;
+      const Tin *cr = cache + (size_t)n * 3 * C + c;
+      r0[m] = cr[0];
+      r1[m] = cr[C];
+      r2[m] = cr[2 * C];
+      xin[m] = x[(size_t)n * C + c];
+      wc[m] = __ldg(reinterpret_cast<const float4 *>(w + (size_t)c * 4));
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kCh; ++m) {
+    const int i = tid + m * Sh::kThreads;
+    if (i < 3 * D) {
+      const int c = (i / D) * H * D + h * D + i % D;
+      float a = wc[m].x * to_f32(r0[m]);
+      a = fmaf(wc[m].y, to_f32(r1[m]), a);
+      a = fmaf(wc[m].z, to_f32(r2[m]), a);
+      a = fmaf(wc[m].w, to_f32(xin[m]), a);
+      qkv[i] = silu(a);
+      Tin *cr = cache + (size_t)n * 3 * C + c;
+      cr[0] = r1[m];
+      cr[C] = r2[m];
+      cr[2 * C] = xin[m];
+    }
   }
   __syncthreads();
   // Every warp reduces |q|^2, |k|^2 and <k, q> itself (the same operations in the
