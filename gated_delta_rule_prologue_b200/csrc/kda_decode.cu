@@ -54,14 +54,6 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
   const int rsub = lane / LPR;         // row within the warp access
   const int dk0 = sub * 4;
 
-  // 1. Issue the state loads first: they do not depend on the prologue.
-  float *base = state + (size_t)nh * D * D;
-  float4 s[Sh::kIters];
-#pragma unroll
-  for (int it = 0; it < Sh::kIters; ++it) {
-    const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
-    s[it] = __ldcs(reinterpret_cast<const float4 *>(base + (size_t)j * D + dk0));
-  }
   float4 g4;
   if constexpr (kGated) {
     const Tin *gr = static_cast<const Tin *>(g) + (size_t)nh * D + dk0;
@@ -77,9 +69,9 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
   }
   const float b = __ldg(beta + nh);
 
-  // 2. Prologue for this head's 3*D channels; the conv cache is shifted in place.
-  //    A thread's channels (two at most) have all their loads issued before any
-  //    is used, so the barrier waits for one round trip, not two.
+  // 1. Prologue for this head's 3*D channels; the conv cache is shifted in place.
+  //    A thread's channels (two at most) have all their loads issued first, before
+  //    the state's, and before any is used: the barrier waits for one round trip.
   const int C = 3 * H * D;
   constexpr int kCh = (3 * D + Sh::kThreads - 1) / Sh::kThreads;
   Tin r0[kCh], r1[kCh], r2[kCh], xin[kCh];
@@ -96,6 +88,15 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
       xin[m] = x[(size_t)n * C + c];
       wc[m] = __ldg(reinterpret_cast<const float4 *>(w + (size_t)c * 4));
     }
+  }
+  // The state loads follow: the prologue is on the path to the barrier, the
+  // state is first needed after it.
+  float *base = state + (size_t)nh * D * D;
+  float4 s[Sh::kIters];
+#pragma unroll
+  for (int it = 0; it < Sh::kIters; ++it) {
+    const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
+    s[it] = __ldcs(reinterpret_cast<const float4 *>(base + (size_t)j * D + dk0));
   }
 #pragma unroll
   for (int m = 0; m < kCh; ++m) {
@@ -137,7 +138,7 @@ decode_kernel(const Tin *__restrict__ x, const float *__restrict__ w, Tin *__res
                                 qkv[D + dk0 + 2] * rk, qkv[D + dk0 + 3] * rk);
   const float4 a4 = make_float4(expf(g4.x), expf(g4.y), expf(g4.z), expf(g4.w));
 
-  // 3. State update, one row of S^T per LPR lanes.
+  // 2. State update, one row of S^T per LPR lanes.
 #pragma unroll
   for (int it = 0; it < Sh::kIters; ++it) {
     const int j = (warp * Sh::kIters + it) * Sh::kRowsPerInstr + rsub;
