@@ -34,6 +34,7 @@ __all__ = [
     "kda_decode_step",
     "kda_prologue_chunk_fwd",
     "kda_get_device_status",
+    "kda_selftest_wait_timeout",
     "kda_version",
     "KDA_OK",
     "KDA_ERR_INVALID_ARG",
@@ -109,13 +110,15 @@ lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
             lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
             lib.kda_state_compose,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_output_epilogue,
-            lib.kda_prologue_chunk_fwd, lib.kda_get_device_status):
+            lib.kda_prologue_chunk_fwd, lib.kda_get_device_status,
+            lib.kda_selftest_wait_timeout):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
 lib.kda_last_error.argtypes = []
@@ -171,6 +174,13 @@ def kda_get_device_status() -> int:
     code = ctypes.c_int(0)
     _check(lib.kda_get_device_status(ctypes.byref(code)))
     return code.value
+
+
+def kda_selftest_wait_timeout(limit_us: int = 1000, stream=None):
+    """Launch one CTA whose bounded mbarrier wait runs out after ``limit_us``
+    microseconds; it records KDA_ERR_DEVICE_TIMEOUT in the status word and
+    returns without faulting (the failure path of every tensor-core kernel)."""
+    _check(lib.kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def kda_prologue(x, conv_w, q, k, v, *, H: int, D: int, cache_in=None, cache_out=None,

@@ -1,12 +1,12 @@
-// Host side of the libkda C ABI: argument validation, the per-device status
-// word, error reporting and dispatch to the kernels.  No entry point
-// allocates memory per call.
+// Host side of the libkda C ABI: argument validation, error reporting and
+// dispatch to the kernels.  No entry point allocates device memory: the status
+// word (kda_status.cu) and the scratch of kda_chunk_fwd_static (kda_static.cu)
+// are file-scope __device__ variables.
 #include <cuda_runtime.h>
 
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 #include <string>
 
 #include "kda_chunk_record.cuh"
@@ -30,49 +30,11 @@ kda_status cuda_fail(cudaError_t e, const char *what) {
   return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-constexpr int kMaxDevices = 64;
-std::mutex g_status_mu;
-int *g_status[kMaxDevices] = {nullptr};
-
-// The status word of the current device, allocated (and zeroed) on first use.
+// The status word of the current device: a __device__ int of kda_status.cu,
+// looked up once per device; nothing is allocated.
 kda_status device_status_word(int **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED, "device index %d", dev);
-  std::lock_guard<std::mutex> lock(g_status_mu);
-  if (g_status[dev] == nullptr) {
-    int *p = nullptr;
-    e = cudaMalloc(&p, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status word)");
-    e = cudaMemset(p, 0, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
-    g_status[dev] = p;
-  }
-  *out = g_status[dev];
-  return KDA_OK;
-}
-
-// Scratch of kda_chunk_fwd_static: a module global, one per device, never
-// allocated or freed by a call.  Its device address is looked up once per
-// device and cached.
-__device__ __align__(256) uint8_t g_static_scratch[KDA_CHUNK_STATIC_SCRATCH_BYTES];
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
-
-kda_status static_scratch(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED, "device index %d", dev);
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  cudaError_t e = kda::status_word_address(out);
+  if (e != cudaSuccess) return cuda_fail(e, "status word address");
   return KDA_OK;
 }
 
@@ -148,6 +110,17 @@ kda_status kda_output_epilogue(const float *o, const void *gate, const float *we
   cudaError_t e = kda::launch_epilogue(o, gate, weight, eps, (long long)T * H, D, dt, out,
                                        (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kda_output_epilogue launch");
+  return KDA_OK;
+}
+
+kda_status kda_selftest_wait_timeout(unsigned limit_us, kda_stream_t stream) {
+  KDA_REQUIRE(limit_us >= 1 && limit_us <= 2000000u, "limit_us=%u outside [1, 2000000]",
+              limit_us);
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  const cudaError_t e = kda::launch_wait_timeout(limit_us, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_wait_timeout launch");
   return KDA_OK;
 }
 
@@ -449,23 +422,12 @@ kda_status kda_chunk_fwd_static(const void *q, const void *k, const void *v, con
                 "buffer holds %zu (use kda_chunk_fwd_ws with a caller workspace)",
                 N, T, H, need, (size_t)KDA_CHUNK_STATIC_SCRATCH_BYTES);
   void *scratch = nullptr;
-  st = static_scratch(&scratch);
-  if (st != KDA_OK) return st;
-  int *status = nullptr;
-  st = device_status_word(&status);
-  if (st != KDA_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaSuccess;
-  const int L = kda::rec::segment_chunks(N, T, H);
-  if (cu_seqlens || L > 0) e = kda::launch_chunk_index(cu_seqlens, N, T, L, scratch, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, scratch, nullptr,
-                               nullptr, 0.f, false, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_state(scratch, cu_seqlens, initial_state, scale, N, T, H, L, o,
-                                final_state, status, s);
-  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_static launch");
-  return KDA_OK;
+  const cudaError_t e = kda::static_scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
+  return chunk_two_pass(q, k, v, g, 4, nullptr, nullptr, 0.f, false, beta, scale, initial_state,
+                        cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, scratch,
+                        KDA_CHUNK_STATIC_SCRATCH_BYTES, (cudaStream_t)stream,
+                        "kda_chunk_fwd_static launch", kda::rec::segment_chunks(N, T, H));
 }
 
 }  // extern "C"

@@ -139,6 +139,7 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
   }
 
   uint32_t pa = 0, pk = 0, pm = 0;
+  bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
   for (int c = nch - 1; c >= 0; --c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
     const uint8_t *rp = rec_of(c);
@@ -184,7 +185,10 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
     const float gl = __ldg(reinterpret_cast<const float *>(rp + rec::GL) + t);
     fence_async_smem();
     tc_fence_before();
-    if (!wait_all(bar_kp, pk, status)) break;  // K', P of this chunk; also a CTA barrier
+    if (!wait_all(bar_kp, pk, status)) {
+      failed = true;
+      break;
+    }  // K', P of this chunk; also a CTA barrier
     pk ^= 1;
 
     // ---- D_u = P^T (scale dO) + K' dS' -------------------------------------------------
@@ -203,7 +207,10 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
         mma_bf16(tmem + TB_DU, desc_kmajor(kp, 64, ks), desc_mn32_sw64(dso, ks), idK, 1);
       mma_commit(bar_mma);
     }
-    if (!wait_all(bar_mma, pm, status)) break;
+    if (!wait_all(bar_mma, pm, status)) {
+      failed = true;
+      break;
+    }
     pm ^= 1;
     tc_fence_after();
     if (tid == 0 && c > 0) load_kp(c - 1);  // K' and P have been read
@@ -230,7 +237,10 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
     }
     fence_async_smem();
     tc_fence_before();
-    if (!wait_all(bar_a1, pa, status)) break;  // [W; Q G] of this chunk; also a CTA barrier
+    if (!wait_all(bar_a1, pa, status)) {
+      failed = true;
+      break;
+    }  // [W; Q G] of this chunk; also a CTA barrier
     pa ^= 1;
 
     // ---- D_s = [W^T | (Q G)^T] [-dU ; scale dO] ----------------------------------------------
@@ -243,7 +253,10 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
         mma_bf16(tmem + TB_DS, desc_mnmajor(a1, 128, ks), desc_mn32_sw64(b2, ks), idT, ks > 0);
       mma_commit(bar_mma);
     }
-    if (!wait_all(bar_mma, pm, status)) break;
+    if (!wait_all(bar_mma, pm, status)) {
+      failed = true;
+      break;
+    }
     pm ^= 1;
     tc_fence_after();
     if (tid == 0 && c > 0) load_a1(c - 1);  // [W; Q G] has been read
@@ -260,9 +273,14 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
     __syncthreads();
   }
 
-  if (ds0) {
+  if (ds0 && !failed) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) ds0[head_off + sbase + (size_t)i * 128] = dS[i];
+  }
+  if (failed && tid == 0) {  // let in-flight record copies and MMAs land first
+    drain(bar_a1);
+    drain(bar_kp);
+    drain(bar_mma);
   }
   tc_fence_before();
   __syncthreads();

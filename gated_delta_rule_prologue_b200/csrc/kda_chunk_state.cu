@@ -257,6 +257,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   }
 
   uint32_t pa = 0, pk = 0, pm = 0, pm2 = 0;
+  bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
   for (int c = c_lo; c < c_hi; ++c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
     if (ckpt) {  // entry state of the chunk, for the backward pass
@@ -266,7 +267,10 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     }
 
     // ---- D1 = [W ; Q G] S ----------------------------------------------------------
-    if (!wait_all(bar_a1, pa, status)) break;
+    if (!wait_all(bar_a1, pa, status)) {
+      failed = true;
+      break;
+    }
     pa ^= 1;
     if (tid == 0) {
       tc_fence_after();
@@ -342,7 +346,10 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       }
     }
     pk ^= 1;
-    if (!wait_all(bar_m2, pm2, status)) break;
+    if (!wait_all(bar_m2, pm2, status)) {
+      failed = true;
+      break;
+    }
     pm2 ^= 1;
     tc_fence_after();
     if (tid == 0 && c + 1 < c_hi) load_kp(c + 1);  // K' and P have been read
@@ -383,9 +390,15 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     // the next chunk's wait on its [W; Q G] tile is the barrier before MMA1 reads S
   }
 
-  if (s_out) {
+  if (s_out && !failed) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) s_out[sbase + (size_t)i * 128] = S[i];
+  }
+  if (failed && tid == 0) {  // let in-flight record copies and MMAs land first
+    drain(bar_a1);
+    drain(bar_kp);
+    drain(bar_mma);
+    drain(bar_m2);
   }
   tc_fence_before();
   __syncthreads();
@@ -543,7 +556,13 @@ state_scan_kernel(const uint8_t *__restrict__ ws, int N, int T, int H, int *stat
 #pragma unroll
     for (int j = 0; j < kScanCols; ++j) bcur[j] = bnext[j];
     if (g + 2 < G) load_b(g + 1);
-    if (!wait_all(bar + b, (phase >> b) & 1, status)) return;
+    if (!wait_all(bar + b, (phase >> b) & 1, status)) {
+      if (r == 0) {  // the other buffer's copy may still be in flight
+        drain(bar);
+        drain(bar + 1);
+      }
+      return;
+    }
     phase ^= 1u << b;
     const float *Ms = reinterpret_cast<const float *>(sm + SC_M + b * 65536);
     float acc[4][kScanCols];

@@ -424,13 +424,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (cur.ok) fetch_gate(cur);
 
   uint32_t tma_par = 0, mma_par = 0;
+  bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
   int c = 0;
   for (; cur.ok; ++c) {
     const Work nxt = work_of(c + 1);
     const int t0 = cur.t0, Lc = cur.Lc, h = cur.h;
 
     // ---- P0: raw tiles of this chunk ---------------------------------------------
-    if (!wait_all(bar_tma, tma_par, status)) break;
+    if (!wait_all(bar_tma, tma_par, status)) {
+      failed = true;
+      break;
+    }
     tma_par ^= 1;
     if constexpr (kGated) {
       ga = ga_next;
@@ -663,7 +667,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       mma_commit(bar_mma);
     }
-    if (!wait_all(bar_mma, mma_par, status)) break;
+    if (!wait_all(bar_mma, mma_par, status)) {
+      failed = true;
+      break;
+    }
     mma_par ^= 1;
     tc_fence_after();
 
@@ -952,7 +959,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
     }
     fence_async_smem();
-    if (!wait_all(bar_mma, mma_par, status)) break;
+    if (!wait_all(bar_mma, mma_par, status)) {
+      failed = true;
+      break;
+    }
     mma_par ^= 1;
     tc_fence_after();
 
@@ -1044,7 +1054,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bvmax = fmaxf(bvmax, fabsf(bvv));
       }
     }
-    if (!wait_all(bar_mma, mma_par, status)) break;
+    if (!wait_all(bar_mma, mma_par, status)) {
+      failed = true;
+      break;
+    }
     mma_par ^= 1;
     tc_fence_after();
 
@@ -1087,7 +1100,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_bf16(tmem + TM_S, desc_kmajor(ut, 128, ks), desc_mnmajor(kp, 64, ks), idS, ks > 0);
       mma_commit(bar_mma);
     }
-    if (!wait_all(bar_mma, mma_par, status)) break;
+    if (!wait_all(bar_mma, mma_par, status)) {
+      failed = true;
+      break;
+    }
     mma_par ^= 1;
     tc_fence_after();
 
@@ -1122,7 +1138,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if constexpr (kPrepM) {
     if (tid == 0) bulk_wait_all();
   }
-  if (sN && !kPrepM) {
+  if (failed && tid == 0) {  // let in-flight tile loads and MMAs land first
+    drain(bar_tma);
+    drain(bar_mma);
+  }
+  if (sN && !kPrepM && !failed) {
     float *dst = sN + (((size_t)n * H + hb) * 128 + j) * 128 + dk0;
 #pragma unroll
     for (int x = 0; x < 32; x += 4)

@@ -185,6 +185,13 @@ __device__ __forceinline__ int seq_of_token(const int32_t *cu, int N, int t) {
 
 // Host-side launchers implemented in the kernel files, called by kda_api.cu.
 namespace kda {
+// Device addresses of the file-scope __device__ status word (kda_status.cu)
+// and of the fixed scratch of kda_chunk_fwd_static (kda_static.cu) on the
+// current device, looked up once per device.
+cudaError_t status_word_address(int **out);
+cudaError_t static_scratch_address(void **out);
+// One CTA whose bounded mbarrier wait runs out after limit_us (kda_selftest.cu).
+cudaError_t launch_wait_timeout(unsigned limit_us, int *status, cudaStream_t s);
 cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in, void *cache_out,
                             const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
                             kda_dtype out_dt, void *q, void *k, void *v, int *status,

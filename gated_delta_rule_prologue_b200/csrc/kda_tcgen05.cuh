@@ -100,6 +100,17 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, int *st
   return true;
 }
 
+// Error exit of a kernel whose wait ran out: one thread waits (bounded) for the
+// current phase of each of the CTA's mbarriers, so that a bulk copy or an MMA
+// that is still in flight lands before the CTA frees its TMEM and exits.  A
+// barrier with nothing in flight simply runs out after limit_ns.  The current
+// phase's parity is read from the barrier itself: try_wait.parity(0) succeeds
+// exactly when the current phase is odd.
+__device__ __forceinline__ void drain(uint64_t *bar, uint64_t limit_ns = 100000000ull) {
+  const uint32_t cur = mbar_try_wait(bar, 0u) ? 1u : 0u;
+  (void)mbar_wait(bar, cur, limit_ns);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor tile loads; no multicast)
 // ---------------------------------------------------------------------------

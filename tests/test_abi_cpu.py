@@ -249,6 +249,22 @@ def test_static_scratch_constant_matches_header(kda):
     assert m and int(m.group(1)) << int(m.group(2)) == kda.KDA_CHUNK_STATIC_SCRATCH_BYTES
 
 
+def test_library_sources_never_allocate_device_memory():
+    """The status word and the static scratch are file-scope __device__
+    variables; no source of the library calls an allocator."""
+    csrc = os.path.join(ROOT, "gated_delta_rule_prologue_b200", "csrc")
+    banned = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cuMemAlloc\w*|cuMemCreate|"
+                        r"cudaHostAlloc|cudaMallocHost)\b")
+    for f in sorted(os.listdir(csrc)):
+        src = open(os.path.join(csrc, f), encoding="utf-8").read()
+        src = re.sub(r"//[^\n]*|/\*.*?\*/", "", src, flags=re.S)  # code only
+        assert not banned.search(src), (f, banned.search(src).group(0))
+    for f, sym in (("kda_status.cu", "g_status_word"), ("kda_static.cu", "g_static_scratch")):
+        src = open(os.path.join(csrc, f), encoding="utf-8").read()
+        assert re.search(r"__device__[^;]*\b%s\b" % sym, src), f
+        assert "cudaGetSymbolAddress" in src, f
+
+
 def test_gated_entry_points_reject_bad_gate_arguments(kda):
     L = kda.lib
     T, H = 128, 2
