@@ -46,6 +46,11 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 D_ = 128
 QKV_DT = 2                                          # q/k/v handed from prologue to chunk: f16
 PROLOGUE_BYTES_PER_TH = 3 * D_ * 2 + 3 * D_ * QKV_DT   # read x (bf16), write q/k/v      = 1536
+# The algorithmic bytes of the chunk call as first planned: q, k, v (16-bit) + g + beta
+# + o in the activation type (16-bit) = 1540 per token-head.  The library writes o in
+# fp32 (its read-out is heavy-tailed: a 16-bit o alone breaks the parity bound), which
+# makes 1796; both fractions are reported.
+CHUNK_BYTES_PER_TH_PLAN = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 2
 CHUNK_BYTES_PER_TH = 3 * D_ * QKV_DT + D_ * 4 + 4 + D_ * 4  # q,k,v + g + beta + o (f32) = 1796
 FUSED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4  # x + g + beta + o: the fused floor = 1796
 GATED_BYTES_PER_TH = 3 * D_ * 2 + D_ * 2 + 4 + D_ * 4  # bf16 q,k,v + bf16 g_raw + beta + o = 1540
@@ -237,12 +242,20 @@ def oracle_sample(n_tokens):
     return wall, max(1, round(cpu / wall))
 
 
-def cpu_baseline(n_tokens=1024):
+# Tokens of the K3-layer workload (all 96 heads) the oracle runs per sample, in the
+# cpu_baseline leg and in every step of the reference arm alike.
+ORACLE_SAMPLE_TOKENS = 768
+ORACLE_NOTE = ("the oracle is single-threaded by construction: a Python loop over tokens "
+               "with float64 NumPy vectorised over heads, so BLAS threading does not engage")
+
+
+def cpu_baseline(n_tokens=ORACLE_SAMPLE_TOKENS):
     wall, cores = oracle_sample(n_tokens)
     return {"value": round(n_tokens / wall, 3), "unit": "tokens/s", "cores": cores,
             "host_cores_available": len(os.sched_getaffinity(0)), "kind": "oracle",
             "sample": f"first {n_tokens} tokens of the K3-layer prefill, all 96 heads "
-                      f"(prologue + token-by-token recurrence, float64 NumPy), {wall:.1f} s"}
+                      f"(prologue + token-by-token recurrence, float64 NumPy), {wall:.1f} s",
+            "note": ORACLE_NOTE}
 
 
 # Bytes of one record of the two-pass prefill and the workspace of one K3 call (the
@@ -268,9 +281,11 @@ def k3_config(world, T=32768, H=96, D=128):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    budget_s = 150.0
+    # the same sample as the cpu_baseline leg, shrunk only if the run would exceed ~5 min
+    budget_s = 300.0
     per_token_s = 0.011
-    n_tok = int(max(16, min(1024, budget_s / max(1, args.steps + args.warmup) / per_token_s)))
+    n_tok = int(max(16, min(ORACLE_SAMPLE_TOKENS,
+                            budget_s / max(1, args.steps + args.warmup) / per_token_s)))
     for _ in range(args.warmup):
         oracle_sample(n_tok)
     times, cores = [], 1
@@ -288,7 +303,8 @@ def run_reference(args, world, rank):
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"first {n_tok} tokens x 96 heads of the K3-layer prefill "
-                                   "per step (prologue + recurrence, float64)"},
+                                   "per step (prologue + recurrence, float64)",
+                         "note": ORACLE_NOTE},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -342,6 +358,101 @@ def seq4k_side(kda, dev, stream, hbm):
     out["speedup"] = round(out["whole"]["ms"] / out["split"]["ms"], 3)
     del q4, k4, v4, g4, b4, s04, o4, f4, flush
     return out
+
+
+def varlen_side(kda, dev, stream, hbm):
+    """The packed varlen prefill: 16 sequences of uniform length in [512, 16384]
+    (93,891 tokens as drawn), H=32, d=128, bf16 q/k/v, an initial state per
+    sequence and every final state returned, through kda_chunk_fwd with
+    cu_seqlens and a preallocated workspace.  Its inputs are larger than L2."""
+    vinp = W.varlen16()
+    Tv, Hv, Dv, Nv = vinp.T, vinp.H, vinp.q.shape[2], vinp.N
+    qv, kv, vv = vinp.q.to(dev), vinp.k.to(dev), vinp.v.to(dev)
+    gv, bv, s0v = vinp.g.to(dev), vinp.beta.to(dev), vinp.initial_state.to(dev)
+    cu = vinp.cu_seqlens.to(dev)
+    ov = torch.empty((Tv, Hv, Dv), dtype=torch.float32, device=dev)
+    fv = torch.empty_like(s0v)
+    wsv = torch.empty(kda.kda_chunk_fwd_workspace_bytes(Nv, Tv, Hv, Dv, Dv, 64, qv.dtype),
+                      dtype=torch.uint8, device=dev)
+    call = lambda: kda.kda_chunk_fwd(qv, kv, vv, gv, bv, ov, scale=vinp.scale,
+                                     initial_state=s0v, final_state=fv, cu_seqlens=cu,
+                                     workspace=wsv, stream=stream)
+    for _ in range(3):
+        call()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(5)]
+    for e in ev:
+        e[0].record(stream)
+        call()
+        e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    th = Tv * Hv
+    states = 2 * Nv * Hv * Dv * Dv * 4  # initial state read, final state written
+    out = {"workload": f"varlen16: {Nv} packed sequences, {Tv} tokens (lengths uniform in "
+                       f"[512, 16384]), H={Hv}, d=128, bf16 q/k/v, initial and final state "
+                       "per sequence", "ms": round(ms, 4),
+           "tokens_per_s": round(Tv / (ms * 1e-3), 1),
+           "segment_chunks": kda.kda_chunk_fwd_segment_chunks(Nv, Tv, Hv),
+           "roofline": dict(roofline("hbm", CHUNK_BYTES_PER_TH_PLAN * th + states, ms, hbm,
+                                     "GB/s", None),
+                            algorithmic_bytes=f"{CHUNK_BYTES_PER_TH_PLAN} B per token-head + "
+                                              "the states (2 x 64 KiB per sequence-head)",
+                            frac_fp32_readout_bytes=roofline(
+                                "hbm", CHUNK_BYTES_PER_TH * th + states, ms, hbm, "GB/s",
+                                None)["frac"])}
+    del qv, kv, vv, gv, bv, s0v, cu, ov, fv, wsv
+    return out
+
+
+def tiny_side(kda, dev, stream):
+    """The tiny fp32 forward (T=64, H=2, d=16, chunk 16: the exact-fp32 CUDA-core
+    path): latency of one kda_chunk_fwd call, median over 200 calls."""
+    t = W.tiny_f32()
+    args_ = [x.to(dev) for x in (t.q, t.k, t.v, t.g, t.beta)]
+    o = torch.empty(t.v.shape, dtype=torch.float32, device=dev)
+    fs = torch.empty((1, t.H, t.q.shape[2], t.q.shape[2]), device=dev)
+    call = lambda: kda.kda_chunk_fwd(*args_, o, scale=t.scale, final_state=fs, chunk=t.chunk,
+                                     stream=stream)
+    for _ in range(10):
+        call()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(200)]
+    for e in ev:
+        e[0].record(stream)
+        call()
+        e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status() == 0
+    us = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    return {"workload": "tiny_f32: T=64, H=2, d_k=d_v=16, chunk 16, fp32 (CUDA-core path)",
+            "latency_us": round(us, 2), "tokens_per_s": round(t.T / (us * 1e-6), 1)}
+
+
+def decode_parity(state, cache, outs_last, steps, ns):
+    """The oracle's run of the same ``steps`` decode steps on sequences ``ns``
+    (all 96 heads), against the GPU's state, cache and last read-out."""
+    import numpy as np
+    from oracle import kda_decode_step, state_from_abi, state_to_abi
+    st0, c0, xs, gs, bs, wr = W.decode256_seqs(ns, steps)
+    c = W.WORKLOADS["decode256"]
+    H, D = c["H"], c["D"]
+    S, cc = state_from_abi(st0), c0
+    t0 = time.perf_counter()
+    for i in range(steps):
+        o_ref, S, cc = kda_decode_step(xs[i], wr, cc, gs[i], bs[i], S, H, D)
+    wall = time.perf_counter() - t0
+    got_o = outs_last[ns].double().cpu().numpy()
+    got_s = state[ns].double().cpu().numpy()
+    rel_o = float(np.max(np.abs(got_o - o_ref)) / np.sqrt(np.mean(o_ref ** 2)))
+    ref_s = state_to_abi(S)
+    rel_s = float(np.linalg.norm(got_s - ref_s) / np.linalg.norm(ref_s))
+    cache_ok = bool(np.array_equal(cache[ns].double().cpu().numpy(), cc))
+    return {"sequences": list(ns), "heads": H, "steps": steps,
+            "o_rel_max": round(rel_o, 6), "state_rel_fro": round(rel_s, 6),
+            "cache_exact": cache_ok, "ok": bool(rel_o <= 2e-2 and rel_s <= 1e-2 and cache_ok),
+            "bounds": "max|o - o_ref| / RMS(o_ref) <= 2e-2 (last step); "
+                      "||S - S_ref||_F / ||S_ref||_F <= 1e-2",
+            "oracle_s": round(wall, 1)}
 
 
 def run_ours(args, world, rank, local):
@@ -462,6 +573,9 @@ def run_ours(args, world, rank, local):
     del d_o, bwd_out, d_beta, bws
     torch.cuda.empty_cache()
     seq4k = seq4k_side(kda, dev, stream, hbm)
+    varlen = varlen_side(kda, dev, stream, hbm)
+    torch.cuda.empty_cache()
+    tiny = tiny_side(kda, dev, stream)
 
     th = T * H
     # the shared workload description assumes the library's record layout
@@ -492,10 +606,14 @@ def run_ours(args, world, rank, local):
     kernels["kda_chunk_fwd"]["tensor_tflops"] = round(
         CHUNK_FLOPS_PER_TH * th / (chk_ms * 1e-3) / 1e12, 2)
     dominant = "kda_chunk_fwd"
-    roof = {k_: kernels[dominant][k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roof = roofline("hbm", CHUNK_BYTES_PER_TH_PLAN * th, chk_ms, hbm, "GB/s",
+                    recorded_traffic("kda_chunk_fwd"))
     roof["kernel"] = dominant + " (one call: prep pass + state pass)"
     roof["peak_source"] = f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-    fused_floor_ms = 1e3 * FUSED_BYTES_PER_TH * th / (hbm * 1e9)
+    roof["algorithmic_bytes_per_token_head"] = CHUNK_BYTES_PER_TH_PLAN
+    roof["frac_fp32_readout_bytes"] = kernels[dominant]["frac"]  # 1796 B: o written as fp32
+    # the whole step against the HBM floor of the fused workload (x in, g, beta, o out)
+    fused_floor_ms = 1e3 * (3 * D_ * 2 + D_ * 4 + 4 + D_ * 2) * th / (hbm * 1e9)
 
     # ---- end to end through the C ABI with host buffers ----
     # Every step copies its inputs in from pinned host memory and its read-out back.
@@ -550,10 +668,12 @@ def run_ours(args, world, rank, local):
     dw = dinp.conv_w.to(dev)
     dx, dg, db = dinp.x.to(dev), dinp.g.to(dev), dinp.beta.to(dev)
     do = torch.empty((Nd, Hd, Dd), dtype=torch.float32, device=dev)
-    for s in range(min(3, args.decode_steps)):
-        kda.kda_decode_step(dx[s], dw, cache, dg[s], db[s], state, do, H=Hd, D=Dd,
+    wstate, wcache = state.clone(), cache.clone()  # warm-up on copies: the timed steps
+    for s in range(min(3, args.decode_steps)):    # start from the workload's state
+        kda.kda_decode_step(dx[s], dw, wcache, dg[s], db[s], wstate, do, H=Hd, D=Dd,
                             scale=dinp.scale, stream=stream)
     torch.cuda.synchronize(dev)
+    del wstate, wcache
     dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
               for _ in range(args.decode_steps)]
     barrier(world)
@@ -583,6 +703,9 @@ def run_ours(args, world, rank, local):
                          kernel="kda_decode_step"),
     }
     launches_total = launches
+    if rank == 0:  # the oracle's run of the same 100 steps on 16 of the 256 sequences
+        decode["parity"] = decode_parity(state, cache, do, args.decode_steps,
+                                         list(range(0, Nd, Nd // 16)))
     del state, cache, dx, dg, db
 
     line = {
@@ -594,8 +717,11 @@ def run_ours(args, world, rank, local):
         "roofline": roof,
         "kernels": kernels,
         "fused_hbm_floor_ms": round(fused_floor_ms, 4),
+        "step_fraction_of_fused_floor": round(fused_floor_ms / ms_step, 4),
         "decode": decode,
         "seq4k": seq4k,
+        "varlen16": varlen,
+        "tiny_f32": tiny,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -672,7 +798,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--e2e-steps", type=int, default=4)
-    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--cpu-tokens", type=int, default=ORACLE_SAMPLE_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", choices=("fused", "prologue", "chunk", "chunk_one_pass", "decode",
                                            "seq4k", "seq4k_whole", "bwd"),

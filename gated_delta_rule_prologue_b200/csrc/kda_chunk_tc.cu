@@ -93,8 +93,8 @@ constexpr uint32_t F_ELB = F_ELA + 512;     //   exp(gamma_last - c_B)
 constexpr uint32_t F_EGC = F_ELB + 512;     //   exp(gamma_last)
 constexpr uint32_t SM_BETA = F_EGC + 512;   // beta of the chunk     [64]
 constexpr uint32_t SM_PDIAG = SM_BETA + 256;// <q_r, k_r> in fp32    [64]
-constexpr uint32_t SM_BAR = SM_PDIAG + 256; // two mbarriers
-constexpr uint32_t SM_SLOT = SM_BAR + 16;   // TMEM base address
+constexpr uint32_t SM_BAR = SM_PDIAG + 256; // three mbarriers (tiles, MMAs, inverse MMAs)
+constexpr uint32_t SM_SLOT = SM_BAR + 32;   // TMEM base address
 constexpr uint32_t SM_TOTAL = SM_SLOT + 16;
 // Fused prologue only: fp32 correction beta*v - f16(beta*v_tile) kept as bf16
 // [64][128], and two conv histories (3 parts x 3 rows x 128 raw values).
@@ -108,6 +108,21 @@ constexpr uint32_t SM_ALLOC_FUSED = SM_TOTAL_FUSED + 1024;
 static_assert(SM_ALLOC_FUSED <= 232448, "shared memory budget");
 static_assert(SM_ALLOC_PREP <= SM_ALLOC_FUSED, "the prep plan is a prefix of the fused one");
 static_assert(SM_GB + 49152 <= SM_ST + 32768, "Gram tiles stay inside X, TOP, POP and ST");
+// The 64 x 64 inverse (P4b / P5) works in the S^T tile and the T tile, both dead
+// from the Gram MMA to P6.  16-bit tiles are 64 rows x 128 bytes, row-major with
+// the 128-byte swizzle: the same bytes serve as a K-major A operand (row = M
+// index) and as an MN-major B operand (row = K index).  An A operand is read as
+// M = 128 rows, so 8 KB past each A tile must be readable (those rows' products
+// land in TMEM lanes 64..127, which nobody reads).
+constexpr uint32_t SM_A16 = SM_ST;           // A = beta-scaled strict lower Gram, fp16; after
+constexpr uint32_t SM_YM = SM_ST;            //   the third product, Y's lower-left block
+constexpr uint32_t SM_D16 = SM_ST + 8192;    // D = inverses of the 16x16 diagonal blocks
+constexpr uint32_t SM_ZM = SM_ST + 16384;    // the two in-half off-diagonal blocks of A D
+constexpr uint32_t SM_ATD = SM_ST + 24576;   // fp32 diagonal 16x16 blocks of A, [blk][col][row]
+constexpr uint32_t SM_T32 = SM_TOP;          // T at the 32x32-block level, then T itself
+static_assert(SM_T32 + 16384 <= SM_ST && SM_D16 + 16384 <= SM_ST + 32768 &&
+              SM_ATD + 4096 <= SM_ST + 32768 && SM_ST + 32768 <= SM_F,
+              "A-operand reads stay inside shared memory");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
 constexpr uint32_t TM_G = 0;     // Gram, 96 columns (first of two partial sums)
@@ -117,7 +132,13 @@ constexpr uint32_t TM_W = 160;   // W^T, 64
 constexpr uint32_t TM_U = 224;   // U^T, 64
 constexpr uint32_t TM_O = 288;   // O^T, 64
 constexpr uint32_t TM_S = 352;   // delta S^T, 128
+// The inverse's MMA stages (during P5 only, before W / Ut / O / delta S are written):
+constexpr uint32_t TM_Z = 96;    // Z = A D, 64 columns; later T32 Y
+constexpr uint32_t TM_T2 = 384;  // D Z, 64 (over delta S, written only after P5)
+constexpr uint32_t TM_Y = 448;   // Y = A T32, 64
 constexpr uint32_t TM_COLS = 512;
+static_assert(TM_Z + 64 <= TM_W && TM_G + 96 <= TM_Z && TM_G2 + 96 <= TM_T2 &&
+              TM_Y + 64 <= TM_COLS, "inverse stages overlap a live accumulator");
 
 constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
@@ -238,12 +259,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int n = blockIdx.x / H, hb = blockIdx.x % H;  // kSingle / kFused
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);
   uint64_t *bar_mma = bar_tma + 1;
+  uint64_t *bar_inv = bar_tma + 2;
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SM_SLOT);
   float *Gf = reinterpret_cast<float *>(sm + SM_G);
   float *beta_s = reinterpret_cast<float *>(sm + SM_BETA);
   float *pdiag = reinterpret_cast<float *>(sm + SM_PDIAG);
-  float *fca = reinterpret_cast<float *>(sm + F_CA);
-  float *fcb = reinterpret_cast<float *>(sm + F_CB);
   float *feca = reinterpret_cast<float *>(sm + F_ECA);
   float *fecb = reinterpret_cast<float *>(sm + F_ECB);
   float *feba = reinterpret_cast<float *>(sm + F_EBA);
@@ -311,6 +331,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_inv, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -423,7 +444,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   };
   if (cur.ok) fetch_gate(cur);
 
-  uint32_t tma_par = 0, mma_par = 0;
+  uint32_t tma_par = 0, mma_par = 0, inv_par = 0;
   bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
   int c = 0;
   for (; cur.ok; ++c) {
@@ -436,6 +457,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       break;
     }
     tma_par ^= 1;
+    if constexpr (!kFused) {
+      // Rows past the chunk's end (the next sequence's tokens, or the zero fill past T)
+      // are zeroed once here, so no later phase has to mask them (the fused prologue
+      // writes zero rows there itself; the cumsum masks the g tile).
+      if (Lc < 64) {
+        for (int x = tid; x < (64 - Lc) * 48; x += kThreads) {
+          const int row = Lc + x / 48, part = (x % 48) >> 4, c = x & 15;
+          st_shared_16(sm + SM_Q + part * 16384, (uint32_t)(row * 256 + c * 16),
+                       make_uint4(0u, 0u, 0u, 0u));
+        }
+      }
+    }
     if constexpr (kGated) {
       ga = ga_next;
       gb = gb_next;
@@ -593,39 +626,37 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       XS[part * 128 + d] = acc;
       __syncthreads();
-      float off = 0.f;
-      for (int pp = 0; pp < part; ++pp) off += XS[pp * 128 + d];
+      // every thread forms the prefix of its 16-row part and the references from the four
+      // part totals: c_A = gamma_15, c_B = gamma_47, gamma_63
+      const float s0 = XS[d], s1 = XS[128 + d], s2 = XS[256 + d], s3 = XS[384 + d];
+      const float s01 = s0 + s1, ca = s0, cb = s01 + s2, cl = cb + s3;
+      const float off = part == 0 ? 0.f : (part == 1 ? s0 : (part == 2 ? s01 : cb));
+      const float ref = part < 2 ? ca : cb;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) vals[r] += off;
-      if (part == 0) fca[d] = vals[15];  // c_A = gamma_15
-      if (part == 2) fcb[d] = vals[15];  // c_B = gamma_47
-      if (part == 3) fegc[d] = vals[15]; // gamma_63 (exponentiated below)
-      __syncthreads();
-      const float ref = part < 2 ? fca[d] : fcb[d];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Gf[(16 * part + r) * 128 + d] = __expf(vals[r] - ref);
+      for (int r = 0; r < 16; ++r) Gf[(16 * part + r) * 128 + d] = __expf((vals[r] + off) - ref);
       if (tid < 128) {
-        const float ca = fca[d], cb = fcb[d], cl = fegc[d];
         feca[d] = __expf(ca);
         fecb[d] = __expf(cb);
         feba[d] = __expf(0.5f * (cb - ca));
         fela[d] = __expf(cl - ca);
         felb[d] = __expf(cl - cb);
+        fegc[d] = __expf(cl);
       }
-      __syncthreads();
-      if (tid < 128) fegc[d] = __expf(fegc[d]);  // every reader of gamma_63 is past the barrier
     }
     if constexpr (kPrepM) {
       if (tid == 0) bulk_wait_read_all();  // the previous record's tiles have left shared memory
     }
     __syncthreads();
 
-    // ---- P2: Gram operands (fp32, rounded to tf32) -----------------------------------------
+    // ---- P2: Gram operands (fp32, rounded to tf32), in two halves of key channels; the
+    //      Gram MMA over the first half starts while the second half is being built ------
+    // G over key channels [0, 64) and G2 over [64, 128): two independent accumulators
+    // summed at read-out, 8 K=8 steps each
+    const uint32_t ga_s = smem_u32(sm + SM_GA), gb_s = smem_u32(sm + SM_GB);
+    constexpr uint32_t id_gram = idesc_tf32(128, 96, false, false);
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      const int p = tid + kThreads * m;
-      const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
-      const bool valid = r < Lc;
+      const int r = tid >> 3, c8 = 8 * m + (tid & 7), d0 = c8 * 8;
       float k8[8], q8[8], e8[8];
       ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
       ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
@@ -633,7 +664,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float a[8], b[8], ki[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f;
+        const float kk = k8[e], qq = q8[e];  // rows past the chunk's end are zero
         a[e] = kk * e8[e];
         b[e] = qq * e8[e];
         ki[e] = __fdividef(kk, e8[e]);  // E in [e^-80, e^75]: inside the intrinsic's range
@@ -648,24 +679,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * hf[e]) * hf[e];
       }
       st_tf32x8(sm + SM_GB, 96, 32 + r, c8, ki);
-    }
-    fence_async_smem();
-    __syncthreads();
-
-    // ---- P3: Gram MMA ------------------------------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
-      constexpr uint32_t id = idesc_tf32(128, 96, false, false);
-      // 16 K=8 steps in two independent accumulation chains, interleaved:
-      // G over key channels [0, 64), G2 over [64, 128)
+      fence_async_smem();
+      __syncthreads();
+      // ---- P3: Gram MMA over this half's key channels (tid 0) --------------------------
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t acc = m == 0 ? TM_G : TM_G2;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        mma_tf32(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
-        mma_tf32(tmem + TM_G2, desc_kmajor(ga, 128, ks + 8), desc_kmajor(gb, 96, ks + 8), id,
-                 ks > 0);
+        for (int ks = 0; ks < 8; ++ks)
+          mma_tf32(tmem + acc, desc_kmajor(ga_s, 128, 8 * m + ks), desc_kmajor(gb_s, 96, 8 * m + ks),
+                   id_gram, ks > 0);
+        if (m == 1) mma_commit(bar_mma);
       }
-      mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, mma_par, status)) {
       failed = true;
@@ -675,15 +700,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
 
     // ---- P4: two warp groups ---------------------------------------------------------------
-    //   warps 0-7:  P4b (Gram read-out -> A^T, strict P), P5 (T = (I + A)^-1)
+    //   warps 0-7:  P4b (Gram read-out -> A as an fp16 tile and its diagonal 16x16 blocks in
+    //               fp32, strict P), P5 (T = (I + A)^-1)
     //   warps 8-15: P4a (the W / Ut / output operands; <q_r, k_r>), which needs neither
-    // A^T and T live over the S^T tile (dead from the Gram MMA to P6), so P4a can
+    // P4b / P5 work in the S^T and T tiles (dead from the Gram MMA to P6), so P4a can
     // still read E from the g tile.
-    float *AT = reinterpret_cast<float *>(sm + SM_ST);  // AT[i*64 + r] = A[r][i]
-    float *TT = AT + 4096;                              // TT[r*64 + c] = T[r][c]
+    bool inv_ok = true;  // warps 0-1: every wait on the inverse's MMA stages completed
     if (tid < kHalf) {
-      // ---- P4b: Gram read-out -> A^T (fp32, strictly lower part only: nothing else of
-      //      it is read), strict P operand ------------------------------------------------
+      float *ATd = reinterpret_cast<float *>(sm + SM_ATD);  // [blk][col][row] of A's diagonal blocks
+      // ---- P4b: Gram read-out -> A (fp16 tile, zero on and above the diagonal; its
+      //      diagonal 16x16 blocks also in fp32), strict P operand -------------------------
       // warp w reads TMEM lanes 32 (w % 4).. and column groups 2 (w / 4) + {0, 1}: the
       // first half of the columns ([0, 32), i = col) in groups of 8, the second
       // ([32, 96), i = col - 32) in groups of 16
@@ -697,12 +723,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int g8 = 0; g8 < 2; ++g8) {
           if (g8 == 1 && !(quad & 1)) break;
           const int i0 = i0s + 8 * g8;
+          float p8[8];
           if (!isP) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (i0 + e < r) AT[(i0 + e) * 64 + r] = br * v[8 * g8 + e];
+            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? br * v[8 * g8 + e] : 0.f;
+            if ((i0 >> 4) == (r >> 4)) {  // a diagonal block: row and columns in one 16-block
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                ATd[((r >> 4) * 16 + ((i0 + e) & 15)) * 16 + (r & 15)] = p8[e];
+            }
+            st_shared_16(sm + SM_A16, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
           } else {  // every chunk of the strict P tile this thread reads is written
-            float p8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
             st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
@@ -742,127 +773,139 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           emit(cg0 + gs, v);
         }
       }
-      if (tid < 128) {  // P rows 0..31, columns 32..63: above the diagonal, not read out
+      if (tid < 128) {  // rows 0..31, columns 32..63 of A and P: above the diagonal, not read out
         const int rz = tid >> 2, cz = 4 + (tid & 3);
         st_shared_16(sm + SM_POP, kmaj_off(64, rz, cz), make_uint4(0u, 0u, 0u, 0u));
+        st_shared_16(sm + SM_A16, kmaj_off(64, rz, cz), make_uint4(0u, 0u, 0u, 0u));
       }
       bar_half();
 
-      // ---- P5: T = (I + A)^{-1} by 16x16 blocks, fp32 ----------------------------------
-      // (i) the four diagonal 16x16 blocks by forward substitution, one column per
-      //     thread; (ii) the two 16x16 blocks under them inside each 32x32 half,
-      //     T_{s+1,s} = -T_{s+1,s+1} A_{s+1,s} T_{s,s}; (iii) the lower-left 32x32
-      //     block T_BL = -T_BR (A_BL T_TL).
-      if (tid < 64) {  // column jj of a diagonal block, swept row by row, stored at the end
-        const int base = 16 * (tid >> 4), jj = tid & 15;
+      // ---- P5: T = (I + A)^{-1} -------------------------------------------------------------
+      // The blocked inverse of a lower triangular matrix.  D = blockdiag of the inverses of
+      // the four 16x16 diagonal blocks of I + A (forward substitution, fp32); then
+      //   T32 = D - D Z      with Z = A D          (T at the 32x32-block level; only the
+      //                                             blocks (1,0) and (3,2) of Z are used)
+      //   T   = T32 - T32 Y  with Y = A T32        (only Y's lower-left 32x32 block)
+      // The four products are tcgen05 MMAs (M = 128: rows 64..127 are not read) with fp16
+      // operands and fp32 accumulation; each piece of T is rounded to fp16 once, for the
+      // W / Ut MMAs.  Warps 0-1 run the substitution and the four stages; warps 2-7 zero
+      // the parts of the 16-bit tiles that nothing else writes, then go on to the join.
+      float amax = 0.f;
+      if (warp < 2) {  // (i) column jj of D_b, swept row by row; fp16 into D16 and T32
+        const int b = tid >> 4, jj = tid & 15, base = 16 * b;
         float acc[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
           acc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -acc[ii]);
-          const float *arow = AT + (base + ii) * 64 + base;  // A[base+rr][base+ii], rr > ii
+          const float *arow = ATd + (b * 16 + ii) * 16;  // A[base + rr][base + ii]
 #pragma unroll
           for (int rr = ii + 1; rr < 16; ++rr) acc[rr] = fmaf(arow[rr], acc[ii], acc[rr]);
         }
+        const uint32_t col = (uint32_t)((base + jj) & 7) * 2;
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) TT[(base + rr) * 64 + base + jj] = acc[rr];
-      }
-      bar_half();
-      // Blocks below the diagonal, 2x2 output tiles per thread.  A is read through
-      // its transpose (columns of A are contiguous), T and Y by rows, so the
-      // operands of one k-step are float2 loads.
-      if (tid < 128) {  // (ii) X = A_{s+1,s} T_{s,s} for s = 0, 2
-        const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
-        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const float2 av = *reinterpret_cast<const float2 *>(AT + (s0b + t) * 64 + s0b + 16 + a);
-          const float2 tv = *reinterpret_cast<const float2 *>(TT + (s0b + t) * 64 + s0b + b);
-          x00 = fmaf(av.x, tv.x, x00); x01 = fmaf(av.x, tv.y, x01);
-          x10 = fmaf(av.y, tv.x, x10); x11 = fmaf(av.y, tv.y, x11);
+        for (int rr = 0; rr < 16; ++rr) {
+          const __half hv = __float2half_rn(acc[rr]);
+          amax = fmaxf(amax, fabsf(acc[rr]));
+          const uint32_t off = kmaj_off(64, base + rr, (base + jj) >> 3) + col;
+          *reinterpret_cast<__half *>(sm + SM_D16 + off) = hv;
+          *reinterpret_cast<__half *>(sm + SM_T32 + off) = hv;
         }
-        *reinterpret_cast<float2 *>(XS + blk * 256 + a * 16 + b) = make_float2(x00, x01);
-        *reinterpret_cast<float2 *>(XS + blk * 256 + (a + 1) * 16 + b) = make_float2(x10, x11);
+      } else {
+        // D16 and T32 outside the diagonal 16x16 blocks, and all of Zm, start at zero
+        // (the diagonal blocks' 16-byte chunks are written whole by the substitution)
+        for (int x = tid - 64; x < 3 * 512; x += kHalf - 64) {
+          const int row = (x & 511) >> 3, c8 = x & 7;
+          if (x < 1024 && (c8 >> 1) == (row >> 4)) continue;
+          const uint32_t tile = x < 512 ? SM_D16 : (x < 1024 ? SM_T32 : SM_ZM);
+          st_shared_16(sm + tile, kmaj_off(64, row, c8), make_uint4(0u, 0u, 0u, 0u));
+        }
       }
+      fence_async_smem();
       bar_half();
-      if (tid < 128) {  // T_{s+1,s} = -T_{s+1,s+1} X
-        const int blk = tid >> 6, a = 2 * ((tid >> 3) & 7), b = 2 * (tid & 7), s0b = 32 * blk;
-        const float *t0r = TT + (s0b + 16 + a) * 64 + s0b + 16;  // row a of T_{s+1,s+1}
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+      if (warp < 2) {
+        auto inv_mma = [&](uint32_t a_tile, uint32_t b_tile, uint32_t dcol) {
+          if (tid == 0 && inv_ok) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc_fp16(128, 64, false, true);
+            const uint32_t a = smem_u32(sm + a_tile), bt = smem_u32(sm + b_tile);
 #pragma unroll
-        for (int t4 = 0; t4 < 16; t4 += 4) {  // diagonal blocks were stored with their zeros
-          const float4 ra = *reinterpret_cast<const float4 *>(t0r + t4);
-          const float4 rb = *reinterpret_cast<const float4 *>(t0r + 64 + t4);
-          const float ta[4] = {ra.x, ra.y, ra.z, ra.w}, tb[4] = {rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xv = *reinterpret_cast<const float2 *>(XS + blk * 256 + (t4 + e) * 16 + b);
-            y00 = fmaf(ta[e], xv.x, y00); y01 = fmaf(ta[e], xv.y, y01);
-            y10 = fmaf(tb[e], xv.x, y10); y11 = fmaf(tb[e], xv.y, y11);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + dcol, desc_kmajor(a, 128, ks), desc_mnmajor(bt, 64, ks), id, ks > 0);
+            mma_commit(bar_inv);
           }
-        }
-        *reinterpret_cast<float2 *>(TT + (s0b + 16 + a) * 64 + s0b + b) = make_float2(-y00, -y01);
-        *reinterpret_cast<float2 *>(TT + (s0b + 17 + a) * 64 + s0b + b) = make_float2(-y10, -y11);
-      }
-      bar_half();
-      {  // (iii) Y = A_BL T_TL  (rows 32..63, cols 0..31)
-        const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-        for (int m = 0; m < 32; ++m) {
-          const float2 av = *reinterpret_cast<const float2 *>(AT + m * 64 + 32 + a);
-          float2 tv = *reinterpret_cast<const float2 *>(TT + m * 64 + cc);  // T_TL[m][cc..cc+1]
-          tv.x = m >= cc ? tv.x : 0.f;                                      // upper blocks unwritten
-          tv.y = m >= cc + 1 ? tv.y : 0.f;
-          y00 = fmaf(av.x, tv.x, y00); y01 = fmaf(av.x, tv.y, y01);
-          y10 = fmaf(av.y, tv.x, y10); y11 = fmaf(av.y, tv.y, y11);
-        }
-        *reinterpret_cast<float2 *>(XS + a * 32 + cc) = make_float2(y00, y01);
-        *reinterpret_cast<float2 *>(XS + (a + 1) * 32 + cc) = make_float2(y10, y11);
-      }
-      bar_half();
-      {  // T_BL = -T_BR Y
-        const int a = 2 * (tid >> 4), cc = 2 * (tid & 15);
-        const float *tr = TT + (32 + a) * 64 + 32;  // row a of T_BR
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 2
-        for (int m4 = 0; m4 < 32; m4 += 4) {
-          const float4 ra = *reinterpret_cast<const float4 *>(tr + m4);
-          const float4 rb = *reinterpret_cast<const float4 *>(tr + 64 + m4);
-          const float ta4[4] = {ra.x, ra.y, ra.z, ra.w}, tb4[4] = {rb.x, rb.y, rb.z, rb.w};
+        };
+        auto inv_wait = [&]() {
+          if (!mbar_wait(bar_inv, inv_par)) inv_ok = false;
+          inv_par ^= 1;
+          tc_fence_after();
+        };
+        auto pair_sync = [&]() {  // warps 0-1: 16-bit tile writes -> the next MMA
+          fence_async_smem();
+          tc_fence_before();
+          asm volatile("bar.sync 3, 64;" ::: "memory");
+        };
+        // the in-half off-diagonal blocks: warp 0 holds rows 16..31 (block column 0),
+        // warp 1 rows 48..63 (block column 32), in its upper 16 lanes
+        auto offdiag16 = [&](uint32_t col, uint32_t tile, float sign) {
+          float z[16];
+          tmem_ld16(tmem + lane_addr + col + 32 * warp, z);
+          if (lane >= 16) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {  // T_BR's upper-right 16x16 block was never written
-            const int m = m4 + e;
-            const float ta = m <= a ? ta4[e] : 0.f, tb = m <= a + 1 ? tb4[e] : 0.f;
-            const float2 yv = *reinterpret_cast<const float2 *>(XS + m * 32 + cc);
-            y00 = fmaf(ta, yv.x, y00); y01 = fmaf(ta, yv.y, y01);
-            y10 = fmaf(tb, yv.x, y10); y11 = fmaf(tb, yv.y, y11);
+            for (int h8 = 0; h8 < 2; ++h8) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                f[e] = sign * z[8 * h8 + e];
+                amax = fmaxf(amax, fabsf(f[e]));
+              }
+              st_shared_16(sm + tile, kmaj_off(64, 32 * warp + lane, 4 * warp + h8), pack8_f16(f));
+            }
           }
-        }
-        *reinterpret_cast<float2 *>(TT + (32 + a) * 64 + cc) = make_float2(-y00, -y01);
-        *reinterpret_cast<float2 *>(TT + (33 + a) * 64 + cc) = make_float2(-y10, -y11);
-      }
-      bar_half();
+        };
+        // the lower-left 32x32 block: warp 1 (TMEM lanes 32..63), 32 columns
+        auto lowerleft = [&](uint32_t col, uint32_t tile, float sign) {
+          if (warp == 1) {
+            float y[32];
+            tmem_ld32(tmem + lane_addr + col, y);
 #pragma unroll
-      for (int task = tid; task < 512; task += kHalf) {  // T as the fp16 operand
-        const int r8 = task >> 3, c8 = task & 7;
-        float f[8];
-        ld8_f32(TT + r8 * 64 + 8 * c8, f);
+            for (int h8 = 0; h8 < 4; ++h8) {
+              float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int cc = 8 * c8 + e;
-          f[e] = cc < r8 ? f[e] : (cc == r8 ? 1.f : 0.f);
-        }
-        st_shared_16(sm + SM_TOP, kmaj_off(64, r8, c8), pack8_f16(f));
+              for (int e = 0; e < 8; ++e) {
+                f[e] = sign * y[8 * h8 + e];
+                amax = fmaxf(amax, fabsf(f[e]));
+              }
+              st_shared_16(sm + tile, kmaj_off(64, 32 + lane, h8), pack8_f16(f));
+            }
+          }
+        };
+        inv_mma(SM_A16, SM_D16, TM_Z);  // Z = A D
+        inv_wait();
+        offdiag16(TM_Z, SM_ZM, 1.f);
+        pair_sync();
+        inv_mma(SM_D16, SM_ZM, TM_T2);  // D Z
+        inv_wait();
+        offdiag16(TM_T2, SM_T32, -1.f);  // T32 = D - D Z
+        pair_sync();
+        inv_mma(SM_A16, SM_T32, TM_Y);  // A T32
+        inv_wait();
+        // Y goes over A (dead): the rest of that tile keeps A's finite values, which meet
+        // only zeros of T32 in the rows read below
+        lowerleft(TM_Y, SM_YM, 1.f);
+        pair_sync();
+        inv_mma(SM_T32, SM_YM, TM_Z);  // T32 Y (its rows 32..63: T_BR Y)
+        inv_wait();
+        lowerleft(TM_Z, SM_T32, -1.f);  // T's lower-left block; the T32 tile is now T
       }
+      if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
     } else {
       // ---- P4a: WY / output operands (the Gram operands are dead) -------------------------
 #pragma unroll 2
       for (int m = 0; m < 4; ++m) {
         const int p = (tid - kHalf) + kHalf * m;
         const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
-        const bool valid = r < Lc;
         const float bt = beta_s[r];
         const float *fec = r < 32 ? feca : fecb;
         const float *fel = r < 32 ? fela : felb;
@@ -876,7 +919,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ld8_f32(fel + d0, el8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float kk = valid ? k8[e] : 0.f, qq = valid ? q8[e] : 0.f, vv = valid ? v8[e] : 0.f;
+          const float kk = k8[e], qq = q8[e], vv = v8[e];  // zero past the chunk's end
           bkg[e] = bt * kk * e8[e] * ec8[e];
           bv[e] = bt * vv;
           qg[e] = qq * e8[e] * ec8[e];
@@ -894,7 +937,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
           acc += __shfl_xor_sync(0xffffffffu, acc, 4);
           acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-          if (c8 == 0) pdiag[r] = valid ? acc : 0.f;
+          if (c8 == 0) pdiag[r] = acc;
         }
         if constexpr (kPrepM && !kFused) {  // fp32 remainder beta v - f16(beta v), kept as bf16
           float cr[8], bvmax = 0.f;
@@ -922,7 +965,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!inv_ok)) {
+      if (tid == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
+      failed = true;
+      break;
+    }
     if constexpr (!kPrepM) {
       if (tid == 0 && nxt.ok) {  // q, k and g are dead (v is read until the U read-out)
         arm_tma(nxt);
@@ -943,6 +990,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_bf16(tmem + TM_U, desc_mnmajor(bv, 64, ks), desc_kmajor(top, 64, ks), id, ks > 0);
       }
       mma_commit(bar_mma);
+      if constexpr (kPrepM) {
+        // the record's tiles that are complete already leave while the MMAs run: each
+        // k-atom of A1 = [W ; Q G] holds the 64 W rows, then the 64 Q G rows
+        uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)cur.ci * H + h) * rec::BYTES;
+        bulk_store(rp + rec::A1 + 8192, sm + SM_QG, 8192);
+        bulk_store(rp + rec::A1 + 24576, sm + SM_QG + 8192, 8192);
+        bulk_store(rp + rec::KP, sm + SM_KP, 16384);
+        bulk_store(rp + rec::P, sm + SM_POP, 8192);
+        bulk_commit();
+      }
     }
     if constexpr (!kPrepM) {
       float amax = 0.f;
@@ -971,36 +1028,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       //      exp(gamma_63), <q_r, k_r>; then the tiles leave by bulk copies -------------
       uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)cur.ci * H + h) * rec::BYTES;
       {
-        float w[16];
-        tmem_ld16(tmem + lane_addr + TM_W + 16 * grp, w);  // W[16 grp + i][j]
+        float w[16], u[16], cr[16];
+        tmem_ld16_nowait(tmem + lane_addr + TM_W + 16 * grp, w);  // W[16 grp + i][j]
+        tmem_ld16_nowait(tmem + lane_addr + TM_U + 16 * grp, u);  // Ut[16 grp + i][j]
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cr[i] = __bfloat162float(corr[(16 * grp + i) * 128 + j]);
+        tmem_wait_ld(w, u);
         __half *wt = reinterpret_cast<__half *>(sm + SM_BKG);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           wt[(kmaj_off(64, 16 * grp + i, j >> 3) >> 1) + (j & 7)] = __float2half_rn(w[i]);
-      }
-      {
-        float u[16];
-        tmem_ld16(tmem + lane_addr + TM_U + 16 * grp, u);  // Ut[16 grp + i][j]
         float *ut = reinterpret_cast<float *>(rp + rec::UT);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int r = 16 * grp + i;
-          ut[r * 128 + j] = u[i] + __bfloat162float(corr[r * 128 + j]);
-        }
+        for (int i = 0; i < 16; ++i) ut[(16 * grp + i) * 128 + j] = u[i] + cr[i];
       }
       if (tid < 128) reinterpret_cast<float *>(rp + rec::GL)[tid] = fegc[tid];
       if (tid < 64) reinterpret_cast<float *>(rp + rec::PD)[tid] = pdiag[tid];
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
-      if (tid == 0) {
-        // A1 = [W ; Q G]: each k-atom holds the 64 W rows, then the 64 Q G rows
+      if (tid == 0) {  // the W rows of A1's two k-atoms
         bulk_store(rp + rec::A1, sm + SM_BKG, 8192);
-        bulk_store(rp + rec::A1 + 8192, sm + SM_QG, 8192);
         bulk_store(rp + rec::A1 + 16384, sm + SM_BKG + 8192, 8192);
-        bulk_store(rp + rec::A1 + 24576, sm + SM_QG + 8192, 8192);
-        bulk_store(rp + rec::KP, sm + SM_KP, 16384);
-        bulk_store(rp + rec::P, sm + SM_POP, 8192);
         bulk_commit();
       }
       cur = nxt;
@@ -1141,6 +1190,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (failed && tid == 0) {  // let in-flight tile loads and MMAs land first
     drain(bar_tma);
     drain(bar_mma);
+    drain(bar_inv);
   }
   if (sN && !kPrepM && !failed) {
     float *dst = sN + (((size_t)n * H + hb) * 128 + j) * 128 + dk0;
