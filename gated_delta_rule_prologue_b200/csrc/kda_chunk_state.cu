@@ -258,6 +258,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 
   uint32_t pa = 0, pk = 0, pm = 0, pm2 = 0;
   bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
+  bool m2_ok = true;    // this thread's waits on the second MMA group completed
   for (int c = c_lo; c < c_hi; ++c) {
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
     if (ckpt) {  // entry state of the chunk, for the backward pass
@@ -267,7 +268,8 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     }
 
     // ---- D1 = [W ; Q G] S ----------------------------------------------------------
-    if (!wait_all(bar_a1, pa, status)) {
+    if (__syncthreads_or(!(mbar_wait(bar_a1, pa) && m2_ok))) {
+      if (tid == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
       failed = true;
       break;
     }
@@ -308,7 +310,6 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       for (int i = 0; i < 32; ++i) {
         y[i] = ut[i] - (y[i] + y2[i]);  // U
         amax = fmaxf(amax, fabsf(y[i]));
-        if (kRole == kOutputs) exch[i * 64 + r] = pd * y[i];  // S operand is dead until the next chunk
       }
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
@@ -318,7 +319,6 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
         st_shared_16(sm + SB_U, mn32_sw64_off(r, x), pack8_f16(f));
       }
       if (!(amax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
-      if (c + 1 < c_hi) fetch_u(c + 1);
       // Only warps 0-1 wrote the U operand and read D1: they alone meet before the
       // issuing thread (warp 0) starts the MMAs that read U and accumulate into D1.
       fence_async_smem();
@@ -344,15 +344,22 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
           report(status, KDA_ERR_DEVICE_TIMEOUT);  // no commit: the wait below times out too
         }
       }
+      // While the second group runs: the token's own term for warps 2-3 (the S operand
+      // is dead until the next chunk) and the next chunk's Ut and <q_r, k_r>.
+      if (kRole == kOutputs) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) exch[i * 64 + r] = pd * y[i];
+        asm volatile("bar.arrive 2, 128;" ::: "memory");  // the exchange is written
+      }
+      if (c + 1 < c_hi) fetch_u(c + 1);
     }
     pk ^= 1;
-    if (!wait_all(bar_m2, pm2, status)) {
-      failed = true;
-      break;
-    }
+    // Each thread waits for the second group by itself; a wait that ran out is acted on
+    // at the next CTA-wide wait (the loop's next tile wait, or the check after the loop).
+    m2_ok = mbar_wait(bar_m2, pm2) && m2_ok;
     pm2 ^= 1;
     tc_fence_after();
-    if (tid == 0 && c + 1 < c_hi) load_kp(c + 1);  // K' and P have been read
+    if (tid == 0 && c + 1 < c_hi && m2_ok) load_kp(c + 1);  // K' and P have been read
 
     // ---- outputs (warps 2-3: TMEM lanes 64..127) and the state update ---------------------
     {
@@ -362,6 +369,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], gl, ds[i]);
       if (c + 1 < c_hi) fetch_gl(c + 1);
     }
+    if (kRole == kOutputs && warp >= 2) asm volatile("bar.sync 2, 128;" ::: "memory");
     if (kRole == kOutputs && warp >= 2 && o) {
       float ov[32], ov2[32];
       tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
@@ -370,7 +378,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 #pragma unroll
       for (int i = 0; i < 32; ++i) ov[i] += ov2[i];
       const int r = tid - 64;
-      if (r < Lc) {
+      if (r < Lc && m2_ok) {
         float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * 128 + slice * 32);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
@@ -390,6 +398,10 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     // the next chunk's wait on its [W; Q G] tile is the barrier before MMA1 reads S
   }
 
+  if (!failed && __syncthreads_or(!m2_ok)) {  // the last chunk's second-group wait
+    if (tid == 0) report(status, KDA_ERR_DEVICE_TIMEOUT);
+    failed = true;
+  }
   if (s_out && !failed) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) s_out[sbase + (size_t)i * 128] = S[i];

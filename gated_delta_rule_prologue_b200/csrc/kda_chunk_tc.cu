@@ -125,9 +125,7 @@ static_assert(SM_T32 + 16384 <= SM_ST && SM_D16 + 16384 <= SM_ST + 32768 &&
               "A-operand reads stay inside shared memory");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) -------------------------------
-constexpr uint32_t TM_G = 0;     // Gram, 96 columns (first of two partial sums)
-constexpr uint32_t TM_G2 = 288;  // second partial sum of the Gram, 96 columns; it lives
-                                 // over O and delta S, which are written only later
+constexpr uint32_t TM_G = 0;     // Gram, 96 columns
 constexpr uint32_t TM_W = 160;   // W^T, 64
 constexpr uint32_t TM_U = 224;   // U^T, 64
 constexpr uint32_t TM_O = 288;   // O^T, 64
@@ -137,8 +135,8 @@ constexpr uint32_t TM_Z = 96;    // Z = A D, 64 columns; later T32 Y
 constexpr uint32_t TM_T2 = 384;  // D Z, 64 (over delta S, written only after P5)
 constexpr uint32_t TM_Y = 448;   // Y = A T32, 64
 constexpr uint32_t TM_COLS = 512;
-static_assert(TM_Z + 64 <= TM_W && TM_G + 96 <= TM_Z && TM_G2 + 96 <= TM_T2 &&
-              TM_Y + 64 <= TM_COLS, "inverse stages overlap a live accumulator");
+static_assert(TM_Z + 64 <= TM_W && TM_G + 96 <= TM_Z && TM_T2 + 64 <= TM_Y &&
+              TM_Y + 64 <= TM_COLS && TM_S + 128 <= TM_COLS, "TMEM column plan");
 
 constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
@@ -648,15 +646,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncthreads();
 
-    // ---- P2: Gram operands (fp32, rounded to tf32), in two halves of key channels; the
-    //      Gram MMA over the first half starts while the second half is being built ------
-    // G over key channels [0, 64) and G2 over [64, 128): two independent accumulators
-    // summed at read-out, 8 K=8 steps each
-    const uint32_t ga_s = smem_u32(sm + SM_GA), gb_s = smem_u32(sm + SM_GB);
-    constexpr uint32_t id_gram = idesc_tf32(128, 96, false, false);
+    // ---- P2: Gram operands (fp32, rounded to tf32) -----------------------------------------
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      const int r = tid >> 3, c8 = 8 * m + (tid & 7), d0 = c8 * 8;
+      const int p = tid + kThreads * m;
+      const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
       float k8[8], q8[8], e8[8];
       ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
       ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
@@ -679,18 +673,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * hf[e]) * hf[e];
       }
       st_tf32x8(sm + SM_GB, 96, 32 + r, c8, ki);
-      fence_async_smem();
-      __syncthreads();
-      // ---- P3: Gram MMA over this half's key channels (tid 0) --------------------------
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t acc = m == 0 ? TM_G : TM_G2;
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---- P3: Gram MMA: one accumulator, 16 K=8 steps --------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ga = smem_u32(sm + SM_GA), gb = smem_u32(sm + SM_GB);
+      constexpr uint32_t id = idesc_tf32(128, 96, false, false);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_tf32(tmem + acc, desc_kmajor(ga_s, 128, 8 * m + ks), desc_kmajor(gb_s, 96, 8 * m + ks),
-                   id_gram, ks > 0);
-        if (m == 1) mma_commit(bar_mma);
-      }
+      for (int ks = 0; ks < 16; ++ks)
+        mma_tf32(tmem + TM_G, desc_kmajor(ga, 128, ks), desc_kmajor(gb, 96, ks), id, ks > 0);
+      mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, mma_par, status)) {
       failed = true;
@@ -708,90 +703,38 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool inv_ok = true;  // warps 0-1: every wait on the inverse's MMA stages completed
     if (tid < kHalf) {
       float *ATd = reinterpret_cast<float *>(sm + SM_ATD);  // [blk][col][row] of A's diagonal blocks
-      // ---- P4b: Gram read-out -> A (fp16 tile, zero on and above the diagonal; its
-      //      diagonal 16x16 blocks also in fp32), strict P operand -------------------------
-      // warp w reads TMEM lanes 32 (w % 4).. and column groups 2 (w / 4) + {0, 1}: the
-      // first half of the columns ([0, 32), i = col) in groups of 8, the second
-      // ([32, 96), i = col - 32) in groups of 16
-      const bool isP = quad >= 2;
-      const int r = 32 * (quad & 1) + lane;
-      const float br = beta_s[r];
-      // one column group: v holds the summed partial Grams of its 8 or 16 columns
-      auto emit = [&](int cg, const float (&v)[16]) {
-        const int i0s = (quad & 1) ? 16 * cg : 8 * cg;
-#pragma unroll
-        for (int g8 = 0; g8 < 2; ++g8) {
-          if (g8 == 1 && !(quad & 1)) break;
-          const int i0 = i0s + 8 * g8;
-          float p8[8];
-          if (!isP) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? br * v[8 * g8 + e] : 0.f;
-            if ((i0 >> 4) == (r >> 4)) {  // a diagonal block: row and columns in one 16-block
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                ATd[((r >> 4) * 16 + ((i0 + e) & 15)) * 16 + (r & 15)] = p8[e];
-            }
-            st_shared_16(sm + SM_A16, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
-          } else {  // every chunk of the strict P tile this thread reads is written
-#pragma unroll
-            for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
-            st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
-          }
-        }
-      };
-      auto load_group = [&](int cg, float (&v)[16], float (&w)[16]) {
-        if (quad & 1) {
-          tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * cg, v);
-          tmem_ld16_nowait(tmem + lane_addr + TM_G2 + 32 + 16 * cg, w);
-        } else {
-          tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * cg, *reinterpret_cast<float(*)[8]>(v));
-          tmem_ld8_nowait(tmem + lane_addr + TM_G2 + 8 * cg, *reinterpret_cast<float(*)[8]>(w));
-        }
-      };
-      const int cg0 = 2 * (warp >> 2);
-      if constexpr (kMode == kPrep) {  // both groups in flight at once (registers allow it)
-        float v[2][16], w[2][16];
-        load_group(cg0, v[0], w[0]);
-        load_group(cg0 + 1, v[1], w[1]);
-        tmem_wait_ld(v[0], v[1]);
-        tmem_wait_ld(w[0], w[1]);
-#pragma unroll
-        for (int gs = 0; gs < 2; ++gs) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[gs][e] += w[gs][e];
-          emit(cg0 + gs, v[gs]);
-        }
-      } else {
-#pragma unroll 1
-        for (int gs = 0; gs < 2; ++gs) {
-          float v[16], w[16];
-          load_group(cg0 + gs, v, w);
-          tmem_wait_ld(v, w);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] += w[e];
-          emit(cg0 + gs, v);
-        }
-      }
-      if (tid < 128) {  // rows 0..31, columns 32..63 of A and P: above the diagonal, not read out
-        const int rz = tid >> 2, cz = 4 + (tid & 3);
-        st_shared_16(sm + SM_POP, kmaj_off(64, rz, cz), make_uint4(0u, 0u, 0u, 0u));
-        st_shared_16(sm + SM_A16, kmaj_off(64, rz, cz), make_uint4(0u, 0u, 0u, 0u));
-      }
-      bar_half();
-
-      // ---- P5: T = (I + A)^{-1} -------------------------------------------------------------
-      // The blocked inverse of a lower triangular matrix.  D = blockdiag of the inverses of
-      // the four 16x16 diagonal blocks of I + A (forward substitution, fp32); then
+      // ---- P4b / P5 (i): warps 0-1 read only the diagonal 16x16 blocks of A out of TMEM and
+      //      run the forward substitution at once, while warps 2-7 read out the whole of A
+      //      (fp16 tile, zero on and above the diagonal) and the strict P operand, then
+      //      zero what the inverse's tiles need zeroed --------------------------------------
+      // TMEM layout of the Gram: rows 0..31 hold columns i in [0, 32) (reference c_A), rows
+      // 32..63 columns i in [0, 64) at TMEM columns 32 + i (reference c_B).
+      // P5: T = (I + A)^{-1}, the blocked inverse of a lower triangular matrix.  D =
+      // blockdiag of the inverses of the four 16x16 diagonal blocks of I + A (forward
+      // substitution, fp32); then
       //   T32 = D - D Z      with Z = A D          (T at the 32x32-block level; only the
       //                                             blocks (1,0) and (3,2) of Z are used)
       //   T   = T32 - T32 Y  with Y = A T32        (only Y's lower-left 32x32 block)
       // The four products are tcgen05 MMAs (M = 128: rows 64..127 are not read) with fp16
       // operands and fp32 accumulation; each piece of T is rounded to fp16 once, for the
-      // W / Ut MMAs.  Warps 0-1 run the substitution and the four stages; warps 2-7 zero
-      // the parts of the 16-bit tiles that nothing else writes, then go on to the join.
+      // W / Ut MMAs.  Warps 0-1 run the substitution and the four stages.
       float amax = 0.f;
-      if (warp < 2) {  // (i) column jj of D_b, swept row by row; fp16 into D16 and T32
+      if (warp < 2) {
+        {  // warp 0: rows 0..31, TMEM columns 0..31; warp 1: rows 32..63, TMEM columns 64..95
+          const int r = 32 * warp + lane;
+          const float br = beta_s[r];
+          float v[32];
+          tmem_ld32(tmem + lane_addr + TM_G + 64 * warp, v);
+          const bool hi = lane >= 16;  // the row's block starts at loaded column 16 * hi
+          const int b = r >> 4, rr = r & 15;
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) {
+            const float g = hi ? v[16 + ii] : v[ii];
+            if (ii < rr) ATd[(b * 16 + ii) * 16 + rr] = br * g;
+          }
+        }
+        asm volatile("bar.sync 3, 64;" ::: "memory");
+        // column jj of D_b, swept row by row; fp16 into D16 and T32
         const int b = tid >> 4, jj = tid & 15, base = 16 * b;
         float acc[16];
 #pragma unroll
@@ -813,9 +756,61 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           *reinterpret_cast<__half *>(sm + SM_T32 + off) = hv;
         }
       } else {
+        // warp 4: A rows 0..31 (quad 0), all four column groups of 8; warp 5: A rows 32..63
+        // (quad 1), all four groups of 16; warps 2, 6 (quad 2) and 3, 7 (quad 3): the P rows,
+        // column groups {0, 1} and {2, 3}
+        const bool isP = quad >= 2;
+        const int r = 32 * (quad & 1) + lane;
+        const float br = beta_s[r];
+        auto emit = [&](int cg, const float (&v)[16]) {
+          const int i0s = (quad & 1) ? 16 * cg : 8 * cg;
+#pragma unroll
+          for (int g8 = 0; g8 < 2; ++g8) {
+            if (g8 == 1 && !(quad & 1)) break;
+            const int i0 = i0s + 8 * g8;
+            float p8[8];
+            if (!isP) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? br * v[8 * g8 + e] : 0.f;
+              st_shared_16(sm + SM_A16, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
+            } else {  // every chunk of the strict P tile this thread reads is written
+#pragma unroll
+              for (int e = 0; e < 8; ++e) p8[e] = i0 + e < r ? v[8 * g8 + e] : 0.f;
+              st_shared_16(sm + SM_POP, kmaj_off(64, r, i0 >> 3), pack8_f16(p8));
+            }
+          }
+        };
+        // two column groups per TMEM wait
+        auto load_group = [&](int cg, float (&v)[16]) {
+          if (quad & 1)
+            tmem_ld16_nowait(tmem + lane_addr + TM_G + 32 + 16 * cg, v);
+          else
+            tmem_ld8_nowait(tmem + lane_addr + TM_G + 8 * cg, *reinterpret_cast<float(*)[8]>(v));
+        };
+        const int ng = warp >= 4 && warp < 6 ? 2 : 1;  // pairs of column groups
+        const int cg0 = warp >= 6 ? 2 : 0;
+#pragma unroll 1
+        for (int pg = 0; pg < ng; ++pg) {
+          const int cga = cg0 + 2 * pg;
+          float v[16], w[16];
+          load_group(cga, v);
+          load_group(cga + 1, w);
+          tmem_wait_ld(v, w);
+          emit(cga, v);
+          emit(cga + 1, w);
+        }
+        const int zt = tid - 64;  // 0..191
+        if (warp >= 6) {  // rows 0..31, columns 32..63 of A and P: above the diagonal, not read out
+          const int t = tid - 192, rz = t >> 1, cz = 4 + 2 * (t & 1);
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            st_shared_16(sm + SM_POP, kmaj_off(64, rz, cz + z), make_uint4(0u, 0u, 0u, 0u));
+            st_shared_16(sm + SM_A16, kmaj_off(64, rz, cz + z), make_uint4(0u, 0u, 0u, 0u));
+          }
+        }
         // D16 and T32 outside the diagonal 16x16 blocks, and all of Zm, start at zero
         // (the diagonal blocks' 16-byte chunks are written whole by the substitution)
-        for (int x = tid - 64; x < 3 * 512; x += kHalf - 64) {
+        for (int x = zt; x < 3 * 512; x += kHalf - 64) {
           const int row = (x & 511) >> 3, c8 = x & 7;
           if (x < 1024 && (c8 >> 1) == (row >> 4)) continue;
           const uint32_t tile = x < 512 ? SM_D16 : (x < 1024 ? SM_T32 : SM_ZM);
