@@ -375,19 +375,25 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
       tmem_ld32_nowait(tmem + lane_addr + TB_D1B, ov2);
       tmem_wait_ld(ov, ov2);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) ov[i] += ov2[i];
       const int r = tid - 64;
-      if (r < Lc && m2_ok) {
-        float4 *dst = reinterpret_cast<float4 *>(o + ((size_t)(t0 + r) * H + h) * 128 + slice * 32);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          float4 f;
-          f.x = scale * (ov[4 * x] + exch[(4 * x) * 64 + r]);
-          f.y = scale * (ov[4 * x + 1] + exch[(4 * x + 1) * 64 + r]);
-          f.z = scale * (ov[4 * x + 2] + exch[(4 * x + 2) * 64 + r]);
-          f.w = scale * (ov[4 * x + 3] + exch[(4 * x + 3) * 64 + r]);
-          dst[x] = f;
+      for (int i = 0; i < 32; ++i) ov[i] = scale * (ov[i] + ov2[i] + exch[i * 64 + r]);
+      // Token r's 32 values go back over the exchange as a row of the read-out tile
+      // (16-byte chunks swizzled by the row), so that the global stores below write whole
+      // 128-byte rows with eight lanes each instead of one lane per row.
+      asm volatile("bar.sync 4, 64;" ::: "memory");  // warps 2-3 have read the exchange
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        reinterpret_cast<float4 *>(exch)[r * 8 + (x ^ (r & 7))] =
+            make_float4(ov[4 * x], ov[4 * x + 1], ov[4 * x + 2], ov[4 * x + 3]);
+      asm volatile("bar.sync 4, 64;" ::: "memory");
+      if (m2_ok) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int id = 64 * k + r, row = id >> 3, x = id & 7;
+          if (row < Lc)
+            __stcs(reinterpret_cast<float4 *>(o + ((size_t)(t0 + row) * H + h) * 128 + slice * 32) + x,
+                   reinterpret_cast<const float4 *>(exch)[row * 8 + (x ^ (row & 7))]);
         }
       }
     }
