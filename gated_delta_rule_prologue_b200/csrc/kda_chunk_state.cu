@@ -57,9 +57,8 @@ constexpr uint32_t SB_S = 57344;         // S slice operand (value-contiguous, 1
 constexpr uint32_t SB_U = 65536;         // U operand (value-contiguous, 64 token rows x 64 B) 4 KB
 constexpr uint32_t SB_BAR = 69632;       // four mbarriers, TMEM slot
 constexpr uint32_t SB_ALLOC = SB_BAR + 64 + 1024;
-// D1 is accumulated as two halves over the key channels (two independent MMA
-// chains), summed at read-out; D2 = K'^T U.
-constexpr uint32_t TB_D1 = 0, TB_D1B = 32, TB_D2 = 64, TB_COLS = 128;
+// D1 is one accumulator over the 128 key channels; D2 = K'^T U.
+constexpr uint32_t TB_D1 = 0, TB_D2 = 64, TB_COLS = 128;
 static_assert(SB_KP + 24576 == SB_S, "K' and P are adjacent");
 
 enum { kOutputs = 0, kTransition = 1, kMap = 2 };
@@ -279,11 +278,8 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       const uint32_t a1 = smem_u32(sm + SB_A1), sop = smem_u32(sm + SB_S);
       constexpr uint32_t id = idesc_fp16(128, 32, false, true);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {  // key channels [0, 64) into D1, [64, 128) into D1B
+      for (int ks = 0; ks < 8; ++ks)  // one accumulator over the 128 key channels
         mma_bf16(tmem + TB_D1, desc_kmajor(a1, 128, ks), desc_mn32_sw64(sop, ks), id, ks > 0);
-        mma_bf16(tmem + TB_D1B, desc_kmajor(a1, 128, ks + 4), desc_mn32_sw64(sop, ks + 4), id,
-                 ks > 0);
-      }
       mma_commit(bar_mma);
     }
     // Only warps 0-1 read this group's result (W S, TMEM lanes 0..63); warps 2-3 go on
@@ -294,21 +290,20 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
       ok1 = mbar_wait(bar_mma, pm);
       if (!ok1) report(status, KDA_ERR_DEVICE_TIMEOUT);
       tc_fence_after();
-      if (tid == 0 && ok1 && c + 1 < c_hi) load_a1(c + 1);  // A1 has been read
+    } else if (tid == 64 && c + 1 < c_hi && mbar_wait(bar_mma, pm)) {
+      load_a1(c + 1);  // A1 has been read (warp 2 is idle until the second group's result)
     }
     pm ^= 1;
 
     // ---- U = Ut - W S (warps 0-1: TMEM lanes 0..63 are the chunk's tokens) -------------
     if (warp < 2) {
-      float y[32], y2[32];
-      tmem_ld32_nowait(tmem + lane_addr + TB_D1, y);
-      tmem_ld32_nowait(tmem + lane_addr + TB_D1B, y2);
-      tmem_wait_ld(y, y2);
+      float y[32];
+      tmem_ld32(tmem + lane_addr + TB_D1, y);
       const int r = tid;
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        y[i] = ut[i] - (y[i] + y2[i]);  // U
+        y[i] = ut[i] - y[i];  // U
         amax = fmaxf(amax, fabsf(y[i]));
       }
 #pragma unroll
@@ -359,7 +354,9 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     m2_ok = mbar_wait(bar_m2, pm2) && m2_ok;
     pm2 ^= 1;
     tc_fence_after();
-    if (tid == 0 && c + 1 < c_hi && m2_ok) load_kp(c + 1);  // K' and P have been read
+    // K' and P have been read: the next chunk's come in.  Warp 1 issues the copy (warp 0's
+    // state update is on the chunk's critical path; warp 1 only waits at the chunk's end).
+    if (tid == 32 && c + 1 < c_hi && m2_ok) load_kp(c + 1);
 
     // ---- outputs (warps 2-3: TMEM lanes 64..127) and the state update ---------------------
     {
@@ -371,13 +368,11 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     }
     if (kRole == kOutputs && warp >= 2) asm volatile("bar.sync 2, 128;" ::: "memory");
     if (kRole == kOutputs && warp >= 2 && o) {
-      float ov[32], ov2[32];
-      tmem_ld32_nowait(tmem + lane_addr + TB_D1, ov);
-      tmem_ld32_nowait(tmem + lane_addr + TB_D1B, ov2);
-      tmem_wait_ld(ov, ov2);
+      float ov[32];
+      tmem_ld32(tmem + lane_addr + TB_D1, ov);
       const int r = tid - 64;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ov[i] = scale * (ov[i] + ov2[i] + exch[i * 64 + r]);
+      for (int i = 0; i < 32; ++i) ov[i] = scale * (ov[i] + exch[i * 64 + r]);
       // Token r's 32 values go back over the exchange as a row of the read-out tile
       // (16-byte chunks swizzled by the row), so that the global stores below write whole
       // 128-byte rows with eight lanes each instead of one lane per row.
