@@ -915,13 +915,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float kk = k8[e], qq = q8[e], vv = v8[e];  // zero past the chunk's end
-          bkg[e] = bt * kk * e8[e] * ec8[e];
+          const float g_abs = e8[e] * ec8[e];               // exp(gamma_r) per channel
+          bkg[e] = (bt * kk) * g_abs;
           bv[e] = bt * vv;
-          qg[e] = qq * e8[e] * ec8[e];
+          qg[e] = qq * g_abs;
           kp[e] = __fdividef(kk, e8[e]) * el8[e];
         }
+        const uint4 bv_h = pack8_f16(bv);
         st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
-        st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), pack8_f16(bv));
+        st_shared_16(sm + SM_BV, mnmaj_off(64, r, c8), bv_h);
         st_shared_16(sm + SM_QG, kmaj_off(64, r, c8), pack8_f16(qg));
         st_shared_16(sm + SM_KP, mnmaj_off(64, r, c8), pack8_f16(kp));
         if constexpr (!kFused) {  // <q_r, k_r> in fp32 over the row's 16 lanes
@@ -936,10 +938,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if constexpr (kPrepM && !kFused) {  // fp32 remainder beta v - f16(beta v), kept as bf16
           float cr[8], bvmax = 0.f;
+          const __half2 *bh = reinterpret_cast<const __half2 *>(&bv_h);  // f16(beta v), packed above
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            cr[e] = bv[e] - __half2float(__float2half_rn(bv[e]));
-            bvmax = fmaxf(bvmax, fabsf(bv[e]));
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __half22float2(bh[e2]);
+            cr[2 * e2] = bv[2 * e2] - f.x;
+            cr[2 * e2 + 1] = bv[2 * e2 + 1] - f.y;
+            bvmax = fmaxf(bvmax, fmaxf(fabsf(bv[2 * e2]), fabsf(bv[2 * e2 + 1])));
           }
           st_shared_16(reinterpret_cast<uint8_t *>(corr), r * 256 + c8 * 16, pack8_bf16(cr));
           if (!(bvmax < 32768.f)) report(status, KDA_ERR_DEVICE_RANGE);
