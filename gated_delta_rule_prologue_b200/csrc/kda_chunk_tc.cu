@@ -25,9 +25,9 @@
 //         A[r,i] = beta_r D_G[r, i] (i < r);  P[r,i] = D_G[64+r, i] (i < r)
 //         P[r,r] = <q_r, k_r> is taken in fp32 from the unscaled tiles.
 //         The Gram operands are fp32 rounded to tf32 (10-bit significand, fp32
-//         range; MMA kind::tf32), over two accumulators (key channels 0..63 and
-//         64..127) summed at read-out.
-//   WY    T = (I + A)^{-1} (fp32, blocked over 16x16 blocks)
+//         range; MMA kind::tf32), one accumulator over the 128 key channels.
+//   WY    T = (I + A)^{-1}: the four 16x16 diagonal blocks inverted by forward
+//         substitution in fp32, the off-diagonal blocks by four fp16 MMA stages
 //         W^T = (beta K G)^T T^T,  Ut^T = (beta V)^T T^T           (G_r = exp(gamma_r))
 //   state U^T = Ut^T - S^T W^T,   O^T = S^T (Q G)^T + U^T P_strict^T
 //         S <- diag(G_last) S + U^T (K * G_last / G)    (value-major registers)
@@ -54,6 +54,20 @@
 #include "kda_tcgen05.cuh"
 
 namespace kda {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
 namespace {
 using namespace tc;
 
@@ -1203,23 +1217,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
-  return fn;
-}
-
 // 3-D map over a [T, H, 128] tensor: box = `rows` tokens x 1 head x 128 channels.
 bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esz, int H, int T,
               unsigned rows = 64) {
-  auto enc = encode_fn();
+  auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
   cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)H * 128 * esz};

@@ -71,8 +71,6 @@ __device__ __forceinline__ void store8(float *p, const float (&in)[8]) {
   reinterpret_cast<float4 *>(p)[1] = make_float4(in[4], in[5], in[6], in[7]);
 }
 
-// SiLU(x) = x * sigmoid(x) with the fast exponential and division intrinsics
-// (a few ulp; for x -> -inf the denominator overflows and the result is 0).
 // Eight consecutive elements kept in their storage type (16 bytes for 16-bit
 // types, 32 bytes for float) until they are used.
 template <typename T> struct Raw8 { uint4 u; };
@@ -127,13 +125,10 @@ __device__ __forceinline__ void store_raw8(float *p, const Raw8<float> &r) {
   reinterpret_cast<float4 *>(p)[1] = r.b;
 }
 
+// SiLU(x) = x * sigmoid(x) with the fast exponential and division intrinsics
+// (a few ulp; for x -> -inf the denominator overflows and the result is 0).
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
-// ---------------------------------------------------------------------------
-// Device status word (one per device, allocated by the host layer)
-// ---------------------------------------------------------------------------
-
-// Record the first fault code; later faults keep the first one.
 // Bounded log-decay gate ("Kimi K3的线性注意力：从源码看懂KDA如何更新记忆", 彩蛋, the
 // gate.py excerpt): g = lb * sigmoid(a * (graw + bias)) with a = exp(A_log[h]),
 // bias = dt_bias[h][channel] and lb the lower bound (-5 in K3), in fp32.
@@ -142,6 +137,11 @@ __device__ __forceinline__ float bounded_gate(float graw, float a, float bias, f
   return lb * __fdividef(1.f, 1.f + __expf(-z));  // 1/(1 + inf) = 0 for very negative z
 }
 
+// ---------------------------------------------------------------------------
+// Device status word (one per device, a file-scope device variable)
+// ---------------------------------------------------------------------------
+
+// Record the first fault code; later faults keep the first one.
 __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }

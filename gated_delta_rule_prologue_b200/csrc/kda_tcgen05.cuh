@@ -23,9 +23,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kda_common.cuh"
 
 namespace kda {
+
+// The driver's tensor-map encoder (cuTensorMapEncodeTiled), looked up once through
+// the runtime; null if the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 namespace tc {
 
 // ---------------------------------------------------------------------------
@@ -117,6 +125,15 @@ __device__ __forceinline__ void drain(uint64_t *bar, uint64_t limit_ns = 1000000
 
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar,
