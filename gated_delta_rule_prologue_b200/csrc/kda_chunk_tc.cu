@@ -519,65 +519,91 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int c8 = tid & 15, d0 = c8 * 8, r0 = 2 * (tid >> 4);
       uint4 packed[3][2];      // q, k, v of rows r0, r0+1 as fp16, written after the barrier
       uint4 corr_pk[2];        // beta*v - f16(beta*f16(v)) as bf16
-      float q32[2][8];         // q in fp32 until k is known
+      float2 q32[2][4];        // q in fp32 (channel pairs) until k is known
       float qk[2] = {0.f, 0.f};
       float vmax = 0.f;
+      // The same arithmetic as the standalone prologue: channel pairs on the packed fp32
+      // instructions, SiLU on the approximate exponential and reciprocal.
 #pragma unroll
       for (int p = 0; p < 3; ++p) {
         const uint8_t *tile = sm + (p == 0 ? SM_Q : (p == 1 ? SM_K : SM_V));
-        float w8[4][8];  // taps x 8 channels
+        float2 w2[4][4];  // taps x 4 channel pairs
 #pragma unroll
-        for (int tp = 0; tp < 4; ++tp) ld8_f32(wconv + (p * 4 + tp) * 128 + d0, w8[tp]);
-        uint4 xraw[5];  // raw rows r0-3 .. r0+1, still packed
+        for (int tp = 0; tp < 4; ++tp) {
+          const float4 *src = reinterpret_cast<const float4 *>(wconv + (p * 4 + tp) * 128 + d0);
+          const float4 lo = src[0], hi = src[1];
+          w2[tp][0] = make_float2(lo.x, lo.y);
+          w2[tp][1] = make_float2(lo.z, lo.w);
+          w2[tp][2] = make_float2(hi.x, hi.y);
+          w2[tp][3] = make_float2(hi.z, hi.w);
+        }
+        // Rows r0-3 .. r0+1 in order, each widened once and applied to both outputs (tap t - q2
+        // of output row r0 + q2), so each output sees its taps in the order w0, w1, w2, w3.
+        float2 acc[2][4];
 #pragma unroll
         for (int t = 0; t < 5; ++t) {
           const int rr = r0 - 3 + t;
-          xraw[t] = *reinterpret_cast<const uint4 *>(
-              rr >= 0 ? tile + rr * 256 + c8 * 16
-                      : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + rr) * 128) + c8 * 16);
+          float2 xr[4];
+          widen_pairs(*reinterpret_cast<const uint4 *>(
+                          rr >= 0 ? tile + rr * 256 + c8 * 16
+                                  : reinterpret_cast<const uint8_t *>(hcur + (p * 3 + 3 + rr) * 128) +
+                                        c8 * 16),
+                      xr, Tin());
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const int tap = t - q2;
+            if (tap < 0 || tap > 3) continue;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              acc[q2][i] = tap == 0 ? __fmul2_rn(w2[0][i], xr[i])
+                                    : __ffma2_rn(w2[tap][i], xr[i], acc[q2][i]);
+          }
         }
 
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-          float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float2 y[4];
+          float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int tp = 0; tp < 4; ++tp) {
-            float xv[8];
-            unpack8(xraw[q2 + tp], xv, Tin());
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = fmaf(w8[tp][e], xv[e], y[e]);
-          }
-          float ss = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            y[e] = silu(y[e]);
-            ss = fmaf(y[e], y[e], ss);
+          for (int i = 0; i < 4; ++i) {
+            y[i] = silu_pair(acc[q2][i]);
+            ss2 = __ffma2_rn(y[i], y[i], ss2);
           }
           if (p < 2) {
+            float ss = ss2.x + ss2.y;
             ss += __shfl_xor_sync(0xffffffffu, ss, 8);
             ss += __shfl_xor_sync(0xffffffffu, ss, 4);
             ss += __shfl_xor_sync(0xffffffffu, ss, 2);
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          }
-          const float sc = p < 2 ? rsqrtf(ss + 1e-6f) : 1.f;
-          const bool valid = r0 + q2 < Lc;
+            const float sc = rsqrtf(ss + 1e-6f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = valid ? y[e] * sc : 0.f;
-          packed[p][q2] = pack8_in<Tact>(y);
+            for (int i = 0; i < 4; ++i) y[i] = __fmul2_rn(y[i], make_float2(sc, sc));
+          }
+          if (r0 + q2 >= Lc) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[i] = make_float2(0.f, 0.f);
+          }
+          packed[p][q2] = pack_pairs(y, Tact());
           if (p == 0) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) q32[q2][e] = y[e];
+            for (int i = 0; i < 4; ++i) q32[q2][i] = y[i];
           } else if (p == 1) {
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qk[q2] = fmaf(q32[q2][e], y[e], qk[q2]);
+            for (int i = 0; i < 4; ++i) acc = __ffma2_rn(q32[q2][i], y[i], acc);
+            qk[q2] = acc.x + acc.y;
           } else {
             const float bt = beta_s[r0 + q2];
             float cr[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              vmax = fmaxf(vmax, fabsf(y[e]));
-              const float stored = to_f32(from_f32<Tact>(y[e]));
-              cr[e] = bt * y[e] - __half2float(__float2half_rn(bt * stored));
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const float ye = hf ? y[i].y : y[i].x;
+                vmax = fmaxf(vmax, fabsf(ye));
+                const float stored = to_f32(from_f32<Tact>(ye));
+                cr[2 * i + hf] = bt * ye - __half2float(__float2half_rn(bt * stored));
+              }
             }
             corr_pk[q2] = pack8_bf16(cr);
           }

@@ -129,6 +129,72 @@ __device__ __forceinline__ void store_raw8(float *p, const Raw8<float> &r) {
 // (a few ulp; for x -> -inf the denominator overflows and the result is 0).
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
+// ---------------------------------------------------------------------------
+// Channel pairs on the packed fp32 instructions (one issue for two lanes, each
+// lane rounded as its scalar operation)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Four channel pairs of a 16-byte segment of 16-bit values.
+__device__ __forceinline__ void widen_pairs(const uint4 &u, float2 (&f)[4], __nv_bfloat16) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+__device__ __forceinline__ void widen_pairs(const uint4 &u, float2 (&f)[4], __half) {
+  const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = __half22float2(h[i]);
+}
+__device__ __forceinline__ uint4 pack_pairs(const float2 (&y)[4], __half) {
+  uint4 u;
+  __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(y[i].x, y[i].y);
+  return u;
+}
+__device__ __forceinline__ uint4 pack_pairs(const float2 (&y)[4], __nv_bfloat16) {
+  uint4 u;
+  __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(y[i].x, y[i].y);
+  return u;
+}
+
+// SiLU of a channel pair from its definition: a * sigma(a) with sigma(a) = 1 / (1 +
+// 2^(-a log2 e)) on the hardware's approximate base-2 exponential and reciprocal
+// (PTX ex2.approx, rcp.approx; relative errors of a few 2^-23).  For a -> -inf the
+// exponential overflows to +inf and the result is -0.  conv4_silu_pair first applies
+// the width-4 causal conv, taps w0..w3 on x[t-3], x[t-2], x[t-1], x[t], in that order.
+__device__ __forceinline__ float2 silu_pair(float2 a) {
+  float2 d = __fmul2_rn(a, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  d.x = ex2_approx(d.x);
+  d.y = ex2_approx(d.y);
+  d = __fadd2_rn(d, make_float2(1.f, 1.f));
+  d.x = rcp_approx(d.x);
+  d.y = rcp_approx(d.y);
+  return __fmul2_rn(a, d);
+}
+__device__ __forceinline__ float2 conv4_silu_pair(float2 w0, float2 w1, float2 w2, float2 w3,
+                                                  float2 x3, float2 x2, float2 x1, float2 x0) {
+  float2 a = __fmul2_rn(w0, x3);
+  a = __ffma2_rn(w1, x2, a);
+  a = __ffma2_rn(w2, x1, a);
+  a = __ffma2_rn(w3, x0, a);
+  return silu_pair(a);
+}
+
 // Bounded log-decay gate ("Kimi K3的线性注意力：从源码看懂KDA如何更新记忆", 彩蛋, the
 // gate.py excerpt): g = lb * sigmoid(a * (graw + bias)) with a = exp(A_log[h]),
 // bias = dt_bias[h][channel] and lb the lower bound (-5 in K3), in fp32.

@@ -207,46 +207,11 @@ constexpr int kStagedSmem = kStagedWarps * kStages * (kBoxBytes + 8);
 static_assert(kStagedTokens % kBoxTokens == 0 && kBoxTokens % 3 == 0 && kBoxBytes % 128 == 0,
               "box plan");
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Four channel pairs of a 16-byte row segment.
-__device__ __forceinline__ void widen_pairs(const uint4 &u, float2 (&f)[4], __nv_bfloat16) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-}
-__device__ __forceinline__ void widen_pairs(const uint4 &u, float2 (&f)[4], __half) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __half2 h;
-    memcpy(&h, &w[i], 4);
-    f[i] = __half22float2(h);
-  }
-}
 __device__ __forceinline__ void store_pairs(__half *p, const float2 (&y)[4]) {
-  uint4 u;
-  __half2 *h = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(y[i].x, y[i].y);
-  *reinterpret_cast<uint4 *>(p) = u;
+  *reinterpret_cast<uint4 *>(p) = pack_pairs(y, __half{});
 }
 __device__ __forceinline__ void store_pairs(__nv_bfloat16 *p, const float2 (&y)[4]) {
-  uint4 u;
-  __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(y[i].x, y[i].y);
-  *reinterpret_cast<uint4 *>(p) = u;
+  *reinterpret_cast<uint4 *>(p) = pack_pairs(y, __nv_bfloat16{});
 }
 __device__ __forceinline__ void store_pairs(float *p, const float2 (&y)[4]) {
   reinterpret_cast<float4 *>(p)[0] = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
@@ -262,22 +227,10 @@ __device__ __forceinline__ void conv_silu_norm_pairs(const float2 (&w)[4][4],
                                                      const float2 (&h1)[4],
                                                      const float2 (&f)[4], bool norm,
                                                      float2 (&y)[4]) {
-  const float2 neg_log2e = make_float2(-1.4426950408889634f, -1.4426950408889634f);
-  const float2 one = make_float2(1.f, 1.f);
   float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float2 a = __fmul2_rn(w[0][i], h3[i]);
-    a = __ffma2_rn(w[1][i], h2[i], a);
-    a = __ffma2_rn(w[2][i], h1[i], a);
-    a = __ffma2_rn(w[3][i], f[i], a);
-    float2 d = __fmul2_rn(a, neg_log2e);
-    d.x = ex2_approx(d.x);
-    d.y = ex2_approx(d.y);
-    d = __fadd2_rn(d, one);
-    d.x = rcp_approx(d.x);
-    d.y = rcp_approx(d.y);
-    y[i] = __fmul2_rn(a, d);
+    y[i] = conv4_silu_pair(w[0][i], w[1][i], w[2][i], w[3][i], h3[i], h2[i], h1[i], f[i]);
     ss2 = __ffma2_rn(y[i], y[i], ss2);
   }
   float ss = ss2.x + ss2.y;
