@@ -5,7 +5,8 @@ and the current CUDA stream of ``torch`` to the C ABI declared in
 ``include/kda.h`` and raises :class:`KdaError` on a non-OK status.  All work
 runs in the library's CUDA kernels; there is no other implementation behind
 these names, and importing fails loudly when ``libkda.so`` has not been built
-(``python -m gated_delta_rule_prologue_b200.build``).
+(``python -m gated_delta_rule_prologue_b200.build``).  With the environment variable
+``KDA_LIB=debug`` the bounds-checked build ``libkda_debug.so`` is loaded instead.
 
 Tensor conventions (all contiguous, on the current CUDA device):
   q, k, v              [T, H, D]       float32, bfloat16 or float16
@@ -35,6 +36,8 @@ __all__ = [
     "kda_prologue_chunk_fwd",
     "kda_get_device_status",
     "kda_selftest_wait_timeout",
+    "kda_selftest_bounds",
+    "kda_debug_build",
     "kda_version",
     "KDA_OK",
     "KDA_ERR_INVALID_ARG",
@@ -45,7 +48,10 @@ __all__ = [
     "KDA_ERR_DEVICE_RANGE",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+# KDA_LIB=debug selects the bounds-checked build (libkda_debug.so, built by
+# ``python -m gated_delta_rule_prologue_b200.build --debug``); anything else, the release build.
+_LIB_NAME = "libkda_debug.so" if os.environ.get("KDA_LIB") == "debug" else "libkda.so"
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIB_NAME)
 
 KDA_OK = 0
 KDA_ERR_INVALID_ARG = 1
@@ -111,6 +117,9 @@ lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _v
                                        _i, _i, _vp, _vp, _vp]
 lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
 lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
+lib.kda_selftest_bounds.argtypes = [_i, _vp]
+lib.kda_debug_build.argtypes = []
+lib.kda_debug_build.restype = ctypes.c_int
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
             lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
             lib.kda_state_compose,
@@ -118,7 +127,7 @@ for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_c
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
             lib.kda_output_epilogue,
             lib.kda_prologue_chunk_fwd, lib.kda_get_device_status,
-            lib.kda_selftest_wait_timeout):
+            lib.kda_selftest_wait_timeout, lib.kda_selftest_bounds):
     _fn.restype = ctypes.c_int
 lib.kda_last_error.restype = ctypes.c_char_p
 lib.kda_last_error.argtypes = []
@@ -181,6 +190,17 @@ def kda_selftest_wait_timeout(limit_us: int = 1000, stream=None):
     microseconds; it records KDA_ERR_DEVICE_TIMEOUT in the status word and
     returns without faulting (the failure path of every tensor-core kernel)."""
     _check(lib.kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def kda_debug_build() -> bool:
+    """True when the loaded library is the bounds-checked build (KDA_LIB=debug)."""
+    return bool(lib.kda_debug_build())
+
+
+def kda_selftest_bounds(index: int, stream=None):
+    """Debug build only: one checked write of a four-slot device probe at ``index``;
+    outside [0, 4) it records KDA_ERR_DEVICE_BOUNDS and skips the write."""
+    _check(lib.kda_selftest_bounds(int(index), _stream(stream)))
 
 
 def kda_prologue(x, conv_w, q, k, v, *, H: int, D: int, cache_in=None, cache_out=None,

@@ -124,6 +124,20 @@ kda_status kda_selftest_wait_timeout(unsigned limit_us, kda_stream_t stream) {
   return KDA_OK;
 }
 
+int kda_debug_build(void) { return kda::kDebugChecks ? 1 : 0; }
+
+kda_status kda_selftest_bounds(int index, kda_stream_t stream) {
+  if (!kda::kDebugChecks)
+    return fail(KDA_ERR_UNSUPPORTED,
+                "kda_selftest_bounds: a release build (the index checks are compiled out)");
+  int *status = nullptr;
+  kda_status st = device_status_word(&status);
+  if (st != KDA_OK) return st;
+  const cudaError_t e = kda::launch_bounds_probe(index, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_bounds launch");
+  return KDA_OK;
+}
+
 kda_status kda_get_device_status(int *code) {
   KDA_REQUIRE(code != nullptr, "code is NULL");
   int *word = nullptr;

@@ -85,6 +85,12 @@ chunk_bwd_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict
     cbase = cprefix[n];
     nch = cprefix[n + 1] - cbase;
   }
+  {  // debug builds: the chain's chunks lie inside the workspace and its tokens inside T
+    const long long cap = rec::chunk_capacity(N, T);
+    if (nch > 0 && !(in_range(status, cbase, cap) && in_range(status, cbase + nch - 1, cap) &&
+                     in_range(status, eos - 1, T)))
+      return;
+  }
   if (warp == 0) tmem_alloc(slot, TB_COLS);
   if (tid == 0) {
     mbar_init(bar_a1, 1);
@@ -386,6 +392,9 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     seq_bounds(cu, n, T, status, bos, eos);
     const int t0 = bos + 64 * c, Lc = min(64, eos - t0);
     if (Lc <= 0) continue;
+    // debug builds: the chunk's record and checkpoints, and its tokens, are in range
+    if (!in_range(status, ci, rec::chunk_capacity(N, T)) || !in_range(status, t0 + Lc - 1, T))
+      continue;
     const int nsub = (Lc + kSub - 1) / kSub;
     const size_t rec_idx = (size_t)ci * H + h;
     const float *S0 = ckpt + rec_idx * (128 * 128);

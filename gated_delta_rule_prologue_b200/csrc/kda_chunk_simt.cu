@@ -66,6 +66,7 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
   const int j0 = slice * DVS;
   int bos, eos;
   seq_bounds(cu, n, T, status, bos, eos);
+  if (!in_range(status, n, N) || (eos > bos && !in_range(status, eos - 1, T))) return;
 
   // Entry state slice: Ss[d][j] = S[d][j0 + j] = state[n][h][j0 + j][d].
   for (int idx = tid; idx < D * DVS; idx += kThreads) {

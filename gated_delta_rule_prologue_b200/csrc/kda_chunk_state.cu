@@ -134,6 +134,13 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     cbase = cprefix[n];
     if (L == 0) c_hi = cprefix[n + 1] - cbase;
   }
+  {  // debug builds: the chain's sequence, chunks and segment slots lie inside the workspace
+    const long long cap = rec::chunk_capacity(N, T);
+    if (!in_range(status, n, N) ||
+        (c_hi > c_lo && !(in_range(status, cbase + c_lo, cap) && in_range(status, cbase + c_hi - 1, cap))) ||
+        (L > 0 && !in_range(status, s, rec::segment_capacity(N, T, L))))
+      return;
+  }
   // Where the state comes from and goes to.  Slot (s, h, kind) of the segment area.
   auto seg_slot = [&](int seg, int kind) -> float * {
     return segbuf + (((size_t)seg * H + h) * 3 + kind) * (128 * 128);
@@ -386,7 +393,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int id = 64 * k + r, row = id >> 3, x = id & 7;
-          if (row < Lc)
+          if (row < Lc && in_range(status, t0 + row, T))
             __stcs(reinterpret_cast<float4 *>(o + ((size_t)(t0 + row) * H + h) * 128 + slice * 32) + x,
                    reinterpret_cast<const float4 *>(exch)[row * 8 + (x ^ (row & 7))]);
         }
@@ -523,6 +530,8 @@ state_scan_kernel(const uint8_t *__restrict__ ws, int N, int T, int H, int *stat
   const int32_t *sprefix = reinterpret_cast<const int32_t *>(ws) + (N + 1);
   const int s0 = sprefix[n], G = sprefix[n + 1] - s0;
   if (G <= 2) return;
+  // debug builds: the sequence's segments are among the batch's sprefix[N]
+  if (!in_range(status, s0, sprefix[N]) || !in_range(status, s0 + G - 1, sprefix[N])) return;
   float *segbuf = reinterpret_cast<float *>(const_cast<uint8_t *>(ws) +
                                             rec::segment_area_offset(N, T, H));
   auto slot = [&](int seg, int kind) -> float * {

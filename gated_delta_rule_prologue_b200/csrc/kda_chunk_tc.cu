@@ -325,7 +325,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       w.n = lo;
       w.bos = sb;
       w.eos = se;
-      w.ok = w.Lc > 0;
+      w.ok = w.Lc > 0 && in_range(status, w.n, N) &&
+             in_range(status, w.ci, rec::chunk_capacity(N, T)) &&
+             in_range(status, w.t0 + w.Lc - 1, T);
     } else {
       w.ok = it < nchunks;
       w.ci = it;
@@ -335,6 +337,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       w.n = n;
       w.bos = bos;
       w.eos = eos;
+      w.ok = w.ok && in_range(status, w.t0 + w.Lc - 1, T);
     }
     return w;
   };

@@ -212,6 +212,29 @@ __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Debug builds (compiled with -DKDA_DEBUG, the library libkda_debug.so): every
+// index a kernel derives from the call's data or arithmetic (sequence, token,
+// chunk, record, segment, state and cache indices) is checked against its extent
+// before the access that uses it.  An index out of range records
+// KDA_ERR_DEVICE_BOUNDS and the access (or the whole item, where the index is
+// the same for the CTA) is skipped, so the fault shows in the status word and
+// never as a memory fault.  In release builds the checks compile to nothing.
+#ifdef KDA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __forceinline__ bool in_range(int *status, long long i, long long n) {
+  if constexpr (kDebugChecks) {
+    if (i < 0 || i >= n) {
+      if (status) atomicCAS(status, 0, KDA_ERR_DEVICE_BOUNDS);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Sequence bounds from cu_seqlens with device-side validation: a malformed
 // entry (decreasing or outside [0, T]) is clamped and recorded.
 __device__ __forceinline__ void seq_bounds(const int32_t *cu, int n, int T, int *status,
@@ -258,6 +281,9 @@ cudaError_t status_word_address(int **out);
 cudaError_t static_scratch_address(void **out);
 // One CTA whose bounded mbarrier wait runs out after limit_us (kda_selftest.cu).
 cudaError_t launch_wait_timeout(unsigned limit_us, int *status, cudaStream_t s);
+// One checked write of a four-slot probe array at `index` (debug builds only;
+// cudaErrorNotSupported in release builds).
+cudaError_t launch_bounds_probe(int index, int *status, cudaStream_t s);
 cudaError_t launch_prologue(const void *x, const float *w, const void *cache_in, void *cache_out,
                             const int32_t *cu, int N, int T, int H, int D, kda_dtype dt,
                             kda_dtype out_dt, void *q, void *k, void *v, int *status,

@@ -101,6 +101,7 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
   }
 
   int n = seq_of_token(cu, N, t0);
+  if (!in_range(status, n, N)) return;
   int bos, eos;
   seq_bounds(cu, n, T, status, bos, eos);
   while (t0 >= eos && n < N - 1) {  // skip empty sequences ending at t0
@@ -118,11 +119,11 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
     for (int j = 0; j < 3; ++j) {
       const int tt = t0 - 3 + j;
       if (tt >= bos) {
-        hv[j] = load_or_zero(x + (size_t)tt * C + c0, active);
+        hv[j] = load_or_zero(x + (size_t)tt * C + c0, active && in_range(status, tt, T));
       } else {
         const int r = 3 - (bos - tt);  // cache row (0 = oldest)
         hv[j] = load_or_zero(cache_in + ((size_t)n * 3 + r) * C + c0,
-                             active && cache_in != nullptr);
+                             active && cache_in != nullptr && in_range(status, r, 3));
       }
     }
     hm3 = hv[0];
@@ -162,7 +163,7 @@ prologue_kernel(const Tin *__restrict__ x, const float *__restrict__ w,
       widen8(xr[i], f);
       conv_silu_norm<G>(wt, fm3, fm2, fm1, f, p < 2, y);
       if (active) {
-        store8(out + ((size_t)t * H + h) * D + d0, y);
+        if (in_range(status, t, T)) store8(out + ((size_t)t * H + h) * D + d0, y);
         if (cache_out != nullptr && t == eos - 1) {
           store_raw8(cache_out + ((size_t)n * 3 + 0) * C + c0, hm2);
           store_raw8(cache_out + ((size_t)n * 3 + 1) * C + c0, hm1);
@@ -315,6 +316,7 @@ prologue_staged_kernel(const __grid_constant__ CUtensorMap tm_x, const Tin *__re
   }
 
   int n = seq_of_token(cu, N, t0);
+  if (!in_range(status, n, N)) n = 0;  // the ring is already loading: no early exit
   int bos, eos;
   seq_bounds(cu, n, T, status, bos, eos);
   while (t0 >= eos && n < N - 1) {
@@ -323,9 +325,9 @@ prologue_staged_kernel(const __grid_constant__ CUtensorMap tm_x, const Tin *__re
   }
   // Raw row tt of the current sequence (tt >= bos - 3): from x, or from the cache before bos.
   auto raw_row = [&](int tt) {
-    if (tt >= bos) return load_or_zero(x + (size_t)tt * C + c0, active);
+    if (tt >= bos) return load_or_zero(x + (size_t)tt * C + c0, active && in_range(status, tt, T));
     return load_or_zero(cache_in + ((size_t)n * 3 + (3 - (bos - tt))) * C + c0,
-                        active && cache_in != nullptr);
+                        active && cache_in != nullptr && in_range(status, bos - tt - 1, 3));
   };
 
   // History ring: before token i of a box, slot i % 3 holds x[t-3], (i+1) % 3 x[t-2] and
@@ -351,6 +353,7 @@ prologue_staged_kernel(const __grid_constant__ CUtensorMap tm_x, const Tin *__re
     const uint8_t *box = ring + slot * kBoxBytes + lane * 16;
     const int tb = t0 + j * kBoxTokens;
     Tout *ob = out + ((size_t)tb * H + h) * D + d0;
+    const bool box_ok = in_range(status, tb, T);
     if (tb + kBoxTokens < eos && tb + kBoxTokens <= t_end) {
       // Inside one sequence, not its last token, and inside the CTA's range.
 #pragma unroll
@@ -358,7 +361,7 @@ prologue_staged_kernel(const __grid_constant__ CUtensorMap tm_x, const Tin *__re
         float2 f[4], y[4];
         widen_pairs(*reinterpret_cast<const uint4 *>(box + i * (kWarpChannels * 2)), f, Tin{});
         conv_silu_norm_pairs<G>(wt, hr[i % 3], hr[(i + 1) % 3], hr[(i + 2) % 3], f, norm, y);
-        if (active) store_pairs(ob + (size_t)i * HD, y);
+        if (active && box_ok) store_pairs(ob + (size_t)i * HD, y);
 #pragma unroll
         for (int e = 0; e < 4; ++e) hr[i % 3][e] = f[e];
       }
@@ -382,7 +385,7 @@ prologue_staged_kernel(const __grid_constant__ CUtensorMap tm_x, const Tin *__re
         float2 f[4], y[4];
         widen_pairs(xu, f, Tin{});
         conv_silu_norm_pairs<G>(wt, hr[i % 3], hr[(i + 1) % 3], hr[(i + 2) % 3], f, norm, y);
-        if (active) {
+        if (active && box_ok) {
           store_pairs(ob + (size_t)i * HD, y);
           if (cache_out != nullptr && t == eos - 1) {
             store_raw8(cache_out + ((size_t)n * 3 + 0) * C + c0, raw_row(t - 2));

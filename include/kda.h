@@ -493,6 +493,28 @@ kda_status kda_get_device_status(int *code);
  */
 kda_status kda_selftest_wait_timeout(unsigned limit_us, kda_stream_t stream);
 
+/*
+ * kda_debug_build -- 1 for the bounds-checked build of this library
+ * (libkda_debug.so, compiled with KDA_DEBUG), 0 for the release build.  In the
+ * debug build every kernel checks the indices it derives from the call's data
+ * and arithmetic (sequence, token, chunk, record, segment, state and conv-cache
+ * indices) against their extents before the access that uses them; an index
+ * out of range records KDA_ERR_DEVICE_BOUNDS in the status word and the access
+ * (or the kernel's whole item, where the index is the same for the CTA) is
+ * skipped instead of made.  Results of valid calls are the same in both builds.
+ */
+int kda_debug_build(void);
+
+/*
+ * kda_selftest_bounds -- exercise the debug build's index check.  One thread
+ * writes slot `index` of a four-slot device probe array through the check the
+ * kernels use: in the debug build an index outside [0, 4) records
+ * KDA_ERR_DEVICE_BOUNDS and skips the write.  KDA_ERR_UNSUPPORTED in the
+ * release build, where the check is compiled out (nothing is launched).
+ * Asynchronous on `stream`; read the outcome with kda_get_device_status.
+ */
+kda_status kda_selftest_bounds(int index, kda_stream_t stream);
+
 /* Message for the last non-OK return on the calling thread (never NULL). */
 const char *kda_last_error(void);
 

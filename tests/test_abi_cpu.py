@@ -22,7 +22,7 @@ def kda():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:kda_status|const char \*|size_t)\s*(kda_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:kda_status|const char \*|size_t|int)\s*(kda_\w+)\s*\(",
                                  text, re.M)))
 
 
@@ -42,6 +42,27 @@ def test_library_exports_every_declared_symbol(kda):
     assert not missing, missing
     for n in declared_functions():
         assert hasattr(kda.lib, n)
+
+
+def _exported(path):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    return {n for n in re.findall(r"\bT (\w+)$", out, re.M) if n.startswith("kda_")}
+
+
+def test_debug_library_matches_the_release_entry_points(kda):
+    """libkda_debug.so (KDA_DEBUG) exports the same C ABI and says which build it is;
+    the release build refuses the index-check self-test without touching a device."""
+    dbg_path = os.path.join(ROOT, "gated_delta_rule_prologue_b200", "libkda_debug.so")
+    assert _exported(dbg_path) == _exported(kda.LIB_PATH)
+    dbg = ctypes.CDLL(dbg_path)
+    for L in (dbg, kda.lib):
+        L.kda_debug_build.restype = ctypes.c_int
+        L.kda_debug_build.argtypes = []
+    assert dbg.kda_debug_build() == 1
+    assert kda.lib.kda_debug_build() == 0
+    assert kda.lib.kda_selftest_bounds(4, None) == kda.KDA_ERR_UNSUPPORTED
+    assert b"release build" in kda.lib.kda_last_error()
 
 
 def test_no_oracle_or_fallback_in_product_package():
