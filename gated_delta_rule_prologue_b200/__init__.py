@@ -32,6 +32,7 @@ __all__ = [
     "lib",
     "kda_prologue",
     "kda_chunk_fwd",
+    "kda_chunk_fwd_windowed_workspace_bytes",
     "kda_decode_step",
     "kda_prologue_chunk_fwd",
     "kda_get_device_status",
@@ -112,6 +113,10 @@ lib.kda_chunk_fwd_segment_chunks.argtypes = [_i, _i, _i]
 lib.kda_chunk_fwd_segment_chunks.restype = ctypes.c_int
 lib.kda_chunk_fwd_segmented_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
                                            _i, _i, _i, _vp, _vp, _i, _vp, ctypes.c_size_t, _vp]
+lib.kda_chunk_fwd_windowed_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
+                                          _i, _i, _i, _vp, _vp, _i, _vp, ctypes.c_size_t, _vp]
+lib.kda_chunk_fwd_windowed_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+lib.kda_chunk_fwd_windowed_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
                                        _i, _i, _vp, _vp, _vp]
@@ -121,7 +126,8 @@ lib.kda_selftest_bounds.argtypes = [_i, _vp]
 lib.kda_debug_build.argtypes = []
 lib.kda_debug_build.restype = ctypes.c_int
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
-            lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
+            lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_fwd_windowed_ws,
+            lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
             lib.kda_state_compose,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
             lib.kda_prologue_chunk_fwd_gated_ws, lib.kda_decode_step_gated,
@@ -241,7 +247,7 @@ def kda_chunk_fwd_segmented_workspace_bytes(N: int, T: int, H: int, Dk: int, Dv:
 
 def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None,
                   final_state=None, cu_seqlens=None, chunk: int = 64, workspace="auto",
-                  segment_chunks=None, stream=None):
+                  segment_chunks=None, window_chunks=None, stream=None):
     """Chunkwise prefill: writes ``o`` [T, H, Dv] and optionally ``final_state``.
 
     ``workspace``: ``"auto"`` allocates the two-pass path's scratch from
@@ -250,7 +256,13 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
     ``segment_chunks``: ``None`` lets the library pick the state pass's segment
     length; an int (0: whole sequences) calls ``kda_chunk_fwd_segmented_ws``
     with it (workspace sized by :func:`kda_chunk_fwd_segmented_workspace_bytes`).
+    ``window_chunks``: an int >= 1 calls ``kda_chunk_fwd_windowed_ws``: the passes run
+    one window of that many chunk numbers at a time, so the workspace (sized by
+    :func:`kda_chunk_fwd_windowed_workspace_bytes`) does not grow with T.
     """
+    if window_chunks is not None:
+        return _chunk_fwd_windowed(q, k, v, g, beta, o, scale, initial_state, final_state,
+                                   cu_seqlens, chunk, workspace, int(window_chunks), stream)
     if segment_chunks is not None:
         return _chunk_fwd_segmented(q, k, v, g, beta, o, scale, initial_state, final_state,
                                     cu_seqlens, chunk, workspace, int(segment_chunks), stream)
@@ -278,6 +290,36 @@ def kda_chunk_fwd(q, k, v, g, beta, o, *, scale: float = 1.0, initial_state=None
                                 _ptr(initial_state), _ptr(cu_seqlens), N, T, H, Dk, Dv, chunk,
                                 _dtype(q), _ptr(o), _ptr(final_state), _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
+
+
+def kda_chunk_fwd_windowed_workspace_bytes(N, T, H, Dk, Dv, chunk, dtype, window_chunks) -> int:
+    return int(lib.kda_chunk_fwd_windowed_workspace_bytes(N, T, H, Dk, Dv, chunk,
+                                                          _DTYPES[dtype], window_chunks))
+
+
+def _chunk_fwd_windowed(q, k, v, g, beta, o, scale, initial_state, final_state, cu_seqlens,
+                        chunk, workspace, window_chunks, stream):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((o, "o"), (g, "g"), (beta, "beta"), (initial_state, "initial_state"),
+                 (final_state, "final_state")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+        nbytes = kda_chunk_fwd_windowed_workspace_bytes(N, T, H, Dk, Dv, chunk, q.dtype,
+                                                        window_chunks)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib.kda_chunk_fwd_windowed_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         float(scale), _ptr(initial_state), _ptr(cu_seqlens), N,
+                                         T, H, Dk, Dv, chunk, _dtype(q), _ptr(o),
+                                         _ptr(final_state), int(window_chunks), _ptr(workspace),
+                                         workspace.numel(), _stream(stream)))
 
 
 def _chunk_fwd_segmented(q, k, v, g, beta, o, scale, initial_state, final_state, cu_seqlens,

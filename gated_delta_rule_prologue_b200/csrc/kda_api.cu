@@ -2,6 +2,7 @@
 // dispatch to the kernels.  No entry point allocates device memory: the status
 // word (kda_status.cu) and the scratch of kda_chunk_fwd_static (kda_static.cu)
 // are file-scope __device__ variables.
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -298,6 +299,13 @@ size_t kda_chunk_fwd_segmented_workspace_bytes(int N, int T, int H, int Dk, int 
   return kda::rec::workspace_bytes(N, T, H, segment_chunks);
 }
 
+size_t kda_chunk_fwd_windowed_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                              kda_dtype dt, int window_chunks) {
+  if (N < 1 || T < 0 || H < 1 || window_chunks < 1 || !chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return 0;
+  return kda::rec::windowed_workspace_bytes(N, H, window_chunks);
+}
+
 int kda_chunk_fwd_segment_chunks(int N, int T, int H) {
   if (N < 1 || T < 0 || H < 1) return 0;
   return kda::rec::segment_chunks(N, T, H);
@@ -316,8 +324,9 @@ kda_status chunk_two_pass(const void *q, const void *k, const void *v, const voi
                           const float *initial_state, const int32_t *cu_seqlens, int N, int T,
                           int H, int Dk, int Dv, kda_dtype dt, float *o, float *final_state,
                           void *workspace, size_t workspace_bytes, cudaStream_t s,
-                          const char *what, int L) {
-  const size_t need = kda::rec::workspace_bytes(N, T, H, L);
+                          const char *what, int L, int window = 0) {
+  const size_t need = window > 0 ? kda::rec::windowed_workspace_bytes(N, H, window)
+                                 : kda::rec::workspace_bytes(N, T, H, L);
   KDA_OPT_PTR(workspace, "workspace");
   KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
               workspace_bytes, need);
@@ -340,6 +349,31 @@ kda_status chunk_two_pass(const void *q, const void *k, const void *v, const voi
   cudaError_t e = cudaSuccess;
   if (cu_seqlens || L > 0)
     e = kda::launch_chunk_index(cu_seqlens, N, T, L, workspace, status, s);
+  if (window > 0) {
+    // One window of chunk numbers at a time: the prep pass writes the window's records,
+    // the state pass consumes them; a sequence crossing a window boundary hands its state
+    // over through the two carry blocks (alternating).  The real chunk total is known on
+    // the device only, so the windows cover the capacity bound; past the total they are
+    // empty and their CTAs exit at once.
+    float *carry = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                             kda::rec::windowed_carry_offset(N, H, window));
+    const size_t carry_floats = (size_t)H * 128 * 128;
+    const long long cap = kda::rec::chunk_capacity(N, T);
+    for (long long lo = 0, w = 0; lo < cap && e == cudaSuccess; lo += window, ++w) {
+      kda::ChunkWindow win;
+      win.lo = (int)lo;
+      win.hi = (int)std::min<long long>(lo + window, 0x7fffffffLL);
+      win.carry_in = carry + (size_t)(w & 1) * carry_floats;
+      win.carry_out = carry + (size_t)((w + 1) & 1) * carry_floats;
+      e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, A_log,
+                                 dt_bias, lower_bound, gated, status, s, win);
+      if (e == cudaSuccess)
+        e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, 0, o,
+                                    final_state, status, s, nullptr, win);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return KDA_OK;
+  }
   if (e == cudaSuccess)
     e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, N, T, H, dt, workspace, A_log,
                                dt_bias, lower_bound, gated, status, s);
@@ -394,6 +428,28 @@ kda_status kda_chunk_fwd_segmented_ws(const void *q, const void *k, const void *
                         cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, workspace,
                         workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_segmented_ws launch",
                         segment_chunks);
+}
+
+kda_status kda_chunk_fwd_windowed_ws(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta, float scale,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt, float *o, float *final_state,
+                                     int window_chunks, void *workspace, size_t workspace_bytes,
+                                     kda_stream_t stream) {
+  kda_status st = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, N, T, H, Dk, Dv,
+                                   chunk, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  if (!chunk_tc_path(T, Dk, Dv, chunk, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "chunk_fwd_windowed: needs bf16/f16, Dk == Dv == 128, "
+                                     "chunk 64 and T > 0 (got dt=%d Dk=%d chunk=%d T=%d)",
+                (int)dt, Dk, chunk, T);
+  KDA_REQUIRE(window_chunks >= 1, "window_chunks=%d must be at least 1", window_chunks);
+  KDA_REQUIRE(workspace != nullptr, "chunk_fwd_windowed: workspace is NULL");
+  return chunk_two_pass(q, k, v, g, 4, nullptr, nullptr, 0.f, false, beta, scale, initial_state,
+                        cu_seqlens, N, T, H, Dk, Dv, dt, o, final_state, workspace,
+                        workspace_bytes, (cudaStream_t)stream, "kda_chunk_fwd_windowed_ws launch",
+                        0, window_chunks);
 }
 
 kda_status kda_chunk_fwd_gated_ws(const void *q, const void *k, const void *v, const void *g_raw,

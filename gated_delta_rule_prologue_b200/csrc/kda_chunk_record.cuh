@@ -45,6 +45,11 @@
 //   E  the entry state of segment s (for the first segment of a split
 //      sequence, a copy of the caller's initial state)
 // With L = 0 every sequence is one segment and there is no segment area.
+//
+// Windowed form: the passes run over windows of `window` consecutive chunk numbers,
+// one window at a time, so the workspace holds the records of one window; a sequence
+// that crosses a window boundary hands its fp32 state over through one of two carry
+// blocks per head (alternating by window), placed after the records.
 #pragma once
 
 #include <stddef.h>
@@ -136,6 +141,16 @@ __host__ __device__ inline size_t segment_area_offset(int N, int T, int H) {
 __host__ __device__ inline size_t workspace_bytes(int N, int T, int H, int L) {
   return segment_area_offset(N, T, H) +
          (L > 0 ? (size_t)segment_capacity(N, T, L) * H * 3 * SEG_BLOCK : 0);
+}
+
+// Windowed two-pass prefill (kda_chunk_fwd_windowed_ws): the header, records for
+// `window` chunks of every head, then two carry states per head ([H][128][128] fp32
+// each) that hand the state of a sequence over a window boundary.
+__host__ __device__ inline size_t windowed_carry_offset(int N, int H, int window) {
+  return header_bytes(N) + (size_t)window * H * BYTES;
+}
+__host__ __device__ inline size_t windowed_workspace_bytes(int N, int H, int window) {
+  return windowed_carry_offset(N, H, window) + 2 * (size_t)H * SEG_BLOCK;
 }
 
 }  // namespace rec

@@ -99,7 +99,8 @@ template <int kRole>
 __global__ void __launch_bounds__(kBT, 3)
 chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ cu,
                    const float *s0, float scale, int N, int T, int H, int L, float *__restrict__ o,
-                   float *sN, float *ckpt, float *map_m, float *map_b, int *status) {
+                   float *sN, float *ckpt, float *map_m, float *map_b, int *status,
+                   ChunkWindow win) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -134,10 +135,28 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     cbase = cprefix[n];
     if (L == 0) c_hi = cprefix[n + 1] - cbase;
   }
+  // A window of chunk numbers [win.lo, win.hi) (whole sequences only): this chain runs the
+  // sequence's chunks inside it, entering from the carry if the sequence began in an
+  // earlier window and leaving its state in the carry if it goes on past this one.  An
+  // empty sequence belongs to the window holding its chunk position.
+  bool from_carry = false, to_carry = false;
+  if (kRole == kOutputs && L == 0) {
+    const int nch = c_hi;
+    const int lo = max(0, win.lo - cbase);
+    const int hi = (int)min((long long)nch, (long long)win.hi - cbase);
+    if (nch > 0 ? lo >= hi : !(win.lo <= cbase && cbase < win.hi)) return;
+    if (nch > 0) {
+      from_carry = lo > 0;
+      to_carry = hi < nch;
+      c_lo = lo;
+      c_hi = hi;
+    }
+  }
   {  // debug builds: the chain's sequence, chunks and segment slots lie inside the workspace
-    const long long cap = rec::chunk_capacity(N, T);
+    const long long cap = min(rec::chunk_capacity(N, T), (long long)win.hi - win.lo);
     if (!in_range(status, n, N) ||
-        (c_hi > c_lo && !(in_range(status, cbase + c_lo, cap) && in_range(status, cbase + c_hi - 1, cap))) ||
+        (c_hi > c_lo && !(in_range(status, cbase + c_lo - win.lo, cap) &&
+                          in_range(status, cbase + c_hi - 1 - win.lo, cap))) ||
         (L > 0 && !in_range(status, s, rec::segment_capacity(N, T, L))))
       return;
   }
@@ -177,6 +196,8 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
     // the initial state by the last segment while the first is still to run.
     s_in = sg.G > 1 ? seg_slot(s, 2) : s0 ? s0 + head_off : nullptr;
     s_out = sg.g == sg.G - 1 && sN ? sN + head_off : nullptr;
+    if (from_carry) s_in = win.carry_in + (size_t)h * 128 * 128;
+    if (to_carry) s_out = win.carry_out + (size_t)h * 128 * 128;
   }
 
   if (warp == 0) tmem_alloc(slot, TB_COLS);
@@ -222,7 +243,7 @@ chunk_state_kernel(const uint8_t *__restrict__ ws, const int32_t *__restrict__ c
   const uint32_t lane_addr = static_cast<uint32_t>(32 * warp) << 16;
 
   auto rec_of = [&](int c) -> const uint8_t * {
-    return recs + ((size_t)(cbase + c) * H + h) * rec::BYTES;
+    return recs + ((size_t)(cbase + c - win.lo) * H + h) * rec::BYTES;
   };
   auto load_a1 = [&](int c) {
     mbar_arrive_expect_tx(bar_a1, 32768);
@@ -676,7 +697,7 @@ template <int kRole>
 cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0, float scale,
                               int N, int T, int H, int L, float *o, float *sN, float *ckpt,
                               int *status, cudaStream_t s, float *map_m = nullptr,
-                              float *map_b = nullptr) {
+                              float *map_b = nullptr, const ChunkWindow &win = ChunkWindow{}) {
   const long long items = L > 0 ? rec::segment_capacity(N, T, L) : N;
   const long long blocks = items * H * kSlices * (kRole == kOutputs ? 1 : 2);
   if (blocks >= (1LL << 31)) return cudaErrorInvalidValue;
@@ -685,7 +706,7 @@ cudaError_t launch_state_role(const void *ws, const int32_t *cu, const float *s0
   if (e != cudaSuccess) return e;
   chunk_state_kernel<kRole><<<(unsigned)blocks, kBT, SB_ALLOC, s>>>(
       static_cast<const uint8_t *>(ws), cu, s0, scale, N, T, H, L, o, sN, ckpt, map_m, map_b,
-      status);
+      status, win);
   return cudaGetLastError();
 }
 }  // namespace
@@ -737,7 +758,7 @@ cudaError_t launch_state_compose(const float *M, const float *B, const float *E_
 
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,
-                               cudaStream_t s, float *ckpt) {
+                               cudaStream_t s, float *ckpt, const ChunkWindow &win) {
   cudaError_t e;
   if (L > 0) {
     e = launch_state_role<kTransition>(ws, cu, s0, scale, N, T, H, L, o, sN, nullptr, status,
@@ -751,7 +772,8 @@ cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_state_role<kOutputs>(ws, cu, s0, scale, N, T, H, L, o, sN, ckpt, status, s);
+  return launch_state_role<kOutputs>(ws, cu, s0, scale, N, T, H, L, o, sN, ckpt, status, s,
+                                     nullptr, nullptr, win);
 }
 
 }  // namespace kda

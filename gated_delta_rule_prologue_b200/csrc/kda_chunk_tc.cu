@@ -253,7 +253,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float *__restrict__ beta, float scale, const float *s0,
                 const int32_t *__restrict__ cu, int T, int H, float *__restrict__ o, float *sN,
                 int *status, const float *__restrict__ conv_w, const Tin *cache_in,
-                Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N, GateArgs gate) {
+                Tin *cache_out, uint8_t *recs, const int32_t *cprefix, int N, GateArgs gate,
+                ChunkWindow win) {
   constexpr bool kFused = kMode == kFusedMode || kMode == kPrepFused || kMode == kPrepFusedGated;
   constexpr bool kGated = kMode == kPrepGated || kMode == kPrepFusedGated;
   constexpr bool kPrepM = kMode == kPrep || kMode == kPrepFused || kGated;
@@ -296,7 +297,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if constexpr (kPrepM) {
     const long long cap = rec::chunk_capacity(N, T);
     total_chunks = cu ? (int)min((long long)cprefix[N], cap) : (T + 63) / 64;
-    items = (long long)total_chunks * H;
+    items = (long long)max(0, min(total_chunks, win.hi) - win.lo) * H;  // the window's items
   } else {
     seq_bounds(cu, n, T, status, bos, eos);
     nchunks = (eos - bos + 63) / 64;
@@ -307,7 +308,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const long long item = (long long)blockIdx.x + (long long)it * gridDim.x;
       w.ok = item < items;
       if (!w.ok) return w;
-      w.ci = (int)(item / H);
+      w.ci = win.lo + (int)(item / H);
       w.h = (int)(item % H);
       int sb = 0, se = T, c0 = 0, lo = 0;
       if (cu) {  // sequence of chunk ci: the last n with cprefix[n] <= ci
@@ -327,6 +328,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       w.eos = se;
       w.ok = w.Lc > 0 && in_range(status, w.n, N) &&
              in_range(status, w.ci, rec::chunk_capacity(N, T)) &&
+             in_range(status, w.ci - win.lo,
+                      min(rec::chunk_capacity(N, T), (long long)win.hi - win.lo)) &&
              in_range(status, w.t0 + w.Lc - 1, T);
     } else {
       w.ok = it < nchunks;
@@ -1036,7 +1039,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if constexpr (kPrepM) {
         // the record's tiles that are complete already leave while the MMAs run: each
         // k-atom of A1 = [W ; Q G] holds the 64 W rows, then the 64 Q G rows
-        uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)cur.ci * H + h) * rec::BYTES;
+        uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)(cur.ci - win.lo) * H + h) * rec::BYTES;
         bulk_store(rp + rec::A1 + 8192, sm + SM_QG, 8192);
         bulk_store(rp + rec::A1 + 24576, sm + SM_QG + 8192, 8192);
         bulk_store(rp + rec::KP, sm + SM_KP, 16384);
@@ -1069,7 +1072,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if constexpr (kPrepM) {
       // ---- record: W (K-major, over the dead beta K G tile), Ut + fp32 remainder,
       //      exp(gamma_63), <q_r, k_r>; then the tiles leave by bulk copies -------------
-      uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)cur.ci * H + h) * rec::BYTES;
+      uint8_t *rp = recs + rec::header_bytes(N) + ((size_t)(cur.ci - win.lo) * H + h) * rec::BYTES;
       {
         float w[16], u[16], cr[16];
         tmem_ld16_nowait(tmem + lane_addr + TM_W + 16 * grp, w);  // W[16 grp + i][j]
@@ -1282,7 +1285,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
                                                       sN, status, nullptr, nullptr, nullptr,
-                                                      nullptr, nullptr, N, GateArgs{});
+                                                      nullptr, nullptr, N, GateArgs{},
+                                                      ChunkWindow{});
   } else {
     auto kern = chunk_tc_kernel<__half, kSingle>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1290,7 +1294,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, kThreads, SM_ALLOC, s>>>(tq, tk, tv, tg, beta, scale, s0, cu, T, H, o,
                                                       sN, status, nullptr, nullptr, nullptr,
-                                                      nullptr, nullptr, N, GateArgs{});
+                                                      nullptr, nullptr, N, GateArgs{},
+                                                      ChunkWindow{});
   }
   return cudaGetLastError();
 }
@@ -1298,12 +1303,14 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 namespace {
 // Grid of a persistent prep launch: one CTA per SM (each takes a whole SM's
 // shared memory), at most one per work item.
-cudaError_t prep_grid(int N, int T, int H, unsigned *grid) {
+cudaError_t prep_grid(int N, int T, int H, const ChunkWindow &win, unsigned *grid) {
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  *grid = (unsigned)std::min<long long>(rec::chunk_capacity(N, T) * H, sms);
+  const long long chunks =
+      std::min<long long>(rec::chunk_capacity(N, T), (long long)win.hi - win.lo);
+  *grid = (unsigned)std::max<long long>(1, std::min<long long>(chunks * H, sms));
   return cudaSuccess;
 }
 
@@ -1311,16 +1318,16 @@ template <typename Tin, int kMode>
 cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                               const CUtensorMap &tg, const float *beta, const int32_t *cu, int N,
                               int T, int H, uint8_t *ws, const GateArgs &gate, int *status,
-                              cudaStream_t s) {
+                              cudaStream_t s, const ChunkWindow &win) {
   auto kern = chunk_tc_kernel<Tin, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SM_ALLOC_PREP);
   if (e != cudaSuccess) return e;
   unsigned grid = 0;
-  if ((e = prep_grid(N, T, H, &grid)) != cudaSuccess) return e;
+  if ((e = prep_grid(N, T, H, win, &grid)) != cudaSuccess) return e;
   kern<<<grid, kThreads, SM_ALLOC_PREP, s>>>(tq, tk, tv, tg, beta, 1.f, nullptr, cu, T, H, nullptr,
                                              nullptr, status, nullptr, nullptr, nullptr, ws,
-                                             reinterpret_cast<const int32_t *>(ws), N, gate);
+                                             reinterpret_cast<const int32_t *>(ws), N, gate, win);
   return cudaGetLastError();
 }
 }  // namespace
@@ -1328,7 +1335,8 @@ cudaError_t launch_prep_typed(const CUtensorMap &tq, const CUtensorMap &tk, cons
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const void *g,
                               const float *beta, const int32_t *cu, int N, int T, int H,
                               kda_dtype dt, void *ws, const float *A_log, const float *dt_bias,
-                              float lower_bound, bool gated, int *status, cudaStream_t s) {
+                              float lower_bound, bool gated, int *status, cudaStream_t s,
+                              const ChunkWindow &win) {
   const CUtensorMapDataType act =
       dt == KDA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv, tg;
@@ -1341,13 +1349,13 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
   const GateArgs gate{A_log, dt_bias, lower_bound};
   if (dt == KDA_BF16)
     return gated ? launch_prep_typed<__nv_bfloat16, kPrepGated>(tq, tk, tv, tg, beta, cu, N, T, H,
-                                                                 w, gate, status, s)
+                                                                 w, gate, status, s, win)
                  : launch_prep_typed<__nv_bfloat16, kPrep>(tq, tk, tv, tg, beta, cu, N, T, H, w,
-                                                            gate, status, s);
+                                                            gate, status, s, win);
   return gated ? launch_prep_typed<__half, kPrepGated>(tq, tk, tv, tg, beta, cu, N, T, H, w, gate,
-                                                        status, s)
+                                                        status, s, win)
                : launch_prep_typed<__half, kPrep>(tq, tk, tv, tg, beta, cu, N, T, H, w, gate,
-                                                   status, s);
+                                                   status, s, win);
 }
 
 namespace {
@@ -1370,7 +1378,7 @@ cudaError_t launch_fused_typed(const void *x, const float *conv_w, const void *c
   kern<<<(unsigned)blocks, kThreads, SM_ALLOC_FUSED, s>>>(
       tx, tx, tx, tg, beta, scale, s0, cu, T, H, o, sN, status, conv_w,
       static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), nullptr, nullptr, N,
-      GateArgs{});
+      GateArgs{}, ChunkWindow{});
   return cudaGetLastError();
 }
 }  // namespace
@@ -1381,7 +1389,7 @@ cudaError_t launch_prep_fused_typed(const void *x, const float *conv_w, const vo
                                     void *cache_out, const void *g, const float *beta,
                                     const int32_t *cu, int N, int T, int H,
                                     CUtensorMapDataType act, void *ws, const GateArgs &gate,
-                                    int *status, cudaStream_t s) {
+                                    int *status, cudaStream_t s, const ChunkWindow &win) {
   constexpr bool kGatedM = kMode == kPrepFusedGated;
   CUtensorMap tx, th, tg;
   if (!make_map(&tx, x, act, 2, 3 * H, T) || !make_map(&th, x, act, 2, 3 * H, T, 3) ||
@@ -1393,12 +1401,12 @@ cudaError_t launch_prep_fused_typed(const void *x, const float *conv_w, const vo
                                        (int)SM_ALLOC_FUSED);
   if (e != cudaSuccess) return e;
   unsigned grid = 0;
-  if ((e = prep_grid(N, T, H, &grid)) != cudaSuccess) return e;
+  if ((e = prep_grid(N, T, H, win, &grid)) != cudaSuccess) return e;
   uint8_t *w = static_cast<uint8_t *>(ws);
   kern<<<grid, kThreads, SM_ALLOC_FUSED, s>>>(
       tx, th, tx, tg, beta, 1.f, nullptr, cu, T, H, nullptr, nullptr, status, conv_w,
       static_cast<const Tin *>(cache_in), static_cast<Tin *>(cache_out), w,
-      reinterpret_cast<const int32_t *>(w), N, gate);
+      reinterpret_cast<const int32_t *>(w), N, gate, win);
   return cudaGetLastError();
 }
 }  // namespace
@@ -1408,20 +1416,20 @@ cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,
                                        void *ws, const float *A_log, const float *dt_bias,
                                        float lower_bound, bool gated, int *status,
-                                       cudaStream_t s) {
+                                       cudaStream_t s, const ChunkWindow &win) {
   const GateArgs gate{A_log, dt_bias, lower_bound};
   if (dt == KDA_BF16) {
     constexpr auto act = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     return gated ? launch_prep_fused_typed<__nv_bfloat16, kPrepFusedGated>(
-                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s)
+                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s, win)
                  : launch_prep_fused_typed<__nv_bfloat16, kPrepFused>(
-                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s);
+                       x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s, win);
   }
   constexpr auto act = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   return gated ? launch_prep_fused_typed<__half, kPrepFusedGated>(
-                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s)
+                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s, win)
                : launch_prep_fused_typed<__half, kPrepFused>(
-                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s);
+                     x, conv_w, cache_in, cache_out, g, beta, cu, N, T, H, act, ws, gate, status, s, win);
 }
 
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,

@@ -309,17 +309,32 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 // transition pass, the entry-state scan and the output pass.
 // g: fp32 log-decay, or (gated) 16-bit gate pre-activations of type dt turned
 // into the log-decay in the kernel (A_log, dt_bias may be null).
+//
+// Windows (kda_chunk_fwd_windowed_ws): the passes may run over a window [lo, hi) of
+// the batch's chunk numbers (all sequences' chunks in order) at a time, with the
+// window's records at slots 0 .. hi - lo of the workspace.  A sequence that starts
+// before the window enters from carry_in and one that continues past it leaves its
+// state in carry_out ([H][Dv][Dk] fp32 each; one sequence at most crosses a window
+// boundary).  The default window is the whole batch.
+struct ChunkWindow {
+  int lo = 0;
+  int hi = 0x7fffffff;
+  const float *carry_in = nullptr;
+  float *carry_out = nullptr;
+};
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const void *g,
                               const float *beta, const int32_t *cu, int N, int T, int H,
                               kda_dtype dt, void *ws, const float *A_log, const float *dt_bias,
-                              float lower_bound, bool gated, int *status, cudaStream_t s);
+                              float lower_bound, bool gated, int *status, cudaStream_t s,
+                              const ChunkWindow &win = ChunkWindow{});
 cudaError_t launch_chunk_index(const int32_t *cu, int N, int T, int L, void *ws, int *status,
                                cudaStream_t s);
 // ckpt (optional, [chunks][H][Dv][Dk] fp32 in record order): the entry state of
 // every chunk, for the backward pass; o may then be NULL.
 cudaError_t launch_chunk_state(const void *ws, const int32_t *cu, const float *s0, float scale,
                                int N, int T, int H, int L, float *o, float *sN, int *status,
-                               cudaStream_t s, float *ckpt = nullptr);
+                               cudaStream_t s, float *ckpt = nullptr,
+                               const ChunkWindow &win = ChunkWindow{});
 // Affine map of every sequence (one segment each; records from the prep pass):
 // map_m [N][H][Dk][Dk] with M[t][k] at k * Dk + t, map_b [N][H][Dv][Dk] like a state.
 cudaError_t launch_chunk_map(const void *ws, const int32_t *cu, int N, int T, int H, float *map_m,
@@ -347,7 +362,7 @@ cudaError_t launch_prologue_chunk_prep(const void *x, const float *conv_w, const
                                        const int32_t *cu, int N, int T, int H, kda_dtype dt,
                                        void *ws, const float *A_log, const float *dt_bias,
                                        float lower_bound, bool gated, int *status,
-                                       cudaStream_t s);
+                                       cudaStream_t s, const ChunkWindow &win = ChunkWindow{});
 cudaError_t launch_cache_pass(const void *ws, int N, int H, const void *cache_in,
                               void *cache_out, cudaStream_t s);
 cudaError_t launch_prologue_chunk_tc(const void *x, const float *conv_w, const void *cache_in,

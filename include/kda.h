@@ -217,6 +217,43 @@ kda_status kda_chunk_fwd_segmented_ws(const void *q, const void *k, const void *
                                       size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_windowed_ws -- kda_chunk_fwd_ws with a workspace that does not
+ * grow with T: the two passes run over windows of `window_chunks` consecutive
+ * chunk numbers (the chunks of all sequences, in order) one window at a time,
+ * so the workspace holds one window's records (88.75 KiB per chunk and head)
+ * plus two fp32 carry states per head, through which a sequence that crosses
+ * a window boundary hands its state to the next window.  This is the same
+ * computation in the same order: every output and final state is bit for bit
+ * that of kda_chunk_fwd_segmented_ws with segment_chunks = 0.  The cost is two
+ * launches per window (ceil((ceil(T/64) + N) / window_chunks) windows).
+ * Source: "KimiK3轻量化复刻实现KDA并行解析，Chunkwise并行与状态压缩机制详解",
+ * Figure 1 (the in-chunk work is state-independent, so it can run ahead of the
+ * state pass a window at a time).
+ *   window_chunks    >= 1, else KDA_ERR_INVALID_ARG
+ *   workspace        >= kda_chunk_fwd_windowed_workspace_bytes(...) bytes,
+ *                    16-byte aligned, caller-owned, as for kda_chunk_fwd_ws
+ * Supported: the tensor-core path only (dt KDA_BF16 or KDA_F16, Dk == Dv ==
+ * 128, chunk 64, T > 0), else KDA_ERR_UNSUPPORTED.  Other arguments as in
+ * kda_chunk_fwd_ws.
+ */
+kda_status kda_chunk_fwd_windowed_ws(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta, float scale,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     int N, int T, int H, int Dk, int Dv, int chunk,
+                                     kda_dtype dt, float *o, float *final_state,
+                                     int window_chunks, void *workspace, size_t workspace_bytes,
+                                     kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_windowed_workspace_bytes -- workspace of kda_chunk_fwd_windowed_ws:
+ * a 1 KiB-aligned chunk index, window_chunks * H records of 88.75 KiB and
+ * 2 * H carry states of 64 KiB.  0 for arguments off the tensor-core path or
+ * window_chunks < 1.
+ */
+size_t kda_chunk_fwd_windowed_workspace_bytes(int N, int T, int H, int Dk, int Dv, int chunk,
+                                              kda_dtype dt, int window_chunks);
+
+/*
  * The *_gated entry points take the gate pre-activations instead of the
  * log-decay and apply the bounded gate inside the kernels ([W1 彩蛋], the
  * gate.py excerpt):

@@ -230,6 +230,37 @@ def test_chunk_fwd_segmented_rejects_bad_arguments(kda):
     assert st == kda.KDA_ERR_UNSUPPORTED
 
 
+def test_chunk_fwd_windowed_workspace_and_bad_arguments(kda):
+    """The windowed workspace is one window of records plus two carry states per
+    head, whatever T is; argument checks run before any device call."""
+    import torch
+    L = kda.lib
+    T, H, W = 640, 2, 3
+    need = kda.kda_chunk_fwd_windowed_workspace_bytes(1, T, H, 128, 128, 64, torch.bfloat16, W)
+    assert need == 1024 + W * H * 90880 + 2 * H * 128 * 128 * 4
+    assert need == kda.kda_chunk_fwd_windowed_workspace_bytes(1, 100 * T, H, 128, 128, 64,
+                                                              torch.bfloat16, W)
+    assert kda.kda_chunk_fwd_windowed_workspace_bytes(1, T, H, 128, 128, 64, torch.bfloat16,
+                                                      0) == 0
+    assert kda.kda_chunk_fwd_windowed_workspace_bytes(1, T, H, 128, 128, 64, torch.float32,
+                                                      W) == 0
+    q, k, v = _vp(0x100000), _vp(0x200000), _vp(0x300000)
+    g, beta, o = _vp(0x400000), _vp(0x800000), _vp(0x900000)
+    ws = _vp(0x1000000)
+    args = (q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 1, o, None)
+    st = L.kda_chunk_fwd_windowed_ws(*args, 0, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"window_chunks" in L.kda_last_error()
+    st = L.kda_chunk_fwd_windowed_ws(*args, W, None, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace is NULL" in L.kda_last_error()
+    st = L.kda_chunk_fwd_windowed_ws(*args, W, ws, need - 16, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace holds" in L.kda_last_error()
+    st = L.kda_chunk_fwd_windowed_ws(*args, W, _vp(0x900000 + 4096), need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"overlaps" in L.kda_last_error()
+    f32 = (q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 0, o, None)
+    st = L.kda_chunk_fwd_windowed_ws(*f32, W, ws, need, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+
+
 def test_chunk_fwd_ws_rejects_bad_workspace(kda):
     import torch
     L = kda.lib
