@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "kda_chunk_bwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu",
                       _CSRC + "kda_chunk_bwd.cu"],
     "kda_decode_step": [_CSRC + "kda_decode.cu"],
+    "kda_chunk_fwd_windowed64": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
 }
 
 
@@ -543,6 +544,21 @@ def run_ours(args, world, rank, local):
         gev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     gated_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in gev[1:])
+    # the windowed call: 64-chunk windows, a workspace that does not grow with T
+    win_chunks = 64
+    win_ws = torch.empty(kda.kda_chunk_fwd_windowed_workspace_bytes(1, T, H, D, D, inp.chunk,
+                                                                    q.dtype, win_chunks),
+                         dtype=torch.uint8, device=dev)
+    wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    for i in range(3):
+        wev[i][0].record(stream)
+        kda.kda_chunk_fwd(q, k, v, g, beta, o2, scale=inp.scale, chunk=inp.chunk,
+                          window_chunks=win_chunks, workspace=win_ws, stream=stream)
+        wev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    windowed_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in wev[1:])
+    win_ws_gb = win_ws.numel() / 1e9
+    del win_ws
     # the output epilogue on the step's read-out (RMSNorm x sigmoid gate, bf16 out)
     ep_out = gq  # reuse a bf16 [T, H, D] buffer
     ep_w = (0.5 + torch.rand((D,), generator=gen)).to(dev)
@@ -599,6 +615,12 @@ def run_ours(args, world, rank, local):
             recorded_traffic("kda_output_epilogue"))),
         "kda_chunk_bwd": dict(ms=round(bwd_ms, 4), launches=4, **roofline(
             "hbm", BWD_BYTES_PER_TH * th, bwd_ms, hbm, "GB/s", recorded_traffic("kda_chunk_bwd"))),
+        "kda_chunk_fwd_windowed64": dict(
+            ms=round(windowed_ms, 4), window_chunks=win_chunks,
+            launches=2 * ((T + 63) // 64 // win_chunks + 1),
+            workspace_gb=round(win_ws_gb, 3), full_workspace_gb=round(ws.numel() / 1e9, 3),
+            **roofline("hbm", CHUNK_BYTES_PER_TH_PLAN * th, windowed_ms, hbm, "GB/s",
+                       recorded_traffic("kda_chunk_fwd_windowed64"))),
         "kda_chunk_fwd_one_pass": dict(ms=round(one_pass_ms, 4), **roofline(
             "hbm", CHUNK_BYTES_PER_TH * th, one_pass_ms, hbm, "GB/s",
             recorded_traffic("kda_chunk_fwd_one_pass"))),
