@@ -325,6 +325,12 @@ struct LocalSmem {
   float xch[2][128];    // per-key partial sums passed between the two row halves
 };
 
+// Pairs of fp32 lanes on the packed instructions (one issue for two lanes, each lane
+// rounded as its scalar fma): the low and high halves of a float4.
+__device__ __forceinline__ float2 lo2(const float4 &v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4 &v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+
 // Persistent grid: one CTA per SM, each with a scratch slot for the entry states of
 // sub-chunks 1..3 of its current chunk (written by the forward walk, read back by the
 // backward walk; 192 KB per CTA, resident in L2).
@@ -487,25 +493,22 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     // E = V - (K G) S;  KK, A, P;  U = (I + A)^{-1} diag(beta) E.
     auto forward_local = [&](bool with_p) {
       {
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc[e] = sm.E[rr * RS + ca + e];
-          acc[4 + e] = sm.E[rr * RS + cb + e];
-        }
+        const float4 e1 = *reinterpret_cast<const float4 *>(&sm.E[rr * RS + ca]);
+        const float4 e2 = *reinterpret_cast<const float4 *>(&sm.E[rr * RS + cb]);
+        float2 acc[4] = {lo2(e1), hi2(e1), lo2(e2), hi2(e2)};
 #pragma unroll 4
         for (int key = 0; key < 128; ++key) {
-          const float a = sm.KG[rr * RS + key];
+          const float2 na = dup2(-sm.KG[rr * RS + key]);
           const float4 s1 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + ca]);
           const float4 s2 = *reinterpret_cast<const float4 *>(&sm.S[key * RS + cb]);
-          acc[0] -= a * s1.x; acc[1] -= a * s1.y; acc[2] -= a * s1.z; acc[3] -= a * s1.w;
-          acc[4] -= a * s2.x; acc[5] -= a * s2.y; acc[6] -= a * s2.z; acc[7] -= a * s2.w;
+          acc[0] = __ffma2_rn(na, lo2(s1), acc[0]);
+          acc[1] = __ffma2_rn(na, hi2(s1), acc[1]);
+          acc[2] = __ffma2_rn(na, lo2(s2), acc[2]);
+          acc[3] = __ffma2_rn(na, hi2(s2), acc[3]);
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {  // each thread rewrites only the entries it read
-          sm.E[rr * RS + ca + e] = acc[e];
-          sm.E[rr * RS + cb + e] = acc[4 + e];
-        }
+        // each thread rewrites only the entries it read
+        *reinterpret_cast<float4 *>(&sm.E[rr * RS + ca]) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        *reinterpret_cast<float4 *>(&sm.E[rr * RS + cb]) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
       }
       {  // 16 x 16 Grams: thread (r, i)
         const int r = tid >> 4, i = tid & 15;
@@ -544,28 +547,28 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
     // S <- diag(G_last) S + K'^T U   (thread (keys kq, kq + 64; value chunks 16 m + 4 q4))
     auto advance_state = [&]() {
-      float st[2][32];
+      float2 st[2][16];
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int key = kq + 64 * kk;
-        const float gck = sm.gc[key];
+        const float2 gck = dup2(sm.gc[key]);
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           const float4 x = *reinterpret_cast<const float4 *>(&sm.S[key * RS + 16 * m + 4 * q4]);
-          st[kk][4 * m] = gck * x.x; st[kk][4 * m + 1] = gck * x.y;
-          st[kk][4 * m + 2] = gck * x.z; st[kk][4 * m + 3] = gck * x.w;
+          st[kk][2 * m] = __fmul2_rn(gck, lo2(x));
+          st[kk][2 * m + 1] = __fmul2_rn(gck, hi2(x));
         }
       }
 #pragma unroll 2
       for (int r = 0; r < kSub; ++r) {
-        const float kp0 = sm.KP[r * RS + kq], kp1 = sm.KP[r * RS + kq + 64];
+        const float2 kp0 = dup2(sm.KP[r * RS + kq]), kp1 = dup2(sm.KP[r * RS + kq + 64]);
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + 16 * m + 4 * q4]);
-          st[0][4 * m] = fmaf(kp0, u.x, st[0][4 * m]); st[0][4 * m + 1] = fmaf(kp0, u.y, st[0][4 * m + 1]);
-          st[0][4 * m + 2] = fmaf(kp0, u.z, st[0][4 * m + 2]); st[0][4 * m + 3] = fmaf(kp0, u.w, st[0][4 * m + 3]);
-          st[1][4 * m] = fmaf(kp1, u.x, st[1][4 * m]); st[1][4 * m + 1] = fmaf(kp1, u.y, st[1][4 * m + 1]);
-          st[1][4 * m + 2] = fmaf(kp1, u.z, st[1][4 * m + 2]); st[1][4 * m + 3] = fmaf(kp1, u.w, st[1][4 * m + 3]);
+          st[0][2 * m] = __ffma2_rn(kp0, lo2(u), st[0][2 * m]);
+          st[0][2 * m + 1] = __ffma2_rn(kp0, hi2(u), st[0][2 * m + 1]);
+          st[1][2 * m] = __ffma2_rn(kp1, lo2(u), st[1][2 * m]);
+          st[1][2 * m + 1] = __ffma2_rn(kp1, hi2(u), st[1][2 * m + 1]);
         }
       }
 #pragma unroll
@@ -573,7 +576,7 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
         for (int m = 0; m < 8; ++m)
           *reinterpret_cast<float4 *>(&sm.S[(kq + 64 * kk) * RS + 16 * m + 4 * q4]) =
-              make_float4(st[kk][4 * m], st[kk][4 * m + 1], st[kk][4 * m + 2], st[kk][4 * m + 3]);
+              make_float4(st[kk][2 * m].x, st[kk][2 * m].y, st[kk][2 * m + 1].x, st[kk][2 * m + 1].y);
       __syncthreads();
     };
 
@@ -601,29 +604,29 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
       // ---- dU = P^T dO' + K' dS'  (thread (r, 8 value columns)) ----------------------------
       {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float2 acc[4] = {dup2(0.f), dup2(0.f), dup2(0.f), dup2(0.f)};
 #pragma unroll
         for (int i = 0; i < kSub; ++i) {
-          const float p = sm.P[i * SS + rr];
+          const float2 p = dup2(sm.P[i * SS + rr]);
           const float4 d1 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + ca]);
           const float4 d2 = *reinterpret_cast<const float4 *>(&sm.dO[i * RS + cb]);
-          acc[0] = fmaf(p, d1.x, acc[0]); acc[1] = fmaf(p, d1.y, acc[1]);
-          acc[2] = fmaf(p, d1.z, acc[2]); acc[3] = fmaf(p, d1.w, acc[3]);
-          acc[4] = fmaf(p, d2.x, acc[4]); acc[5] = fmaf(p, d2.y, acc[5]);
-          acc[6] = fmaf(p, d2.z, acc[6]); acc[7] = fmaf(p, d2.w, acc[7]);
+          acc[0] = __ffma2_rn(p, lo2(d1), acc[0]);
+          acc[1] = __ffma2_rn(p, hi2(d1), acc[1]);
+          acc[2] = __ffma2_rn(p, lo2(d2), acc[2]);
+          acc[3] = __ffma2_rn(p, hi2(d2), acc[3]);
         }
 #pragma unroll 4
         for (int key = 0; key < 128; ++key) {
-          const float a = sm.KP[rr * RS + key];
+          const float2 a = dup2(sm.KP[rr * RS + key]);
           const float4 s1 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + ca]);
           const float4 s2 = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + cb]);
-          acc[0] = fmaf(a, s1.x, acc[0]); acc[1] = fmaf(a, s1.y, acc[1]);
-          acc[2] = fmaf(a, s1.z, acc[2]); acc[3] = fmaf(a, s1.w, acc[3]);
-          acc[4] = fmaf(a, s2.x, acc[4]); acc[5] = fmaf(a, s2.y, acc[5]);
-          acc[6] = fmaf(a, s2.z, acc[6]); acc[7] = fmaf(a, s2.w, acc[7]);
+          acc[0] = __ffma2_rn(a, lo2(s1), acc[0]);
+          acc[1] = __ffma2_rn(a, hi2(s1), acc[1]);
+          acc[2] = __ffma2_rn(a, lo2(s2), acc[2]);
+          acc[3] = __ffma2_rn(a, hi2(s2), acc[3]);
         }
-        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + ca]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + cb]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + ca]) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        *reinterpret_cast<float4 *>(&sm.dU[rr * RS + cb]) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
       }
       {  // dP = lower(dO' U^T)   (thread (r, i))
         const int r = tid >> 4, i = tid & 15;
@@ -694,29 +697,41 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
       {
         const int rb = 8 * rh;
         float dqg[8], dkg[8], dkp[8];
+        float sds;  // rowsum(S * dS') of key kt
+        {
+          // Dot products over the 128 value columns, as two interleaved partial sums (even
+          // and odd columns) on the packed instructions, added at the end.
+          float2 q2[8], k2[8], p2[8], sd2 = dup2(0.f);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) dqg[x] = dkg[x] = dkp[x] = 0.f;
-        float sds = 0.f;  // rowsum(S * dS') of key kt
-        const float *srow = &sm.S[kt * RS], *dsrow = &sm.dS[kt * RS];
+          for (int x = 0; x < 8; ++x) q2[x] = k2[x] = p2[x] = dup2(0.f);
+          const float *srow = &sm.S[kt * RS], *dsrow = &sm.dS[kt * RS];
 #pragma unroll 2
-        for (int j = 0; j < 128; j += 4) {
-          const float4 sv = *reinterpret_cast<const float4 *>(srow + j);
-          const float4 dv4 = *reinterpret_cast<const float4 *>(dsrow + j);
-          sds = fmaf(sv.x, dv4.x, sds); sds = fmaf(sv.y, dv4.y, sds);
-          sds = fmaf(sv.z, dv4.z, sds); sds = fmaf(sv.w, dv4.w, sds);
+          for (int j = 0; j < 128; j += 4) {
+            const float4 sv = *reinterpret_cast<const float4 *>(srow + j);
+            const float4 dv4 = *reinterpret_cast<const float4 *>(dsrow + j);
+            sd2 = __ffma2_rn(lo2(sv), lo2(dv4), sd2);
+            sd2 = __ffma2_rn(hi2(sv), hi2(dv4), sd2);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const int r = rb + x;  // the same row for the whole warp: broadcast reads
+              const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
+              const float4 rr4 = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
+              const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + j]);
+              q2[x] = __ffma2_rn(lo2(o), lo2(sv), q2[x]);
+              q2[x] = __ffma2_rn(hi2(o), hi2(sv), q2[x]);
+              k2[x] = __ffma2_rn(lo2(rr4), lo2(sv), k2[x]);
+              k2[x] = __ffma2_rn(hi2(rr4), hi2(sv), k2[x]);
+              p2[x] = __ffma2_rn(lo2(u), lo2(dv4), p2[x]);
+              p2[x] = __ffma2_rn(hi2(u), hi2(dv4), p2[x]);
+            }
+          }
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
-            const int r = rb + x;  // the same row for the whole warp: broadcast reads
-            const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + j]);
-            const float4 rr4 = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + j]);
-            const float4 u = *reinterpret_cast<const float4 *>(&sm.U[r * RS + j]);
-            dqg[x] = fmaf(o.x, sv.x, dqg[x]); dqg[x] = fmaf(o.y, sv.y, dqg[x]);
-            dqg[x] = fmaf(o.z, sv.z, dqg[x]); dqg[x] = fmaf(o.w, sv.w, dqg[x]);
-            dkg[x] = fmaf(rr4.x, sv.x, dkg[x]); dkg[x] = fmaf(rr4.y, sv.y, dkg[x]);
-            dkg[x] = fmaf(rr4.z, sv.z, dkg[x]); dkg[x] = fmaf(rr4.w, sv.w, dkg[x]);
-            dkp[x] = fmaf(u.x, dv4.x, dkp[x]); dkp[x] = fmaf(u.y, dv4.y, dkp[x]);
-            dkp[x] = fmaf(u.z, dv4.z, dkp[x]); dkp[x] = fmaf(u.w, dv4.w, dkp[x]);
+            dqg[x] = q2[x].x + q2[x].y;
+            dkg[x] = k2[x].x + k2[x].y;
+            dkp[x] = p2[x].x + p2[x].y;
           }
+          sds = sd2.x + sd2.y;
         }
         float dgam[8], dkd[8];
         float kps = 0.f;  // sum over this thread's rows of dK' K'
@@ -783,35 +798,31 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
       // ---- dS <- diag(G_last) dS' + (Q G)^T dO' - (diag(beta) K G)^T dR  (keys kq, kq + 64) --
       {
-        float st[2][32];
+        float2 st[2][16];
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           const int key = kq + 64 * kk;
-          const float gck = sm.gc[key];
+          const float2 gck = dup2(sm.gc[key]);
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             const float4 x = *reinterpret_cast<const float4 *>(&sm.dS[key * RS + 16 * m + 4 * q4]);
-            st[kk][4 * m] = gck * x.x; st[kk][4 * m + 1] = gck * x.y;
-            st[kk][4 * m + 2] = gck * x.z; st[kk][4 * m + 3] = gck * x.w;
+            st[kk][2 * m] = __fmul2_rn(gck, lo2(x));
+            st[kk][2 * m + 1] = __fmul2_rn(gck, hi2(x));
           }
         }
 #pragma unroll 2
         for (int r = 0; r < kSub; ++r) {
           const float nb = -sm.beta[r];
-          const float a0 = sm.QG[r * RS + kq], a1 = sm.QG[r * RS + kq + 64];
-          const float b0 = nb * sm.KG[r * RS + kq], b1 = nb * sm.KG[r * RS + kq + 64];
+          const float2 a0 = dup2(sm.QG[r * RS + kq]), a1 = dup2(sm.QG[r * RS + kq + 64]);
+          const float2 b0 = dup2(nb * sm.KG[r * RS + kq]), b1 = dup2(nb * sm.KG[r * RS + kq + 64]);
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             const float4 o = *reinterpret_cast<const float4 *>(&sm.dO[r * RS + 16 * m + 4 * q4]);
             const float4 d = *reinterpret_cast<const float4 *>(&sm.dU[r * RS + 16 * m + 4 * q4]);
-            st[0][4 * m] = fmaf(a0, o.x, fmaf(b0, d.x, st[0][4 * m]));
-            st[0][4 * m + 1] = fmaf(a0, o.y, fmaf(b0, d.y, st[0][4 * m + 1]));
-            st[0][4 * m + 2] = fmaf(a0, o.z, fmaf(b0, d.z, st[0][4 * m + 2]));
-            st[0][4 * m + 3] = fmaf(a0, o.w, fmaf(b0, d.w, st[0][4 * m + 3]));
-            st[1][4 * m] = fmaf(a1, o.x, fmaf(b1, d.x, st[1][4 * m]));
-            st[1][4 * m + 1] = fmaf(a1, o.y, fmaf(b1, d.y, st[1][4 * m + 1]));
-            st[1][4 * m + 2] = fmaf(a1, o.z, fmaf(b1, d.z, st[1][4 * m + 2]));
-            st[1][4 * m + 3] = fmaf(a1, o.w, fmaf(b1, d.w, st[1][4 * m + 3]));
+            st[0][2 * m] = __ffma2_rn(a0, lo2(o), __ffma2_rn(b0, lo2(d), st[0][2 * m]));
+            st[0][2 * m + 1] = __ffma2_rn(a0, hi2(o), __ffma2_rn(b0, hi2(d), st[0][2 * m + 1]));
+            st[1][2 * m] = __ffma2_rn(a1, lo2(o), __ffma2_rn(b1, lo2(d), st[1][2 * m]));
+            st[1][2 * m + 1] = __ffma2_rn(a1, hi2(o), __ffma2_rn(b1, hi2(d), st[1][2 * m + 1]));
           }
         }
 #pragma unroll
@@ -819,7 +830,7 @@ chunk_bwd_local_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
           for (int m = 0; m < 8; ++m)
             *reinterpret_cast<float4 *>(&sm.dS[(kq + 64 * kk) * RS + 16 * m + 4 * q4]) =
-                make_float4(st[kk][4 * m], st[kk][4 * m + 1], st[kk][4 * m + 2], st[kk][4 * m + 3]);
+                make_float4(st[kk][2 * m].x, st[kk][2 * m].y, st[kk][2 * m + 1].x, st[kk][2 * m + 1].y);
       }
     }
     __syncthreads();  // before the next item overwrites the shared matrices
