@@ -155,27 +155,6 @@ static_assert(TM_Z + 64 <= TM_W && TM_G + 96 <= TM_Z && TM_T2 + 64 <= TM_Y &&
 constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
 
-// Eight 16-bit values packed in a uint4, widened to floats.
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8], __nv_bfloat16) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8], __half) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __half2 hh;
-    memcpy(&hh, &w[i], 4);
-    const float2 t = __half22float2(hh);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
-
 // 8 consecutive 16-bit activations of a raw tile (bf16 or fp16) as floats.
 template <typename Tin>
 __device__ __forceinline__ void ld8_in(const uint8_t *p, float (&f)[8]) {
@@ -782,15 +761,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         asm volatile("bar.sync 3, 64;" ::: "memory");
         // column jj of D_b, swept row by row; fp16 into D16 and T32
         const int b = tid >> 4, jj = tid & 15, base = 16 * b;
-        float acc[16];
+        // Rows in pairs on the packed fp32 instructions: every entry gets the same fma
+        // sequence as a row-by-row sweep (so the same values), with half the issues.
+        float2 acc2[8];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
+        for (int p = 0; p < 8; ++p) acc2[p] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
-          acc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -acc[ii]);
+          float &aii = (ii & 1) ? acc2[ii >> 1].y : acc2[ii >> 1].x;
+          aii = ii == jj ? 1.f : (ii < jj ? 0.f : -aii);
           const float *arow = ATd + (b * 16 + ii) * 16;  // A[base + rr][base + ii]
+          if (!(ii & 1)) acc2[ii >> 1].y = fmaf(arow[ii + 1], aii, acc2[ii >> 1].y);
+          const float2 a2 = make_float2(aii, aii);
 #pragma unroll
-          for (int rr = ii + 1; rr < 16; ++rr) acc[rr] = fmaf(arow[rr], acc[ii], acc[rr]);
+          for (int p = (ii >> 1) + 1; p < 8; ++p)
+            acc2[p] = __ffma2_rn(reinterpret_cast<const float2 *>(arow)[p], a2, acc2[p]);
+        }
+        float acc[16];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          acc[2 * p] = acc2[p].x;
+          acc[2 * p + 1] = acc2[p].y;
         }
         const uint32_t col = (uint32_t)((base + jj) & 7) * 2;
 #pragma unroll
