@@ -171,6 +171,13 @@ __device__ __forceinline__ void ld8_f32(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+__device__ __forceinline__ void ld8_f32_pairs(const float *p, float2 (&f)[4]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0];
+  const float4 b = reinterpret_cast<const float4 *>(p)[1];
+  f[0] = make_float2(a.x, a.y); f[1] = make_float2(a.z, a.w);
+  f[2] = make_float2(b.x, b.y); f[3] = make_float2(b.z, b.w);
+}
+
 // 8 consecutive K-elements [8*c8, 8*c8+8) of `row` of a K-major fp32 tile of `rows`
 // rows, rounded to tf32: two 16-byte chunks.
 __device__ __forceinline__ void st_tf32x8(uint8_t *tile, int rows, int row, int c8,
@@ -676,26 +683,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int m = 0; m < 2; ++m) {
       const int p = tid + kThreads * m;
       const int r = p >> 4, c8 = p & 15, d0 = c8 * 8;
-      float k8[8], q8[8], e8[8];
-      ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
-      ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
-      ld8_f32(Gf + r * 128 + d0, e8);
+      // channel pairs on the packed fp32 instructions (each lane rounded as its scalar op)
+      float2 k2[4], q2[4], e2[4];
+      widen_pairs(*reinterpret_cast<const uint4 *>(sm + SM_K + r * 256 + c8 * 16), k2, Tact());
+      widen_pairs(*reinterpret_cast<const uint4 *>(sm + SM_Q + r * 256 + c8 * 16), q2, Tact());
+      ld8_f32_pairs(Gf + r * 128 + d0, e2);
       float a[8], b[8], ki[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float kk = k8[e], qq = q8[e];  // rows past the chunk's end are zero
-        a[e] = kk * e8[e];
-        b[e] = qq * e8[e];
-        ki[e] = __fdividef(kk, e8[e]);  // E in [e^-80, e^75]: inside the intrinsic's range
+      for (int i = 0; i < 4; ++i) {  // rows past the chunk's end are zero
+        const float2 ap = __fmul2_rn(k2[i], e2[i]), bp = __fmul2_rn(q2[i], e2[i]);
+        a[2 * i] = ap.x; a[2 * i + 1] = ap.y;
+        b[2 * i] = bp.x; b[2 * i + 1] = bp.y;
+        // E in [e^-80, e^75]: inside the intrinsic's range
+        ki[2 * i] = __fdividef(k2[i].x, e2[i].x);
+        ki[2 * i + 1] = __fdividef(k2[i].y, e2[i].y);
       }
       st_tf32x8(sm + SM_GA, 128, r, c8, a);
       st_tf32x8(sm + SM_GA, 128, 64 + r, c8, b);
       if (r < 32) {
         st_tf32x8(sm + SM_GB, 96, r, c8, ki);
-        float hf[8];
-        ld8_f32(feba + d0, hf);
+        float2 hf[4];
+        ld8_f32_pairs(feba + d0, hf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ki[e] = (ki[e] * hf[e]) * hf[e];
+        for (int i = 0; i < 4; ++i) {
+          const float2 kp = __fmul2_rn(__fmul2_rn(make_float2(ki[2 * i], ki[2 * i + 1]), hf[i]), hf[i]);
+          ki[2 * i] = kp.x; ki[2 * i + 1] = kp.y;
+        }
       }
       st_tf32x8(sm + SM_GB, 96, 32 + r, c8, ki);
     }
@@ -941,22 +954,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float bt = beta_s[r];
         const float *fec = r < 32 ? feca : fecb;
         const float *fel = r < 32 ? fela : felb;
-        float k8[8], q8[8], v8[8], e8[8];
-        ld8_in<Tact>(sm + SM_K + r * 256 + c8 * 16, k8);
-        ld8_in<Tact>(sm + SM_Q + r * 256 + c8 * 16, q8);
-        ld8_in<Tact>(sm + SM_V + r * 256 + c8 * 16, v8);
-        ld8_f32(Gf + r * 128 + d0, e8);
-        float bkg[8], bv[8], qg[8], kp[8], ec8[8], el8[8];
-        ld8_f32(fec + d0, ec8);
-        ld8_f32(fel + d0, el8);
+        // channel pairs on the packed fp32 instructions (each lane rounded as its scalar op)
+        float2 k2[4], q2[4], v2[4], e2[4], ec2[4], el2[4];
+        widen_pairs(*reinterpret_cast<const uint4 *>(sm + SM_K + r * 256 + c8 * 16), k2, Tact());
+        widen_pairs(*reinterpret_cast<const uint4 *>(sm + SM_Q + r * 256 + c8 * 16), q2, Tact());
+        widen_pairs(*reinterpret_cast<const uint4 *>(sm + SM_V + r * 256 + c8 * 16), v2, Tact());
+        ld8_f32_pairs(Gf + r * 128 + d0, e2);
+        ld8_f32_pairs(fec + d0, ec2);
+        ld8_f32_pairs(fel + d0, el2);
+        float k8[8], q8[8], bkg[8], bv[8], qg[8], kp[8];
+        const float2 bt2 = make_float2(bt, bt);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float kk = k8[e], qq = q8[e], vv = v8[e];  // zero past the chunk's end
-          const float g_abs = e8[e] * ec8[e];               // exp(gamma_r) per channel
-          bkg[e] = (bt * kk) * g_abs;
-          bv[e] = bt * vv;
-          qg[e] = qq * g_abs;
-          kp[e] = __fdividef(kk, e8[e]) * el8[e];
+        for (int i = 0; i < 4; ++i) {  // zero past the chunk's end
+          const float2 g_abs = __fmul2_rn(e2[i], ec2[i]);  // exp(gamma_r) per channel
+          const float2 bk = __fmul2_rn(__fmul2_rn(bt2, k2[i]), g_abs);
+          const float2 bvp = __fmul2_rn(bt2, v2[i]);
+          const float2 qgp = __fmul2_rn(q2[i], g_abs);
+          const float2 kpp = __fmul2_rn(make_float2(__fdividef(k2[i].x, e2[i].x),
+                                                    __fdividef(k2[i].y, e2[i].y)), el2[i]);
+          k8[2 * i] = k2[i].x; k8[2 * i + 1] = k2[i].y;
+          q8[2 * i] = q2[i].x; q8[2 * i + 1] = q2[i].y;
+          bkg[2 * i] = bk.x; bkg[2 * i + 1] = bk.y;
+          bv[2 * i] = bvp.x; bv[2 * i + 1] = bvp.y;
+          qg[2 * i] = qgp.x; qg[2 * i + 1] = qgp.y;
+          kp[2 * i] = kpp.x; kp[2 * i + 1] = kpp.y;
         }
         const uint4 bv_h = pack8_f16(bv);
         st_shared_16(sm + SM_BKG, mnmaj_off(64, r, c8), pack8_f16(bkg));
