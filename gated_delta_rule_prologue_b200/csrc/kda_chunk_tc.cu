@@ -771,7 +771,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (ii < rr) ATd[(b * 16 + ii) * 16 + rr] = br * g;
           }
         }
-        asm volatile("bar.sync 3, 64;" ::: "memory");
+        // Each warp's rows hold exactly the two diagonal blocks its own threads invert
+        // (warp 0: blocks 0, 1; warp 1: blocks 2, 3), so the warps need not meet here.
+        __syncwarp();
         // column jj of D_b, swept row by row; fp16 into D16 and T32
         const int b = tid >> 4, jj = tid & 15, base = 16 * b;
         // Rows in pairs on the packed fp32 instructions: every entry gets the same fma
