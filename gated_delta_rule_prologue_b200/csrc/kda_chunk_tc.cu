@@ -71,6 +71,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 namespace {
 using namespace tc;
 
+// Zeros for the inverse's 16-bit tiles (D16 + Zm, 16 KB; T32, 8 KB), copied in by the
+// bulk-copy engine instead of written by threads.
+__device__ __align__(128) uint8_t g_zero_tiles[16384];
+
 constexpr int kThreads = 512;
 constexpr int kHalf = kThreads / 2;
 
@@ -107,7 +111,7 @@ constexpr uint32_t F_ELB = F_ELA + 512;     //   exp(gamma_last - c_B)
 constexpr uint32_t F_EGC = F_ELB + 512;     //   exp(gamma_last)
 constexpr uint32_t SM_BETA = F_EGC + 512;   // beta of the chunk     [64]
 constexpr uint32_t SM_PDIAG = SM_BETA + 256;// <q_r, k_r> in fp32    [64]
-constexpr uint32_t SM_BAR = SM_PDIAG + 256; // three mbarriers (tiles, MMAs, inverse MMAs)
+constexpr uint32_t SM_BAR = SM_PDIAG + 256; // four mbarriers (tiles, MMAs, inverse MMAs, zero fill)
 constexpr uint32_t SM_SLOT = SM_BAR + 32;   // TMEM base address
 constexpr uint32_t SM_TOTAL = SM_SLOT + 16;
 // Fused prologue only: fp32 correction beta*v - f16(beta*v_tile) kept as bf16
@@ -259,6 +263,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);
   uint64_t *bar_mma = bar_tma + 1;
   uint64_t *bar_inv = bar_tma + 2;
+  uint64_t *bar_zero = bar_tma + 3;
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + SM_SLOT);
   float *Gf = reinterpret_cast<float *>(sm + SM_G);
   float *beta_s = reinterpret_cast<float *>(sm + SM_BETA);
@@ -336,6 +341,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
     mbar_init(bar_inv, 1);
+    mbar_init(bar_zero, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -448,7 +454,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   };
   if (cur.ok) fetch_gate(cur);
 
-  uint32_t tma_par = 0, mma_par = 0, inv_par = 0;
+  uint32_t tma_par = 0, mma_par = 0, inv_par = 0, zero_par = 0;
   bool failed = false;  // a wait ran out: copies or MMAs may still be in flight
   int c = 0;
   for (; cur.ok; ++c) {
@@ -731,6 +737,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     mma_par ^= 1;
     tc_fence_after();
+    if (tid == 0) {  // the Gram's operands are dead: D16, Zm and T32 start at zero
+      mbar_arrive_expect_tx(bar_zero, 16384 + 8192);
+      bulk_load(sm + SM_D16, g_zero_tiles, 16384, bar_zero);
+      bulk_load(sm + SM_T32, g_zero_tiles, 8192, bar_zero);
+    }
 
     // ---- P4: two warp groups ---------------------------------------------------------------
     //   warps 0-7:  P4b (Gram read-out -> A as an fp16 tile and its diagonal 16x16 blocks in
@@ -743,8 +754,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float *ATd = reinterpret_cast<float *>(sm + SM_ATD);  // [blk][col][row] of A's diagonal blocks
       // ---- P4b / P5 (i): warps 0-1 read only the diagonal 16x16 blocks of A out of TMEM and
       //      run the forward substitution at once, while warps 2-7 read out the whole of A
-      //      (fp16 tile, zero on and above the diagonal) and the strict P operand, then
-      //      zero what the inverse's tiles need zeroed --------------------------------------
+      //      (fp16 tile, zero on and above the diagonal) and the strict P operand
+      //      (the inverse's 16-bit tiles start at zero: a bulk copy of zeros issued when
+      //      the Gram MMA completed) -----------------------------------------------------
       // TMEM layout of the Gram: rows 0..31 hold columns i in [0, 32) (reference c_A), rows
       // 32..63 columns i in [0, 64) at TMEM columns 32 + i (reference c_B).
       // P5: T = (I + A)^{-1}, the blocked inverse of a lower triangular matrix.  D =
@@ -799,6 +811,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           acc[2 * p + 1] = acc2[p].y;
         }
         const uint32_t col = (uint32_t)((base + jj) & 7) * 2;
+        if (!mbar_wait(bar_zero, zero_par)) inv_ok = false;  // the zeros landed first
+        zero_par ^= 1;
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
           const __half hv = __float2half_rn(acc[rr]);
@@ -851,7 +865,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           emit(cga, v);
           emit(cga + 1, w);
         }
-        const int zt = tid - 64;  // 0..191
         if (warp >= 6) {  // rows 0..31, columns 32..63 of A and P: above the diagonal, not read out
           const int t = tid - 192, rz = t >> 1, cz = 4 + 2 * (t & 1);
 #pragma unroll
@@ -860,14 +873,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             st_shared_16(sm + SM_A16, kmaj_off(64, rz, cz + z), make_uint4(0u, 0u, 0u, 0u));
           }
         }
-        // D16 and T32 outside the diagonal 16x16 blocks, and all of Zm, start at zero
-        // (the diagonal blocks' 16-byte chunks are written whole by the substitution)
-        for (int x = zt; x < 3 * 512; x += kHalf - 64) {
-          const int row = (x & 511) >> 3, c8 = x & 7;
-          if (x < 1024 && (c8 >> 1) == (row >> 4)) continue;
-          const uint32_t tile = x < 512 ? SM_D16 : (x < 1024 ? SM_T32 : SM_ZM);
-          st_shared_16(sm + tile, kmaj_off(64, row, c8), make_uint4(0u, 0u, 0u, 0u));
-        }
+
       }
       fence_async_smem();
       bar_half();
@@ -1251,6 +1257,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     drain(bar_tma);
     drain(bar_mma);
     drain(bar_inv);
+    drain(bar_zero);
   }
   if (sN && !kPrepM && !failed) {
     float *dst = sN + (((size_t)n * H + hb) * 128 + j) * 128 + dk0;
