@@ -159,22 +159,6 @@ static_assert(TM_Z + 64 <= TM_W && TM_G + 96 <= TM_Z && TM_T2 + 64 <= TM_Y &&
 constexpr uint32_t kHaloBytes = 3 * 3 * 128 * 2;  // three raw rows of the q, k, v parts
 
 
-// 8 consecutive 16-bit activations of a raw tile (bf16 or fp16) as floats.
-template <typename Tin>
-__device__ __forceinline__ void ld8_in(const uint8_t *p, float (&f)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4 *>(p);
-  const Tin *h = reinterpret_cast<const Tin *>(&u);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = to_f32(h[i]);
-}
-
-__device__ __forceinline__ void ld8_f32(const float *p, float (&f)[8]) {
-  const float4 a = reinterpret_cast<const float4 *>(p)[0];
-  const float4 b = reinterpret_cast<const float4 *>(p)[1];
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
 __device__ __forceinline__ void ld8_f32_pairs(const float *p, float2 (&f)[4]) {
   const float4 a = reinterpret_cast<const float4 *>(p)[0];
   const float4 b = reinterpret_cast<const float4 *>(p)[1];
