@@ -202,7 +202,8 @@ constexpr int kBoxTokens = 6;    // a multiple of the 3-row history ring
 constexpr int kStages = 3;
 constexpr int kWarpChannels = 256;
 constexpr int kBoxBytes = kBoxTokens * kWarpChannels * 2;
-constexpr int kStagedTokens = 288;  // tokens per CTA: 48 boxes (K3: 2052 CTAs, 6.9 waves of 296)
+constexpr int kStagedTokens = 288;  // tokens per CTA: 48 boxes (32768 tokens x 96 heads: 2052
+                                    // CTAs, 6.9 waves of 2 x 148)
 constexpr int kStagedWarps = kThreads / 32;
 constexpr int kStagedSmem = kStagedWarps * kStages * (kBoxBytes + 8);
 static_assert(kStagedTokens % kBoxTokens == 0 && kBoxTokens % 3 == 0 && kBoxBytes % 128 == 0,
