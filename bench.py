@@ -617,7 +617,7 @@ def run_ours(args, world, rank, local):
             "hbm", BWD_BYTES_PER_TH * th, bwd_ms, hbm, "GB/s", recorded_traffic("kda_chunk_bwd"))),
         "kda_chunk_fwd_windowed64": dict(
             ms=round(windowed_ms, 4), window_chunks=win_chunks,
-            launches=2 * ((T + 63) // 64 // win_chunks + 1),
+            launches=2 * (((T + 63) // 64 + 1 + win_chunks - 1) // win_chunks),
             workspace_gb=round(win_ws_gb, 3), full_workspace_gb=round(ws.numel() / 1e9, 3),
             **roofline("hbm", CHUNK_BYTES_PER_TH_PLAN * th, windowed_ms, hbm, "GB/s",
                        recorded_traffic("kda_chunk_fwd_windowed64"))),
