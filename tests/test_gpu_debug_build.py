@@ -7,7 +7,8 @@ word (KDA_ERR_DEVICE_BOUNDS) instead of making the access.  Two checks:
 * the check itself: a checked write of a four-slot probe at an index outside it
   records BOUNDS and leaves the context usable;
 * no false alarms and unchanged results: the small-shape parity tests (the
-  oracle comparisons of tests/test_gpu_*.py, config-1-sized and ragged inputs)
+  oracle comparisons of tests/test_gpu_*.py, config-1-sized and ragged inputs,
+  the segmented and windowed state passes)
   pass when run against the debug library, with a clean status word after every
   call that checks it.
 
@@ -62,7 +63,7 @@ def test_small_parity_suite_on_the_debug_build():
     env = dict(os.environ, KDA_LIB="debug")
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            "tests/test_gpu_debug_build.py", "tests/test_gpu_parity.py",
-           "tests/test_gpu_segmented.py", "tests/test_gpu_backward.py",
+           "tests/test_gpu_segmented.py", "tests/test_gpu_windowed.py", "tests/test_gpu_backward.py",
            "tests/test_gpu_degenerate.py", "tests/test_gpu_gate.py",
            "-k", "not full_size and not long_sequence and not k3"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
