@@ -116,6 +116,9 @@ lib.kda_chunk_fwd_segmented_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp
 lib.kda_chunk_fwd_windowed_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
                                           _i, _i, _i, _vp, _vp, _i, _vp, ctypes.c_size_t, _vp]
 lib.kda_chunk_fwd_windowed_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+lib.kda_prologue_chunk_fwd_windowed_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                                   _i, _i, _i, _i, _i, _vp, _vp, _i, _vp,
+                                                   ctypes.c_size_t, _vp]
 lib.kda_chunk_fwd_windowed_workspace_bytes.restype = ctypes.c_size_t
 lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp]
 lib.kda_prologue_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i,
@@ -127,6 +130,7 @@ lib.kda_debug_build.argtypes = []
 lib.kda_debug_build.restype = ctypes.c_int
 for _fn in (lib.kda_prologue, lib.kda_chunk_fwd, lib.kda_chunk_fwd_ws, lib.kda_chunk_fwd_static,
             lib.kda_chunk_fwd_segmented_ws, lib.kda_chunk_fwd_windowed_ws,
+            lib.kda_prologue_chunk_fwd_windowed_ws,
             lib.kda_chunk_bwd_ws, lib.kda_chunk_map_ws,
             lib.kda_state_compose,
             lib.kda_prologue_chunk_fwd_ws, lib.kda_decode_step, lib.kda_chunk_fwd_gated_ws,
@@ -463,13 +467,14 @@ def kda_chunk_fwd_static(q, k, v, g, beta, o, *, scale: float = 1.0, initial_sta
 
 def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: float = 1.0,
                            cache_in=None, cache_out=None, initial_state=None, final_state=None,
-                           cu_seqlens=None, workspace="auto", stream=None):
+                           cu_seqlens=None, workspace="auto", window_chunks=None, stream=None):
     """Prologue fused into the chunkwise prefill (chunk 64): ``x`` [T, 3*H*D]
     bf16/fp16 projections in, ``o`` [T, H, D] float32 out; q, k, v stay on chip.
 
     ``workspace`` as in :func:`kda_chunk_fwd`: ``"auto"`` (two passes, scratch
     from torch's caching allocator), a uint8 CUDA tensor, or ``None`` (the
-    one-pass kernel)."""
+    one-pass kernel).  ``window_chunks``: an int >= 1 calls
+    ``kda_prologue_chunk_fwd_windowed_ws`` (a workspace that does not grow with T)."""
     for t, n in ((x, "x"), (cache_in, "cache_in"), (cache_out, "cache_out")):
         _need(t, n, x.dtype)
     for t, n in ((conv_w, "conv_w"), (o, "o"), (g, "g"), (beta, "beta"),
@@ -478,6 +483,20 @@ def kda_prologue_chunk_fwd(x, conv_w, g, beta, o, *, H: int, D: int, scale: floa
     _need(cu_seqlens, "cu_seqlens", torch.int32)
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     T = x.shape[0]
+    if window_chunks is not None:
+        if isinstance(workspace, str):
+            if workspace != "auto":
+                raise ValueError(f"workspace must be 'auto' or a tensor, not {workspace!r}")
+            nbytes = kda_chunk_fwd_windowed_workspace_bytes(N, T, H, D, D, 64, x.dtype,
+                                                            int(window_chunks))
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        _need(workspace, "workspace", torch.uint8)
+        _check(lib.kda_prologue_chunk_fwd_windowed_ws(
+            _ptr(x), _ptr(conv_w), _ptr(cache_in), _ptr(cache_out), _ptr(g), _ptr(beta),
+            float(scale), _ptr(initial_state), _ptr(cu_seqlens), N, T, H, D, _dtype(x), _ptr(o),
+            _ptr(final_state), int(window_chunks), _ptr(workspace), workspace.numel(),
+            _stream(stream)))
+        return
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError(f"workspace must be 'auto', None or a tensor, not {workspace!r}")

@@ -575,8 +575,9 @@ kda_status fused_two_pass(const void *x, const float *conv_w, const void *cache_
                           const float *beta, float scale, const float *initial_state,
                           const int32_t *cu_seqlens, int N, int T, int H, int D, kda_dtype dt,
                           float *o, float *final_state, void *workspace, size_t workspace_bytes,
-                          cudaStream_t s, const char *what) {
-  const size_t need = kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt);
+                          cudaStream_t s, const char *what, int window = 0) {
+  const size_t need = window > 0 ? kda::rec::windowed_workspace_bytes(N, H, window)
+                                 : kda_chunk_fwd_workspace_bytes(N, T, H, D, D, 64, dt);
   KDA_OPT_PTR(workspace, "workspace");
   KDA_REQUIRE(workspace_bytes >= need, "workspace holds %zu bytes, these sizes need %zu",
               workspace_bytes, need);
@@ -599,16 +600,36 @@ kda_status fused_two_pass(const void *x, const float *conv_w, const void *cache_
   kda_status st = device_status_word(&status);
   if (st != KDA_OK) return st;
   cudaError_t e = cudaSuccess;
-  const int L = kda::rec::segment_chunks(N, T, H);
+  const int L = window > 0 ? 0 : kda::rec::segment_chunks(N, T, H);
   if (cu_seqlens || L > 0)
     e = kda::launch_chunk_index(cu_seqlens, N, T, L, workspace, status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N, T,
-                                        H, dt, workspace, A_log, dt_bias, lower_bound, gated,
-                                        status, s);
-  if (e == cudaSuccess)
-    e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, L, o,
-                                final_state, status, s);
+  if (window > 0) {  // one window of chunk numbers at a time (see chunk_two_pass)
+    float *carry = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                             kda::rec::windowed_carry_offset(N, H, window));
+    const size_t carry_floats = (size_t)H * 128 * 128;
+    const long long cap = kda::rec::chunk_capacity(N, T);
+    for (long long lo = 0, w = 0; lo < cap && e == cudaSuccess; lo += window, ++w) {
+      kda::ChunkWindow win;
+      win.lo = (int)lo;
+      win.hi = (int)std::min<long long>(lo + window, 0x7fffffffLL);
+      win.carry_in = carry + (size_t)(w & 1) * carry_floats;
+      win.carry_out = carry + (size_t)((w + 1) & 1) * carry_floats;
+      e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N,
+                                          T, H, dt, workspace, A_log, dt_bias, lower_bound, gated,
+                                          status, s, win);
+      if (e == cudaSuccess)
+        e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, 0, o,
+                                    final_state, status, s, nullptr, win);
+    }
+  } else {
+    if (e == cudaSuccess)
+      e = kda::launch_prologue_chunk_prep(x, conv_w, cache_in, cache_out, g, beta, cu_seqlens, N,
+                                          T, H, dt, workspace, A_log, dt_bias, lower_bound, gated,
+                                          status, s);
+    if (e == cudaSuccess)
+      e = kda::launch_chunk_state(workspace, cu_seqlens, initial_state, scale, N, T, H, L, o,
+                                  final_state, status, s);
+  }
   if (e == cudaSuccess && cu_seqlens && cache_out)
     e = kda::launch_cache_pass(workspace, N, H, cache_in, cache_out, s);
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -636,6 +657,28 @@ kda_status kda_prologue_chunk_fwd_ws(const void *x, const float *conv_w, const v
                         scale, initial_state, cu_seqlens, N, T, H, D, dt, o, final_state,
                         workspace, workspace_bytes, (cudaStream_t)stream,
                         "kda_prologue_chunk_fwd_ws launch");
+}
+
+kda_status kda_prologue_chunk_fwd_windowed_ws(const void *x, const float *conv_w,
+                                              const void *cache_in, void *cache_out,
+                                              const float *g, const float *beta, float scale,
+                                              const float *initial_state,
+                                              const int32_t *cu_seqlens, int N, int T, int H,
+                                              int D, kda_dtype dt, float *o, float *final_state,
+                                              int window_chunks, void *workspace,
+                                              size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_fused_args(x, conv_w, cache_in, cache_out, g, beta, initial_state,
+                                   cu_seqlens, N, T, H, D, dt, o, final_state);
+  if (st != KDA_OK) return st;
+  if (!chunk_tc_path(T, D, D, 64, dt))
+    return fail(KDA_ERR_UNSUPPORTED, "prologue_chunk_fwd_windowed: needs bf16/f16, D == 128 "
+                                     "and T > 0 (got dt=%d D=%d T=%d)", (int)dt, D, T);
+  KDA_REQUIRE(window_chunks >= 1, "window_chunks=%d must be at least 1", window_chunks);
+  KDA_REQUIRE(workspace != nullptr, "prologue_chunk_fwd_windowed: workspace is NULL");
+  return fused_two_pass(x, conv_w, cache_in, cache_out, g, 4, nullptr, nullptr, 0.f, false, beta,
+                        scale, initial_state, cu_seqlens, N, T, H, D, dt, o, final_state,
+                        workspace, workspace_bytes, (cudaStream_t)stream,
+                        "kda_prologue_chunk_fwd_windowed_ws launch", window_chunks);
 }
 
 kda_status kda_prologue_chunk_fwd_gated_ws(const void *x, const float *conv_w,

@@ -245,6 +245,27 @@ kda_status kda_chunk_fwd_windowed_ws(const void *q, const void *k, const void *v
                                      kda_stream_t stream);
 
 /*
+ * kda_prologue_chunk_fwd_windowed_ws -- kda_prologue_chunk_fwd_ws (the prologue
+ * inside the prep pass) one window of `window_chunks` chunk numbers at a time,
+ * as kda_chunk_fwd_windowed_ws: the workspace
+ * (kda_chunk_fwd_windowed_workspace_bytes(N, T, H, D, D, 64, dt, window_chunks))
+ * does not grow with T.  The conv cache out is written as by the unwindowed call;
+ * o and final_state are bit for bit those of kda_prologue_chunk_fwd_ws when it
+ * runs whole sequences (kda_chunk_fwd_segment_chunks(N, T, H) == 0).
+ * Supported: dt KDA_BF16 or KDA_F16, D == 128, T > 0 (else KDA_ERR_UNSUPPORTED);
+ * window_chunks >= 1 and a non-NULL workspace (else KDA_ERR_INVALID_ARG).
+ * Other arguments as in kda_prologue_chunk_fwd_ws.
+ */
+kda_status kda_prologue_chunk_fwd_windowed_ws(const void *x, const float *conv_w,
+                                              const void *cache_in, void *cache_out,
+                                              const float *g, const float *beta, float scale,
+                                              const float *initial_state,
+                                              const int32_t *cu_seqlens, int N, int T, int H,
+                                              int D, kda_dtype dt, float *o, float *final_state,
+                                              int window_chunks, void *workspace,
+                                              size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_windowed_workspace_bytes -- workspace of kda_chunk_fwd_windowed_ws:
  * a 1 KiB-aligned chunk index, window_chunks * H records of 88.75 KiB and
  * 2 * H carry states of 64 KiB.  0 for arguments off the tensor-core path or

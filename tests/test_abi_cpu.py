@@ -259,6 +259,15 @@ def test_chunk_fwd_windowed_workspace_and_bad_arguments(kda):
     f32 = (q, k, v, g, beta, 1.0, None, None, 1, T, H, 128, 128, 64, 0, o, None)
     st = L.kda_chunk_fwd_windowed_ws(*f32, W, ws, need, None)
     assert st == kda.KDA_ERR_UNSUPPORTED
+    # the fused form: x [T, 3*H*128] bf16, conv weights, g, beta, o
+    x, cw = _vp(0x2000000), _vp(0x3000000)
+    fargs = (x, cw, None, None, g, beta, 1.0, None, None, 1, T, H, 128, 1, o, None)
+    st = L.kda_prologue_chunk_fwd_windowed_ws(*fargs, 0, ws, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"window_chunks" in L.kda_last_error()
+    st = L.kda_prologue_chunk_fwd_windowed_ws(*fargs, W, None, need, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace is NULL" in L.kda_last_error()
+    st = L.kda_prologue_chunk_fwd_windowed_ws(*fargs, W, ws, need - 16, None)
+    assert st == kda.KDA_ERR_INVALID_ARG and b"workspace holds" in L.kda_last_error()
 
 
 def test_chunk_fwd_ws_rejects_bad_workspace(kda):

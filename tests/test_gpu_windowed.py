@@ -103,3 +103,35 @@ def test_windowed_dirty_workspace_is_deterministic(kda):
     ws.random_(0, 256, generator=g)
     second = run(kda, inp, window=3, workspace=ws)
     assert torch.equal(first[0], second[0]) and torch.equal(first[1], second[1])
+
+
+@pytest.mark.parametrize("window", [1, 3, 17])
+def test_windowed_fused_matches_unsplit(kda, window):
+    """The prologue inside the prep pass, one window at a time: read-out, final state and
+    conv cache equal the two-pass fused call's.  Five sequences x 32 heads give 640 state
+    chains, so the unwindowed call runs whole sequences too."""
+    lengths = [300, 0, 1, 700, 129]
+    H, D = 32, 128
+    assert kda.lib.kda_chunk_fwd_segment_chunks(len(lengths), sum(lengths), H) == 0
+    T, N, C = sum(lengths), len(lengths), 3 * H * D
+    r = torch.Generator().manual_seed(75)
+    x = torch.randn((T, C), generator=r).to(torch.bfloat16).to(DEV)
+    w = (0.5 * torch.randn((C, 4), generator=r)).to(DEV)
+    g = (-5.0 * torch.sigmoid(torch.randn((T, H, D), generator=r) - 3.0)).to(DEV)
+    beta = torch.sigmoid(torch.randn((T, H), generator=r)).to(DEV)
+    cache_in = torch.randn((N, 3, C), generator=r).to(torch.bfloat16).to(DEV)
+    s0 = (0.1 * torch.randn((N, H, D, D), generator=r)).to(DEV)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32).to(DEV)
+    outs = []
+    for win in (None, window):
+        o = torch.full((T, H, D), float("nan"), device=DEV)
+        fs = torch.empty((N, H, D, D), device=DEV)
+        cache_out = torch.empty_like(cache_in)
+        kda.kda_prologue_chunk_fwd(x, w, g, beta, o, H=H, D=D, scale=0.5, cache_in=cache_in,
+                                   cache_out=cache_out, initial_state=s0, final_state=fs,
+                                   cu_seqlens=cu, window_chunks=win)
+        torch.cuda.synchronize()
+        assert kda.kda_get_device_status() == 0
+        outs.append((o.cpu(), fs.cpu(), cache_out.cpu()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
