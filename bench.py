@@ -62,18 +62,20 @@ CHUNK_FLOPS_PER_TH = 139392                        # chunk form, d=128, C=64
 DECODE_BYTES_PER_SH = 2 * D_ * D_ * 4 + 3 * D_ * 2 + 2 * 3 * 3 * D_ * 2 + D_ * 4 + 4 + D_ * 4
 
 _CSRC = "gated_delta_rule_prologue_b200/csrc/"
+# the device headers every kernel file includes
+_HDRS = [_CSRC + "kda_common.cuh", _CSRC + "kda_tcgen05.cuh", _CSRC + "kda_chunk_record.cuh"]
 KERNEL_SOURCES = {
-    "kda_prologue_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
-    "kda_prologue_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
-    "kda_prologue": [_CSRC + "kda_prologue.cu"],
-    "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
-    "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"],
-    "kda_chunk_fwd_gated": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
-    "kda_output_epilogue": [_CSRC + "kda_epilogue.cu"],
+    "kda_prologue_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"] + _HDRS,
+    "kda_prologue_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"] + _HDRS,
+    "kda_prologue": [_CSRC + "kda_prologue.cu"] + _HDRS,
+    "kda_chunk_fwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"] + _HDRS,
+    "kda_chunk_fwd_one_pass": [_CSRC + "kda_chunk_tc.cu"] + _HDRS,
+    "kda_chunk_fwd_gated": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"] + _HDRS,
+    "kda_output_epilogue": [_CSRC + "kda_epilogue.cu"] + _HDRS,
     "kda_chunk_bwd": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu",
-                      _CSRC + "kda_chunk_bwd.cu"],
-    "kda_decode_step": [_CSRC + "kda_decode.cu"],
-    "kda_chunk_fwd_windowed64": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"],
+                      _CSRC + "kda_chunk_bwd.cu"] + _HDRS,
+    "kda_decode_step": [_CSRC + "kda_decode.cu"] + _HDRS,
+    "kda_chunk_fwd_windowed64": [_CSRC + "kda_chunk_tc.cu", _CSRC + "kda_chunk_state.cu"] + _HDRS,
 }
 
 
